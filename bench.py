@@ -1,0 +1,405 @@
+#!/usr/bin/env python3
+"""Benchmark of the shifted-window attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl native|reference]
+
+A step is one call of swin_window_attn_fwd (the whole hot path: CPB
+evaluation where the workload has one, then the attention kernel) over one
+batch of the workload, inputs resident in HBM.  L2 is flushed (a 256 MB
+write) before every timed step; each step is timed with CUDA events on the
+library's stream.  For N > 1 (torchrun) every rank runs its own batch (weak
+scaling, no collective on the data path) and the time is the max over ranks.
+
+Prints one JSON line.  ``--impl reference`` times the CPU oracle (the
+project's plain double-precision statement of the method) on the host cores
+on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vision_transformer_shifted_window_b200 import synthetic as syn  # noqa: E402
+
+METRIC = "window-attn fwd tokens/s and TFLOP/s (bf16, 1 B200) as % of tensor roofline"
+DEFAULT_WORKLOAD = 3  # FlashSwin dense tokens, M=32: the tensor-bound workload
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per workload
+# ---------------------------------------------------------------------------
+def _seg_lengths(L, M, s):
+    if s == 0:
+        starts = list(range(0, L, M))
+    else:
+        starts = [0] + list(range(s, L, M))
+    ends = starts[1:] + [L]
+    return [b - a for a, b in zip(starts, ends) if b > a]
+
+
+def _window_counts(L, M, s):
+    """Real tokens per rolled-frame window along one axis (Swin's count)."""
+    Lp = -(-L // M) * M
+    out = []
+    for w in range(Lp // M):
+        out.append(sum(1 for u in range(w * M, w * M + M) if (u + s) % Lp < L))
+    return out
+
+
+def work(w: syn.Workload, B=None):
+    B = w.B if B is None else B
+    s = w.shifts[0]
+    win = sum(n * n for n in _window_counts(w.H, w.M, s)) * sum(n * n for n in _window_counts(w.W, w.M, s))
+    exact = sum(n * n for n in _seg_lengths(w.H, w.M, s)) * sum(n * n for n in _seg_lengths(w.W, w.M, s))
+    C = w.heads * w.d
+    esz = 4 if w.dtype == "f32" else 2
+    return {
+        "tokens": B * w.H * w.W,
+        "flops_std": 4.0 * w.d * w.heads * B * win,      # masked pairs in a window included
+        "flops_exact": 4.0 * w.d * w.heads * B * exact,  # only pairs that enter a softmax
+        "exps": float(w.heads * B * exact),
+        "bytes": float(4 * esz * C * B * w.H * w.W),     # Q, K, V read once, O written once
+    }
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def read_traffic(kernel: str, workload: syn.Workload):
+    """dram read+write bytes per launch from a committed ncu summary, if the
+    summary was taken on the current kernel source (else None)."""
+    fn = os.path.join(ROOT, "profiles", "%s_%s.txt" % (kernel, workload.name))
+    if not os.path.exists(fn):
+        return None
+    kv = {}
+    for line in open(fn):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    src = os.path.join(ROOT, "vision_transformer_shifted_window_b200", "csrc", kv.get("source_file", ""))
+    if not os.path.isfile(src) or "source_sha1" not in kv or "dram_bytes_per_launch" not in kv:
+        return None
+    if hashlib.sha1(open(src, "rb").read()).hexdigest() != kv["source_sha1"]:
+        return None
+    return float(kv["dram_bytes_per_launch"])
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", "swin_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons, n = [], None, set(), 0
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            n += 1
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+def make_device_inputs(w: syn.Workload, device, rank: int):
+    import torch
+    inp = syn.make_inputs(w, seed=1000 + w.index + 7919 * rank)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    q, k, v = (dev(inp[n]).to(dt) for n in ("q", "k", "v"))
+    kw = {}
+    if "tau" in inp:
+        kw["tau"] = dev(inp["tau"])
+    if "table" in inp:
+        kw["bias_table"] = dev(inp["table"])
+    if "w1" in inp:
+        kw["cpb"] = tuple(dev(inp[n]) for n in ("w1", "b1", "w2", "b2"))
+    if "rope_freqs" in inp:
+        kw["rope_freqs"] = dev(inp["rope_freqs"])
+    return q, k, v, kw
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_native(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from vision_transformer_shifted_window_b200 import swin_attn as sa
+    from vision_transformer_shifted_window_b200 import build as swin_build
+
+    swin_build.build()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    w = syn.WORKLOADS[args.workload]
+    s = w.shifts[0]
+    q, k, v, kw = make_device_inputs(w, device, rank)
+    out = torch.empty_like(q)
+    ws_bytes = sa.swin_window_attn_workspace_size(w.M, w.heads, w.mode, "bias_table" in kw)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.Stream(device)
+    launches_per_step = 2 if "cpb" in kw else 1
+
+    def step():
+        sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, workspace=ws, stream=stream, **kw)
+
+    def timed_loop(fn, n, flush_l2=True):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        with torch.cuda.stream(stream):
+            for i in range(n):
+                if flush_l2:
+                    flush.fill_(i & 0xFF)
+                evs[i][0].record(stream)
+                fn()
+                evs[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        return [a.elapsed_time(b) for a, b in evs]
+
+    # warm-up (untimed)
+    timed_loop(step, max(args.warmup, 3))
+    assert sa.swin_stream_status(stream) == 0
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    times = timed_loop(step, args.steps)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        dist.barrier()
+    # keep the GPU busy a little longer for the clock record when the timed loop was short
+    t_soak = time.time()
+    while sum(times) < 1500.0 and time.time() - t_soak < 2.0:
+        timed_loop(step, 20)
+    clocks = sampler.stop()
+    st = sa.swin_stream_status(stream)
+    if st != 0:
+        raise RuntimeError("device status %d after timed loop" % st)
+
+    ms = max_over_ranks(sum(times) / len(times), world, device)
+    wk = work(w)
+    tokens = wk["tokens"] * world
+    value = tokens / (ms * 1e-3)
+    tflops = wk["flops_std"] * world / (ms * 1e-3) / 1e12
+    peaks = read_peaks()
+
+    # dominant kernel alone: the attention kernel with the bias table given
+    if "cpb" in kw:
+        table = sa.swin_cpb_eval(w.M, w.heads, *kw["cpb"])
+        kw_k = {kk: vv for kk, vv in kw.items() if kk != "cpb"}
+        kw_k["bias_table"] = table
+
+        def kstep():
+            sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, stream=stream, **kw_k)
+        timed_loop(kstep, 5)
+        ktimes = timed_loop(kstep, max(10, min(args.steps, 200)))
+    else:
+        ktimes = times
+    k_ms = max_over_ranks(sum(ktimes) / len(ktimes), world, device)
+    achieved = wk["flops_std"] / (k_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+                "traffic": read_traffic("attn", w), "peak_source": peaks["source"] + " (burst)",
+                "kernel_ms": round(k_ms, 5),
+                "hbm_achieved_gbs": round(wk["bytes"] / (k_ms * 1e-3) / 1e9, 1),
+                "hbm_frac": round(wk["bytes"] / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "attainable_frac": round(achieved / min(peaks["bf16_tflops"],
+                                                        peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3), 4)}
+
+    # end to end through host buffers: H2D of q/k/v, the call, D2H of out
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        step()
+        hout.copy_(out, non_blocking=True)
+    timed_loop(e2e_step, 3, flush_l2=False)
+    n_e2e = max(3, min(args.steps, 20))
+    etimes = timed_loop(e2e_step, n_e2e, flush_l2=False)
+    e_ms = max_over_ranks(sum(etimes) / len(etimes), world, device)
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = out.numel() * out.element_size()
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d,
+                   "M": w.M, "shift": s, "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode],
+                   "global_batch": w.B * world, "parallelism": "replicas x%d" % world,
+                   "l2": "flushed before every timed step (256 MB write)"},
+        "tflops": round(tflops, 2), "tflops_exact_pairs": round(wk["flops_exact"] * world / (ms * 1e-3) / 1e12, 2),
+        "roofline": roofline,
+        "e2e": {"value": round(tokens / (e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
+        "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+    }
+    return line, w
+
+
+def run_cpu_baseline(w: syn.Workload, budget_s: float):
+    """Time the oracle on a bounded, seeded sample of the workload's queries."""
+    import oracle
+    inp = syn.make_inputs(w, B=1)
+    s = w.shifts[0]
+    table = None
+    if "table" in inp:
+        table = inp["table"]
+    elif "w1" in inp:
+        table = oracle.cpb_table(w.M, w.heads, inp["w1"], inp["b1"], inp["w2"], inp["b2"])
+    rng = np.random.default_rng(99)
+
+    def run(nq):
+        ids = rng.integers(0, w.H * w.W, nq)
+        t0 = time.perf_counter()
+        oracle.window_attn(inp["q"], inp["k"], inp["v"], w.M, s, w.mode, tau=inp.get("tau"), table=table,
+                           rope_freqs=inp.get("rope_freqs"), queries=ids)
+        return time.perf_counter() - t0
+
+    nq = 64
+    t = run(nq)
+    while t < 0.5 and nq < w.H * w.W:
+        nq *= 4
+        t = run(nq)
+    nq = int(min(w.H * w.W * w.B, max(nq, nq * budget_s / max(t, 1e-6))))
+    t = run(nq)
+    return {"value": round(nq / t, 2), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d random query tokens (all %d heads) of one %dx%d image, %.1f s" % (nq, w.heads, w.H, w.W, t),
+            "seconds": round(t, 2)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=("native", "reference"))
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work to time")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--others", action="store_true", help="also time the other bf16 workloads")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = syn.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        budget = max(1.0, min(60.0, args.cpu_budget * max(1, args.steps) / 10.0))
+        cb = run_cpu_baseline(w, budget)
+        line = {"metric": METRIC, "impl": "reference", "value": cb["value"], "unit": "tokens/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d,
+                           "M": w.M, "shift": w.shifts[0]},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    line, w = run_native(args, rank, world, local_rank)
+    if args.others and rank == 0:
+        others = []
+        for idx in sorted(syn.WORKLOADS):
+            if idx == args.workload or syn.WORKLOADS[idx].dtype != "bf16":
+                continue
+            a2 = argparse.Namespace(**vars(args))
+            a2.workload = idx
+            a2.steps = min(args.steps, 100)
+            l2, _ = run_native(a2, 0, 1, local_rank)
+            others.append({"workload": l2["config"]["workload"], "tokens_per_s": l2["value"],
+                           "tflops": l2["tflops"], "ms_per_step": l2["ms_per_step"],
+                           "kernel_frac_of_tensor_peak": l2["roofline"]["frac"],
+                           "kernel_hbm_frac": l2["roofline"]["hbm_frac"]})
+        line["other_workloads"] = others
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = run_cpu_baseline(w, args.cpu_budget)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

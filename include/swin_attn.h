@@ -1,0 +1,165 @@
+/*
+ * swin_attn.h — C ABI of libswinattn.so: shifted-window multi-head
+ * self-attention (forward) on a 2-D token grid, for NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For an image b, head h and query token i at grid
+ * position (y_i, x_i), the attended keys are the tokens j that share i's
+ * segment on both axes, where each axis of length L is cut at s + kM
+ * (k integer) and clipped to [0, L).  This is the attention that Swin's
+ * cyclic shift by s, MxM window partition and region mask give; here the
+ * shift and partition are index arithmetic, nothing is rolled or copied.
+ * Padding never exists: a grid side that M does not divide ends in a shorter
+ * segment.  The score of a pair (i, j) is
+ *   SWIN_MODE_DOT_BIAS   q.k / sqrt(d) + T[r(i,j)][h]
+ *        "Swin Transformer V2: Scaling Up Capacity and Resolution", eq. 1;
+ *   SWIN_MODE_COSINE_CPB cos(q, k) / max(tau_h, 0.01) + T[r(i,j)][h]
+ *        same page, §3.2 / eq. 2 and the window_attention pseudocode; T is
+ *        either given or produced by the Log-CPB meta network G of §3.3
+ *        (eq. 3, eq. 4), see swin_cpb_eval;
+ *   SWIN_MODE_ROPE       (R(p_i) q).(R(p_j) k) / sqrt(d), no bias
+ *        "FLASHSWIN ..." abstract: window-local learnable 2-D RoPE with exact
+ *        softmax attention and no materialised score matrix.
+ * followed by a softmax over the attended keys and a weighted sum of v.
+ * r(i,j) = (dy + M - 1) * (2M - 1) + (dx + M - 1) with (dy, dx) = query
+ * position minus key position.  RoPE: channels [0, d/2) rotate pairs
+ * (2t, 2t+1) by p_y * w[0][t], channels [d/2, d) by p_x * w[1][t], t < d/4,
+ * with window-local coordinates p = (coordinate - s) mod M.
+ *
+ * Memory.  Every tensor pointer is DEVICE memory owned by the caller.  Q, K,
+ * V and O are dense row-major [B][H][W][heads][d] (channel fastest), Q, K, V
+ * of one dtype (fp32 or bf16), O of the same dtype or fp32; 16-byte aligned;
+ * O must not overlap Q, K or V.
+ * The library allocates no device memory for a call; scratch comes from the
+ * caller's workspace (size from swin_window_attn_workspace_size).
+ *
+ * Streams and errors.  Calls are asynchronous on the given stream (NULL =
+ * legacy default stream) and return after enqueueing.  Argument errors return
+ * SWIN_ERR_INVALID_ARG or SWIN_ERR_UNSUPPORTED without launching anything;
+ * launch failures return SWIN_ERR_CUDA.  Kernels never trap: a bounded wait
+ * that runs out records SWIN_ERR_TIMEOUT in a device status word, which
+ * swin_stream_status reads (after synchronising the stream) and clears.
+ * swin_last_error returns a message for the last failure on this host thread.
+ */
+#ifndef SWIN_ATTN_H
+#define SWIN_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Binary-compatible with cudaStream_t / CUstream. */
+typedef struct CUstream_st* swin_stream_t;
+
+typedef enum {
+  SWIN_OK = 0,
+  SWIN_ERR_INVALID_ARG = 1, /* bad shape, pointer, alignment or value */
+  SWIN_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels cover */
+  SWIN_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed */
+  SWIN_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out */
+} swin_status;
+
+typedef enum {
+  SWIN_MODE_DOT_BIAS = 0,
+  SWIN_MODE_COSINE_CPB = 1,
+  SWIN_MODE_ROPE = 2
+} swin_mode;
+
+typedef enum { SWIN_F32 = 0, SWIN_BF16 = 1 } swin_dtype;
+
+/* Weights of the Log-CPB meta network G ("Swin Transformer V2", §3.3, eq. 3):
+ *   G(dx_hat, dy_hat) = w2 . relu(w1 . (dx_hat, dy_hat) + b1) + b2
+ * with dx_hat = sign(dx) * ln(1 + |dx|) (eq. 4).  All device fp32:
+ *   w1 [hidden][2], b1 [hidden] or NULL (zero), w2 [heads][hidden],
+ *   b2 [heads] or NULL (zero).  The page's code uses hidden = 512. */
+typedef struct {
+  int hidden;
+  const float* w1;
+  const float* b1;
+  const float* w2;
+  const float* b2;
+} swin_cpb_weights;
+
+/* swin_cpb_eval — evaluate G once for every offset of an MxM window and store
+ * the bias table ("Swin Transformer V2", §3.3: precompute the biases for
+ * inference; eq. 3, eq. 4).
+ *   M          window size, 1 <= M <= 64
+ *   heads      1 <= heads <= 64
+ *   g          weights (device pointers), 1 <= g->hidden <= 4096
+ *   table_out  device fp32 [(2M-1)^2][heads], row (dy+M-1)*(2M-1)+(dx+M-1)
+ * Computed in fp32 with the CUDA math library's logarithm. */
+swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* table_out,
+                          swin_stream_t stream);
+
+/* swin_window_attn_fwd — the shifted-window attention forward pass.
+ *   q, k, v, out   device [B][H][W][heads][d]; q, k, v of dtype dt, out of
+ *                  dtype out_dt (out_dt == dt, or SWIN_F32 output for SWIN_BF16
+ *                  inputs: the same fp32 result before its final rounding;
+ *                  a bf16 output is that fp32 result rounded to nearest even)
+ *   B, H, W        batch and grid, each >= 1; B*H*W*heads*d < 2^31
+ *   heads, d       heads >= 1; d in {8, 16, 32, 64} for SWIN_F32; d == 32 for
+ *                  SWIN_BF16 (the tensor-core path); RoPE needs d % 4 == 0
+ *   M, shift       window size 1 <= M <= 64, shift 0 <= shift < M
+ *   mode           a swin_mode
+ *   tau            device fp32 [heads], SWIN_MODE_COSINE_CPB only (else NULL);
+ *                  the kernel uses max(tau, 0.01)
+ *   bias_table     device fp32 [(2M-1)^2][heads] or NULL (modes 0 and 1;
+ *                  NULL in mode 1 means "evaluate cpb"; NULL in mode 0 means
+ *                  no bias); must be NULL in SWIN_MODE_ROPE
+ *   cpb            mode 1 with bias_table == NULL: G's weights (host struct,
+ *                  device arrays); the table is evaluated into the workspace
+ *                  on the same stream; may be NULL otherwise
+ *   rope_freqs     device fp32 [2][d/4] (row axis, then column axis),
+ *                  SWIN_MODE_ROPE only
+ *   workspace      device scratch of at least
+ *                  swin_window_attn_workspace_size(...) bytes, 256-byte
+ *                  aligned (may be NULL when that size is 0)
+ *   stream         CUDA stream
+ * Asynchronous; q/k/v must stay valid until the stream reaches the call. */
+swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                 swin_dtype dt, swin_dtype out_dt, int B, int H, int W,
+                                 int heads, int d,
+                                 int M, int shift, swin_mode mode,
+                                 const float* tau, const float* bias_table,
+                                 const swin_cpb_weights* cpb, const float* rope_freqs,
+                                 void* workspace, size_t workspace_bytes,
+                                 swin_stream_t stream);
+
+/* Bytes of workspace swin_window_attn_fwd needs for these arguments
+ * (have_table: whether bias_table is non-NULL).  0 when none is needed. */
+size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int have_table);
+
+/* swin_index_tables — Swin's bookkeeping for an HxW grid in the rolled frame
+ * (pad to Hp = ceil(H/M)*M, Wp likewise; roll by -shift; cut MxM windows), as
+ * the kernels' index arithmetic sees it.  For testing; any output may be NULL.
+ *   tok_window [H][W]  window id (u / M) * (Wp / M) + (v / M), with
+ *                      u = (y - shift) mod Hp, v = (x - shift) mod Wp
+ *   tok_region [H][W]  band label ry * 3 + rx; along an axis the band is 0
+ *                      for u < Hp - M, 1 for u < Hp - shift, else 2 (0 when
+ *                      shift == 0)
+ *   tok_local  [H][W]  (u mod M) * M + (v mod M)
+ *   rel_index  [M*M][M*M]  r(i, j) for window-local positions i, j
+ * All int32 device arrays.  1 <= M <= 64, 0 <= shift < M, H, W >= 1. */
+swin_status swin_index_tables(int H, int W, int M, int shift, int32_t* tok_window,
+                              int32_t* tok_region, int32_t* tok_local, int32_t* rel_index,
+                              swin_stream_t stream);
+
+/* Synchronise the stream, then return and clear the device status word of the
+ * current device (SWIN_OK, or SWIN_ERR_TIMEOUT if a kernel's bounded wait ran
+ * out since the last call); SWIN_ERR_CUDA if the synchronisation failed. */
+swin_status swin_stream_status(swin_stream_t stream);
+
+/* Message describing the last non-OK status returned on this host thread
+ * ("" if none).  The pointer stays valid until the next call on the thread. */
+const char* swin_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int swin_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWIN_ATTN_H */

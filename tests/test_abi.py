@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI (no GPU needed): the library builds, loads,
+exports every function include/swin_attn.h declares, and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vision_transformer_shifted_window_b200 import build as swin_build
+from vision_transformer_shifted_window_b200 import swin_attn as sa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    swin_build.build()
+    return sa.lib()
+
+
+def declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            src = open(os.path.join(inc, fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(swin_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert names, "no declarations found"
+    assert names == set(sa.EXPORTED)
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.swin_version() >= 100
+
+
+def test_workspace_size_rules(L):
+    assert sa.swin_window_attn_workspace_size(16, 3, sa.SWIN_MODE_COSINE_CPB, False) == 31 * 31 * 3 * 4 + 244
+    assert sa.swin_window_attn_workspace_size(16, 3, sa.SWIN_MODE_COSINE_CPB, True) == 0
+    assert sa.swin_window_attn_workspace_size(16, 3, sa.SWIN_MODE_ROPE, False) == 0
+    assert sa.swin_window_attn_workspace_size(16, 3, sa.SWIN_MODE_DOT_BIAS, False) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def call_fwd(L, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, out=FAKE * 64, dt=sa.SWIN_BF16, B=1, H=8, W=8, heads=1,
+             d=32, M=4, shift=2, mode=sa.SWIN_MODE_DOT_BIAS, tau=None, table=None, cpb=None,
+             rope=None, ws=None, wsb=0)
+    a.update(kw)
+    return L.swin_window_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["dt"], a.get("odt", a["dt"]), a["B"], a["H"], a["W"],
+                                  a["heads"], a["d"], a["M"], a["shift"], a["mode"], a["tau"],
+                                  a["table"], a["cpb"], a["rope"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(q=None), "NULL"), (dict(shift=4), "shift"), (dict(shift=-1), "shift"), (dict(M=0), "M"),
+    (dict(M=65, shift=0), "M"), (dict(B=0), ">= 1"), (dict(q=FAKE + 8), "aligned"),
+    (dict(out=FAKE * 2), "overlaps"), (dict(mode=1), "tau"), (dict(mode=2), "rope"),
+    (dict(mode=2, rope=FAKE * 5, d=30), "d % 4"), (dict(mode=2, rope=FAKE * 5, table=FAKE * 6), "no bias"),
+    (dict(mode=7), "mode"), (dict(dt=5), "dtype"), (dict(dt=0, odt=1), "output dtype"),
+])
+def test_rejects_bad_arguments(L, kw, why):
+    rc = call_fwd(L, **kw)
+    assert rc == sa.SWIN_ERR_INVALID_ARG
+    assert why in L.swin_last_error().decode()
+
+
+def test_cpu_entry_points_reject_before_launch(L):
+    assert L.swin_index_tables(8, 8, 4, 4, None, None, None, None, None) == sa.SWIN_ERR_INVALID_ARG
+    assert L.swin_cpb_eval(0, 3, None, FAKE, None) == sa.SWIN_ERR_INVALID_ARG
+    w = sa.swin_cpb_weights(0, FAKE, None, FAKE, None)
+    assert L.swin_cpb_eval(8, 3, ctypes.byref(w), FAKE, None) == sa.SWIN_ERR_INVALID_ARG
+    assert "hidden" in L.swin_last_error().decode()
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 4, 1, 32)
+    with pytest.raises(ValueError):
+        sa.swin_window_attn_fwd(x, x, x, 4, 0, 0)

@@ -1,0 +1,224 @@
+// Shifted-window attention on the CUDA cores, in fp32 arithmetic.
+//
+// This is the path for fp32 tensors (and for bf16 tensors with d != 32),
+// where the tensor cores' bf16/tf32 inputs would not meet fp32 accuracy.
+// Scores follow "Swin Transformer V2" eq. 1 (mode 0) and eq. 2 (mode 1,
+// tau clamped at 0.01, §3.2), or FlashSwin's window-local 2-D RoPE
+// (mode 2); the softmax is the exact online form FlashSwin relies on: a
+// running maximum and rescaled running sums, so no score row is stored.
+//
+// Decomposition: one CTA of 128 threads per (image, head, rectangle, block of
+// 128 queries); a rectangle is one segment per axis of the shifted partition
+// (see swin_index.cuh), i.e. one independent attention problem of up to M*M
+// tokens.  Each thread owns one query row; keys and values stream through
+// shared memory 32 at a time (normalised or rotated once per key), and
+// every thread reads them as broadcasts.
+#include "swin_common.cuh"
+
+namespace swin {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kKeyTile = 32;
+constexpr int kMaxM = 64;
+
+template <typename T>
+__device__ __forceinline__ float load_elem(const T* p);
+template <>
+__device__ __forceinline__ float load_elem<float>(const float* p) {
+  return __ldg(p);
+}
+template <>
+__device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+template <typename T>
+__device__ __forceinline__ T store_conv(float x);
+template <>
+__device__ __forceinline__ float store_conv<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 store_conv<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Rotate channel pairs of one half (row or column axis) by position p.
+template <int D>
+__device__ __forceinline__ void rope_rotate(float* x, int half, int p, const float* cs,
+                                            const float* sn) {
+  constexpr int Q = D / 4;
+#pragma unroll
+  for (int t = 0; t < Q; ++t) {
+    float c = cs[p * Q + t], s = sn[p * Q + t];
+    float a = x[half * (D / 2) + 2 * t], b = x[half * (D / 2) + 2 * t + 1];
+    x[half * (D / 2) + 2 * t] = a * c - b * s;
+    x[half * (D / 2) + 2 * t + 1] = a * s + b * c;
+  }
+}
+
+template <typename T, typename TO, int D, int MODE>
+__global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx, int chunks) {
+  __shared__ float ks[kKeyTile][D];
+  __shared__ float vs[kKeyTile][D];
+  // RoPE tables: [axis][p][t] for p < M, t < D/4
+  __shared__ float rcos[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
+  __shared__ float rsin[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
+
+  const int M = a.M, s = a.shift;
+  const int rect = blockIdx.x / chunks, chunk = blockIdx.x % chunks;
+  const int sy = rect / nsx, sx = rect % nsx;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int y0 = swin_seg_start(sy, M, s), ly = swin_seg_len(sy, a.H, M, s);
+  const int x0 = swin_seg_start(sx, M, s), lx = swin_seg_len(sx, a.W, M, s);
+  const int n = ly * lx;
+  if (chunk * kThreads >= n) return;  // whole CTA idle (uniform)
+  const int C = a.heads * D;
+  const T* Q = static_cast<const T*>(a.q);
+  const T* K = static_cast<const T*>(a.k);
+  const T* V = static_cast<const T*>(a.v);
+  TO* O = static_cast<TO*>(a.out);
+
+  if (MODE == 2) {
+    constexpr int Qd = D / 4;
+    for (int i = threadIdx.x; i < 2 * M * Qd; i += kThreads) {
+      int axis = i / (M * Qd), p = (i / Qd) % M, t = i % Qd;
+      float sv, cv;
+      sincosf((float)p * a.rope[axis * Qd + t], &sv, &cv);
+      rcos[axis * kMaxM * Qd + p * Qd + t] = cv;
+      rsin[axis * kMaxM * Qd + p * Qd + t] = sv;
+    }
+    __syncthreads();
+  }
+
+  const int qi = chunk * kThreads + threadIdx.x;
+  const bool active = qi < n;
+  const int yq = y0 + (active ? qi / lx : 0), xq = x0 + (active ? qi % lx : 0);
+  float q[D], o[D];
+  float inv_tau = 0.0f;
+  {
+    const T* src = Q + (((size_t)b * a.H + yq) * a.W + xq) * C + (size_t)h * D;
+#pragma unroll
+    for (int e = 0; e < D; ++e) q[e] = active ? load_elem(src + e) : 0.0f;
+  }
+  if (MODE == 1) {
+    float ss = 0.0f;
+#pragma unroll
+    for (int e = 0; e < D; ++e) ss = fmaf(q[e], q[e], ss);
+    float nrm = fmaxf(sqrtf(ss), kNormEps);
+#pragma unroll
+    for (int e = 0; e < D; ++e) q[e] = q[e] / nrm;
+    inv_tau = 1.0f / fmaxf(__ldg(a.tau + h), kTauMin);
+  }
+  if (MODE == 2) {
+    rope_rotate<D>(q, 0, swin_local_coord(yq, M, s), rcos, rsin);
+    rope_rotate<D>(q, 1, swin_local_coord(xq, M, s), rcos + kMaxM * (D / 4), rsin + kMaxM * (D / 4));
+  }
+  const float rsd = rsqrtf((float)D);
+#pragma unroll
+  for (int e = 0; e < D; ++e) o[e] = 0.0f;
+  float m = -INFINITY, l = 0.0f;
+
+  for (int j0 = 0; j0 < n; j0 += kKeyTile) {
+    const int nk = min(kKeyTile, n - j0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nk * D; i += kThreads) {
+      int j = i / D, e = i % D, kk = j0 + j;
+      size_t off = (((size_t)b * a.H + y0 + kk / lx) * a.W + x0 + kk % lx) * C + (size_t)h * D + e;
+      ks[j][e] = load_elem(K + off);
+      vs[j][e] = load_elem(V + off);
+    }
+    __syncthreads();
+    if (MODE != 0 && threadIdx.x < nk) {
+      float* kr = ks[threadIdx.x];
+      if (MODE == 1) {
+        float ss = 0.0f;
+        for (int e = 0; e < D; ++e) ss = fmaf(kr[e], kr[e], ss);
+        float nrm = fmaxf(sqrtf(ss), kNormEps);
+        for (int e = 0; e < D; ++e) kr[e] = kr[e] / nrm;
+      } else {
+        int kk = j0 + threadIdx.x;
+        float tmp[D];
+        for (int e = 0; e < D; ++e) tmp[e] = kr[e];
+        rope_rotate<D>(tmp, 0, swin_local_coord(y0 + kk / lx, M, s), rcos, rsin);
+        rope_rotate<D>(tmp, 1, swin_local_coord(x0 + kk % lx, M, s), rcos + kMaxM * (D / 4),
+                       rsin + kMaxM * (D / 4));
+        for (int e = 0; e < D; ++e) kr[e] = tmp[e];
+      }
+    }
+    __syncthreads();
+    if (!active) continue;
+    for (int j = 0; j < nk; ++j) {
+      float dot = 0.0f;
+#pragma unroll
+      for (int e = 0; e < D; ++e) dot = fmaf(q[e], ks[j][e], dot);
+      float lg;
+      if (MODE == 1)
+        lg = dot * inv_tau;
+      else
+        lg = dot * rsd;
+      if (MODE != 2 && a.table) {
+        int kk = j0 + j;
+        int r = swin_rel_row(yq - (y0 + kk / lx), xq - (x0 + kk % lx), M);
+        lg += __ldg(a.table + (size_t)r * a.heads + h);
+      }
+      if (lg > m) {
+        float c = expf(m - lg);
+        l = fmaf(l, c, 1.0f);
+#pragma unroll
+        for (int e = 0; e < D; ++e) o[e] = fmaf(o[e], c, vs[j][e]);
+        m = lg;
+      } else {
+        float p = expf(lg - m);
+        l += p;
+#pragma unroll
+        for (int e = 0; e < D; ++e) o[e] = fmaf(p, vs[j][e], o[e]);
+      }
+    }
+  }
+  if (active) {
+    float inv = 1.0f / l;
+    TO* dst = O + (((size_t)b * a.H + yq) * a.W + xq) * C + (size_t)h * D;
+#pragma unroll
+    for (int e = 0; e < D; ++e) dst[e] = store_conv<TO>(o[e] * inv);
+  }
+}
+
+template <typename T, typename TO, int D>
+swin_status launch_typed(const AttnArgs& a, cudaStream_t stream) {
+  const int nsy = swin_nseg(a.H, a.M, a.shift), nsx = swin_nseg(a.W, a.M, a.shift);
+  const int chunks = (a.M * a.M + kThreads - 1) / kThreads;
+  dim3 grid(nsy * nsx * chunks, a.heads, a.B);
+  switch (a.mode) {
+    case 0: attn_simt_kernel<T, TO, D, 0><<<grid, kThreads, 0, stream>>>(a, nsx, chunks); break;
+    case 1: attn_simt_kernel<T, TO, D, 1><<<grid, kThreads, 0, stream>>>(a, nsx, chunks); break;
+    default:
+      if constexpr (D % 4 == 0) attn_simt_kernel<T, TO, D, 2><<<grid, kThreads, 0, stream>>>(a, nsx, chunks);
+      break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_simt launch: %s", cudaGetErrorString(e));
+  return SWIN_OK;
+}
+
+template <typename T, typename TO>
+swin_status launch_d(const AttnArgs& a, cudaStream_t stream) {
+  switch (a.d) {
+    case 8: return launch_typed<T, TO, 8>(a, stream);
+    case 16: return launch_typed<T, TO, 16>(a, stream);
+    case 32: return launch_typed<T, TO, 32>(a, stream);
+    case 64: return launch_typed<T, TO, 64>(a, stream);
+    default: return fail(SWIN_ERR_UNSUPPORTED, "CUDA-core path supports d in {8,16,32,64}, got %d", a.d);
+  }
+}
+
+}  // namespace
+
+swin_status launch_attn_simt(const AttnArgs& a, bool bf16_in, bool f32_out, cudaStream_t stream) {
+  if (a.M > kMaxM) return fail(SWIN_ERR_UNSUPPORTED, "M=%d above %d", a.M, kMaxM);
+  if (!bf16_in) return launch_d<float, float>(a, stream);
+  return f32_out ? launch_d<__nv_bfloat16, float>(a, stream)
+                 : launch_d<__nv_bfloat16, __nv_bfloat16>(a, stream);
+}
+
+}  // namespace swin

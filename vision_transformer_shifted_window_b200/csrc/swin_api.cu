@@ -1,0 +1,165 @@
+// Host side of the C ABI declared in include/swin_attn.h: argument checks,
+// workspace layout, kernel selection and the device status word.
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "swin_common.cuh"
+
+namespace swin {
+
+namespace {
+thread_local std::string g_last_error;
+
+// One status word per device; kernels OR error codes into it, never trap.
+__device__ int g_status_word;
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_status_mu;
+
+}  // namespace
+
+swin_status fail(swin_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+int* status_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_status_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    g_status_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_status_ptr[dev];
+}
+
+}  // namespace swin
+
+using swin::fail;
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
+extern "C" {
+
+const char* swin_last_error(void) { return swin::g_last_error.c_str(); }
+
+int swin_version(void) { return 100; }
+
+swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* table_out,
+                          swin_stream_t stream) {
+  if (M < 1 || M > 64) return fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
+  if (heads < 1 || heads > 64) return fail(SWIN_ERR_INVALID_ARG, "heads=%d outside [1, 64]", heads);
+  if (!g) return fail(SWIN_ERR_INVALID_ARG, "cpb weights struct is NULL");
+  if (g->hidden < 1 || g->hidden > 4096)
+    return fail(SWIN_ERR_INVALID_ARG, "hidden=%d outside [1, 4096]", g->hidden);
+  if (!g->w1 || !g->w2 || !table_out)
+    return fail(SWIN_ERR_INVALID_ARG, "w1, w2 and table_out must be non-NULL");
+  return swin::launch_cpb_eval(M, heads, *g, table_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int have_table) {
+  if (mode != SWIN_MODE_COSINE_CPB || have_table || M < 1 || heads < 1) return 0;
+  size_t bytes = sizeof(float) * (size_t)(2 * M - 1) * (2 * M - 1) * heads;
+  return (bytes + 255) & ~size_t(255);
+}
+
+swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                 swin_dtype dt, swin_dtype out_dt, int B, int H, int W, int heads,
+                                 int d, int M,
+                                 int shift, swin_mode mode, const float* tau,
+                                 const float* bias_table, const swin_cpb_weights* cpb,
+                                 const float* rope_freqs, void* workspace,
+                                 size_t workspace_bytes, swin_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (!q || !k || !v || !out) return fail(SWIN_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  if (dt != SWIN_F32 && dt != SWIN_BF16) return fail(SWIN_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (out_dt != dt && !(dt == SWIN_BF16 && out_dt == SWIN_F32))
+    return fail(SWIN_ERR_INVALID_ARG, "output dtype %d not allowed for input dtype %d", (int)out_dt, (int)dt);
+  if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1)
+    return fail(SWIN_ERR_INVALID_ARG, "B, H, W, heads and d must be >= 1");
+  if (M < 1 || M > 64) return fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
+  if (shift < 0 || shift >= M) return fail(SWIN_ERR_INVALID_ARG, "shift=%d outside [0, M)", shift);
+  if (mode != SWIN_MODE_DOT_BIAS && mode != SWIN_MODE_COSINE_CPB && mode != SWIN_MODE_ROPE)
+    return fail(SWIN_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+  const long long elems = (long long)B * H * W * heads * d;
+  if (elems >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "B*H*W*heads*d must be < 2^31");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SWIN_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  const size_t bytes = (size_t)elems * (dt == SWIN_F32 ? 4 : 2);
+  const size_t obytes = (size_t)elems * (out_dt == SWIN_F32 ? 4 : 2);
+  if (overlaps(out, obytes, q, bytes) || overlaps(out, obytes, k, bytes) || overlaps(out, obytes, v, bytes))
+    return fail(SWIN_ERR_INVALID_ARG, "out overlaps q, k or v");
+  if (mode == SWIN_MODE_COSINE_CPB && !tau) return fail(SWIN_ERR_INVALID_ARG, "cosine mode needs tau");
+  if (mode == SWIN_MODE_ROPE) {
+    if (!rope_freqs) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode needs rope_freqs");
+    if (d % 4 != 0) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode needs d %% 4 == 0, got %d", d);
+    if (bias_table) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode takes no bias table");
+  }
+  if (cpb && (cpb->hidden < 1 || cpb->hidden > 4096 || !cpb->w1 || !cpb->w2))
+    return fail(SWIN_ERR_INVALID_ARG, "cpb weights incomplete or hidden outside [1, 4096]");
+  if (heads > 64 && mode == SWIN_MODE_COSINE_CPB && !bias_table && cpb)
+    return fail(SWIN_ERR_INVALID_ARG, "cpb evaluation supports heads <= 64");
+
+  const float* table = bias_table;
+  if (mode == SWIN_MODE_COSINE_CPB && !bias_table && cpb) {
+    size_t need = swin_window_attn_workspace_size(M, heads, mode, 0);
+    if (!workspace || workspace_bytes < need)
+      return fail(SWIN_ERR_INVALID_ARG, "workspace of %zu bytes needed, got %zu", need, workspace_bytes);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return fail(SWIN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    float* ws_table = static_cast<float*>(workspace);
+    swin_status s = swin::launch_cpb_eval(M, heads, *cpb, ws_table, st);
+    if (s != SWIN_OK) return s;
+    table = ws_table;
+  }
+  if (mode == SWIN_MODE_ROPE) table = nullptr;
+
+  swin::AttnArgs a;
+  a.q = q; a.k = k; a.v = v; a.out = out;
+  a.B = B; a.H = H; a.W = W; a.heads = heads; a.d = d; a.M = M; a.shift = shift; a.mode = (int)mode;
+  a.tau = tau; a.table = table; a.rope = rope_freqs;
+  a.status = swin::status_word();
+  if (!a.status) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
+  return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
+}
+
+swin_status swin_index_tables(int H, int W, int M, int shift, int32_t* tok_window,
+                              int32_t* tok_region, int32_t* tok_local, int32_t* rel_index,
+                              swin_stream_t stream) {
+  if (H < 1 || W < 1) return fail(SWIN_ERR_INVALID_ARG, "H and W must be >= 1");
+  if (M < 1 || M > 64) return fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
+  if (shift < 0 || shift >= M) return fail(SWIN_ERR_INVALID_ARG, "shift=%d outside [0, M)", shift);
+  if ((long long)H * W >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "H*W must be < 2^31");
+  return swin::launch_index_tables(H, W, M, shift, tok_window, tok_region, tok_local, rel_index,
+                                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+swin_status swin_stream_status(swin_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  int* w = swin::status_word();
+  if (!w) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
+  int val = 0, zero = 0;
+  if (cudaMemcpy(&val, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return fail(SWIN_ERR_CUDA, "reading the device status word failed");
+  if (val != 0) return fail((swin_status)val, "a kernel reported status %d (bounded wait ran out)", val);
+  return SWIN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,45 @@
+// Shared declarations of libswinattn's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/swin_attn.h"
+#include "swin_index.cuh"
+
+namespace swin {
+
+// Records a failure message for swin_last_error() and returns st.
+swin_status fail(swin_status st, const char* fmt, ...);
+
+// Device address of this device's status word (set up once per device).
+int* status_word();
+
+// fp32 RoPE tables are built in the kernels from the caller's frequencies.
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kTauMin = 0.01f;
+constexpr float kNormEps = 1e-12f;
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  int B, H, W, heads, d, M, shift, mode;
+  const float* tau;
+  const float* table;  // [(2M-1)^2][heads] or nullptr
+  const float* rope;   // [2][d/4] or nullptr
+  int* status;
+};
+
+// Launchers (one per translation unit).
+swin_status launch_cpb_eval(int M, int heads, const swin_cpb_weights& g, float* table,
+                            cudaStream_t stream);
+swin_status launch_index_tables(int H, int W, int M, int shift, int32_t* tw, int32_t* tr,
+                                int32_t* tl, int32_t* ri, cudaStream_t stream);
+swin_status launch_attn_simt(const AttnArgs& a, bool bf16_in, bool f32_out, cudaStream_t stream);
+
+}  // namespace swin

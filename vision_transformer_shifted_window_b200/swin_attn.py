@@ -1,0 +1,195 @@
+"""Python binding of libswinattn.so (include/swin_attn.h), argument marshalling only.
+
+Every function keeps its C name.  Tensors are torch CUDA tensors used as plain
+device buffers; the computation happens in the library's kernels on the
+current torch stream (or the stream passed in).  There is no fallback: if the
+shared library is missing or a call fails, a RuntimeError is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libswinattn.so")
+
+SWIN_OK = 0
+SWIN_ERR_INVALID_ARG = 1
+SWIN_ERR_UNSUPPORTED = 2
+SWIN_ERR_CUDA = 3
+SWIN_ERR_TIMEOUT = 4
+
+SWIN_MODE_DOT_BIAS = 0
+SWIN_MODE_COSINE_CPB = 1
+SWIN_MODE_ROPE = 2
+
+SWIN_F32 = 0
+SWIN_BF16 = 1
+
+#: every symbol include/swin_attn.h declares
+EXPORTED = ("swin_cpb_eval", "swin_window_attn_fwd", "swin_window_attn_workspace_size",
+            "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version")
+
+
+class SwinError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__("swin status %d: %s" % (status, msg))
+        self.status = status
+
+
+class swin_cpb_weights(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("w1", ctypes.c_void_p), ("b1", ctypes.c_void_p),
+                ("w2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """Load the shared library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libswinattn.so is not built; run "
+                               "`python -m vision_transformer_shifted_window_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
+        L.swin_cpb_eval.argtypes = [i, i, ctypes.POINTER(swin_cpb_weights), vp, st]
+        L.swin_cpb_eval.restype = i
+        L.swin_window_attn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp,
+                                           ctypes.POINTER(swin_cpb_weights), vp, vp,
+                                           ctypes.c_size_t, st]
+        L.swin_window_attn_fwd.restype = i
+        L.swin_window_attn_workspace_size.argtypes = [i, i, i, i]
+        L.swin_window_attn_workspace_size.restype = ctypes.c_size_t
+        L.swin_index_tables.argtypes = [i, i, i, i, vp, vp, vp, vp, st]
+        L.swin_index_tables.restype = i
+        L.swin_stream_status.argtypes = [st]
+        L.swin_stream_status.restype = i
+        L.swin_last_error.argtypes = []
+        L.swin_last_error.restype = ctypes.c_char_p
+        L.swin_version.argtypes = []
+        L.swin_version.restype = i
+        _lib = L
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != SWIN_OK:
+        raise SwinError(rc, lib().swin_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _f32(t: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if t is None:
+        return None
+    if t.dtype != torch.float32:
+        raise ValueError("parameter tensors must be float32")
+    return t.contiguous()
+
+
+def _cpb_struct(cpb: Optional[Tuple[torch.Tensor, ...]]):
+    if cpb is None:
+        return None, ()
+    w1, b1, w2, b2 = (_f32(t) for t in cpb)
+    s = swin_cpb_weights(int(w1.shape[0]), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
+    return s, (w1, b1, w2, b2)
+
+
+def swin_version() -> int:
+    return int(lib().swin_version())
+
+
+def swin_last_error() -> str:
+    return lib().swin_last_error().decode()
+
+
+def swin_window_attn_workspace_size(M: int, heads: int, mode: int, have_table: bool) -> int:
+    return int(lib().swin_window_attn_workspace_size(M, heads, mode, int(bool(have_table))))
+
+
+def swin_cpb_eval(M: int, heads: int, w1, b1, w2, b2, out: Optional[torch.Tensor] = None,
+                  stream=None) -> torch.Tensor:
+    """Evaluate the Log-CPB MLP for every offset -> fp32 [(2M-1)^2, heads]."""
+    R = 2 * M - 1
+    if out is None:
+        out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
+    s, keep = _cpb_struct((w1, b1, w2, b2))
+    _check(lib().swin_cpb_eval(M, heads, ctypes.byref(s), _ptr(out), _stream(stream)))
+    del keep
+    return out
+
+
+def swin_window_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int,
+                         mode: int, tau: Optional[torch.Tensor] = None,
+                         bias_table: Optional[torch.Tensor] = None, cpb=None,
+                         rope_freqs: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None, stream=None,
+                         out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
+    """Shifted-window attention forward; q, k, v, out are [B, H, W, heads, d].
+
+    ``out_dtype`` (or the dtype of ``out``) may be float32 for bfloat16 inputs."""
+    if q.dtype == torch.float32:
+        dt = SWIN_F32
+    elif q.dtype == torch.bfloat16:
+        dt = SWIN_BF16
+    else:
+        raise ValueError("q, k, v must be float32 or bfloat16")
+    if k.dtype != q.dtype or v.dtype != q.dtype or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share dtype and shape")
+    if q.dim() != 5:
+        raise ValueError("q, k, v must be [B, H, W, heads, d]")
+    B, H, W, heads, d = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if out.shape != q.shape:
+        raise ValueError("out must have q's shape")
+    odt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(out.dtype)
+    if odt is None:
+        raise ValueError("out must be float32 or bfloat16")
+    tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
+    cs, keep = _cpb_struct(cpb)
+    need = swin_window_attn_workspace_size(M, heads, mode, bias_table is not None) if cs else 0
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().swin_window_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
+        _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
+        _ptr(rope_freqs), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc)
+    del keep
+    return out
+
+
+def swin_index_tables(H: int, W: int, M: int, shift: int, device="cuda", stream=None):
+    """(tok_window, tok_region, tok_local) int32 [H, W] and rel_index int32 [M*M, M*M]."""
+    mk = lambda *s: torch.empty(s, dtype=torch.int32, device=device)
+    tw, tr, tl, ri = mk(H, W), mk(H, W), mk(H, W), mk(M * M, M * M)
+    _check(lib().swin_index_tables(H, W, M, shift, _ptr(tw), _ptr(tr), _ptr(tl), _ptr(ri),
+                                   _stream(stream)))
+    return tw, tr, tl, ri
+
+
+def swin_stream_status(stream=None) -> int:
+    """Synchronise and return/clear the device status word (0 = OK)."""
+    return int(lib().swin_stream_status(_stream(stream)))
