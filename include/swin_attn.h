@@ -127,6 +127,27 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
                                  void* workspace, size_t workspace_bytes,
                                  swin_stream_t stream);
 
+/* swin_window_attn_fwd_noalloc — the same forward pass for callers that
+ * cannot allocate device memory (a framework that owns every device byte
+ * through its own pool, code running under stream capture, an embedding that
+ * forbids allocation after start-up).  The pages have no counterpart: it only
+ * changes where scratch lives.  Arguments as swin_window_attn_fwd, without a
+ * workspace.  When the cosine mode must evaluate the CPB meta network, the
+ * table goes into a fixed device array of the library (131072 floats, 512 KiB,
+ * held on every GPU that loads the library until exit) instead of caller
+ * scratch; (2M-1)^2 * heads above 131072 returns SWIN_ERR_UNSUPPORTED.  The
+ * first call on a device looks the array's address up (cudaGetSymbolAddress)
+ * and should come before any stream capture.  All calls share the array, and
+ * calls whose kernels overlap on the GPU race on it: serialise them.  Every
+ * table entry is rewritten on each call; the array keeps the last call's
+ * table.  Allocates nothing. */
+swin_status swin_window_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                         swin_dtype dt, swin_dtype out_dt, int B, int H, int W,
+                                         int heads, int d, int M, int shift, swin_mode mode,
+                                         const float* tau, const float* bias_table,
+                                         const swin_cpb_weights* cpb, const float* rope_freqs,
+                                         swin_stream_t stream);
+
 /* Bytes of workspace swin_window_attn_fwd needs for these arguments
  * (have_table: whether bias_table is non-NULL).  0 when none is needed. */
 size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int have_table);

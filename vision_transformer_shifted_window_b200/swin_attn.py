@@ -30,7 +30,8 @@ SWIN_F32 = 0
 SWIN_BF16 = 1
 
 #: every symbol include/swin_attn.h declares
-EXPORTED = ("swin_cpb_eval", "swin_window_attn_fwd", "swin_window_attn_workspace_size",
+EXPORTED = ("swin_cpb_eval", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
+            "swin_window_attn_workspace_size",
             "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version")
 
 
@@ -63,6 +64,9 @@ def lib():
                                            ctypes.POINTER(swin_cpb_weights), vp, vp,
                                            ctypes.c_size_t, st]
         L.swin_window_attn_fwd.restype = i
+        L.swin_window_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp,
+                                                   vp, ctypes.POINTER(swin_cpb_weights), vp, st]
+        L.swin_window_attn_fwd_noalloc.restype = i
         L.swin_window_attn_workspace_size.argtypes = [i, i, i, i]
         L.swin_window_attn_workspace_size.restype = ctypes.c_size_t
         L.swin_index_tables.argtypes = [i, i, i, i, vp, vp, vp, vp, st]
@@ -176,6 +180,36 @@ def swin_window_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: i
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
         _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
         _ptr(rope_freqs), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc)
+    del keep
+    return out
+
+
+def swin_window_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int,
+                                 mode: int, tau: Optional[torch.Tensor] = None,
+                                 bias_table: Optional[torch.Tensor] = None, cpb=None,
+                                 rope_freqs: Optional[torch.Tensor] = None,
+                                 out: Optional[torch.Tensor] = None, stream=None,
+                                 out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
+    """Forward pass for callers that cannot allocate device memory: the CPB
+    table lives in a fixed device array of the library, not in a workspace.
+    ``out`` must be given by such callers (this wrapper allocates it only when
+    it is None, as a convenience for Python users)."""
+    dt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(q.dtype)
+    if dt is None or k.dtype != q.dtype or v.dtype != q.dtype or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must share a float32/bfloat16 dtype and shape")
+    B, H, W, heads, d = q.shape
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    odt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(out.dtype)
+    if odt is None or out.shape != q.shape:
+        raise ValueError("out must be float32 or bfloat16 with q's shape")
+    tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
+    cs, keep = _cpb_struct(cpb)
+    rc = lib().swin_window_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
+        _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
+        _ptr(rope_freqs), _stream(stream))
     _check(rc)
     del keep
     return out
