@@ -176,6 +176,14 @@ swin_status swin_stream_status(swin_stream_t stream);
  * ("" if none).  The pointer stays valid until the next call on the thread. */
 const char* swin_last_error(void);
 
+/* Test hook for the failure path (no counterpart in the pages).  flags bit 0
+ * makes every later tensor-core launch wait on a barrier that nothing
+ * completes, so its bounded wait runs out, the kernel records
+ * SWIN_ERR_TIMEOUT and returns cleanly; wait_limit_cycles (<= 0: default of
+ * about two seconds) bounds every wait of those launches.  flags = 0 restores
+ * normal operation.  Process-wide; not thread-safe against concurrent calls. */
+swin_status swin_debug_set(int flags, long long wait_limit_cycles);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int swin_version(void);
 

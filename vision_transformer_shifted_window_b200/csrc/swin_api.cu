@@ -135,6 +135,7 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
   a.tau = tau; a.table = table; a.rope = rope_freqs;
   a.status = swin::status_word();
   if (!a.status) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
+  if (dt == SWIN_BF16 && d == 32) return swin::launch_attn_tc(a, out_dt == SWIN_F32, st);
   return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
 }
 
@@ -147,6 +148,12 @@ swin_status swin_index_tables(int H, int W, int M, int shift, int32_t* tok_windo
   if ((long long)H * W >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "H*W must be < 2^31");
   return swin::launch_index_tables(H, W, M, shift, tok_window, tok_region, tok_local, rel_index,
                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+swin_status swin_debug_set(int flags, long long wait_limit_cycles) {
+  if (flags & ~1) return fail(SWIN_ERR_INVALID_ARG, "unknown debug flags 0x%x", flags);
+  swin::tc_set_debug(flags, wait_limit_cycles);
+  return SWIN_OK;
 }
 
 swin_status swin_stream_status(swin_stream_t stream) {

@@ -40,6 +40,8 @@ swin_status launch_cpb_eval(int M, int heads, const swin_cpb_weights& g, float* 
                             cudaStream_t stream);
 swin_status launch_index_tables(int H, int W, int M, int shift, int32_t* tw, int32_t* tr,
                                 int32_t* tl, int32_t* ri, cudaStream_t stream);
+swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream);
+void tc_set_debug(int flags, long long wait_limit);
 swin_status launch_attn_simt(const AttnArgs& a, bool bf16_in, bool f32_out, cudaStream_t stream);
 
 }  // namespace swin

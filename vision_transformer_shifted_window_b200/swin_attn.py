@@ -32,7 +32,8 @@ SWIN_BF16 = 1
 #: every symbol include/swin_attn.h declares
 EXPORTED = ("swin_cpb_eval", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
             "swin_window_attn_workspace_size",
-            "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version")
+            "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version",
+            "swin_debug_set")
 
 
 class SwinError(RuntimeError):
@@ -75,6 +76,8 @@ def lib():
         L.swin_stream_status.restype = i
         L.swin_last_error.argtypes = []
         L.swin_last_error.restype = ctypes.c_char_p
+        L.swin_debug_set.argtypes = [i, ctypes.c_longlong]
+        L.swin_debug_set.restype = i
         L.swin_version.argtypes = []
         L.swin_version.restype = i
         _lib = L
@@ -116,6 +119,11 @@ def _cpb_struct(cpb: Optional[Tuple[torch.Tensor, ...]]):
     w1, b1, w2, b2 = (_f32(t) for t in cpb)
     s = swin_cpb_weights(int(w1.shape[0]), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
     return s, (w1, b1, w2, b2)
+
+
+def swin_debug_set(flags: int, wait_limit_cycles: int = 0) -> None:
+    """Failure-path test hook (see include/swin_attn.h)."""
+    _check(lib().swin_debug_set(int(flags), int(wait_limit_cycles)))
 
 
 def swin_version() -> int:
