@@ -117,7 +117,15 @@ swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* ta
  *                  swin_window_attn_workspace_size(...) bytes, 256-byte
  *                  aligned (may be NULL when that size is 0)
  *   stream         CUDA stream
- * Asynchronous; q/k/v must stay valid until the stream reaches the call. */
+ * Asynchronous; q/k/v must stay valid until the stream reaches the call.
+ *
+ * Arithmetic of the bf16, d == 32 path (tcgen05 tensor cores): q.k products
+ * of the bf16 inputs accumulate in fp32 (modes 0 and 1; mode 1 applies 1/|q|,
+ * 1/|k| and 1/tau in fp32 afterwards); mode 2 rotates q and k in fp32 and
+ * multiplies them as fp16 scaled by powers of two.  Probabilities and V are
+ * carried in fp16 (V scaled by a power of two per 96-key block), sums in
+ * fp32.  V entries of magnitude 2^22 or more saturate; the kernel then
+ * records SWIN_ERR_UNSUPPORTED, which swin_stream_status reports. */
 swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
                                  swin_dtype dt, swin_dtype out_dt, int B, int H, int W,
                                  int heads, int d,

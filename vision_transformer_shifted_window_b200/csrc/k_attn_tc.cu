@@ -9,9 +9,9 @@
 // — without ever storing a score matrix: FlashSwin's point is that the
 // per-window score matrix is the memory problem; here S lives only in TMEM.
 //
-// Work unit: a pair of 128-row query tiles of one rectangle (tile = R whole
-// rectangle rows, R = floor(128 / lx)), one per softmax warpgroup; both
-// warpgroups stream the same K/V blocks of R rectangle rows.
+// Work unit: a pair of query tiles of one rectangle (tile = floor(128 / lx)
+// whole rectangle rows), one per softmax warpgroup; both warpgroups stream
+// the same K/V blocks of floor(96 / lx) rectangle rows (at most 96 keys).
 //
 // Warp roles (384 threads, one persistent CTA per SM):
 //   warp 0      TMA producer: Q tiles and K/V blocks, 5-D tensor maps over
@@ -21,17 +21,21 @@
 //               RoPE rotation of Q and K (mode 2), per-row 1/(tau |q|) (mode 1)
 //   warps 4-7   softmax of warpgroup 0 (one TMEM lane = one query row)
 //   warps 8-11  softmax of warpgroup 1
-// TMEM per softmax warpgroup g (128 lanes): S [g*256, +128) fp32 scores,
-// P [g*256+128, +64) bf16x2 probabilities, O [g*256+192, +48) fp32: 32 output
-// columns and, in column 32, the row sum of P.
-// Per K/V block: S = Q K^T (2 MMAs, K-dim 32); softmax on S with the exact
-// running maximum (O is rescaled whenever it grows, so the largest weight of
-// a row is exactly 1 in bf16); P written to TMEM; O += P [V | 1] (8 MMAs,
-// N = 48, A from TMEM): a constant block with a one in the first column
-// appended to V makes the tensor core add up the same bf16-rounded P that
-// multiplies V, so the normalisation is consistent and costs no ALU work.
-// S of the next block is issued as soon as the softmax has copied the
-// current S to registers.
+// TMEM per softmax warpgroup g (128 lanes): two score buffers X0, X1 of 96
+// fp32 columns and O (48 columns: 32 outputs and, in column 32, the row sum
+// of P).  Block b's scores S = Q K^T land in X[b % 2]; the softmax turns them
+// into fp16 probabilities P written over the same columns, and O += P [V | c]
+// (6 MMAs, N = 48, A from TMEM) reads them there.  With two buffers the
+// softmax never waits for the previous block's PV; the tensor core executes
+// in order, so S(b+2) cannot overwrite P(b) before PV(b) has read it.
+//
+// Softmax: online, with the running maximum kept until a block exceeds it by
+// more than 8 (log2 units), so O is rescaled rarely; P in fp16 (values up to
+// 2^15) keeps that accurate.  V is converted to fp16 by the prep warps with a
+// power-of-two scale 2^-k per block (k = 0 unless |v| >= 2^15, at most 7);
+// the same block's P carries 2^k in its exponent and its ones column holds
+// 2^-k, so O and the row sum stay exact.  V entries of 2^22 or more saturate
+// and record SWIN_ERR_UNSUPPORTED in the status word.
 //
 // Precision of the score operands: mode 0 multiplies the bf16 inputs as they
 // are; mode 1 also multiplies the raw inputs and applies 1/|q| (per row),
@@ -43,17 +47,23 @@
 // the status word, every role leaves its loop, in-flight copies and MMAs are
 // drained with bounded waits, TMEM is freed and the kernel returns.
 #include <cuda.h>
+#include <cuda_fp16.h>
 
 #include <cstring>
 
 #include "sm100_ptx.cuh"
 #include "swin_common.cuh"
 
+// Phase markers for external timing builds; they compile to nothing here.
+#ifndef SWIN_TC_MARK
+#define SWIN_TC_MARK(k)
+#endif
+
 namespace swin {
 
 struct TcParams {
   CUtensorMap tmap[3][3];  // [tensor q/k/v][x-class first/middle/last]
-  int lx[3], R[3];         // per x-class: segment width, rows per tile
+  int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
   void* out;
   int B, H, W, heads, M, s, nsy, nsx, pmax;
   long long n_items;
@@ -69,26 +79,32 @@ namespace {
 
 constexpr int kThreads = 384;
 constexpr int kStages = 6;                  // K/V ring
-constexpr int kTileBytes = 128 * 64;        // 128 rows x 32 bf16
+constexpr int kTileBytes = 128 * 64;        // 128 rows x 32 16-bit values
+constexpr int kBlk = 96;                    // keys per K/V block (TMEM: 2 x 96 + 48 columns per warpgroup)
 constexpr int kQOff = 0;                    // [2 wg][2 buf] Q tiles
 constexpr int kKVOff = kQOff + 4 * kTileBytes;
-constexpr int kOnesOff = kKVOff + kStages * 2 * kTileBytes;    // 16 rows of [1, 0...] (1 KB)
-constexpr int kScaleOff = kOnesOff + 1024;                      // [2][2][128] f32
-constexpr int kRopeOff = kScaleOff + 2 * 2 * 128 * 4;         // cos,sin [2][64][8] f32
-constexpr int kKofsOff = kRopeOff + 2 * 2 * 64 * 8 * 4;       // [3][128] int
-constexpr int kKscOff = kKofsOff + 3 * 128 * 4;                 // [kStages] f32 + reduction [2][2]
-constexpr int kKcolOff = kKscOff + 256;                          // [kStages][128] f32, 1/|k| (mode 1)
-constexpr int kBarOff = kKcolOff + kStages * 128 * 4;
-constexpr int kNumBars = 12 + 3 * kStages + 8 + 2;
+constexpr int kOnesOff = kKVOff + kStages * 2 * kTileBytes;   // per stage: 16 rows of [c, 0...] (1 KB)
+constexpr int kScaleOff = kOnesOff + kStages * 1024;         // [2][2][128] f32
+constexpr int kRopeOff = kScaleOff + 2 * 2 * 128 * 4;        // cos,sin [2][64][8] f32
+constexpr int kKofsOff = kRopeOff + 2 * 2 * 64 * 8 * 4;      // [3][128] int
+constexpr int kRposOff = kKofsOff + 3 * 128 * 4;             // [3][128] int: (r / lx) | (r % lx) << 16
+constexpr int kKcolOff = kRposOff + 3 * 128 * 4;             // [kStages][128] f32, 1/|k| (mode 1)
+constexpr int kBiasFloats = 16384;                           // bias tables of all heads if they fit
+constexpr int kBiasOff = kKcolOff + kStages * 128 * 4;
+constexpr int kBarOff = kBiasOff + kBiasFloats * 4;
+constexpr int kNumBars = 12 + 3 * kStages + 12 + 2;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 
 constexpr float kLog2eF = 1.4426950408889634f;
 
 struct Bars {
   uint64_t q_full[2][2], q_ready[2][2], q_empty[2][2];
   uint64_t kv_full[kStages], kv_ready[kStages], kv_empty[kStages];
-  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  // per warpgroup and score buffer: a barrier's next phase (block b + 2) can
+  // only start after its current one was consumed, so parity tests never alias
+  uint64_t s_full[2][2], p_full[2][2], o_done[2][2];
   uint64_t never, drain;
 };
 static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
@@ -96,7 +112,7 @@ static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
 struct Task {
   bool any;       // item has work for warpgroup 0
   bool valid[2];  // per warpgroup
-  int b, h, cls, lx, R, y0, x0, ly, n, nb;
+  int b, h, cls, lx, R, Rk, y0, x0, ly, n, nb;
   int tile[2], nq[2];
 };
 
@@ -114,14 +130,16 @@ __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
   t.cls = sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1);
   t.lx = p.lx[t.cls];
   t.R = p.R[t.cls];
+  t.Rk = p.Rk[t.cls];
   t.y0 = swin_seg_start(sy, p.M, p.s);
   t.ly = swin_seg_len(sy, p.H, p.M, p.s);
   t.x0 = swin_seg_start(sx, p.M, p.s);
   t.n = t.ly * t.lx;
-  t.nb = (t.ly + t.R - 1) / t.R;
+  t.nb = (t.ly + t.Rk - 1) / t.Rk;
+  const int ntiles = (t.ly + t.R - 1) / t.R;
   for (int g = 0; g < 2; ++g) {
     t.tile[g] = 2 * pr + g;
-    t.valid[g] = t.tile[g] < t.nb;
+    t.valid[g] = t.tile[g] < ntiles;
     int rows = t.ly - t.tile[g] * t.R;
     t.nq[g] = t.valid[g] ? (rows < t.R ? rows : t.R) * t.lx : 0;
   }
@@ -179,6 +197,17 @@ __device__ __forceinline__ void load_row_bf16(const uint8_t* tile, int row, floa
   }
 }
 
+// Store v * sc as fp16 with saturation into the same row.
+__device__ __forceinline__ void store_row_f16_sat(uint8_t* tile, int row, const float (&v)[32], float sc) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t u[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) u[e] = ptx::pack_f16x2_sat(v[8 * c + 2 * e] * sc, v[8 * c + 2 * e + 1] * sc);
+    *reinterpret_cast<uint4*>(tile + swz64(row, c)) = make_uint4(u[0], u[1], u[2], u[3]);
+  }
+}
+
 // Store v * sc as fp16 into the same row.
 __device__ __forceinline__ void store_row_f16(uint8_t* tile, int row, const float (&v)[32], float sc) {
 #pragma unroll
@@ -202,14 +231,18 @@ __device__ __forceinline__ void rope_rotate(float (&v)[32], int py, int px, cons
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const int pos = half ? px : py;
-    const float* cs = rc + (half * 64 + pos) * 8;
-    const float* sn = rs + (half * 64 + pos) * 8;
+    const float4* cs4 = reinterpret_cast<const float4*>(rc + (half * 64 + pos) * 8);
+    const float4* sn4 = reinterpret_cast<const float4*>(rs + (half * 64 + pos) * 8);
+    const float4 c0 = cs4[0], c1 = cs4[1], s0 = sn4[0], s1 = sn4[1];
+    const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       const float a = v[16 * half + 2 * t], b = v[16 * half + 2 * t + 1];
       const float co = cs[t], si = sn[t];
-      v[16 * half + 2 * t] = a * co - b * si;
-      v[16 * half + 2 * t + 1] = a * si + b * co;
+      // explicit roundings: every instantiation of the kernel computes the same bits
+      v[16 * half + 2 * t] = __fmaf_rn(a, co, -__fmul_rn(b, si));
+      v[16 * half + 2 * t + 1] = __fmaf_rn(a, si, __fmul_rn(b, co));
     }
   }
 }
@@ -219,6 +252,22 @@ __device__ __forceinline__ float absmax(const float (&v)[32]) {
 #pragma unroll
   for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(v[e]));
   return m;
+}
+
+// Largest |value| of one 32-element bf16 row (packed bf16x2 arithmetic).
+__device__ __forceinline__ float row_absmax_bf16(const uint8_t* tile, int row) {
+  __nv_bfloat162 m = __float2bfloat162_rn(0.f);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + swz64(row, c));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
+      m = __hmax2(m, __habs2(x));
+    }
+  }
+  return fmaxf(__bfloat162float(m.x), __bfloat162float(m.y));
 }
 
 // Power of two that brings a row maximum m below 2^15 (fp16 max is 65504).
@@ -236,14 +285,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* qbuf = smem + kQOff;
   uint8_t* kvbuf = smem + kKVOff;
+  uint8_t* ones = smem + kOnesOff;
   float* qscale = reinterpret_cast<float*>(smem + kScaleOff);
   float* rcos = reinterpret_cast<float*>(smem + kRopeOff);
   float* rsin = rcos + 2 * 64 * 8;
   int* kofs = reinterpret_cast<int*>(smem + kKofsOff);
-  float* kscale = reinterpret_cast<float*>(smem + kKscOff);          // per K/V stage
-  float* kred = kscale + 32;                                         // [2 parity][2 warps]
+  int* rpos = reinterpret_cast<int*>(smem + kRposOff);
   float* kcol = reinterpret_cast<float*>(smem + kKcolOff);
-  uint8_t* ones = smem + kOnesOff;
+  float* sbias = reinterpret_cast<float*>(smem + kBiasOff);  // [heads][(2M-1)^2], times log2(e)
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -251,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = p.M, s = p.s;
 
-  // ---- set-up: barriers, RoPE tables, bias column offsets, TMEM
+  // ---- set-up: barriers, RoPE tables, bias tables and column offsets, TMEM
   if (threadIdx.x == 0) {
     for (int g = 0; g < 2; ++g)
       for (int b = 0; b < 2; ++b) {
@@ -265,10 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       ptx::mbar_init(&bars->kv_empty[i], 1);
     }
     for (int g = 0; g < 2; ++g) {
-      ptx::mbar_init(&bars->s_full[g], 1);
-      ptx::mbar_init(&bars->s_free[g], 128);
-      ptx::mbar_init(&bars->p_full[g], 128);
-      ptx::mbar_init(&bars->o_done[g], 1);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(&bars->s_full[g][b], 1);
+        ptx::mbar_init(&bars->p_full[g][b], 128);
+        ptx::mbar_init(&bars->o_done[g][b], 1);
+      }
     }
     ptx::mbar_init(&bars->never, 1);
     ptx::mbar_init(&bars->drain, 1);
@@ -277,26 +327,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     ptx::fence_mbar_init();
   }
   if (MODE == 2) {
-    for (int i = threadIdx.x; i < 2 * M * 8; i += kThreads) {
-      const int axis = i / (M * 8), pos = (i / 8) % M, t = i % 8;
-      float sv, cv;
-      sincosf((float)pos * p.rope[axis * 8 + t], &sv, &cv);
+    // all 64 positions (rows past a rectangle's end, which are masked, read up to 63)
+    for (int i = threadIdx.x; i < 2 * 64 * 8; i += kThreads) {
+      const int axis = i / (64 * 8), pos = (i / 8) % 64, t = i % 8;
+      float sv = 0.f, cv = 1.f;
+      if (pos < M) sincosf((float)pos * p.rope[axis * 8 + t], &sv, &cv);
       rcos[(axis * 64 + pos) * 8 + t] = cv;
       rsin[(axis * 64 + pos) * 8 + t] = sv;
     }
   }
-  if (MODE != 2) {
-    for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
-      const int c = i / 128, col = i % 128, lx = p.lx[c];
-      kofs[i] = (col / lx) * (2 * M - 1) + (col % lx);
+  const int R2sq = (2 * M - 1) * (2 * M - 1);
+  const bool bias_in_smem = MODE != 2 && p.table != nullptr && p.heads * R2sq <= kBiasFloats;
+  if (bias_in_smem) {
+    // table [(2M-1)^2][heads] -> shared [heads][(2M-1)^2], pre-scaled by log2(e)
+    for (int i = threadIdx.x; i < p.heads * R2sq; i += kThreads) {
+      const int h = i / R2sq, r = i % R2sq;
+      sbias[i] = __ldg(p.table + (size_t)r * p.heads + h) * kLog2eF;
     }
   }
-  // zero the K/V ring once so rows a tile never writes hold finite values;
-  // the ones block: 16 rows of 64 bytes (64B swizzle), bf16 1.0 at element 0
-  for (int i = threadIdx.x; i < (kStages * 2 * kTileBytes + 1024) / 16; i += kThreads)
+  for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
+    const int c = i / 128, col = i % 128, lx = p.lx[c];
+    kofs[i] = (col / lx) * (2 * M - 1) + (col % lx);
+    rpos[i] = (col / lx) | ((col % lx) << 16);
+  }
+  // zero the K/V ring and the ones blocks once, so rows a tile never writes
+  // hold finite values
+  for (int i = threadIdx.x; i < (kStages * 2 * kTileBytes + kStages * 1024) / 16; i += kThreads)
     reinterpret_cast<uint4*>(kvbuf)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  if (threadIdx.x < 16) *reinterpret_cast<uint16_t*>(ones + swz64(threadIdx.x, 0)) = 0x3F80;
+  // the constant column block of every stage: fp16 1.0 in the first column of 16 rows
+  if (threadIdx.x < 16 * kStages)
+    *reinterpret_cast<uint16_t*>(ones + (threadIdx.x / 16) * 1024 + swz64(threadIdx.x % 16, 0)) = 0x3C00;
   if (warp == 1) {
     ptx::tmem_alloc(tmem_holder, 512);
     ptx::tmem_relinquish();
@@ -310,46 +371,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   Ctl ctl{abort_flag, &p};
-  // Register split: warps 0-3 (producer, MMA, prep) give registers to the two
-  // softmax warpgroups: 384 x 168 = 128 x 72 + 256 x 216.
-
   const long long first = blockIdx.x, step = gridDim.x;
 
+  // Register split: warps 0-3 (producer, MMA, prep) give registers to the two
+  // softmax warpgroups: 384 x 168 = 128 x 88 + 256 x 208.
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
-  if (warp == 0) {
-    // ================================================================ producer
-    if (lane == 0) {
-      uint32_t qu[2] = {0, 0};
-      uint32_t ku = 0;
-      bool ok = true;
-      for (long long it = first; it < p.n_items && ok; it += step) {
-        const Task t = decode(p, it);
-        if (!t.any) continue;
-        const uint32_t box_bytes = (uint32_t)(64 * t.lx * t.R);
-        for (int g = 0; g < 2 && ok; ++g) {
-          if (!t.valid[g]) continue;
-          const int qs = qu[g] & 1;
-          if (qu[g] >= 2) ok = wait_bar(&bars->q_empty[g][qs], ((qu[g] >> 1) - 1) & 1, ctl);
-          if (!ok) break;
-          ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], box_bytes);
-          ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][t.cls], &bars->q_full[g][qs], 0, t.h,
-                           t.x0, t.y0 + t.tile[g] * t.R, t.b);
-          ++qu[g];
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+    if (warp == 0) {
+      // ============================================================== producer
+      if (lane == 0) {
+        uint32_t qu[2] = {0, 0};
+        uint32_t ku = 0;
+        bool ok = true;
+        for (long long it = first; it < p.n_items && ok; it += step) {
+          const Task t = decode(p, it);
+          if (!t.any) continue;
+          const uint32_t qbytes = (uint32_t)(64 * t.lx * t.R), kbytes = (uint32_t)(64 * t.lx * t.Rk);
+          for (int g = 0; g < 2 && ok; ++g) {
+            if (!t.valid[g]) continue;
+            const int qs = qu[g] & 1;
+            if (qu[g] >= 2) ok = wait_bar(&bars->q_empty[g][qs], ((qu[g] >> 1) - 1) & 1, ctl);
+            if (!ok) break;
+            ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], qbytes);
+            ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][t.cls], &bars->q_full[g][qs], 0, t.h,
+                             t.x0, t.y0 + t.tile[g] * t.R, t.b);
+            ++qu[g];
+          }
+          for (int j = 0; j < t.nb && ok; ++j) {
+            const int st = ku % kStages;
+            if (ku >= (uint32_t)kStages) ok = wait_bar(&bars->kv_empty[st], ((ku / kStages) - 1) & 1, ctl);
+            if (!ok) break;
+            uint8_t* kb = kvbuf + st * 2 * kTileBytes;
+            ptx::mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kbytes);
+            ptx::tma_load_5d(kb, &p.tmap[1][t.cls], &bars->kv_full[st], 0, t.h, t.x0, t.y0 + j * t.Rk, t.b);
+            ptx::tma_load_5d(kb + kTileBytes, &p.tmap[2][t.cls], &bars->kv_full[st], 0, t.h, t.x0,
+                             t.y0 + j * t.Rk, t.b);
+            ++ku;
+          }
         }
-        for (int j = 0; j < t.nb && ok; ++j) {
-          const int st = ku % kStages;
-          if (ku >= (uint32_t)kStages) ok = wait_bar(&bars->kv_empty[st], ((ku / kStages) - 1) & 1, ctl);
-          if (!ok) break;
-          uint8_t* kb = kvbuf + st * 2 * kTileBytes;
-          ptx::mbar_arrive_expect_tx(&bars->kv_full[st], 2 * box_bytes);
-          ptx::tma_load_5d(kb, &p.tmap[1][t.cls], &bars->kv_full[st], 0, t.h, t.x0, t.y0 + j * t.R, t.b);
-          ptx::tma_load_5d(kb + kTileBytes, &p.tmap[2][t.cls], &bars->kv_full[st], 0, t.h, t.x0,
-                           t.y0 + j * t.R, t.b);
-          ++ku;
-        }
-      }
-      {
         // drain copies that may still be landing in shared memory (after an
         // abort; in a normal exit every phase waited here has completed)
         Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
@@ -359,223 +418,261 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (uint32_t u = (qu[g] > 2 ? qu[g] - 2 : 0); u < qu[g]; ++u)
             wait_bar(&bars->q_full[g][u & 1], (u >> 1) & 1, drain);
       }
-    }
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0) {
-      // mode 2 feeds fp16 operands (see prep), modes 0 and 1 the bf16 inputs
-      constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
-      constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, 128, 128);
-      constexpr uint32_t idPV = ptx::idesc_f16(1, 1, 0, 1, 48, 128);
-      const uint32_t ones_addr = ptx::smem_addr(ones);
-      uint32_t qu[2] = {0, 0}, s_iss[2] = {0, 0}, pv_cnt[2] = {0, 0};
-      uint32_t ku = 0;  // K/V block uses consumed
-      bool ok = true;
-      if (p.debug_flags & 1) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
+    } else if (warp == 1) {
+      // ============================================================== MMA issuer
+      // Event-driven: each warpgroup's next S and next PV are probed without
+      // blocking and issued as soon as their inputs are ready.
+      if (lane == 0) {
+        // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
+        constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
+        constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlk, 128);
+        constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
+        bool ok = true;
+        if (p.debug_flags & 1) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
 
-      auto issue_S = [&](int g, int qs, int st) -> bool {
-        if (s_iss[g] > 0 && !wait_bar(&bars->s_free[g], (s_iss[g] - 1) & 1, ctl)) return false;
-        ptx::tc_fence_after();
-        const uint32_t qa = ptx::smem_addr(qbuf + (g * 2 + qs) * kTileBytes);
-        const uint32_t ka = ptx::smem_addr(kvbuf + st * 2 * kTileBytes);
-        const uint64_t ad = ptx::smem_desc(qa, 16, 512, ptx::kSwizzle64B);
-        const uint64_t bd = ptx::smem_desc(ka, 16, 512, ptx::kSwizzle64B);
-        const uint32_t dS = tmem_base + g * 256;
-        ptx::mma_ss(dS, ad, bd, idS, 0);
-        ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
-        ptx::mma_commit(&bars->s_full[g]);
-        ++s_iss[g];
-        return true;
-      };
-
-      // Find the first item with work.
-      long long it = first;
-      Task cur;
-      cur.any = false;
-      for (; it < p.n_items; it += step) {
-        cur = decode(p, it);
-        if (cur.any) break;
-      }
-      int cur_qs[2] = {0, 0};
-      uint32_t cur_k0 = 0;
-      if (ok && it < p.n_items) {
-        // prologue: S of block 0 of the first item
-        for (int g = 0; g < 2 && ok; ++g)
-          if (cur.valid[g]) {
-            cur_qs[g] = qu[g] & 1;
-            ok = wait_bar(&bars->q_ready[g][cur_qs[g]], (qu[g] >> 1) & 1, ctl);
-            ++qu[g];
+        struct Cur {
+          long long it_next;  // next item to examine
+          uint32_t u_next;    // K/V use index of the next item's first block
+          uint32_t qcnt;      // Q tiles taken so far
+          uint32_t u0, qpar;  // first K/V use of the current item; Q buffer phase
+          int j, nb, qs, nvalid;
+          bool live;
+        };
+        auto next_item = [&](Cur& c, int g) {
+          c.live = false;
+          while (c.it_next < p.n_items) {
+            const Task t = decode(p, c.it_next);
+            c.it_next += step;
+            if (!t.any) continue;
+            const uint32_t u0 = c.u_next;
+            c.u_next += t.nb;
+            if (!t.valid[g]) continue;
+            c.nb = t.nb;
+            c.nvalid = (int)t.valid[0] + (int)t.valid[1];
+            c.j = 0;
+            c.u0 = u0;
+            c.qs = c.qcnt & 1;
+            c.qpar = (c.qcnt >> 1) & 1;
+            ++c.qcnt;
+            c.live = true;
+            return;
           }
-        cur_k0 = ku;
-        if (ok) ok = wait_bar(&bars->kv_ready[ku % kStages], (ku / kStages) & 1, ctl);
-        for (int g = 0; g < 2 && ok; ++g)
-          if (cur.valid[g]) {
-            ok = issue_S(g, cur_qs[g], ku % kStages);
-            if (ok && cur.nb == 1) ptx::mma_commit(&bars->q_empty[g][cur_qs[g]]);
-          }
-        ++ku;
-      }
-      while (ok && it < p.n_items) {
-        long long nit = it + step;
-        Task nxt;
-        nxt.any = false;
-        int nxt_qs[2] = {0, 0};
-        for (int j = 0; j < cur.nb && ok; ++j) {
-          const int st = (cur_k0 + j) % kStages;
-          if (j + 1 < cur.nb) {
-            ok = wait_bar(&bars->kv_ready[ku % kStages], (ku / kStages) & 1, ctl);
-            for (int g = 0; g < 2 && ok; ++g)
-              if (cur.valid[g]) {
-                ok = issue_S(g, cur_qs[g], ku % kStages);
-                if (ok && j + 1 == cur.nb - 1) ptx::mma_commit(&bars->q_empty[g][cur_qs[g]]);
+        };
+        Cur cs[2], cp[2];
+        for (int g = 0; g < 2; ++g) {
+          cs[g].it_next = first;
+          cs[g].u_next = 0;
+          cs[g].qcnt = 0;
+          cs[g].live = false;
+          cp[g] = cs[g];
+          next_item(cs[g], g);
+          next_item(cp[g], g);
+        }
+        uint32_t s_iss[2] = {0, 0}, pv_iss[2] = {0, 0};
+        uint32_t rem[kStages], tag[kStages];
+        for (int i = 0; i < kStages; ++i) {
+          rem[i] = 0;
+          tag[i] = 0xffffffffu;
+        }
+        long long idle_since = clock64();
+        while (ok && (cs[0].live || cs[1].live || cp[0].live || cp[1].live)) {
+          bool progress = false;
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            // ---- S = Q K^T of warpgroup g's next block, into X[b % 2]
+            Cur& c = cs[g];
+            if (c.live && (s_iss[g] < 2 || pv_iss[g] + 1 >= s_iss[g])) {
+              const uint32_t u = c.u0 + c.j, st = u % kStages;
+              const bool ready = (c.j > 0 || ptx::mbar_test(&bars->q_ready[g][c.qs], c.qpar)) &&
+                                 ptx::mbar_test(&bars->kv_ready[st], (u / kStages) & 1);
+              if (ready) {
+                ptx::tc_fence_after();
+                if (tag[st] != u) {  // first use of this K/V block: count its consumers
+                  tag[st] = u;
+                  rem[st] = (uint32_t)c.nvalid;
+                }
+                const uint32_t qa = ptx::smem_addr(qbuf + (g * 2 + c.qs) * kTileBytes);
+                const uint32_t ka = ptx::smem_addr(kvbuf + st * 2 * kTileBytes);
+                const uint64_t ad = ptx::smem_desc(qa, 16, 512, ptx::kSwizzle64B);
+                const uint64_t bd = ptx::smem_desc(ka, 16, 512, ptx::kSwizzle64B);
+                const uint32_t dS = tmem_base + g * 256 + (s_iss[g] & 1) * kBlk;
+                ptx::mma_ss(dS, ad, bd, idS, 0);
+                ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
+                ptx::mma_commit(&bars->s_full[g][s_iss[g] & 1]);
+                ++s_iss[g];
+                if (c.j == c.nb - 1) ptx::mma_commit(&bars->q_empty[g][c.qs]);
+                if (++c.j == c.nb) next_item(c, g);
+                progress = true;
               }
-            ++ku;
+            }
+            // ---- O += P [V | c] of warpgroup g's next block
+            Cur& d = cp[g];
+            if (d.live && pv_iss[g] < s_iss[g] &&
+                ptx::mbar_test(&bars->p_full[g][pv_iss[g] & 1], (pv_iss[g] >> 1) & 1)) {
+              ptx::tc_fence_after();
+              const uint32_t u = d.u0 + d.j, st = u % kStages;
+              const uint32_t va = ptx::smem_addr(kvbuf + st * 2 * kTileBytes + kTileBytes);
+              const uint32_t oa = ptx::smem_addr(ones + st * 1024);
+              const uint32_t dO = tmem_base + g * 256 + 2 * kBlk;
+              const uint32_t aP = tmem_base + g * 256 + (pv_iss[g] & 1) * kBlk;
+#pragma unroll
+              for (int kk = 0; kk < kBlk / 16; ++kk) {
+                // N columns 0-31: V rows; 32-47: the stage's constant block (LBO = its distance)
+                const uint32_t vk = va + kk * 1024;
+                const uint64_t bd = ptx::smem_desc(vk, oa - vk, 512, ptx::kSwizzle64B);
+                ptx::mma_ts(dO, aP + kk * 8, bd, idPV, (d.j > 0 || kk > 0) ? 1u : 0u);
+              }
+              ptx::mma_commit(&bars->o_done[g][pv_iss[g] & 1]);
+              ++pv_iss[g];
+              if (--rem[st] == 0) ptx::mma_commit(&bars->kv_empty[st]);
+              if (++d.j == d.nb) next_item(d, g);
+              progress = true;
+            }
+          }
+          if (progress) {
+            idle_since = clock64();
           } else {
-            // look ahead into the next item with work
-            for (; nit < p.n_items; nit += step) {
-              nxt = decode(p, nit);
-              if (nxt.any) break;
-            }
-            if (nit < p.n_items) {
-              for (int g = 0; g < 2 && ok; ++g)
-                if (nxt.valid[g]) {
-                  nxt_qs[g] = qu[g] & 1;
-                  ok = wait_bar(&bars->q_ready[g][nxt_qs[g]], (qu[g] >> 1) & 1, ctl);
-                  ++qu[g];
-                }
-              if (ok) ok = wait_bar(&bars->kv_ready[ku % kStages], (ku / kStages) & 1, ctl);
-              for (int g = 0; g < 2 && ok; ++g)
-                if (nxt.valid[g]) {
-                  ok = issue_S(g, nxt_qs[g], ku % kStages);
-                  if (ok && nxt.nb == 1) ptx::mma_commit(&bars->q_empty[g][nxt_qs[g]]);
-                }
-              ++ku;
+            if (*abort_flag) break;
+            if (clock64() - idle_since > p.wait_limit) {
+              atomicOr(p.status, (int)SWIN_ERR_TIMEOUT);
+              *abort_flag = 1;
+              break;
             }
           }
-          // O += P V for block j
-          const uint32_t va = ptx::smem_addr(kvbuf + st * 2 * kTileBytes + kTileBytes);
-          for (int g = 0; g < 2 && ok; ++g) {
-            if (!cur.valid[g]) continue;
-            ok = wait_bar(&bars->p_full[g], pv_cnt[g] & 1, ctl);
-            ++pv_cnt[g];
-            if (!ok) break;
-            ptx::tc_fence_after();
-            const uint32_t dO = tmem_base + g * 256 + 192, aP = tmem_base + g * 256 + 128;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              // N columns 0-31: V rows; 32-47: the ones block (LBO = its distance)
-              const uint32_t vk = va + kk * 1024;
-              const uint64_t bd = ptx::smem_desc(vk, ones_addr - vk, 512, ptx::kSwizzle64B);
-              ptx::mma_ts(dO, aP + kk * 8, bd, idPV, (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            ptx::mma_commit(&bars->o_done[g]);
-          }
-          if (ok) ptx::mma_commit(&bars->kv_empty[st]);
         }
-        cur = nxt;
-        cur_qs[0] = nxt_qs[0];
-        cur_qs[1] = nxt_qs[1];
-        cur_k0 = ku - 1;
-        it = nit;
+        // drain: every MMA this thread issued has completed before TMEM is freed
+        ptx::mma_commit(&bars->drain);
+        Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
+        wait_bar(&bars->drain, 0, drain);
       }
-      // drain: every MMA this thread issued has completed before TMEM is freed
-      ptx::mma_commit(&bars->drain);
-      Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
-      wait_bar(&bars->drain, 0, drain);
-    }
-  } else if (warp < 4) {
-    // ================================================================ prep
-    const int pt = threadIdx.x - 64;  // 0..63
-    uint32_t qu[2] = {0, 0}, ku = 0;
-    bool ok = true;
-    for (long long it = first; it < p.n_items && ok; it += step) {
-      const Task t = decode(p, it);
-      if (!t.any) continue;
-      const int rows = t.lx * t.R;
-      for (int g = 0; g < 2 && ok; ++g) {
-        if (!t.valid[g]) continue;
-        const int qs = qu[g] & 1;
-        ok = wait_bar(&bars->q_full[g][qs], (qu[g] >> 1) & 1, ctl);
-        ++qu[g];
-        if (!ok) break;
-        uint8_t* tile = qbuf + (g * 2 + qs) * kTileBytes;
-        const float te = MODE == 1 ? fmaxf(__ldg(p.tau + t.h), kTauMin) : 1.f;
-        if (MODE != 0) {
-          for (int r = pt; r < rows; r += 64) {
-            float v[32];
-            load_row_bf16(tile, r, v);
-            if (MODE == 1) {
-              qscale[(g * 2 + qs) * 128 + r] = kLog2eF * inv_norm(v) / te;
-            } else {
-              const int qy = t.tile[g] * t.R + r / t.lx, qx = r % t.lx;
-              rope_rotate(v, swin_local_coord(t.y0 + qy, M, s), swin_local_coord(t.x0 + qx, M, s), rcos, rsin);
-              const float sc = pow2_scale(absmax(v));
-              store_row_f16(tile, r, v, sc);
-              qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
+    } else {
+      // ============================================================== prep
+      const int pt = threadIdx.x - 64;  // 0..63
+      uint32_t qu[2] = {0, 0}, ku = 0;
+      bool ok = true;
+      bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
+      for (long long it = first; it < p.n_items && ok; it += step) {
+        const Task t = decode(p, it);
+        if (!t.any) continue;
+        const int qrows = t.lx * t.R, krows = t.lx * t.Rk;
+        const int* rp = rpos + t.cls * 128;
+        // window-local coordinates of the rectangle's first row and column
+        const int py0 = swin_local_coord(t.y0, M, s), px0 = swin_local_coord(t.x0, M, s);
+        for (int g = 0; g < 2 && ok; ++g) {
+          if (!t.valid[g]) continue;
+          const int qs = qu[g] & 1;
+          ok = wait_bar(&bars->q_full[g][qs], (qu[g] >> 1) & 1, ctl);
+          ++qu[g];
+          if (!ok) break;
+          uint8_t* tile = qbuf + (g * 2 + qs) * kTileBytes;
+          const float te = MODE == 1 ? fmaxf(__ldg(p.tau + t.h), kTauMin) : 1.f;
+          if (MODE != 0) {
+            for (int r = pt; r < qrows; r += 64) {
+              float v[32];
+              load_row_bf16(tile, r, v);
+              if (MODE == 1) {
+                qscale[(g * 2 + qs) * 128 + r] = kLog2eF * inv_norm(v) / te;
+              } else {
+                const int pr = rp[r];
+                rope_rotate(v, min(py0 + t.tile[g] * t.R + (pr & 0xFFFF), 63), px0 + (pr >> 16), rcos, rsin);
+                const float sc = pow2_scale(absmax(v));  // exact per-row scale, undone in the softmax
+                store_row_f16(tile, r, v, sc);
+                qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
+              }
+            }
+            ptx::fence_proxy_async_smem();
+          }
+          ptx::mbar_arrive(&bars->q_ready[g][qs]);
+        }
+        for (int j = 0; j < t.nb && ok; ++j) {
+          const int st = ku % kStages;
+          ok = wait_bar(&bars->kv_full[st], (ku / kStages) & 1, ctl);
+          ++ku;
+          if (!ok) break;
+          uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
+          uint8_t* vtile = ktile + kTileBytes;
+          // K rows pt, pt + 64 and V rows 63 - pt, 127 - pt (rows < krows <= 96):
+          // each prep warp carries 1.5 rows of each.  Rows are independent: fp16
+          // with saturation, a saturated entry is reported after the loop.
+#pragma unroll 1
+          for (int i = 0; i < 2; ++i) {
+            const int krow = pt + 64 * i, vrow = 63 - pt + 64 * i;
+            if (MODE != 0 && krow < krows) {
+              float v[32];
+              load_row_bf16(ktile, krow, v);
+              if (MODE == 1) {
+                kcol[st * 128 + krow] = inv_norm(v);
+              } else {
+                const int pr = rp[krow];
+                rope_rotate(v, min(py0 + j * t.Rk + (pr & 0xFFFF), 63), px0 + (pr >> 16), rcos, rsin);
+                range_hit |= absmax(v) >= 65504.0f;
+                store_row_f16_sat(ktile, krow, v, 1.0f);
+              }
+            }
+            if (vrow < krows) {
+              range_hit |= row_absmax_bf16(vtile, vrow) >= 65504.0f;
+              float v[32];
+              load_row_bf16(vtile, vrow, v);
+              store_row_f16_sat(vtile, vrow, v, 1.0f);
             }
           }
           ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&bars->kv_ready[st]);
         }
-        ptx::mbar_arrive(&bars->q_ready[g][qs]);
       }
-      for (int j = 0; j < t.nb && ok; ++j) {
-        const int st = ku % kStages;
-        ok = wait_bar(&bars->kv_full[st], (ku / kStages) & 1, ctl);
-        ++ku;
-        if (!ok) break;
-        uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
-        if (MODE == 1) {
-          for (int r = pt; r < rows; r += 64) {
-            float v[32];
-            load_row_bf16(ktile, r, v);
-            kcol[st * 128 + r] = inv_norm(v);
-          }
-        }
-        if (MODE == 2) {
-          // rotate this thread's rows (at most two), then one power-of-two
-          // scale for the whole block from the block's largest component
-          float v0[32], v1[32];
-          float mx = 0.f;
-          const int r0 = pt, r1 = pt + 64;
-          if (r0 < rows) {
-            load_row_bf16(ktile, r0, v0);
-            rope_rotate(v0, swin_local_coord(t.y0 + j * t.R + r0 / t.lx, M, s),
-                        swin_local_coord(t.x0 + r0 % t.lx, M, s), rcos, rsin);
-            mx = absmax(v0);
-          }
-          if (r1 < rows) {
-            load_row_bf16(ktile, r1, v1);
-            rope_rotate(v1, swin_local_coord(t.y0 + j * t.R + r1 / t.lx, M, s),
-                        swin_local_coord(t.x0 + r1 % t.lx, M, s), rcos, rsin);
-            mx = fmaxf(mx, absmax(v1));
-          }
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const int par = (ku - 1) & 1;
-          if (lane == 0) kred[par * 2 + (warp - 2)] = mx;
-          ptx::named_bar_sync(1, 64);
-          const float sc = pow2_scale(fmaxf(kred[par * 2], kred[par * 2 + 1]));
-          if (r0 < rows) store_row_f16(ktile, r0, v0, sc);
-          if (r1 < rows) store_row_f16(ktile, r1, v1, sc);
-          if (pt == 0) kscale[st] = 1.0f / sc;
-          ptx::fence_proxy_async_smem();
-        }
-        ptx::mbar_arrive(&bars->kv_ready[st]);
-      }
+      if (range_hit) atomicOr(p.status, (int)SWIN_ERR_UNSUPPORTED);
     }
-  }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
     // ================================================================ softmax
-    const int g = (warp - 4) >> 2;            // warpgroup 0 or 1
+    const int g = (warp - 4) >> 2;              // warpgroup 0 or 1
     const int t = threadIdx.x - 128 - g * 128;  // row of the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem_base + g * 256 + lane_off;
-    const uint32_t tP = tS + 128, tO = tS + 192;
+    const uint32_t tX = tmem_base + g * 256 + lane_off;  // X0; X1 = tX + kBlk
+    const uint32_t tO = tX + 2 * kBlk;
     const float cscale = kLog2eF * rsqrtf(32.0f);
     const int R2 = 2 * M - 1;
-    uint32_t qu = 0, s_cnt = 0, o_cnt = 0, ku = 0;
+    uint32_t qu = 0, ku = 0, blk = 0;  // Q tiles, K/V uses, blocks of this warpgroup
     bool ok = true;
+    bool pend = false, pend_ok = false;  // an item's O still waiting in TMEM
+    size_t pend_off = 0;
+    // O / l of one row to global memory (32 values; column 32 holds l)
+    auto store_rows = [&](const uint32_t (&o)[32], const uint32_t (&o2)[16], size_t off, bool row_valid) {
+      if (!row_valid) return;
+      const float inv = 1.0f / __uint_as_float(o2[0]);  // row sum of the fp16 P
+      if (OUT_F32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
+                               __uint_as_float(o[4 * c + 2]) * inv, __uint_as_float(o[4 * c + 3]) * inv);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = ptx::pack_bf16x2(__uint_as_float(o[8 * c + 2 * e]) * inv,
+                                    __uint_as_float(o[8 * c + 2 * e + 1]) * inv);
+          dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    };
+    // PV completions are consumed strictly in order, one barrier per PV
+    // parity: PV(b + 2) needs P(b + 2), which is written only after PV(b)
+    // was consumed, so no parity test can alias another phase.
+    uint32_t o_cons = 0;  // PVs of this warpgroup known complete
+    auto consume_pv = [&](uint32_t upto) -> bool {  // PV(0..upto) complete
+      bool r = true;
+      while (r && o_cons <= upto) {
+        r = wait_bar(&bars->o_done[g][o_cons & 1], (o_cons >> 1) & 1, ctl);
+        r = __all_sync(0xffffffffu, r);
+        ++o_cons;
+      }
+      ptx::tc_fence_after();
+      return r;
+    };
     for (long long it = first; it < p.n_items && ok; it += step) {
       const Task tk = decode(p, it);
       const uint32_t ku0 = ku;
@@ -594,142 +691,188 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int qy = tk.tile[g] * tk.R + t / tk.lx, qx = t % tk.lx;
       const int bbase = (qy + M - 1) * R2 + (qx + M - 1);
       const int* kof = kofs + tk.cls * 128;
-      const float* tab = p.table;
       float m_run = -INFINITY;
-      for (int j = 0; j < tk.nb; ++j) {
-        ok = wait_bar(&bars->s_full[g], s_cnt & 1, ctl);
+      for (int j = 0; j < tk.nb; ++j, ++blk) {
+        SWIN_TC_MARK(0);
+        ok = wait_bar(&bars->s_full[g][blk & 1], (blk >> 1) & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
-        ++s_cnt;
         if (!ok) break;
+        SWIN_TC_MARK(1);
         ptx::tc_fence_after();
-        float x[128];
+        const uint32_t tS = tX + (blk & 1) * kBlk;
+        float2 x[kBlk / 2];  // scores as packed pairs (keys 2c, 2c+1)
         {
-          uint32_t r0[32], r1[32], r2[32], r3[32];
+          uint32_t r0[32], r1[32], r2[32];
           ptx::tmem_ld32(tS, r0);
           ptx::tmem_ld32(tS + 32, r1);
           ptx::tmem_ld32(tS + 64, r2);
-          ptx::tmem_ld32(tS + 96, r3);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            x[e] = __uint_as_float(r0[e]);
-            x[32 + e] = __uint_as_float(r1[e]);
-            x[64 + e] = __uint_as_float(r2[e]);
-            x[96 + e] = __uint_as_float(r3[e]);
+          for (int e = 0; e < 16; ++e) {
+            x[e] = make_float2(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+            x[16 + e] = make_float2(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+            x[32 + e] = make_float2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1]));
           }
         }
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->s_free[g]);
-        float ascale = alpha;
+        SWIN_TC_MARK(2);
         const uint32_t u = ku0 + j, ust = u % kStages;
-        if (MODE != 0) {
-          // the block's K scales (mode 2: one per block, mode 1: 1/|k| per
-          // column) were written by prep before it released kv_ready
+        if (MODE == 1) {
+          // 1/|k| of the block's keys was written by prep before it released kv_ready
           ok = wait_bar(&bars->kv_ready[ust], (u / kStages) & 1, ctl);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          if (MODE == 2) ascale = alpha * kscale[ust];
         }
-        const float4* kc4 = reinterpret_cast<const float4*>(kcol + ust * 128);
-        const int nk_all = tk.n - j * tk.R * tk.lx;
-        const int nk = nk_all < tk.R * tk.lx ? nk_all : tk.R * tk.lx;
-        const int jb = bbase - j * tk.R * R2;
-        float mb = -INFINITY;
+        const float ascale = alpha;
+        const int nk_all = tk.n - j * tk.Rk * tk.lx;
+        const int nk = nk_all < tk.Rk * tk.lx ? nk_all : tk.Rk * tk.lx;
+        // x = log2-domain logits.  Mode 2: the scale is applied inside the
+        // exponent below (max over raw scores, scale > 0).
+        if (MODE == 1) {
+          const float4* kc4 = reinterpret_cast<const float4*>(kcol + ust * 128);
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float v;
-          if (MODE == 1) {
-            const float4 kc = kc4[c >> 2];  // same address in every lane: broadcast
-            const float kcv = (c & 3) == 0 ? kc.x : (c & 3) == 1 ? kc.y : (c & 3) == 2 ? kc.z : kc.w;
-            v = (x[c] * kcv) * ascale;
-          } else {
-            v = x[c] * ascale;
+          for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+            const float4 kc = kc4[c4];  // same address in every lane: broadcast
+            x[2 * c4] = __fmul2_rn(x[2 * c4], make_float2(kc.x * ascale, kc.y * ascale));
+            x[2 * c4 + 1] = __fmul2_rn(x[2 * c4 + 1], make_float2(kc.z * ascale, kc.w * ascale));
           }
-          if (MODE != 2) {
-            if (tab != nullptr && row_ok && c < nk)
-              v = fmaf(__ldg(tab + (size_t)(jb - kof[c]) * p.heads + tk.h), kLog2eF, v);
-          }
-          v = c < nk ? v : -INFINITY;
-          x[c] = v;
-          mb = fmaxf(mb, v);
+        } else if (MODE == 0) {
+          const float2 a2 = make_float2(ascale, ascale);
+#pragma unroll
+          for (int c = 0; c < kBlk / 2; ++c) x[c] = __fmul2_rn(x[c], a2);
         }
+        if (MODE != 2 && p.table != nullptr) {
+          const int jb = bbase - j * tk.Rk * R2;
+          const int lim = row_ok ? nk : 0;
+          if (bias_in_smem) {
+            const int4* kof4 = reinterpret_cast<const int4*>(kof);
+            const float* hb = sbias + tk.h * R2sq + jb;
+#pragma unroll
+            for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+              const int4 ko = kof4[c4];  // broadcast
+              if (4 * c4 + 0 < lim) x[2 * c4].x += hb[-ko.x];
+              if (4 * c4 + 1 < lim) x[2 * c4].y += hb[-ko.y];
+              if (4 * c4 + 2 < lim) x[2 * c4 + 1].x += hb[-ko.z];
+              if (4 * c4 + 3 < lim) x[2 * c4 + 1].y += hb[-ko.w];
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < kBlk; ++c) {
+              if (c < lim) {
+                const float tv = __ldg(p.table + (size_t)(jb - kof[c]) * p.heads + tk.h);
+                if (c & 1)
+                  x[c >> 1].y = __fmaf_rn(tv, kLog2eF, x[c >> 1].y);
+                else
+                  x[c >> 1].x = __fmaf_rn(tv, kLog2eF, x[c >> 1].x);
+              }
+            }
+          }
+        }
+        if (nk < kBlk) {  // partial block (uniform across the warpgroup): mask the tail keys
+#pragma unroll
+          for (int c = 0; c < kBlk / 2; ++c) {
+            if (2 * c >= nk) x[c].x = -INFINITY;
+            if (2 * c + 1 >= nk) x[c].y = -INFINITY;
+          }
+        }
+        // block maximum: four independent 3-input max chains
+        float mq[4] = {x[0].x, x[0].y, x[1].x, x[1].y};
+#pragma unroll
+        for (int c = 2; c < kBlk / 2; c += 4) {
+          mq[0] = ptx::max3(mq[0], x[c].x, x[c + 2].x);
+          mq[1] = ptx::max3(mq[1], x[c].y, x[c + 2].y);
+          mq[2] = ptx::max3(mq[2], x[c + 1].x, x[c + 3].x);
+          mq[3] = ptx::max3(mq[3], x[c + 1].y, x[c + 3].y);
+        }
+        float mb = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        if (MODE == 2) mb *= ascale;
+        SWIN_TC_MARK(3);
+        // running maximum, kept unless this block exceeds it by more than 8
         float factor = 1.f;
         bool rescale = false;
         if (j == 0) {
           m_run = mb;
-        } else if (mb > m_run) {
+        } else if (mb > m_run + 8.0f) {
           factor = ptx::ex2_approx(m_run - mb);
           m_run = mb;
           rescale = true;
         }
-        if (j > 0) {
-          // PV of the previous block must be done: it reads P and writes O
-          ok = wait_bar(&bars->o_done[g], o_cnt & 1, ctl);
-          ok = __all_sync(0xffffffffu, ok);
-          ++o_cnt;
+        // keep PV completions consumed in order (PV(blk - 2) was issued two
+        // blocks ago, so this rarely waits)
+        if (blk >= 2) {
+          ok = consume_pv(blk - 2);
           if (!ok) break;
-          ptx::tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {
-            // O and its row-sum column follow the new maximum
-            uint32_t o[32], o2[16];
-            ptx::tmem_ld32(tO, o);
-            ptx::tmem_ld16(tO + 32, o2);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o2[e] = __float_as_uint(__uint_as_float(o2[e]) * factor);
-            ptx::tmem_st32(tO, o);
-            ptx::tmem_st16(tO + 32, o2);
-          }
         }
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O and its row-sum column follow the new maximum
+          ok = consume_pv(blk - 1);
+          if (!ok) break;
+          uint32_t o[32], o2[16];
+          ptx::tmem_ld32(tO, o);
+          ptx::tmem_ld16(tO + 32, o2);
+          ptx::tmem_wait_ld();
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t pk[32];
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) o2[e] = __float_as_uint(__uint_as_float(o2[e]) * factor);
+          ptx::tmem_st32(tO, o);
+          ptx::tmem_st16(tO + 32, o2);
+        }
+        SWIN_TC_MARK(4);
+        // probabilities, fp16, written over the scores
+        // exponent argument: mode 2  x * ascale - m,  modes 0/1  x - m
+        const float ea = MODE == 2 ? ascale : 1.0f, eb = -m_run;
+        {
+          uint32_t pa[32], pb[16];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const float p0 = ptx::ex2_approx(x[64 * hf + 2 * c] - m_run);
-            const float p1 = ptx::ex2_approx(x[64 * hf + 2 * c + 1] - m_run);
-            pk[c] = ptx::pack_bf16x2(p0, p1);
+            const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
+            pa[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
           }
-          ptx::tmem_st32(tP + 32 * hf, pk);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float2 e = __ffma2_rn(x[32 + c], make_float2(ea, ea), make_float2(eb, eb));
+            pb[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+          }
+          SWIN_TC_MARK(5);
+          uint32_t po[32], po2[16];  // previous item's O (deferred epilogue)
+          const bool epi = j == 0 && pend;
+          if (epi) {
+            ok = consume_pv(blk - 1);
+            if (!ok) break;
+            ptx::tmem_ld32(tO, po);
+            ptx::tmem_ld16(tO + 32, po2);
+          }
+          ptx::tmem_st32(tS, pa);
+          ptx::tmem_st16(tS + 32, pb);
+          if (epi) ptx::tmem_wait_ld();
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bars->p_full[g][blk & 1]);
+          SWIN_TC_MARK(6);
+          if (epi) {
+            store_rows(po, po2, pend_off, pend_ok);
+            pend = false;
+          }
         }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&bars->p_full[g]);
+        SWIN_TC_MARK(7);
       }
       if (!ok) break;
-      // epilogue: O / l to global memory
-      ok = wait_bar(&bars->o_done[g], o_cnt & 1, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-      ++o_cnt;
-      if (!ok) break;
-      ptx::tc_fence_after();
-      uint32_t o[32], o2[16];
-      ptx::tmem_ld32(tO, o);
-      ptx::tmem_ld16(tO + 32, o2);
-      ptx::tmem_wait_ld();
-      if (row_ok) {
-        const float inv = 1.0f / __uint_as_float(o2[0]);  // row sum of the bf16 P
-        const size_t tok = ((size_t)tk.b * p.H + (tk.y0 + qy)) * p.W + (tk.x0 + qx);
-        const size_t off = tok * (size_t)(p.heads * 32) + (size_t)tk.h * 32;
-        if (OUT_F32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            dst[c] = make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
-                                 __uint_as_float(o[4 * c + 2]) * inv, __uint_as_float(o[4 * c + 3]) * inv);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + off);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = ptx::pack_bf16x2(__uint_as_float(o[8 * c + 2 * e]) * inv, __uint_as_float(o[8 * c + 2 * e + 1]) * inv);
-            dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        }
+      // this item's O is read in the next item's first block (or after the loop)
+      SWIN_TC_MARK(8);
+      pend = true;
+      pend_ok = row_ok;
+      pend_off = (((size_t)tk.b * p.H + (tk.y0 + qy)) * p.W + (tk.x0 + qx)) * (size_t)(p.heads * 32) +
+                 (size_t)tk.h * 32;
+      SWIN_TC_MARK(10);
+    }
+    if (ok && pend) {
+      ok = consume_pv(blk - 1);
+      if (ok) {
+        uint32_t po[32], po2[16];
+        ptx::tmem_ld32(tO, po);
+        ptx::tmem_ld16(tO + 32, po2);
+        ptx::tmem_wait_ld();
+        store_rows(po, po2, pend_off, pend_ok);
       }
     }
   }
@@ -811,12 +954,13 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   int tiles_max = 1;
   for (int c = 0; c < 3; ++c) {
     p.lx[c] = lxs[c];
-    p.R[c] = 128 / lxs[c];
-    if (p.R[c] > 256) p.R[c] = 256;
+    p.R[c] = 128 / lxs[c];    // query tile: whole rectangle rows, at most 128 queries
+    p.Rk[c] = kBlk / lxs[c];  // K/V block: whole rectangle rows, at most 96 keys
     const int tl = (a.M + p.R[c] - 1) / p.R[c];
     if (tl > tiles_max) tiles_max = tl;
-    if (!encode_map(&p.tmap[0][c], a.q, a, p.lx[c], p.R[c]) || !encode_map(&p.tmap[1][c], a.k, a, p.lx[c], p.R[c]) ||
-        !encode_map(&p.tmap[2][c], a.v, a, p.lx[c], p.R[c]))
+    if (!encode_map(&p.tmap[0][c], a.q, a, p.lx[c], p.R[c]) ||
+        !encode_map(&p.tmap[1][c], a.k, a, p.lx[c], p.Rk[c]) ||
+        !encode_map(&p.tmap[2][c], a.v, a, p.lx[c], p.Rk[c]))
       return fail(SWIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (lx=%d, R=%d)", p.lx[c], p.R[c]);
   }
   p.pmax = (tiles_max + 1) / 2;

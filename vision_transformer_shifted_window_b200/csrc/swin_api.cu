@@ -165,7 +165,10 @@ swin_status swin_stream_status(swin_stream_t stream) {
   if (cudaMemcpy(&val, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(SWIN_ERR_CUDA, "reading the device status word failed");
-  if (val != 0) return fail((swin_status)val, "a kernel reported status %d (bounded wait ran out)", val);
+  if (val & SWIN_ERR_TIMEOUT) return fail(SWIN_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+  if (val & SWIN_ERR_UNSUPPORTED)
+    return fail(SWIN_ERR_UNSUPPORTED, "a V entry of magnitude >= 2^22 was saturated on the tensor-core path");
+  if (val != 0) return fail(SWIN_ERR_CUDA, "unknown device status %d", val);
   return SWIN_OK;
 }
 
