@@ -61,8 +61,29 @@
 
 namespace swin {
 
+// Division by a launch constant with a multiply and a shift (Granlund and
+// Montgomery's method): n / d = (umulhi(m, n) + n) >> l for n < 2^31, with
+// l = ceil(log2 d) and m = floor(2^32 (2^l - d) / d) + 1.
+struct FastDiv {
+  uint32_t d, m, l;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.l = 0;
+  while ((1ull << f.l) < d) ++f.l;
+  f.m = (uint32_t)(((1ull << 32) * ((1ull << f.l) - d)) / d + 1);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return (__umulhi(f.m, n) + n) >> f.l;
+}
+
 struct TcParams {
   CUtensorMap tmap[3][3];  // [tensor q/k/v][x-class first/middle/last]
+  FastDiv div_pmax, div_nsx, div_nsy, div_heads;
   int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
   void* out;
   int B, H, W, heads, M, s, nsy, nsx, pmax;
@@ -77,7 +98,8 @@ struct TcParams {
 
 namespace {
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+constexpr int kPrepThreads = 192;  // warps 2-3 and 12-15
 constexpr int kStages = 6;                  // K/V ring
 constexpr int kTileBytes = 128 * 64;        // 128 rows x 32 16-bit values
 constexpr int kBlk = 96;                    // keys per K/V block (TMEM: 2 x 96 + 48 columns per warpgroup)
@@ -91,7 +113,8 @@ constexpr int kRposOff = kKofsOff + 3 * 128 * 4;             // [3][128] int: (r
 constexpr int kKcolOff = kRposOff + 3 * 128 * 4;             // [kStages][128] f32, 1/|k| (mode 1)
 constexpr int kBiasFloats = 16384;                           // bias tables of all heads if they fit
 constexpr int kBiasOff = kKcolOff + kStages * 128 * 4;
-constexpr int kBarOff = kBiasOff + kBiasFloats * 4;
+constexpr int kDescOff = kBiasOff + kBiasFloats * 4;          // MMA operand descriptors, counters (256 B)
+constexpr int kBarOff = kDescOff + 256;
 constexpr int kNumBars = 12 + 3 * kStages + 12 + 2;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
@@ -118,15 +141,19 @@ struct Task {
 
 __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
   Task t;
-  long long i = item;
-  const int pr = (int)(i % p.pmax);
-  i /= p.pmax;
-  const int sx = (int)(i % p.nsx);
-  i /= p.nsx;
-  const int sy = (int)(i % p.nsy);
-  i /= p.nsy;
-  t.h = (int)(i % p.heads);
-  t.b = (int)(i / p.heads);
+  uint32_t i = (uint32_t)item;
+  uint32_t q = fdiv(i, p.div_pmax);
+  const int pr = (int)(i - q * p.div_pmax.d);
+  i = q;
+  q = fdiv(i, p.div_nsx);
+  const int sx = (int)(i - q * p.div_nsx.d);
+  i = q;
+  q = fdiv(i, p.div_nsy);
+  const int sy = (int)(i - q * p.div_nsy.d);
+  i = q;
+  q = fdiv(i, p.div_heads);
+  t.h = (int)(i - q * p.div_heads.d);
+  t.b = (int)q;
   t.cls = sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1);
   t.lx = p.lx[t.cls];
   t.R = p.R[t.cls];
@@ -254,6 +281,61 @@ __device__ __forceinline__ float absmax(const float (&v)[32]) {
   return m;
 }
 
+// Half rows: channels [16 h, 16 h + 16) = 16-byte chunks 2h and 2h + 1.
+__device__ __forceinline__ void load_half_bf16(const uint8_t* tile, int row, int h, float (&v)[16]) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const uint4 w = *reinterpret_cast<const uint4*>(tile + swz64(row, 2 * h + c));
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * c + 2 * e] = bf_lo(u[e]);
+      v[8 * c + 2 * e + 1] = bf_hi(u[e]);
+    }
+  }
+}
+
+__device__ __forceinline__ void store_half_f16(uint8_t* tile, int row, int h, const float (&v)[16], float sc) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t u[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) u[e] = ptx::pack_f16x2_sat(v[8 * c + 2 * e] * sc, v[8 * c + 2 * e + 1] * sc);
+    *reinterpret_cast<uint4*>(tile + swz64(row, 2 * h + c)) = make_uint4(u[0], u[1], u[2], u[3]);
+  }
+}
+
+// Rotate the 8 channel pairs of one half by position pos of its axis (half 0:
+// rows, half 1: columns).
+__device__ __forceinline__ void rope_half(float (&v)[16], int h, int pos, const float* rc, const float* rs) {
+  const float4* cs4 = reinterpret_cast<const float4*>(rc + (h * 64 + pos) * 8);
+  const float4* sn4 = reinterpret_cast<const float4*>(rs + (h * 64 + pos) * 8);
+  const float4 c0 = cs4[0], c1 = cs4[1], s0 = sn4[0], s1 = sn4[1];
+  const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const float a = v[2 * t], b = v[2 * t + 1];
+    // explicit roundings: every instantiation of the kernel computes the same bits
+    v[2 * t] = __fmaf_rn(a, cs[t], -__fmul_rn(b, sn[t]));
+    v[2 * t + 1] = __fmaf_rn(a, sn[t], __fmul_rn(b, cs[t]));
+  }
+}
+
+__device__ __forceinline__ float half_absmax(const float (&v)[16]) {
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
+  return m;
+}
+
+__device__ __forceinline__ float half_sumsq(const float (&v)[16]) {
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) ss = fmaf(v[e], v[e], ss);
+  return ss;
+}
+
 // Largest |value| of one 32-element bf16 row (packed bf16x2 arithmetic).
 __device__ __forceinline__ float row_absmax_bf16(const uint8_t* tile, int row) {
   __nv_bfloat162 m = __float2bfloat162_rn(0.f);
@@ -293,6 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   int* rpos = reinterpret_cast<int*>(smem + kRposOff);
   float* kcol = reinterpret_cast<float*>(smem + kKcolOff);
   float* sbias = reinterpret_cast<float*>(smem + kBiasOff);  // [heads][(2M-1)^2], times log2(e)
+  uint64_t* mdesc = reinterpret_cast<uint64_t*>(smem + kDescOff);  // q[2][2], k[S], v[S]
+  uint32_t* mrem = reinterpret_cast<uint32_t*>(mdesc + 4 + 2 * kStages);  // [S] consumers left, [S] tag
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -305,12 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int g = 0; g < 2; ++g)
       for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(&bars->q_full[g][b], 1);
-        ptx::mbar_init(&bars->q_ready[g][b], 64);
+        ptx::mbar_init(&bars->q_ready[g][b], kPrepThreads);
         ptx::mbar_init(&bars->q_empty[g][b], 1 + 4);
       }
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(&bars->kv_full[i], 1);
-      ptx::mbar_init(&bars->kv_ready[i], 64);
+      ptx::mbar_init(&bars->kv_ready[i], kPrepThreads);
       ptx::mbar_init(&bars->kv_empty[i], 1);
     }
     for (int g = 0; g < 2; ++g) {
@@ -362,6 +446,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     ptx::tmem_alloc(tmem_holder, 512);
     ptx::tmem_relinquish();
   }
+  if (threadIdx.x < 4 + 2 * kStages) {
+    // operand descriptors (64-byte swizzle): Q tiles and K blocks K-major
+    // (SBO 512), V blocks MN-major with the stage's constant column block at
+    // leading-byte distance (N columns 32-47)
+    const int i = threadIdx.x;
+    if (i < 4) {
+      mdesc[i] = ptx::smem_desc(ptx::smem_addr(qbuf + i * kTileBytes), 16, 512, ptx::kSwizzle64B);
+    } else if (i < 4 + kStages) {
+      mdesc[i] = ptx::smem_desc(ptx::smem_addr(kvbuf + (i - 4) * 2 * kTileBytes), 16, 512, ptx::kSwizzle64B);
+    } else {
+      const int st = i - 4 - kStages;
+      const uint32_t va = ptx::smem_addr(kvbuf + st * 2 * kTileBytes + kTileBytes);
+      const uint32_t oa = ptx::smem_addr(ones + st * 1024);
+      mdesc[i] = ptx::smem_desc(va, oa - va, 512, ptx::kSwizzle64B);
+    }
+  }
+  if (threadIdx.x < kStages) {
+    mrem[threadIdx.x] = 0;
+    mrem[kStages + threadIdx.x] = 0xffffffffu;
+  }
   if (warp == 0 && lane == 0)
     for (int t = 0; t < 3; ++t)
       for (int c = 0; c < 3; ++c) ptx::prefetch_tmap(&p.tmap[t][c]);
@@ -373,10 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   Ctl ctl{abort_flag, &p};
   const long long first = blockIdx.x, step = gridDim.x;
 
-  // Register split: warps 0-3 (producer, MMA, prep) give registers to the two
-  // softmax warpgroups: 384 x 168 = 128 x 88 + 256 x 208.
-  if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+  // Register split: warpgroups 0 (producer, MMA, prep) and 3 (prep) give
+  // registers to the two softmax warpgroups: 512 x 128 = 256 x 64 + 256 x 192.
+  if (warp < 4 || warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
     if (warp == 0) {
       // ============================================================== producer
       if (lane == 0) {
@@ -427,6 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
         constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlk, 128);
         constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
+        (void)ones;
         bool ok = true;
         if (p.debug_flags & 1) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
 
@@ -469,11 +574,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           next_item(cp[g], g);
         }
         uint32_t s_iss[2] = {0, 0}, pv_iss[2] = {0, 0};
-        uint32_t rem[kStages], tag[kStages];
-        for (int i = 0; i < kStages; ++i) {
-          rem[i] = 0;
-          tag[i] = 0xffffffffu;
-        }
         long long idle_since = clock64();
         while (ok && (cs[0].live || cs[1].live || cp[0].live || cp[1].live)) {
           bool progress = false;
@@ -487,14 +587,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                                  ptx::mbar_test(&bars->kv_ready[st], (u / kStages) & 1);
               if (ready) {
                 ptx::tc_fence_after();
-                if (tag[st] != u) {  // first use of this K/V block: count its consumers
-                  tag[st] = u;
-                  rem[st] = (uint32_t)c.nvalid;
+                if (mrem[kStages + st] != u) {  // first use of this K/V block: count its consumers
+                  mrem[kStages + st] = u;
+                  mrem[st] = (uint32_t)c.nvalid;
                 }
-                const uint32_t qa = ptx::smem_addr(qbuf + (g * 2 + c.qs) * kTileBytes);
-                const uint32_t ka = ptx::smem_addr(kvbuf + st * 2 * kTileBytes);
-                const uint64_t ad = ptx::smem_desc(qa, 16, 512, ptx::kSwizzle64B);
-                const uint64_t bd = ptx::smem_desc(ka, 16, 512, ptx::kSwizzle64B);
+                const uint64_t ad = mdesc[g * 2 + c.qs], bd = mdesc[4 + st];
                 const uint32_t dS = tmem_base + g * 256 + (s_iss[g] & 1) * kBlk;
                 ptx::mma_ss(dS, ad, bd, idS, 0);
                 ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
@@ -511,20 +608,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 ptx::mbar_test(&bars->p_full[g][pv_iss[g] & 1], (pv_iss[g] >> 1) & 1)) {
               ptx::tc_fence_after();
               const uint32_t u = d.u0 + d.j, st = u % kStages;
-              const uint32_t va = ptx::smem_addr(kvbuf + st * 2 * kTileBytes + kTileBytes);
-              const uint32_t oa = ptx::smem_addr(ones + st * 1024);
+              const uint64_t vd = mdesc[4 + kStages + st];
               const uint32_t dO = tmem_base + g * 256 + 2 * kBlk;
               const uint32_t aP = tmem_base + g * 256 + (pv_iss[g] & 1) * kBlk;
+              // k-step kk: V rows 16 kk.. (+1024 bytes) with the constant block at
+              // the same place (leading byte offset 1024 bytes shorter)
+              constexpr uint64_t kStep = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
+              ptx::mma_ts(dO, aP, vd, idPV, d.j > 0 ? 1u : 0u);
 #pragma unroll
-              for (int kk = 0; kk < kBlk / 16; ++kk) {
-                // N columns 0-31: V rows; 32-47: the stage's constant block (LBO = its distance)
-                const uint32_t vk = va + kk * 1024;
-                const uint64_t bd = ptx::smem_desc(vk, oa - vk, 512, ptx::kSwizzle64B);
-                ptx::mma_ts(dO, aP + kk * 8, bd, idPV, (d.j > 0 || kk > 0) ? 1u : 0u);
-              }
+              for (int kk = 1; kk < kBlk / 16; ++kk) ptx::mma_ts(dO, aP + kk * 8, vd + kk * kStep, idPV, 1u);
               ptx::mma_commit(&bars->o_done[g][pv_iss[g] & 1]);
               ++pv_iss[g];
-              if (--rem[st] == 0) ptx::mma_commit(&bars->kv_empty[st]);
+              if (--mrem[st] == 0) ptx::mma_commit(&bars->kv_empty[st]);
               if (++d.j == d.nb) next_item(d, g);
               progress = true;
             }
@@ -547,7 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
     } else {
       // ============================================================== prep
-      const int pt = threadIdx.x - 64;  // 0..63
+      // 192 threads (warps 2-3 and 12-15); work in half rows (16 channels):
+      // the two halves of a row sit in adjacent lanes, and each half of a
+      // RoPE row rotates along one axis only.
+      const int pt = warp < 4 ? (int)threadIdx.x - 64 : (int)threadIdx.x - 384 + 64;  // 0..191
       uint32_t qu[2] = {0, 0}, ku = 0;
       bool ok = true;
       bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
@@ -567,17 +665,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           uint8_t* tile = qbuf + (g * 2 + qs) * kTileBytes;
           const float te = MODE == 1 ? fmaxf(__ldg(p.tau + t.h), kTauMin) : 1.f;
           if (MODE != 0) {
-            for (int r = pt; r < qrows; r += 64) {
-              float v[32];
-              load_row_bf16(tile, r, v);
+#pragma unroll 1
+            for (int u = pt; u < 2 * 128; u += kPrepThreads) {  // uniform trip count per lane pair
+              const int r = u >> 1, h = u & 1;
+              const bool act = r < qrows;
+              float v[16];
+              if (act) load_half_bf16(tile, r, h, v);
+              else for (int e = 0; e < 16; ++e) v[e] = 0.f;
               if (MODE == 1) {
-                qscale[(g * 2 + qs) * 128 + r] = kLog2eF * inv_norm(v) / te;
+                float ss = half_sumsq(v);
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                if (act && h == 0)
+                  qscale[(g * 2 + qs) * 128 + r] = kLog2eF / (fmaxf(sqrtf(ss), kNormEps) * te);
               } else {
-                const int pr = rp[r];
-                rope_rotate(v, min(py0 + t.tile[g] * t.R + (pr & 0xFFFF), 63), px0 + (pr >> 16), rcos, rsin);
-                const float sc = pow2_scale(absmax(v));  // exact per-row scale, undone in the softmax
-                store_row_f16(tile, r, v, sc);
-                qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
+                if (act) {
+                  const int pr = rp[r];
+                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + t.tile[g] * t.R + (pr & 0xFFFF), 63), rcos,
+                            rsin);
+                }
+                float m = half_absmax(v);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                const float sc = pow2_scale(m);  // exact per-row scale, undone in the softmax
+                if (act) {
+                  store_half_f16(tile, r, h, v, sc);
+                  if (h == 0) qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
+                }
               }
             }
             ptx::fence_proxy_async_smem();
@@ -591,30 +703,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!ok) break;
           uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
           uint8_t* vtile = ktile + kTileBytes;
-          // K rows pt, pt + 64 and V rows 63 - pt, 127 - pt (rows < krows <= 96):
-          // each prep warp carries 1.5 rows of each.  Rows are independent: fp16
-          // with saturation, a saturated entry is reported after the loop.
-#pragma unroll 1
-          for (int i = 0; i < 2; ++i) {
-            const int krow = pt + 64 * i, vrow = 63 - pt + 64 * i;
-            if (MODE != 0 && krow < krows) {
-              float v[32];
-              load_row_bf16(ktile, krow, v);
-              if (MODE == 1) {
-                kcol[st * 128 + krow] = inv_norm(v);
-              } else {
-                const int pr = rp[krow];
-                rope_rotate(v, min(py0 + j * t.Rk + (pr & 0xFFFF), 63), px0 + (pr >> 16), rcos, rsin);
-                range_hit |= absmax(v) >= 65504.0f;
-                store_row_f16_sat(ktile, krow, v, 1.0f);
-              }
+          // this thread: half h of K row r and half h of V row r (r < krows <= 96);
+          // fp16 with saturation, a saturated entry is reported after the loop
+          const int r = pt >> 1, h = pt & 1;
+          const bool act = r < krows;
+          if (MODE != 0) {
+            float v[16];
+            if (act) load_half_bf16(ktile, r, h, v);
+            else for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            if (MODE == 1) {
+              float ss = half_sumsq(v);
+              ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+              if (act && h == 0) kcol[st * 128 + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
+            } else if (act) {
+              const int pr = rp[r];
+              rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + j * t.Rk + (pr & 0xFFFF), 63), rcos, rsin);
+              range_hit |= half_absmax(v) >= 65504.0f;
+              store_half_f16(ktile, r, h, v, 1.0f);
             }
-            if (vrow < krows) {
-              range_hit |= row_absmax_bf16(vtile, vrow) >= 65504.0f;
-              float v[32];
-              load_row_bf16(vtile, vrow, v);
-              store_row_f16_sat(vtile, vrow, v, 1.0f);
-            }
+          }
+          if (act) {
+            float v[16];
+            load_half_bf16(vtile, r, h, v);
+            range_hit |= half_absmax(v) >= 65504.0f;
+            store_half_f16(vtile, r, h, v, 1.0f);
           }
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(&bars->kv_ready[st]);
@@ -623,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (range_hit) atomicOr(p.status, (int)SWIN_ERR_UNSUPPORTED);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
     // ================================================================ softmax
     const int g = (warp - 4) >> 2;              // warpgroup 0 or 1
     const int t = threadIdx.x - 128 - g * 128;  // row of the tile = TMEM lane
@@ -965,6 +1077,11 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   }
   p.pmax = (tiles_max + 1) / 2;
   p.n_items = (long long)a.B * a.heads * p.nsy * p.nsx * p.pmax;
+  if (p.n_items >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "too many work items (%lld)", p.n_items);
+  p.div_pmax = make_fastdiv((uint32_t)p.pmax);
+  p.div_nsx = make_fastdiv((uint32_t)p.nsx);
+  p.div_nsy = make_fastdiv((uint32_t)p.nsy);
+  p.div_heads = make_fastdiv((uint32_t)a.heads);
   p.out = a.out;
   p.tau = a.tau;
   p.table = a.table;
