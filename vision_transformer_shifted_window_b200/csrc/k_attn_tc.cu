@@ -13,12 +13,14 @@
 // whole rectangle rows), one per softmax warpgroup; both warpgroups stream
 // the same K/V blocks of floor(96 / lx) rectangle rows (at most 96 keys).
 //
-// Warp roles (384 threads, one persistent CTA per SM):
+// Warp roles (512 threads, one persistent CTA per SM):
 //   warp 0      TMA producer: Q tiles and K/V blocks, 5-D tensor maps over
 //               [B][H][W][heads][d] with 64-byte swizzle, no multicast
-//   warp 1      tcgen05.mma issuer (one thread) and TMEM owner
-//   warps 2-3   operand prep in shared memory: K unit-normalisation (mode 1),
-//               RoPE rotation of Q and K (mode 2), per-row 1/(tau |q|) (mode 1)
+//   warps 1, 2  tcgen05.mma issuers, one thread each: warp 1 + g issues the
+//               MMAs of softmax warpgroup g; warp 1 owns TMEM
+//   warps 3, 12-15  operand prep in shared memory: K unit-normalisation
+//               (mode 1), RoPE rotation of Q and K (mode 2), per-row
+//               1/(tau |q|) (mode 1), V to fp16
 //   warps 4-7   softmax of warpgroup 0 (one TMEM lane = one query row)
 //   warps 8-11  softmax of warpgroup 1
 // TMEM per softmax warpgroup g (128 lanes): two score buffers X0, X1 of 96
@@ -26,16 +28,16 @@
 // of P).  Block b's scores S = Q K^T land in X[b % 2]; the softmax turns them
 // into fp16 probabilities P written over the same columns, and O += P [V | c]
 // (6 MMAs, N = 48, A from TMEM) reads them there.  With two buffers the
-// softmax never waits for the previous block's PV; the tensor core executes
-// in order, so S(b+2) cannot overwrite P(b) before PV(b) has read it.
+// softmax never waits for the previous block's PV; a thread's MMAs execute
+// in issue order, so S(b+2) cannot overwrite P(b) before PV(b) has read it.
 //
 // Softmax: online, with the running maximum kept until a block exceeds it by
 // more than 8 (log2 units), so O is rescaled rarely; P in fp16 (values up to
-// 2^15) keeps that accurate.  V is converted to fp16 by the prep warps with a
-// power-of-two scale 2^-k per block (k = 0 unless |v| >= 2^15, at most 7);
-// the same block's P carries 2^k in its exponent and its ones column holds
-// 2^-k, so O and the row sum stay exact.  V entries of 2^22 or more saturate
-// and record SWIN_ERR_UNSUPPORTED in the status word.
+// 2^8) keeps that accurate.  V is converted to fp16 by the prep warps; the
+// constant column c = 1 of [V | c] makes the same MMAs accumulate the row sum
+// of the fp16 P, so O / l uses exactly the probabilities that weighted V.
+// V entries of magnitude 65504 or more saturate and record
+// SWIN_ERR_UNSUPPORTED in the status word.
 //
 // Precision of the score operands: mode 0 multiplies the bf16 inputs as they
 // are; mode 1 also multiplies the raw inputs and applies 1/|q| (per row),
@@ -99,7 +101,7 @@ struct TcParams {
 namespace {
 
 constexpr int kThreads = 512;
-constexpr int kPrepThreads = 192;  // warps 2-3 and 12-15
+constexpr int kPrepThreads = 160;  // warps 3 and 12-15
 constexpr int kStages = 6;                  // K/V ring
 constexpr int kTileBytes = 128 * 64;        // 128 rows x 32 16-bit values
 constexpr int kBlk = 96;                    // keys per K/V block (TMEM: 2 x 96 + 48 columns per warpgroup)
@@ -113,9 +115,8 @@ constexpr int kRposOff = kKofsOff + 3 * 128 * 4;             // [3][128] int: (r
 constexpr int kKcolOff = kRposOff + 3 * 128 * 4;             // [kStages][128] f32, 1/|k| (mode 1)
 constexpr int kBiasFloats = 16384;                           // bias tables of all heads if they fit
 constexpr int kBiasOff = kKcolOff + kStages * 128 * 4;
-constexpr int kDescOff = kBiasOff + kBiasFloats * 4;          // MMA operand descriptors, counters (256 B)
-constexpr int kBarOff = kDescOff + 256;
-constexpr int kNumBars = 12 + 3 * kStages + 12 + 2;
+constexpr int kBarOff = kBiasOff + kBiasFloats * 4;
+constexpr int kNumBars = 12 + 3 * kStages + 12 + 3;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
@@ -128,15 +129,20 @@ struct Bars {
   // per warpgroup and score buffer: a barrier's next phase (block b + 2) can
   // only start after its current one was consumed, so parity tests never alias
   uint64_t s_full[2][2], p_full[2][2], o_done[2][2];
-  uint64_t never, drain;
+  uint64_t never, drain[2];
 };
 static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
 
 struct Task {
-  bool any;       // item has work for warpgroup 0
-  bool valid[2];  // per warpgroup
-  int b, h, cls, lx, R, Rk, y0, x0, ly, n, nb;
-  int tile[2], nq[2];
+  bool any;  // item has work (a query tile for warpgroup 0)
+  int b, h, cls, lx, R, Rk, y0, x0, ly, n, nb, pr, ntiles;
+  // warpgroup g's query tile: rectangle rows [tile(g) R, tile(g) R + R)
+  __device__ __forceinline__ int tile(int g) const { return 2 * pr + g; }
+  __device__ __forceinline__ bool valid(int g) const { return tile(g) < ntiles; }
+  __device__ __forceinline__ int nq(int g) const {  // queries of warpgroup g's tile
+    const int rows = ly - tile(g) * R;
+    return valid(g) ? (rows < R ? rows : R) * lx : 0;
+  }
 };
 
 __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
@@ -163,14 +169,9 @@ __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
   t.x0 = swin_seg_start(sx, p.M, p.s);
   t.n = t.ly * t.lx;
   t.nb = (t.ly + t.Rk - 1) / t.Rk;
-  const int ntiles = (t.ly + t.R - 1) / t.R;
-  for (int g = 0; g < 2; ++g) {
-    t.tile[g] = 2 * pr + g;
-    t.valid[g] = t.tile[g] < ntiles;
-    int rows = t.ly - t.tile[g] * t.R;
-    t.nq[g] = t.valid[g] ? (rows < t.R ? rows : t.R) * t.lx : 0;
-  }
-  t.any = t.valid[0];
+  t.pr = pr;
+  t.ntiles = (t.ly + t.R - 1) / t.R;
+  t.any = t.valid(0);
   return t;
 }
 
@@ -375,8 +376,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   int* rpos = reinterpret_cast<int*>(smem + kRposOff);
   float* kcol = reinterpret_cast<float*>(smem + kKcolOff);
   float* sbias = reinterpret_cast<float*>(smem + kBiasOff);  // [heads][(2M-1)^2], times log2(e)
-  uint64_t* mdesc = reinterpret_cast<uint64_t*>(smem + kDescOff);  // q[2][2], k[S], v[S]
-  uint32_t* mrem = reinterpret_cast<uint32_t*>(mdesc + 4 + 2 * kStages);  // [S] consumers left, [S] tag
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -395,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(&bars->kv_full[i], 1);
       ptx::mbar_init(&bars->kv_ready[i], kPrepThreads);
-      ptx::mbar_init(&bars->kv_empty[i], 1);
+      ptx::mbar_init(&bars->kv_empty[i], 2);  // one release per softmax warpgroup
     }
     for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < 2; ++b) {
@@ -405,7 +404,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
     }
     ptx::mbar_init(&bars->never, 1);
-    ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->drain[0], 1);
+    ptx::mbar_init(&bars->drain[1], 1);
     *abort_flag = 0;
     tmem_holder[2] = 0;  // abort flag of the drain waits (never set by a role)
     ptx::fence_mbar_init();
@@ -446,26 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     ptx::tmem_alloc(tmem_holder, 512);
     ptx::tmem_relinquish();
   }
-  if (threadIdx.x < 4 + 2 * kStages) {
-    // operand descriptors (64-byte swizzle): Q tiles and K blocks K-major
-    // (SBO 512), V blocks MN-major with the stage's constant column block at
-    // leading-byte distance (N columns 32-47)
-    const int i = threadIdx.x;
-    if (i < 4) {
-      mdesc[i] = ptx::smem_desc(ptx::smem_addr(qbuf + i * kTileBytes), 16, 512, ptx::kSwizzle64B);
-    } else if (i < 4 + kStages) {
-      mdesc[i] = ptx::smem_desc(ptx::smem_addr(kvbuf + (i - 4) * 2 * kTileBytes), 16, 512, ptx::kSwizzle64B);
-    } else {
-      const int st = i - 4 - kStages;
-      const uint32_t va = ptx::smem_addr(kvbuf + st * 2 * kTileBytes + kTileBytes);
-      const uint32_t oa = ptx::smem_addr(ones + st * 1024);
-      mdesc[i] = ptx::smem_desc(va, oa - va, 512, ptx::kSwizzle64B);
-    }
-  }
-  if (threadIdx.x < kStages) {
-    mrem[threadIdx.x] = 0;
-    mrem[kStages + threadIdx.x] = 0xffffffffu;
-  }
   if (warp == 0 && lane == 0)
     for (int t = 0; t < 3; ++t)
       for (int c = 0; c < 3; ++c) ptx::prefetch_tmap(&p.tmap[t][c]);
@@ -492,13 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!t.any) continue;
           const uint32_t qbytes = (uint32_t)(64 * t.lx * t.R), kbytes = (uint32_t)(64 * t.lx * t.Rk);
           for (int g = 0; g < 2 && ok; ++g) {
-            if (!t.valid[g]) continue;
+            if (!t.valid(g)) continue;
             const int qs = qu[g] & 1;
             if (qu[g] >= 2) ok = wait_bar(&bars->q_empty[g][qs], ((qu[g] >> 1) - 1) & 1, ctl);
             if (!ok) break;
             ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], qbytes);
             ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][t.cls], &bars->q_full[g][qs], 0, t.h,
-                             t.x0, t.y0 + t.tile[g] * t.R, t.b);
+                             t.x0, t.y0 + t.tile(g) * t.R, t.b);
             ++qu[g];
           }
           for (int j = 0; j < t.nb && ok; ++j) {
@@ -522,130 +502,99 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (uint32_t u = (qu[g] > 2 ? qu[g] - 2 : 0); u < qu[g]; ++u)
             wait_bar(&bars->q_full[g][u & 1], (u >> 1) & 1, drain);
       }
-    } else if (warp == 1) {
-      // ============================================================== MMA issuer
-      // Event-driven: each warpgroup's next S and next PV are probed without
-      // blocking and issued as soon as their inputs are ready.
+    } else if (warp == 1 || warp == 2) {
+      // ============================================================== MMA issuers
+      // One thread per softmax warpgroup g (warp 1 + g) issues that group's
+      // MMAs in program order: S(0), S(1), then for every later block b first
+      // PV(b - 2), as soon as P(b - 2) is in TMEM, and then S(b).  A thread's
+      // MMAs execute in issue order, so S(b) cannot overwrite P(b - 2) before
+      // PV(b - 2) has read it.
       if (lane == 0) {
+        const int g = warp - 1;
         // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
         constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
         constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlk, 128);
         constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
-        (void)ones;
+        // Operand descriptors (64-byte swizzle) of Q buffer 0 and K/V stage 0;
+        // the others differ only in the start-address field (16-byte units)
+        // and, for [V | c], in the leading byte offset to the stage's constant
+        // column block, which sits outside the ring (N columns 32-47).
+        const uint64_t qd0 = ptx::smem_desc(ptx::smem_addr(qbuf + g * 2 * kTileBytes), 16, 512, ptx::kSwizzle64B);
+        const uint64_t kd0 = ptx::smem_desc(ptx::smem_addr(kvbuf), 16, 512, ptx::kSwizzle64B);
+        const uint32_t va0 = ptx::smem_addr(kvbuf + kTileBytes), oa0 = ptx::smem_addr(ones);
+        const uint64_t vd0 = ptx::smem_desc(va0, oa0 - va0, 512, ptx::kSwizzle64B);
+        constexpr uint64_t kQBuf = kTileBytes >> 4;
+        constexpr uint64_t kStageK = (2 * kTileBytes) >> 4;
+        constexpr uint64_t kStageV = kStageK - ((uint64_t)((2 * kTileBytes - 1024) >> 4) << 16);
+        // k-step kk of PV: V rows 16 kk.. (+1024 bytes), constant block unchanged
+        constexpr uint64_t kStepV = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
+        const uint32_t tg = tmem_base + g * 256;
         bool ok = true;
         if (p.debug_flags & 1) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
-
-        struct Cur {
-          long long it_next;  // next item to examine
-          uint32_t u_next;    // K/V use index of the next item's first block
-          uint32_t qcnt;      // Q tiles taken so far
-          uint32_t u0, qpar;  // first K/V use of the current item; Q buffer phase
-          int j, nb, qs, nvalid;
-          bool live;
-        };
-        auto next_item = [&](Cur& c, int g) {
-          c.live = false;
-          while (c.it_next < p.n_items) {
-            const Task t = decode(p, c.it_next);
-            c.it_next += step;
-            if (!t.any) continue;
-            const uint32_t u0 = c.u_next;
-            c.u_next += t.nb;
-            if (!t.valid[g]) continue;
-            c.nb = t.nb;
-            c.nvalid = (int)t.valid[0] + (int)t.valid[1];
-            c.j = 0;
-            c.u0 = u0;
-            c.qs = c.qcnt & 1;
-            c.qpar = (c.qcnt >> 1) & 1;
-            ++c.qcnt;
-            c.live = true;
-            return;
-          }
-        };
-        Cur cs[2], cp[2];
-        for (int g = 0; g < 2; ++g) {
-          cs[g].it_next = first;
-          cs[g].u_next = 0;
-          cs[g].qcnt = 0;
-          cs[g].live = false;
-          cp[g] = cs[g];
-          next_item(cs[g], g);
-          next_item(cp[g], g);
-        }
-        uint32_t s_iss[2] = {0, 0}, pv_iss[2] = {0, 0};
-        long long idle_since = clock64();
-        while (ok && (cs[0].live || cs[1].live || cp[0].live || cp[1].live)) {
-          bool progress = false;
+        // blocks whose PV is still to be issued, by b & 1: stage | accumulate << 8 | second release << 9
+        uint32_t pend0 = 0, pend1 = 0;
+        auto issue_pv = [&](uint32_t k) -> bool {
+          if (!wait_bar(&bars->p_full[g][k & 1], (k >> 1) & 1, ctl)) return false;
+          ptx::tc_fence_after();
+          const uint32_t info = (k & 1) ? pend1 : pend0;
+          const uint32_t st = info & 0xffu;
+          const uint64_t vd = vd0 + st * kStageV;
+          const uint32_t aP = tg + (k & 1) * kBlk;
+          ptx::mma_ts(tg + 2 * kBlk, aP, vd, idPV, (info >> 8) & 1u);
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            // ---- S = Q K^T of warpgroup g's next block, into X[b % 2]
-            Cur& c = cs[g];
-            if (c.live && (s_iss[g] < 2 || pv_iss[g] + 1 >= s_iss[g])) {
-              const uint32_t u = c.u0 + c.j, st = u % kStages;
-              const bool ready = (c.j > 0 || ptx::mbar_test(&bars->q_ready[g][c.qs], c.qpar)) &&
-                                 ptx::mbar_test(&bars->kv_ready[st], (u / kStages) & 1);
-              if (ready) {
-                ptx::tc_fence_after();
-                if (mrem[kStages + st] != u) {  // first use of this K/V block: count its consumers
-                  mrem[kStages + st] = u;
-                  mrem[st] = (uint32_t)c.nvalid;
-                }
-                const uint64_t ad = mdesc[g * 2 + c.qs], bd = mdesc[4 + st];
-                const uint32_t dS = tmem_base + g * 256 + (s_iss[g] & 1) * kBlk;
-                ptx::mma_ss(dS, ad, bd, idS, 0);
-                ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
-                ptx::mma_commit(&bars->s_full[g][s_iss[g] & 1]);
-                ++s_iss[g];
-                if (c.j == c.nb - 1) ptx::mma_commit(&bars->q_empty[g][c.qs]);
-                if (++c.j == c.nb) next_item(c, g);
-                progress = true;
-              }
-            }
-            // ---- O += P [V | c] of warpgroup g's next block
-            Cur& d = cp[g];
-            if (d.live && pv_iss[g] < s_iss[g] &&
-                ptx::mbar_test(&bars->p_full[g][pv_iss[g] & 1], (pv_iss[g] >> 1) & 1)) {
-              ptx::tc_fence_after();
-              const uint32_t u = d.u0 + d.j, st = u % kStages;
-              const uint64_t vd = mdesc[4 + kStages + st];
-              const uint32_t dO = tmem_base + g * 256 + 2 * kBlk;
-              const uint32_t aP = tmem_base + g * 256 + (pv_iss[g] & 1) * kBlk;
-              // k-step kk: V rows 16 kk.. (+1024 bytes) with the constant block at
-              // the same place (leading byte offset 1024 bytes shorter)
-              constexpr uint64_t kStep = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
-              ptx::mma_ts(dO, aP, vd, idPV, d.j > 0 ? 1u : 0u);
-#pragma unroll
-              for (int kk = 1; kk < kBlk / 16; ++kk) ptx::mma_ts(dO, aP + kk * 8, vd + kk * kStep, idPV, 1u);
-              ptx::mma_commit(&bars->o_done[g][pv_iss[g] & 1]);
-              ++pv_iss[g];
-              if (--mrem[st] == 0) ptx::mma_commit(&bars->kv_empty[st]);
-              if (++d.j == d.nb) next_item(d, g);
-              progress = true;
-            }
-          }
-          if (progress) {
-            idle_since = clock64();
-          } else {
-            if (*abort_flag) break;
-            if (clock64() - idle_since > p.wait_limit) {
-              atomicOr(p.status, (int)SWIN_ERR_TIMEOUT);
-              *abort_flag = 1;
-              break;
-            }
+          for (int kk = 1; kk < kBlk / 16; ++kk) ptx::mma_ts(tg + 2 * kBlk, aP + kk * 8, vd + kk * kStepV, idPV, 1u);
+          ptx::mma_commit(&bars->o_done[g][k & 1]);
+          ptx::mma_commit(&bars->kv_empty[st]);
+          if (info >> 9) ptx::mma_commit(&bars->kv_empty[st]);  // the other warpgroup has no tile here
+          return true;
+        };
+        // K/V uses (all items), Q tiles, S and PV issued by this group, K/V use of S(b - 1)
+        uint32_t u = 0, qcnt = 0, b = 0, npv = 0, u_last = 0;
+        for (long long it = first; it < p.n_items && ok; it += step) {
+          const Task t = decode(p, it);
+          if (!t.any) continue;
+          const uint32_t u0 = u;
+          u += t.nb;
+          if (!t.valid(g)) continue;
+          const uint32_t qs = qcnt & 1, qpar = (qcnt >> 1) & 1;
+          ++qcnt;
+          const uint64_t ad = qd0 + qs * kQBuf;
+          const uint32_t rel2 = (g == 0 && !t.valid(1)) ? 512u : 0u;
+          for (int j = 0; j < t.nb; ++j, ++b) {
+            const uint32_t uu = u0 + j, st = uu % kStages;
+            // S(b) overwrites P(b - 2): PV(b - 2) first
+            while (ok && npv + 2 <= b) ok = issue_pv(npv++);
+            // A pending PV(b - 1) whose K/V use is a whole ring behind block
+            // uu holds a slot the producer needs before it can load uu (or
+            // the next Q tile): issue it before waiting for either.
+            if (ok && npv < b && u_last + kStages <= uu) ok = issue_pv(npv++);
+            ok = ok && (j > 0 || wait_bar(&bars->q_ready[g][qs], qpar, ctl)) &&
+                 wait_bar(&bars->kv_ready[st], (uu / kStages) & 1, ctl);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint64_t bd = kd0 + st * kStageK;
+            const uint32_t dS = tg + (b & 1) * kBlk;
+            ptx::mma_ss(dS, ad, bd, idS, 0);
+            ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
+            ptx::mma_commit(&bars->s_full[g][b & 1]);
+            if (j == t.nb - 1) ptx::mma_commit(&bars->q_empty[g][qs]);
+            const uint32_t info = st | (j > 0 ? 256u : 0u) | rel2;
+            if (b & 1) pend1 = info; else pend0 = info;
+            u_last = uu;
           }
         }
+        while (ok && npv < b) ok = issue_pv(npv++);
         // drain: every MMA this thread issued has completed before TMEM is freed
-        ptx::mma_commit(&bars->drain);
+        ptx::mma_commit(&bars->drain[g]);
         Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
-        wait_bar(&bars->drain, 0, drain);
+        wait_bar(&bars->drain[g], 0, drain);
       }
     } else {
       // ============================================================== prep
-      // 192 threads (warps 2-3 and 12-15); work in half rows (16 channels):
+      // 160 threads (warps 3 and 12-15); work in half rows (16 channels):
       // the two halves of a row sit in adjacent lanes, and each half of a
       // RoPE row rotates along one axis only.
-      const int pt = warp < 4 ? (int)threadIdx.x - 64 : (int)threadIdx.x - 384 + 64;  // 0..191
+      const int pt = warp < 4 ? (int)threadIdx.x - 96 : (int)threadIdx.x - 384 + 32;  // 0..159
       uint32_t qu[2] = {0, 0}, ku = 0;
       bool ok = true;
       bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
@@ -657,7 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // window-local coordinates of the rectangle's first row and column
         const int py0 = swin_local_coord(t.y0, M, s), px0 = swin_local_coord(t.x0, M, s);
         for (int g = 0; g < 2 && ok; ++g) {
-          if (!t.valid[g]) continue;
+          if (!t.valid(g)) continue;
           const int qs = qu[g] & 1;
           ok = wait_bar(&bars->q_full[g][qs], (qu[g] >> 1) & 1, ctl);
           ++qu[g];
@@ -680,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               } else {
                 if (act) {
                   const int pr = rp[r];
-                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + t.tile[g] * t.R + (pr & 0xFFFF), 63), rcos,
+                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + t.tile(g) * t.R + (pr & 0xFFFF), 63), rcos,
                             rsin);
                 }
                 float m = half_absmax(v);
@@ -703,9 +652,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!ok) break;
           uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
           uint8_t* vtile = ktile + kTileBytes;
-          // this thread: half h of K row r and half h of V row r (r < krows <= 96);
-          // fp16 with saturation, a saturated entry is reported after the loop
-          const int r = pt >> 1, h = pt & 1;
+          // units: half h of K row r and half h of V row r (r < krows <= 96);
+          // fp16 with saturation, a saturated entry is reported after the loop.
+          // Trip counts are uniform per warp (the shuffle below needs all lanes).
+#pragma unroll 1
+          for (int un = pt; un < 2 * kBlk; un += kPrepThreads) {
+          const int r = un >> 1, h = un & 1;
           const bool act = r < krows;
           if (MODE != 0) {
             float v[16];
@@ -728,6 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             range_hit |= half_absmax(v) >= 65504.0f;
             store_half_f16(vtile, r, h, v, 1.0f);
           }
+          }
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(&bars->kv_ready[st]);
         }
@@ -749,9 +702,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     bool pend = false, pend_ok = false;  // an item's O still waiting in TMEM
     size_t pend_off = 0;
     // O / l of one row to global memory (32 values; column 32 holds l)
-    auto store_rows = [&](const uint32_t (&o)[32], const uint32_t (&o2)[16], size_t off, bool row_valid) {
+    auto store_rows = [&](const uint32_t (&o)[32], uint32_t l, size_t off, bool row_valid) {
       if (!row_valid) return;
-      const float inv = 1.0f / __uint_as_float(o2[0]);  // row sum of the fp16 P
+      const float inv = 1.0f / __uint_as_float(l);  // row sum of the fp16 P
       if (OUT_F32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
 #pragma unroll
@@ -789,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const Task tk = decode(p, it);
       const uint32_t ku0 = ku;
       if (tk.any) ku += tk.nb;  // K/V block uses of this item (both warpgroups)
-      if (!tk.valid[g]) continue;
+      if (!tk.valid(g)) continue;
       const int qs = qu & 1;
       ok = wait_bar(&bars->q_ready[g][qs], (qu >> 1) & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
@@ -799,8 +752,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const float alpha = MODE == 0 ? cscale : qscale[(g * 2 + qs) * 128 + t];
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
-      const bool row_ok = t < tk.nq[g];
-      const int qy = tk.tile[g] * tk.R + t / tk.lx, qx = t % tk.lx;
+      const bool row_ok = t < tk.nq(g);
+      const int qy = tk.tile(g) * tk.R + t / tk.lx, qx = t % tk.lx;
       const int bbase = (qy + M - 1) * R2 + (qx + M - 1);
       const int* kof = kofs + tk.cls * 128;
       float m_run = -INFINITY;
@@ -914,57 +867,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           ok = consume_pv(blk - 2);
           if (!ok) break;
         }
-        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-          // O and its row-sum column follow the new maximum
-          ok = consume_pv(blk - 1);
-          if (!ok) break;
-          uint32_t o[32], o2[16];
-          ptx::tmem_ld32(tO, o);
-          ptx::tmem_ld16(tO + 32, o2);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o2[e] = __float_as_uint(__uint_as_float(o2[e]) * factor);
-          ptx::tmem_st32(tO, o);
-          ptx::tmem_st16(tO + 32, o2);
-        }
         SWIN_TC_MARK(4);
-        // probabilities, fp16, written over the scores
+        // probabilities, fp16; written over the scores after O is brought up to
+        // date, so the scores' registers are free by then.
         // exponent argument: mode 2  x * ascale - m,  modes 0/1  x - m
         const float ea = MODE == 2 ? ascale : 1.0f, eb = -m_run;
-        {
-          uint32_t pa[32], pb[16];
+        uint32_t pa[32], pb[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
-            pa[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
-          }
+        for (int c = 0; c < 32; ++c) {
+          const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
+          pa[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+        }
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float2 e = __ffma2_rn(x[32 + c], make_float2(ea, ea), make_float2(eb, eb));
-            pb[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+        for (int c = 0; c < 16; ++c) {
+          const float2 e = __ffma2_rn(x[32 + c], make_float2(ea, ea), make_float2(eb, eb));
+          pb[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+        }
+        SWIN_TC_MARK(5);
+        // O (32 columns) and its row sum (column 32): rescaled to the new
+        // maximum, or, in an item's first block, the previous item's result
+        // read for the deferred store.  Both need PV(blk - 1) complete.
+        uint32_t po[32], pl = 0;
+        const bool epi = j == 0 && pend;
+        const bool resc = j > 0 && __any_sync(0xffffffffu, rescale);
+        if (epi || resc) {
+          ok = consume_pv(blk - 1);
+          if (!ok) break;
+          ptx::tmem_ld32(tO, po);
+          pl = ptx::tmem_ld1(tO + 32);
+          ptx::tmem_wait_ld();
+          if (resc) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) po[e] = __float_as_uint(__uint_as_float(po[e]) * factor);
+            ptx::tmem_st32(tO, po);
+            ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
           }
-          SWIN_TC_MARK(5);
-          uint32_t po[32], po2[16];  // previous item's O (deferred epilogue)
-          const bool epi = j == 0 && pend;
-          if (epi) {
-            ok = consume_pv(blk - 1);
-            if (!ok) break;
-            ptx::tmem_ld32(tO, po);
-            ptx::tmem_ld16(tO + 32, po2);
-          }
-          ptx::tmem_st32(tS, pa);
-          ptx::tmem_st16(tS + 32, pb);
-          if (epi) ptx::tmem_wait_ld();
-          ptx::tmem_wait_st();
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(&bars->p_full[g][blk & 1]);
-          SWIN_TC_MARK(6);
-          if (epi) {
-            store_rows(po, po2, pend_off, pend_ok);
-            pend = false;
-          }
+        }
+        ptx::tmem_st32(tS, pa);
+        ptx::tmem_st16(tS + 32, pb);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_full[g][blk & 1]);
+        SWIN_TC_MARK(6);
+        if (epi) {
+          store_rows(po, pl, pend_off, pend_ok);
+          pend = false;
         }
         SWIN_TC_MARK(7);
       }
@@ -980,11 +927,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     if (ok && pend) {
       ok = consume_pv(blk - 1);
       if (ok) {
-        uint32_t po[32], po2[16];
+        uint32_t po[32];
         ptx::tmem_ld32(tO, po);
-        ptx::tmem_ld16(tO + 32, po2);
+        const uint32_t pl = ptx::tmem_ld1(tO + 32);
         ptx::tmem_wait_ld();
-        store_rows(po, po2, pend_off, pend_ok);
+        store_rows(po, pl, pend_off, pend_ok);
       }
     }
   }
