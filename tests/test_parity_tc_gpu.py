@@ -70,3 +70,19 @@ def test_tc_forced_timeout_reports_status_and_recovers():
     assert sa.swin_stream_status() == sa.SWIN_OK
     want = oracle_run(inp, w, 8)
     assert rel_err(out.cpu().numpy(), want) <= TOL_BF16
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("B,H,W,heads,M,s", [(3, 32, 32, 12, 8, 4), (2, 35, 30, 9, 7, 3), (1, 48, 40, 6, 24, 12)])
+def test_tc_bias_head_changes(B, H, W, heads, M, s, mode):
+    """More work items than SMs and many heads: every CTA walks several items
+    and reloads its warpgroups' bias-table slots when the head changes; even
+    rectangle widths take the paired-load path, odd ones the general path."""
+    w = syn.Workload(83, "tc", "bf16", B, H, W, heads, 32, M, (s,), mode, tau=(0.05, 0.2),
+                     cpb_hidden=64 if mode == 1 else 0)
+    inp = syn.make_inputs(w, seed=11 * heads + M + mode)
+    if mode == 0:
+        inp["table"] = (0.5 * np.random.default_rng(4).standard_normal(((2 * M - 1) ** 2, heads))).astype(np.float32)
+    got = gpu_run_bf16_checked(inp, w, s).cpu().numpy()
+    want = oracle_run(inp, w, s)
+    assert rel_err(got, want) <= TOL_BF16

@@ -85,7 +85,7 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
 
 struct TcParams {
   CUtensorMap tmap[3][3];  // [tensor q/k/v][x-class first/middle/last]
-  FastDiv div_pmax, div_nsx, div_nsy, div_heads;
+  FastDiv div_pmax, div_nsx, div_nsy, div_B;
   int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
   void* out;
   int B, H, W, heads, M, s, nsy, nsx, pmax;
@@ -113,10 +113,13 @@ constexpr int kRopeOff = kScaleOff + 2 * 2 * 128 * 4;        // cos,sin [2][64][
 constexpr int kKofsOff = kRopeOff + 2 * 2 * 64 * 8 * 4;      // [3][128] int
 constexpr int kRposOff = kKofsOff + 3 * 128 * 4;             // [3][128] int: (r / lx) | (r % lx) << 16
 constexpr int kKcolOff = kRposOff + 3 * 128 * 4;             // [kStages][128] f32, 1/|k| (mode 1)
-constexpr int kBiasFloats = 16384;                           // bias tables of all heads if they fit
+// Relative-bias table of the current head, one slot per softmax warpgroup:
+// rows dy padded to an even stride 2M, stored twice (the second copy one
+// float ahead) so that every pair of adjacent keys is one aligned 8-byte load.
+constexpr int kSlotFloats = 8192;                            // 2 (2M-1) 2M + 2 <= 8192 for M <= 32
 constexpr int kBiasOff = kKcolOff + kStages * 128 * 4;
-constexpr int kBarOff = kBiasOff + kBiasFloats * 4;
-constexpr int kNumBars = 12 + 3 * kStages + 12 + 3;
+constexpr int kBarOff = kBiasOff + 2 * kSlotFloats * 4;
+constexpr int kNumBars = 12 + 3 * kStages + 12 + 3 + 4;
 constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
@@ -130,6 +133,7 @@ struct Bars {
   // only start after its current one was consumed, so parity tests never alias
   uint64_t s_full[2][2], p_full[2][2], o_done[2][2];
   uint64_t never, drain[2];
+  uint64_t tab_free[2], tab_ready[2];  // bias-table slot handshake of each softmax warpgroup (4 warps)
 };
 static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
 
@@ -157,9 +161,9 @@ __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
   q = fdiv(i, p.div_nsy);
   const int sy = (int)(i - q * p.div_nsy.d);
   i = q;
-  q = fdiv(i, p.div_heads);
-  t.h = (int)(i - q * p.div_heads.d);
-  t.b = (int)q;
+  q = fdiv(i, p.div_B);
+  t.b = (int)(i - q * p.div_B.d);
+  t.h = (int)q;  // heads outermost: a CTA keeps one head's bias table for many items
   t.cls = sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1);
   t.lx = p.lx[t.cls];
   t.R = p.R[t.cls];
@@ -365,7 +369,9 @@ __device__ __forceinline__ float pow2_scale(float m) {
 template <int MODE, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte alignment by pointer arithmetic on the shared array itself, so
+  // that every access below stays a shared-space load or store
+  uint8_t* smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
   uint8_t* qbuf = smem + kQOff;
   uint8_t* kvbuf = smem + kKVOff;
   uint8_t* ones = smem + kOnesOff;
@@ -375,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   int* kofs = reinterpret_cast<int*>(smem + kKofsOff);
   int* rpos = reinterpret_cast<int*>(smem + kRposOff);
   float* kcol = reinterpret_cast<float*>(smem + kKcolOff);
-  float* sbias = reinterpret_cast<float*>(smem + kBiasOff);  // [heads][(2M-1)^2], times log2(e)
+  float* sbias = reinterpret_cast<float*>(smem + kBiasOff);  // [2 warpgroups][kSlotFloats]
   Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -406,6 +412,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     ptx::mbar_init(&bars->never, 1);
     ptx::mbar_init(&bars->drain[0], 1);
     ptx::mbar_init(&bars->drain[1], 1);
+    for (int g = 0; g < 2; ++g) {
+      ptx::mbar_init(&bars->tab_free[g], 4);
+      ptx::mbar_init(&bars->tab_ready[g], 4);
+    }
     *abort_flag = 0;
     tmem_holder[2] = 0;  // abort flag of the drain waits (never set by a role)
     ptx::fence_mbar_init();
@@ -420,18 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       rsin[(axis * 64 + pos) * 8 + t] = sv;
     }
   }
-  const int R2sq = (2 * M - 1) * (2 * M - 1);
-  const bool bias_in_smem = MODE != 2 && p.table != nullptr && p.heads * R2sq <= kBiasFloats;
-  if (bias_in_smem) {
-    // table [(2M-1)^2][heads] -> shared [heads][(2M-1)^2], pre-scaled by log2(e)
-    for (int i = threadIdx.x; i < p.heads * R2sq; i += kThreads) {
-      const int h = i / R2sq, r = i % R2sq;
-      sbias[i] = __ldg(p.table + (size_t)r * p.heads + h) * kLog2eF;
-    }
-  }
+  const int R2e = 2 * M;  // padded row stride of the bias slot
+  const bool has_table = MODE != 2 && p.table != nullptr;
   for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
     const int c = i / 128, col = i % 128, lx = p.lx[c];
-    kofs[i] = (col / lx) * (2 * M - 1) + (col % lx);
+    kofs[i] = (col / lx) * R2e + (col % lx);  // slot offset of key col
     rpos[i] = (col / lx) | ((col % lx) << 16);
   }
   // zero the K/V ring and the ones blocks once, so rows a tile never writes
@@ -696,7 +699,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t tX = tmem_base + g * 256 + lane_off;  // X0; X1 = tX + kBlk
     const uint32_t tO = tX + 2 * kBlk;
     const float cscale = kLog2eF * rsqrtf(32.0f);
-    const int R2 = 2 * M - 1;
+    float* slot = sbias + g * kSlotFloats;
+    constexpr int kCopy1 = kSlotFloats / 2;  // second copy: slot[kCopy1 + i] = slot[i + 1]
+    int cur_h = -1;
+    uint32_t tabn = 0;  // table loads of this warpgroup
     uint32_t qu = 0, ku = 0, blk = 0;  // Q tiles, K/V uses, blocks of this warpgroup
     bool ok = true;
     bool pend = false, pend_ok = false;  // an item's O still waiting in TMEM
@@ -743,6 +749,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const uint32_t ku0 = ku;
       if (tk.any) ku += tk.nb;  // K/V block uses of this item (both warpgroups)
       if (!tk.valid(g)) continue;
+      if (has_table && tk.h != cur_h) {
+        // new head: once all four warps are done with the old table, each
+        // loads a quarter of the new one (times log2 e, zero padding column)
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->tab_free[g]);
+        ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_free[g], tabn & 1, ctl));
+        if (!ok) break;
+        const int n = (2 * M - 1) * R2e;
+        for (int i = (warp & 3) * 32 + lane; i < n; i += 128) {
+          const int dy = i / R2e, c = i - dy * R2e;
+          const float v = c < 2 * M - 1 ? __ldg(p.table + (size_t)(dy * (2 * M - 1) + c) * p.heads + tk.h) * kLog2eF : 0.f;
+          slot[i] = v;
+          if (i > 0) slot[kCopy1 + i - 1] = v;
+        }
+        if (warp == 4 + 4 * g && lane == 0) slot[kCopy1 + n - 1] = 0.f;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->tab_ready[g]);
+        ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_ready[g], tabn & 1, ctl));
+        ++tabn;
+        if (!ok) break;
+        cur_h = tk.h;
+      }
       const int qs = qu & 1;
       ok = wait_bar(&bars->q_ready[g][qs], (qu >> 1) & 1, ctl);
       ok = __all_sync(0xffffffffu, ok);
@@ -754,7 +782,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
       const bool row_ok = t < tk.nq(g);
       const int qy = tk.tile(g) * tk.R + t / tk.lx, qx = t % tk.lx;
-      const int bbase = (qy + M - 1) * R2 + (qx + M - 1);
+      // Slot index of this row's bias for key (0, 0) of the rectangle; the
+      // pair load for keys (2c, 2c+1) of a row starts one float earlier, in
+      // copy 0 when that index is even, else in copy 1 (the parity is fixed
+      // per query: row stride and even key offsets do not change it).
+      // Bias loads are unconditional: rows past the tile use row M - 1, and
+      // keys past the block (masked below) read other slot entries, at
+      // most 95 rows of 2M floats before slot 0, inside shared memory.
+      const int bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
+      const float* pbase = slot + (((bbase - 1) & 1) ? kCopy1 - 1 : 0) + bbase - 1;
+      const bool pair_ok = (tk.lx & 1) == 0;
       const int* kof = kofs + tk.cls * 128;
       float m_run = -INFINITY;
       for (int j = 0; j < tk.nb; ++j, ++blk) {
@@ -787,51 +824,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
         }
+        SWIN_TC_MARK(11);
         const float ascale = alpha;
         const int nk_all = tk.n - j * tk.Rk * tk.lx;
         const int nk = nk_all < tk.Rk * tk.lx ? nk_all : tk.Rk * tk.lx;
         // x = log2-domain logits.  Mode 2: the scale is applied inside the
-        // exponent below (max over raw scores, scale > 0).
-        if (MODE == 1) {
+        // exponent below (max over raw scores, scale > 0).  Modes 0/1:
+        // x = S * scale + bias in one rounding; the bias slot already holds
+        // T * log2(e), and mode 1's scale is log2e / (tau |q| |k|).
+        if (MODE != 2) {
           const float4* kc4 = reinterpret_cast<const float4*>(kcol + ust * 128);
-#pragma unroll
-          for (int c4 = 0; c4 < kBlk / 4; ++c4) {
-            const float4 kc = kc4[c4];  // same address in every lane: broadcast
-            x[2 * c4] = __fmul2_rn(x[2 * c4], make_float2(kc.x * ascale, kc.y * ascale));
-            x[2 * c4 + 1] = __fmul2_rn(x[2 * c4 + 1], make_float2(kc.z * ascale, kc.w * ascale));
-          }
-        } else if (MODE == 0) {
-          const float2 a2 = make_float2(ascale, ascale);
-#pragma unroll
-          for (int c = 0; c < kBlk / 2; ++c) x[c] = __fmul2_rn(x[c], a2);
-        }
-        if (MODE != 2 && p.table != nullptr) {
-          const int jb = bbase - j * tk.Rk * R2;
-          const int lim = row_ok ? nk : 0;
-          if (bias_in_smem) {
-            const int4* kof4 = reinterpret_cast<const int4*>(kof);
-            const float* hb = sbias + tk.h * R2sq + jb;
+          const int4* kof4 = reinterpret_cast<const int4*>(kof);
+          const int jo = j * tk.Rk * R2e;  // block j starts Rk rectangle rows further
+          if (!has_table) {
+            const float2 a2 = make_float2(ascale, ascale);
 #pragma unroll
             for (int c4 = 0; c4 < kBlk / 4; ++c4) {
-              const int4 ko = kof4[c4];  // broadcast
-              if (4 * c4 + 0 < lim) x[2 * c4].x += hb[-ko.x];
-              if (4 * c4 + 1 < lim) x[2 * c4].y += hb[-ko.y];
-              if (4 * c4 + 2 < lim) x[2 * c4 + 1].x += hb[-ko.z];
-              if (4 * c4 + 3 < lim) x[2 * c4 + 1].y += hb[-ko.w];
+              float2 s0 = a2, s1 = a2;
+              if (MODE == 1) {
+                const float4 kc = kc4[c4];
+                s0 = __fmul2_rn(make_float2(kc.x, kc.y), a2);
+                s1 = __fmul2_rn(make_float2(kc.z, kc.w), a2);
+              }
+              x[2 * c4] = __fmul2_rn(x[2 * c4], s0);
+              x[2 * c4 + 1] = __fmul2_rn(x[2 * c4 + 1], s1);
+            }
+          } else if (pair_ok) {
+            const float* pb = pbase - jo;
+#pragma unroll
+            for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+              float2 s0 = make_float2(ascale, ascale), s1 = s0;
+              if (MODE == 1) {
+                const float4 kc = kc4[c4];  // same address in every lane: broadcast
+                s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
+                s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
+              }
+              const int4 ko = kof4[c4];  // broadcast; keys 4 c4 .. 4 c4 + 3 share a row pairwise
+              const float2 b0 = *reinterpret_cast<const float2*>(pb - ko.x);  // (bias key+1, bias key)
+              const float2 b1 = *reinterpret_cast<const float2*>(pb - ko.z);
+              x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(b0.y, b0.x));
+              x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(b1.y, b1.x));
             }
           } else {
+            // odd rectangle widths: one load per key
+            const float* hb = slot + bbase - jo;
 #pragma unroll
-            for (int c = 0; c < kBlk; ++c) {
-              if (c < lim) {
-                const float tv = __ldg(p.table + (size_t)(jb - kof[c]) * p.heads + tk.h);
-                if (c & 1)
-                  x[c >> 1].y = __fmaf_rn(tv, kLog2eF, x[c >> 1].y);
-                else
-                  x[c >> 1].x = __fmaf_rn(tv, kLog2eF, x[c >> 1].x);
+            for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+              float2 s0 = make_float2(ascale, ascale), s1 = s0;
+              if (MODE == 1) {
+                const float4 kc = kc4[c4];
+                s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
+                s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
               }
+              const int4 ko = kof4[c4];
+              x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(hb[-ko.x], hb[-ko.y]));
+              x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(hb[-ko.z], hb[-ko.w]));
             }
           }
         }
+        SWIN_TC_MARK(12);
         if (nk < kBlk) {  // partial block (uniform across the warpgroup): mask the tail keys
 #pragma unroll
           for (int c = 0; c < kBlk / 2; ++c) {
@@ -1002,6 +1053,8 @@ void tc_set_debug(int flags, long long wait_limit) {
 swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream) {
   if (a.d != 32) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs d == 32, got %d", a.d);
   if (a.M > 64) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs M <= 64");
+  if (a.mode != 2 && a.table && 2 * (2 * a.M - 1) * (2 * a.M) + 2 > kSlotFloats)
+    return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path keeps a bias table only for M <= 32");
   TcParams p;
   memset(&p, 0, sizeof(p));
   p.B = a.B; p.H = a.H; p.W = a.W; p.heads = a.heads; p.M = a.M; p.s = a.shift;
@@ -1028,7 +1081,7 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   p.div_pmax = make_fastdiv((uint32_t)p.pmax);
   p.div_nsx = make_fastdiv((uint32_t)p.nsx);
   p.div_nsy = make_fastdiv((uint32_t)p.nsy);
-  p.div_heads = make_fastdiv((uint32_t)a.heads);
+  p.div_B = make_fastdiv((uint32_t)a.B);
   p.out = a.out;
   p.tau = a.tau;
   p.table = a.table;

@@ -135,7 +135,9 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
   a.tau = tau; a.table = table; a.rope = rope_freqs;
   a.status = swin::status_word();
   if (!a.status) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
-  if (dt == SWIN_BF16 && d == 32) return swin::launch_attn_tc(a, out_dt == SWIN_F32, st);
+  // tensor-core path: bf16, d = 32; a bias table must fit its shared-memory slot (M <= 32)
+  if (dt == SWIN_BF16 && d == 32 && (table == nullptr || M <= 32))
+    return swin::launch_attn_tc(a, out_dt == SWIN_F32, st);
   return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
 }
 
