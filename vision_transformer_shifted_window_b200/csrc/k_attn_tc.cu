@@ -190,7 +190,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, const C
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (ptx::mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (*c.abort) return false;
     if (clock64() - t0 > c.p->wait_limit) {
       atomicOr(c.p->status, (int)SWIN_ERR_TIMEOUT);
@@ -211,80 +211,10 @@ __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 
 // ------------------------------------------------------------------ prep
 // Score-prep operands go to the tensor core as fp16 (both Q and K, so the MMA
 // sees one type): fp16 keeps 3 more mantissa bits than bf16, and rounding the
-// rotated / normalised operands is the largest error term of the path.  Unit
-// vectors cannot overflow fp16; rotated rows are first scaled by an exact power
-// of two (per query row, per K block) that is divided out in the softmax.
-
-// Load one 32-element bf16 row (64-byte swizzled tile row) as fp32.
-__device__ __forceinline__ void load_row_bf16(const uint8_t* tile, int row, float (&v)[32]) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 w = *reinterpret_cast<const uint4*>(tile + swz64(row, c));
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      v[8 * c + 2 * e] = bf_lo(u[e]);
-      v[8 * c + 2 * e + 1] = bf_hi(u[e]);
-    }
-  }
-}
-
-// Store v * sc as fp16 with saturation into the same row.
-__device__ __forceinline__ void store_row_f16_sat(uint8_t* tile, int row, const float (&v)[32], float sc) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t u[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) u[e] = ptx::pack_f16x2_sat(v[8 * c + 2 * e] * sc, v[8 * c + 2 * e + 1] * sc);
-    *reinterpret_cast<uint4*>(tile + swz64(row, c)) = make_uint4(u[0], u[1], u[2], u[3]);
-  }
-}
-
-// Store v * sc as fp16 into the same row.
-__device__ __forceinline__ void store_row_f16(uint8_t* tile, int row, const float (&v)[32], float sc) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t u[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) u[e] = ptx::pack_f16x2(v[8 * c + 2 * e] * sc, v[8 * c + 2 * e + 1] * sc);
-    *reinterpret_cast<uint4*>(tile + swz64(row, c)) = make_uint4(u[0], u[1], u[2], u[3]);
-  }
-}
-
-__device__ __forceinline__ float inv_norm(const float (&v)[32]) {
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) ss = fmaf(v[e], v[e], ss);
-  return 1.0f / fmaxf(sqrtf(ss), kNormEps);
-}
-
-// Rotate channels [0,16) by py and [16,32) by px (pairs (2t, 2t+1), t < 8).
-__device__ __forceinline__ void rope_rotate(float (&v)[32], int py, int px, const float* rc, const float* rs) {
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int pos = half ? px : py;
-    const float4* cs4 = reinterpret_cast<const float4*>(rc + (half * 64 + pos) * 8);
-    const float4* sn4 = reinterpret_cast<const float4*>(rs + (half * 64 + pos) * 8);
-    const float4 c0 = cs4[0], c1 = cs4[1], s0 = sn4[0], s1 = sn4[1];
-    const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const float a = v[16 * half + 2 * t], b = v[16 * half + 2 * t + 1];
-      const float co = cs[t], si = sn[t];
-      // explicit roundings: every instantiation of the kernel computes the same bits
-      v[16 * half + 2 * t] = __fmaf_rn(a, co, -__fmul_rn(b, si));
-      v[16 * half + 2 * t + 1] = __fmaf_rn(a, si, __fmul_rn(b, co));
-    }
-  }
-}
-
-__device__ __forceinline__ float absmax(const float (&v)[32]) {
-  float m = 0.f;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(v[e]));
-  return m;
-}
+// rotated operands is the largest error term of the path.  A rotated Q row is
+// first scaled by an exact power of two that brings it below 2^15 (divided
+// out in the softmax); rotated K rows and V are converted with saturation,
+// and an entry at or beyond the fp16 range is reported as unsupported.
 
 // Half rows: channels [16 h, 16 h + 16) = 16-byte chunks 2h and 2h + 1.
 __device__ __forceinline__ void load_half_bf16(const uint8_t* tile, int row, int h, float (&v)[16]) {
@@ -327,6 +257,26 @@ __device__ __forceinline__ void rope_half(float (&v)[16], int h, int pos, const 
   }
 }
 
+// 2^e for a pair on the FMA pipe, so that part of the exponentials leave the
+// MUFU: e = j + f with j = rint(e) read from the low mantissa bits of
+// e + 1.5 * 2^23 and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by
+// the Remez exchange algorithm for minimax relative error on [-1/2, 1/2]
+// (7.5e-5, below half an fp16 ulp), and j is added to its exponent field.
+// Arguments below -125 are clamped (the result then rounds to 0 in fp16).
+__device__ __forceinline__ float2 exp2_poly2(float2 e) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  e.x = fmaxf(e.x, -125.0f);
+  e.y = fmaxf(e.y, -125.0f);
+  const float2 t = __fadd2_rn(e, make_float2(kRound, kRound));
+  const float2 r = __fadd2_rn(t, make_float2(-kRound, -kRound));     // rint(e), exact
+  const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), e);      // e - rint(e), exact
+  float2 q = __ffma2_rn(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.2426111251f, 0.2426111251f));
+  q = __ffma2_rn(q, f, make_float2(0.6932609677f, 0.6932609677f));
+  q = __ffma2_rn(q, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 __device__ __forceinline__ float half_absmax(const float (&v)[16]) {
   float m = 0.f;
 #pragma unroll
@@ -341,21 +291,6 @@ __device__ __forceinline__ float half_sumsq(const float (&v)[16]) {
   return ss;
 }
 
-// Largest |value| of one 32-element bf16 row (packed bf16x2 arithmetic).
-__device__ __forceinline__ float row_absmax_bf16(const uint8_t* tile, int row) {
-  __nv_bfloat162 m = __float2bfloat162_rn(0.f);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 w = *reinterpret_cast<const uint4*>(tile + swz64(row, c));
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
-      m = __hmax2(m, __habs2(x));
-    }
-  }
-  return fmaxf(__bfloat162float(m.x), __bfloat162float(m.y));
-}
 
 // Power of two that brings a row maximum m below 2^15 (fp16 max is 65504).
 __device__ __forceinline__ float pow2_scale(float m) {
@@ -923,16 +858,25 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // date, so the scores' registers are free by then.
         // exponent argument: mode 2  x * ascale - m,  modes 0/1  x - m
         const float ea = MODE == 2 ? ascale : 1.0f, eb = -m_run;
+        // keys 0-63 on the MUFU, stored to TMEM while keys 64-95 are done;
+        // mode 2 (no bias work, MUFU-bound) takes those through the
+        // polynomial on the FMA pipe
         uint32_t pa[32], pb[16];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
           pa[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
         }
+        ptx::tmem_st32(tS, pa);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const float2 e = __ffma2_rn(x[32 + c], make_float2(ea, ea), make_float2(eb, eb));
-          pb[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+          if (MODE == 2) {
+            const float2 pe = exp2_poly2(e);
+            pb[c] = ptx::pack_f16x2(pe.x, pe.y);
+          } else {
+            pb[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+          }
         }
         SWIN_TC_MARK(5);
         // O (32 columns) and its row sum (column 32): rescaled to the new
@@ -954,7 +898,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
           }
         }
-        ptx::tmem_st32(tS, pa);
         ptx::tmem_st16(tS + 32, pb);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
