@@ -262,7 +262,7 @@ def run_native(args, rank: int, world: int, local_rank: int):
     achieved = wk["flops_std"] / (k_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": read_traffic("attn", w), "peak_source": peaks["source"] + " (burst)",
+                "traffic": read_traffic("attn_tc", w), "peak_source": peaks["source"] + " (burst)",
                 "kernel_ms": round(k_ms, 5),
                 "hbm_achieved_gbs": round(wk["bytes"] / (k_ms * 1e-3) / 1e9, 1),
                 "hbm_frac": round(wk["bytes"] / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
