@@ -119,12 +119,15 @@ swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* ta
  *   stream         CUDA stream
  * Asynchronous; q/k/v must stay valid until the stream reaches the call.
  *
- * Arithmetic of the bf16, d == 32 path (tcgen05 tensor cores): q.k products
- * of the bf16 inputs accumulate in fp32 (modes 0 and 1; mode 1 applies 1/|q|,
- * 1/|k| and 1/tau in fp32 afterwards); mode 2 rotates q and k in fp32 and
- * multiplies them as fp16 scaled by powers of two.  Probabilities and V are
- * carried in fp16 (V scaled by a power of two per 96-key block), sums in
- * fp32.  V entries of magnitude 2^22 or more saturate; the kernel then
+ * Arithmetic of the bf16, d == 32 path (tcgen05 tensor cores; taken when
+ * there is no bias table or M <= 32, else the CUDA-core path runs): q.k
+ * products of the bf16 inputs accumulate in fp32 (modes 0 and 1; mode 1
+ * applies 1/|q|, 1/|k| and 1/tau in fp32 afterwards, and the bias is added in
+ * fp32); mode 2 rotates q and k in fp32 and multiplies them as fp16, q scaled
+ * by an exact power of two.  Probabilities (at most 2^8 times the running
+ * maximum's) and V are carried in fp16, sums in fp32, and the row sum is
+ * accumulated from the same fp16 probabilities that weight V.  A rotated k
+ * entry or a V entry of magnitude 65504 or more saturates; the kernel then
  * records SWIN_ERR_UNSUPPORTED, which swin_stream_status reports. */
 swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, void* out,
                                  swin_dtype dt, swin_dtype out_dt, int B, int H, int W,

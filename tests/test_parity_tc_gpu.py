@@ -86,3 +86,19 @@ def test_tc_bias_head_changes(B, H, W, heads, M, s, mode):
     got = gpu_run_bf16_checked(inp, w, s).cpu().numpy()
     want = oracle_run(inp, w, s)
     assert rel_err(got, want) <= TOL_BF16
+
+
+def test_tc_v_out_of_fp16_range_reports_unsupported():
+    """V is carried in fp16 on the tensor-core path: an entry at or beyond
+    65504 saturates and the call reports SWIN_ERR_UNSUPPORTED (no fault); the
+    next call with in-range inputs is clean."""
+    w = syn.Workload(84, "tc", "bf16", 1, 16, 16, 1, 32, 8, (4,), 0)
+    inp = syn.make_inputs(w, seed=3)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    q, k, v = (dev(inp[n]).to(torch.bfloat16) for n in ("q", "k", "v"))
+    v_big = v.clone()
+    v_big[0, 5, 7, 0, 3] = 70000.0
+    sa.swin_window_attn_fwd(q, k, v_big, 8, 4, 0)
+    assert sa.swin_stream_status() == sa.SWIN_ERR_UNSUPPORTED
+    sa.swin_window_attn_fwd(q, k, v, 8, 4, 0)
+    assert sa.swin_stream_status() == sa.SWIN_OK

@@ -1,0 +1,262 @@
+"""The tensor-core kernel's barrier protocol, replayed on the host.
+
+Every role of attn_tc_kernel (TMA producer, operand prep, one MMA issuer per
+softmax warpgroup, two softmax warpgroups) is modelled as a program of
+mbarrier arrivals and parity waits in the kernel's order; TMA copies complete
+in any order, each issuer's MMA commits complete in issue order, and the
+online-softmax rescale happens at random.  Random interleavings over the real
+per-CTA work-item sequences of every workload must finish with no deadlock and
+with no wait whose parity could match a phase two or more completions old.
+"""
+import random
+
+import pytest
+
+S = 6  # K/V ring stages of the kernel
+KBLK = 96  # keys per K/V block
+
+
+# segment geometry of the shifted partition (cut at s + kM, clipped)
+def nseg(L, M, s):
+    if s == 0: return (L + M - 1) // M
+    if L <= s: return 1
+    return 1 + (L - s + M - 1) // M
+
+
+def seg_start(k, M, s):
+    if s == 0: return k * M
+    return 0 if k == 0 else s + (k - 1) * M
+
+
+def seg_len(k, L, M, s):
+    a = seg_start(k, M, s)
+    b = (k + 1) * M if s == 0 else s + k * M
+    return min(b, L) - a
+
+
+def items_for(B, H, W, heads, M, s, cta, grid):
+    """(has work, tile of warpgroup 0, tile of warpgroup 1, K/V blocks) of the
+    items CTA `cta` walks, in the kernel's order (tile pair fastest, then
+    segment x, segment y, image, head)."""
+    nsy, nsx = nseg(H, M, s), nseg(W, M, s)
+    lxs = [seg_len(0, W, M, s), seg_len(1, W, M, s) if nsx > 2 else seg_len(0, W, M, s), seg_len(nsx - 1, W, M, s)]
+    R = [128 // l for l in lxs]
+    Rk = [KBLK // l for l in lxs]
+    tiles_max = max((M + r - 1) // r for r in R)
+    pmax = (tiles_max + 1) // 2
+    n_items = B * heads * nsy * nsx * pmax
+    out = []
+    for it in range(cta, n_items, grid):
+        i = it
+        pr = i % pmax; i //= pmax
+        sx = i % nsx; i //= nsx
+        sy = i % nsy; i //= nsy
+        cls = 0 if sx == 0 else (2 if sx == nsx - 1 else 1)
+        ly = seg_len(sy, H, M, s)
+        nb = (ly + Rk[cls] - 1) // Rk[cls]
+        ntiles = (ly + R[cls] - 1) // R[cls]
+        v0 = 2 * pr < ntiles
+        v1 = 2 * pr + 1 < ntiles
+        out.append((v0, v0, v1, nb))
+    return out
+
+
+class Bar:
+    def __init__(self, name, count):
+        self.name, self.count, self.pending, self.done = name, count, 0, 0
+
+    def arrive(self, n=1):
+        self.pending += n
+        assert self.pending <= self.count, self.name
+        if self.pending == self.count:
+            self.pending = 0
+            self.done += 1
+
+
+class Deadlock(Exception):
+    pass
+
+
+def run(items, mode, seed, rescale_p=0.2, early_pv=True):
+    rng = random.Random(seed)
+    bars = {}
+
+    def bar(name, count):
+        if name not in bars: bars[name] = Bar(name, count)
+        return bars[name]
+    for g in range(2):
+        for b in range(2):
+            bar(("q_full", g, b), 1); bar(("q_ready", g, b), 1); bar(("q_empty", g, b), 5)
+            bar(("s_full", g, b), 1); bar(("p_full", g, b), 1); bar(("o_done", g, b), 1)
+    for i in range(S):
+        bar(("kv_full", i), 1); bar(("kv_ready", i), 1); bar(("kv_empty", i), 2)
+
+    def W(name, k):
+        """wait for completion k (0-based) of a barrier, by parity"""
+        return ("wait", name, k)
+
+    tma = []  # pending async TMA completions (any order)
+    mmaq = {0: [], 1: []}  # per issuer FIFO of commit lists
+
+    def producer():
+        qu = [0, 0]; ku = 0
+        for (any_, v0, v1, nb) in items:
+            if not any_: continue
+            for g, v in ((0, v0), (1, v1)):
+                if not v: continue
+                qs = qu[g] & 1
+                if qu[g] >= 2: yield W(("q_empty", g, qs), (qu[g] >> 1) - 1)
+                tma.append(("q_full", g, qs)); qu[g] += 1
+            for j in range(nb):
+                st = ku % S
+                if ku >= S: yield W(("kv_empty", st), ku // S - 1)
+                tma.append(("kv_full", st)); ku += 1
+
+    def prep():
+        qu = [0, 0]; ku = 0
+        for (any_, v0, v1, nb) in items:
+            if not any_: continue
+            for g, v in ((0, v0), (1, v1)):
+                if not v: continue
+                qs = qu[g] & 1
+                yield W(("q_full", g, qs), qu[g] >> 1); qu[g] += 1
+                bars[("q_ready", g, qs)].arrive()
+            for j in range(nb):
+                st = ku % S
+                yield W(("kv_full", st), ku // S); ku += 1
+                bars[("kv_ready", st)].arrive()
+
+    def issuer(g):
+        u = qcnt = b = npv = u_last = 0
+        pend = [0, 0]
+
+        def issue_pv(k):
+            yield W(("p_full", g, k & 1), k >> 1)
+            st, acc, rel2 = pend[k & 1]
+            c = [("o_done", g, k & 1), ("kv_empty", st)]
+            if rel2: c.append(("kv_empty", st))
+            mmaq[g].append(c)
+        for (any_, v0, v1, nb) in items:
+            if not any_: continue
+            u0 = u; u += nb
+            if not (v0 if g == 0 else v1): continue
+            qs, qpar = qcnt & 1, (qcnt >> 1)
+            qcnt += 1
+            rel2 = g == 0 and not v1
+            for j in range(nb):
+                uu = u0 + j; st = uu % S
+                while npv + 2 <= b:
+                    yield from issue_pv(npv); npv += 1
+                if early_pv and npv < b and u_last + S <= uu:
+                    yield from issue_pv(npv); npv += 1
+                if j == 0: yield W(("q_ready", g, qs), qpar)
+                yield W(("kv_ready", st), uu // S)
+                c = [("s_full", g, b & 1)]
+                if j == nb - 1: c.append(("q_empty", g, qs))
+                mmaq[g].append(c)
+                pend[b & 1] = (st, j > 0, rel2)
+                u_last = uu
+                b += 1
+        while npv < b:
+            yield from issue_pv(npv); npv += 1
+
+    def softmax(g):
+        qu = ku = blk = 0
+        o_cons = [0]
+        pend = False
+
+        def consume(upto):
+            while o_cons[0] <= upto:
+                yield W(("o_done", g, o_cons[0] & 1), o_cons[0] >> 1)
+                o_cons[0] += 1
+        for (any_, v0, v1, nb) in items:
+            ku0 = ku
+            if any_: ku += nb
+            if not (v0 if g == 0 else v1): continue
+            qs = qu & 1
+            yield W(("q_ready", g, qs), qu >> 1); qu += 1
+            bars[("q_empty", g, qs)].arrive(4)
+            for j in range(nb):
+                yield W(("s_full", g, blk & 1), blk >> 1)
+                uu = ku0 + j
+                if mode == 1: yield W(("kv_ready", uu % S), uu // S)
+                if blk >= 2: yield from consume(blk - 2)
+                epi = j == 0 and pend
+                resc = j > 0 and rng.random() < rescale_p
+                if epi or resc: yield from consume(blk - 1)
+                bars[("p_full", g, blk & 1)].arrive()
+                if epi: pend = False
+                blk += 1
+            pend = True
+        if pend: yield from consume(blk - 1)
+
+    roles = {"producer": producer(), "prep": prep(), "iss0": issuer(0), "iss1": issuer(1),
+             "sm0": softmax(0), "sm1": softmax(1)}
+    waiting = {k: None for k in roles}
+    alive = set(roles)
+
+    def ready(w):
+        _, name, k = w
+        c = bars[name].done
+        if c >= k + 2:
+            raise AssertionError("parity alias on %s: waiting for completion %d, %d done" % (name, k, c))
+        return c >= k + 1
+    steps = 0
+    while alive or tma or mmaq[0] or mmaq[1]:
+        steps += 1
+        cands = []
+        for r in alive:
+            w = waiting[r]
+            if w is None or ready(w): cands.append(("role", r))
+        if tma: cands.append(("tma", None))
+        for g in (0, 1):
+            if mmaq[g]: cands.append(("mma", g))
+        if not cands:
+            raise Deadlock({r: waiting[r] for r in alive})
+        kind, x = rng.choice(cands)
+        if kind == "role":
+            try:
+                waiting[x] = next(roles[x])
+            except StopIteration:
+                alive.discard(x)
+        elif kind == "tma":
+            i = rng.randrange(len(tma))
+            bars[tma.pop(i)].arrive()
+        else:
+            for c in mmaq[x].pop(0): bars[c].arrive()
+    return steps
+
+
+
+
+WORKLOADS = {  # B, H, W, heads, M, shift, mode
+    "swin-t-M7": (32, 56, 56, 3, 7, 3, 0),
+    "swinv2-t-M16": (64, 64, 64, 3, 16, 8, 1),
+    "flashswin-t-M32": (16, 112, 112, 3, 32, 16, 2),
+    "swinv2-g-M24": (2, 384, 384, 16, 24, 12, 1),
+    "ragged-M7": (1, 20, 37, 2, 7, 3, 1),
+    "ragged-M32": (3, 17, 64, 3, 32, 16, 1),
+    "M24-no-shift-odd": (1, 100, 60, 5, 24, 0, 0),
+    "M16-shift0": (2, 33, 33, 1, 16, 0, 2),
+    "thin-M8": (1, 9, 200, 4, 8, 4, 1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_protocol_no_deadlock_no_parity_alias(name):
+    B, H, W, heads, M, s, mode = WORKLOADS[name]
+    grid = 148 if B * H * W > 20000 else 8
+    for cta in (0, 1, grid // 3, grid - 1):
+        items = items_for(B, H, W, heads, M, s, cta, grid)
+        for seed in range(4):
+            run(items, mode, seed)
+
+
+def test_model_catches_the_deadlock_it_guards_against():
+    """Without the early PV issue (a pending PV whose K/V slot is a whole
+    ring behind the block being waited for) the model deadlocks on the M=16
+    workload, where most items have one query tile."""
+    items = items_for(64, 64, 64, 3, 16, 8, 0, 148)
+    with pytest.raises(Deadlock):
+        for seed in range(8):
+            run(items, 1, seed, early_pv=False)
