@@ -180,7 +180,7 @@ def run(items, mode, seed, rescale_p=0.2, early_pv=True):
                 yield W(("s_full", g, blk & 1), blk >> 1)
                 uu = ku0 + j
                 if mode == 1: yield W(("kv_ready", uu % S), uu // S)
-                if blk >= 2: yield from consume(blk - 2)
+                if blk >= 2: o_cons[0] = max(o_cons[0], blk - 1)  # implied by s_full(blk)
                 epi = j == 0 and pend
                 resc = j > 0 and rng.random() < rescale_p
                 if epi or resc: yield from consume(blk - 1)

@@ -665,9 +665,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
     };
-    // PV completions are consumed strictly in order, one barrier per PV
-    // parity: PV(b + 2) needs P(b + 2), which is written only after PV(b)
-    // was consumed, so no parity test can alias another phase.
+    // PV completion: o_done[parity] completes once per PV of that parity.
+    // The softmax waits on it only where O is read (rescale, deferred
+    // epilogue); every other completion is inferred: S(b)'s commit follows
+    // PV(b - 2)'s MMAs in the issuing thread, so s_full(b) implies that
+    // PV(0..b-2) are complete.  A parity wait for PV(k) cannot alias:
+    // PV(k + 2) needs P(k + 2), which this warpgroup has not written yet.
     uint32_t o_cons = 0;  // PVs of this warpgroup known complete
     auto consume_pv = [&](uint32_t upto) -> bool {  // PV(0..upto) complete
       bool r = true;
@@ -847,12 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           m_run = mb;
           rescale = true;
         }
-        // keep PV completions consumed in order (PV(blk - 2) was issued two
-        // blocks ago, so this rarely waits)
-        if (blk >= 2) {
-          ok = consume_pv(blk - 2);
-          if (!ok) break;
-        }
+        if (blk >= 2 && o_cons < blk - 1) o_cons = blk - 1;  // PV(0..blk-2) done: s_full(blk) seen
         SWIN_TC_MARK(4);
         // probabilities, fp16; written over the scores after O is brought up to
         // date, so the scores' registers are free by then.
