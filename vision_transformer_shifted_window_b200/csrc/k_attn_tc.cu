@@ -89,6 +89,7 @@ struct TcParams {
   int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
   void* out;
   int B, H, W, heads, M, s, nsy, nsx, pmax;
+  int R2e;  // row stride of the bias slot (even, >= 2M - 1, chosen against bank conflicts)
   long long n_items;
   const float* tau;
   const float* table;
@@ -116,7 +117,8 @@ constexpr int kKcolOff = kRposOff + 3 * 128 * 4;             // [kStages][128] f
 // Relative-bias table of the current head, one slot per softmax warpgroup:
 // rows dy padded to an even stride 2M, stored twice (the second copy one
 // float ahead) so that every pair of adjacent keys is one aligned 8-byte load.
-constexpr int kSlotFloats = 8192;                            // 2 (2M-1) 2M + 2 <= 8192 for M <= 32
+constexpr int kSlotFloats = 8192;                            // two copies of (2M-1) rows fit for M <= 32
+constexpr int kCopy1 = kSlotFloats / 2 + 16;
 constexpr int kBiasOff = kKcolOff + kStages * 128 * 4;
 constexpr int kBarOff = kBiasOff + 2 * kSlotFloats * 4;
 constexpr int kNumBars = 12 + 3 * kStages + 12 + 3 + 4;
@@ -300,8 +302,13 @@ __device__ __forceinline__ float pow2_scale(float m) {
   return ldexpf(1.0f, 15 - e);
 }
 
+// How a launch adds the relative bias (a template argument, so that each
+// kernel carries only the code it runs): no table; pair loads (every
+// rectangle width of the launch even); one load per key (some width odd).
+enum BiasKind { kBiasNone = 0, kBiasPairs = 1, kBiasKeys = 2 };
+
 // ------------------------------------------------------------------ kernel
-template <int MODE, bool OUT_F32>
+template <int MODE, bool OUT_F32, int BIAS>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment by pointer arithmetic on the shared array itself, so
@@ -365,8 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       rsin[(axis * 64 + pos) * 8 + t] = sv;
     }
   }
-  const int R2e = 2 * M;  // padded row stride of the bias slot
-  const bool has_table = MODE != 2 && p.table != nullptr;
+  const int R2e = p.R2e;
+  constexpr bool has_table = MODE != 2 && BIAS != kBiasNone;
   for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
     const int c = i / 128, col = i % 128, lx = p.lx[c];
     kofs[i] = (col / lx) * R2e + (col % lx);  // slot offset of key col
@@ -635,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const uint32_t tO = tX + 2 * kBlk;
     const float cscale = kLog2eF * rsqrtf(32.0f);
     float* slot = sbias + g * kSlotFloats;
-    constexpr int kCopy1 = kSlotFloats / 2;  // second copy: slot[kCopy1 + i] = slot[i + 1]
+    // second copy: slot[kCopy1 + i] = slot[i + 1], 16 banks away from the first
     int cur_h = -1;
     uint32_t tabn = 0;  // table loads of this warpgroup
     uint32_t qu = 0, ku = 0, blk = 0;  // Q tiles, K/V uses, blocks of this warpgroup
@@ -729,7 +736,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // most 95 rows of 2M floats before slot 0, inside shared memory.
       const int bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
       const float* pbase = slot + (((bbase - 1) & 1) ? kCopy1 - 1 : 0) + bbase - 1;
-      const bool pair_ok = (tk.lx & 1) == 0;
       const int* kof = kofs + tk.cls * 128;
       float m_run = -INFINITY;
       for (int j = 0; j < tk.nb; ++j, ++blk) {
@@ -787,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               x[2 * c4] = __fmul2_rn(x[2 * c4], s0);
               x[2 * c4 + 1] = __fmul2_rn(x[2 * c4 + 1], s1);
             }
-          } else if (pair_ok) {
+          } else if (BIAS == kBiasPairs) {
             const float* pb = pbase - jo;
 #pragma unroll
             for (int c4 = 0; c4 < kBlk / 4; ++c4) {
@@ -970,9 +976,9 @@ bool encode_map(CUtensorMap* m, const void* base, const AttnArgs& a, int lx, int
   return r == CUDA_SUCCESS;
 }
 
-template <int MODE, bool F32>
+template <int MODE, bool F32, int BIAS>
 swin_status launch_mode(const TcParams& p, int grid, cudaStream_t stream) {
-  auto k = attn_tc_kernel<MODE, F32>;
+  auto k = attn_tc_kernel<MODE, F32, BIAS>;
   cudaError_t ea = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (ea != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_tc smem attribute: %s", cudaGetErrorString(ea));
   k<<<grid, kThreads, kSmemAlloc, stream>>>(p);
@@ -994,7 +1000,7 @@ void tc_set_debug(int flags, long long wait_limit) {
 swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream) {
   if (a.d != 32) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs d == 32, got %d", a.d);
   if (a.M > 64) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs M <= 64");
-  if (a.mode != 2 && a.table && 2 * (2 * a.M - 1) * (2 * a.M) + 2 > kSlotFloats)
+  if (a.mode != 2 && a.table && (2 * a.M - 1) * (2 * a.M) > kSlotFloats - kCopy1)
     return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path keeps a bias table only for M <= 32");
   TcParams p;
   memset(&p, 0, sizeof(p));
@@ -1016,6 +1022,39 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
         !encode_map(&p.tmap[2][c], a.v, a, p.lx[c], p.Rk[c]))
       return fail(SWIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (lx=%d, R=%d)", p.lx[c], p.R[c]);
   }
+  // Bias-slot row stride: the even value in [2M, 2M + 14] (whose two copies fit
+  // the slot) with the fewest shared-memory wavefronts for the paired bias
+  // loads of this launch's rectangle widths.  A warp's 32 queries load 8
+  // bytes each in two 16-lane phases; query (qy, qx) of a width-lx rectangle
+  // reads floats qy R2e + qx - 1 (+ kCopy1 - 1 when that is odd) and on.
+  p.R2e = 2 * a.M;
+  if (a.mode != 2 && a.table) {
+    long best = -1;
+    for (int r2 = 2 * a.M; r2 <= 2 * a.M + 14; r2 += 2) {
+      if ((2 * a.M - 1) * r2 > kSlotFloats - kCopy1) break;
+      long cost = 0;
+      for (int c = 0; c < 3; ++c) {
+        const int lx = p.lx[c];
+        if (lx & 1) continue;
+        for (int w0 = 0; w0 < 128; w0 += 32)
+          for (int ph = 0; ph < 2; ++ph) {
+            int hits[16] = {0}, mx = 0;
+            for (int l = 0; l < 16; ++l) {
+              const int t = w0 + 16 * ph + l, qy = t / lx, qx = t % lx;
+              int idx = qy * r2 + qx + a.M - 2;  // parity as in the kernel's bbase - 1
+              if (idx & 1) idx += kCopy1 - 1;
+              const int bank2 = (idx >> 1) & 15;
+              mx = ++hits[bank2] > mx ? hits[bank2] : mx;
+            }
+            cost += mx;
+          }
+      }
+      if (best < 0 || cost < best) {
+        best = cost;
+        p.R2e = r2;
+      }
+    }
+  }
   p.pmax = (tiles_max + 1) / 2;
   p.n_items = (long long)a.B * a.heads * p.nsy * p.nsx * p.pmax;
   if (p.n_items >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "too many work items (%lld)", p.n_items);
@@ -1035,9 +1074,28 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)(p.n_items < sms ? p.n_items : sms);
   switch (a.mode) {
-    case 0: return f32_out ? launch_mode<0, true>(p, grid, stream) : launch_mode<0, false>(p, grid, stream);
-    case 1: return f32_out ? launch_mode<1, true>(p, grid, stream) : launch_mode<1, false>(p, grid, stream);
-    default: return f32_out ? launch_mode<2, true>(p, grid, stream) : launch_mode<2, false>(p, grid, stream);
+    case 0:
+    case 1: {
+      const bool all_even = !(p.lx[0] & 1) && !(p.lx[1] & 1) && !(p.lx[2] & 1);
+      const int kind = !a.table ? kBiasNone : (all_even ? kBiasPairs : kBiasKeys);
+#define SWIN_TC_LAUNCH(MD)                                                                               \
+  switch (kind) {                                                                                       \
+    case kBiasNone:                                                                                     \
+      return f32_out ? launch_mode<MD, true, kBiasNone>(p, grid, stream)                                \
+                     : launch_mode<MD, false, kBiasNone>(p, grid, stream);                              \
+    case kBiasPairs:                                                                                    \
+      return f32_out ? launch_mode<MD, true, kBiasPairs>(p, grid, stream)                               \
+                     : launch_mode<MD, false, kBiasPairs>(p, grid, stream);                             \
+    default:                                                                                            \
+      return f32_out ? launch_mode<MD, true, kBiasKeys>(p, grid, stream)                                \
+                     : launch_mode<MD, false, kBiasKeys>(p, grid, stream);                              \
+  }
+      if (a.mode == 0) SWIN_TC_LAUNCH(0)
+      SWIN_TC_LAUNCH(1)
+#undef SWIN_TC_LAUNCH
+    }
+    default:
+      return f32_out ? launch_mode<2, true, kBiasNone>(p, grid, stream) : launch_mode<2, false, kBiasNone>(p, grid, stream);
   }
 }
 
