@@ -183,6 +183,15 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def whole_job(wk: dict, world: int, ms_max: float) -> dict:
+    """Whole-job rates of `world` replica ranks that each processed one
+    workload `wk` (weak scaling), timed as the slowest rank's ms per step."""
+    sec = ms_max * 1e-3
+    return {"tokens_per_s": wk["tokens"] * world / sec,
+            "tflops": wk["flops_std"] * world / sec / 1e12,
+            "tflops_exact": wk["flops_exact"] * world / sec / 1e12}
+
+
 def run_native(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -242,8 +251,8 @@ def run_native(args, rank: int, world: int, local_rank: int):
     ms = max_over_ranks(sum(times) / len(times), world, device)
     wk = work(w)
     tokens = wk["tokens"] * world
-    value = tokens / (ms * 1e-3)
-    tflops = wk["flops_std"] * world / (ms * 1e-3) / 1e12
+    job = whole_job(wk, world, ms)
+    value, tflops = job["tokens_per_s"], job["tflops"]
     peaks = read_peaks()
 
     # dominant kernel alone: the attention kernel with the bias table given
@@ -295,7 +304,7 @@ def run_native(args, rank: int, world: int, local_rank: int):
                    "M": w.M, "shift": s, "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode],
                    "global_batch": w.B * world, "parallelism": "replicas x%d" % world,
                    "l2": "flushed before every timed step (256 MB write)"},
-        "tflops": round(tflops, 2), "tflops_exact_pairs": round(wk["flops_exact"] * world / (ms * 1e-3) / 1e12, 2),
+        "tflops": round(tflops, 2), "tflops_exact_pairs": round(job["tflops_exact"], 2),
         "roofline": roofline,
         "e2e": {"value": round(tokens / (e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
