@@ -340,7 +340,7 @@ def run_cpu_baseline(w: syn.Workload, budget_s: float):
     nq = int(min(w.H * w.W * w.B, max(nq, nq * budget_s / max(t, 1e-6))))
     t = run(nq)
     return {"value": round(nq / t, 2), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d random query tokens (all %d heads) of one %dx%d image, %.1f s" % (nq, w.heads, w.H, w.W, t),
+            "sample": "%d query tokens drawn with replacement from one %dx%d image (all %d heads), %.1f s" % (nq, w.H, w.W, w.heads, t),
             "seconds": round(t, 2)}
 
 
