@@ -35,29 +35,47 @@ def seg_len(k, L, M, s):
 
 
 def items_for(B, H, W, heads, M, s, cta, grid):
-    """(has work, tile of warpgroup 0, tile of warpgroup 1, K/V blocks) of the
-    items CTA `cta` walks, in the kernel's order (tile pair fastest, then
-    segment x, segment y, image, head)."""
+    """Work items of CTA `cta` in the kernel's order: heads outermost, then
+    image, then rows of rectangles; item i of a row takes tiles 2i and 2i+1 of
+    the row's tile list (rectangles left to right, each split into query
+    tiles of floor(128 / lx) rows).  Returns (nb0, nb1, shared) per item: K/V
+    blocks of warpgroup 0's and 1's rectangles (nb1 = 0: no second tile) and
+    whether both tiles are in one rectangle (K/V blocks shared)."""
     nsy, nsx = nseg(H, M, s), nseg(W, M, s)
+    cls = lambda sx: 0 if sx == 0 else (2 if sx == nsx - 1 else 1)
     lxs = [seg_len(0, W, M, s), seg_len(1, W, M, s) if nsx > 2 else seg_len(0, W, M, s), seg_len(nsx - 1, W, M, s)]
     R = [128 // l for l in lxs]
     Rk = [KBLK // l for l in lxs]
-    tiles_max = max((M + r - 1) // r for r in R)
-    pmax = (tiles_max + 1) // 2
-    n_items = B * heads * nsy * nsx * pmax
-    out = []
-    for it in range(cta, n_items, grid):
-        i = it
-        pr = i % pmax; i //= pmax
-        sx = i % nsx; i //= nsx
-        sy = i % nsy; i //= nsy
-        cls = 0 if sx == 0 else (2 if sx == nsx - 1 else 1)
+    per_hb = []
+    for sy in range(nsy):
         ly = seg_len(sy, H, M, s)
-        nb = (ly + Rk[cls] - 1) // Rk[cls]
-        ntiles = (ly + R[cls] - 1) // R[cls]
-        v0 = 2 * pr < ntiles
-        v1 = 2 * pr + 1 < ntiles
-        out.append((v0, v0, v1, nb))
+        tiles = []
+        for sx in range(nsx):
+            c = cls(sx)
+            nt = (ly + R[c] - 1) // R[c]
+            tiles += [(sx, (ly + Rk[c] - 1) // Rk[c])] * nt
+        for i in range(0, len(tiles), 2):
+            a = tiles[i]
+            if i + 1 < len(tiles):
+                b = tiles[i + 1]
+                per_hb.append((a[1], b[1], a[0] == b[0]))
+            else:
+                per_hb.append((a[1], 0, False))
+    n_items = B * heads * len(per_hb)
+    return [per_hb[it % len(per_hb)] for it in range(cta, n_items, grid)]
+
+
+def kv_order(nb0, nb1, shared):
+    """Consumers of the item's K/V loads in ring order: shared blocks go to
+    both warpgroups; otherwise the two rectangles' blocks alternate, then the
+    longer one's remainder follows."""
+    if shared:
+        return [(0, 1)] * nb0
+    mn = min(nb0, nb1)
+    out = []
+    for j in range(mn):
+        out += [(0,), (1,)]
+    out += [(0,)] * (nb0 - mn) + [(1,)] * (nb1 - mn)
     return out
 
 
@@ -100,28 +118,26 @@ def run(items, mode, seed, rescale_p=0.2, early_pv=True):
 
     def producer():
         qu = [0, 0]; ku = 0
-        for (any_, v0, v1, nb) in items:
-            if not any_: continue
-            for g, v in ((0, v0), (1, v1)):
+        for (nb0, nb1, shared) in items:
+            for g, v in ((0, True), (1, nb1 > 0)):
                 if not v: continue
                 qs = qu[g] & 1
                 if qu[g] >= 2: yield W(("q_empty", g, qs), (qu[g] >> 1) - 1)
                 tma.append(("q_full", g, qs)); qu[g] += 1
-            for j in range(nb):
+            for _ in kv_order(nb0, nb1, shared):
                 st = ku % S
                 if ku >= S: yield W(("kv_empty", st), ku // S - 1)
                 tma.append(("kv_full", st)); ku += 1
 
     def prep():
         qu = [0, 0]; ku = 0
-        for (any_, v0, v1, nb) in items:
-            if not any_: continue
-            for g, v in ((0, v0), (1, v1)):
+        for (nb0, nb1, shared) in items:
+            for g, v in ((0, True), (1, nb1 > 0)):
                 if not v: continue
                 qs = qu[g] & 1
                 yield W(("q_full", g, qs), qu[g] >> 1); qu[g] += 1
                 bars[("q_ready", g, qs)].arrive()
-            for j in range(nb):
+            for _ in kv_order(nb0, nb1, shared):
                 st = ku % S
                 yield W(("kv_full", st), ku // S); ku += 1
                 bars[("kv_ready", st)].arrive()
@@ -136,15 +152,16 @@ def run(items, mode, seed, rescale_p=0.2, early_pv=True):
             c = [("o_done", g, k & 1), ("kv_empty", st)]
             if rel2: c.append(("kv_empty", st))
             mmaq[g].append(c)
-        for (any_, v0, v1, nb) in items:
-            if not any_: continue
-            u0 = u; u += nb
-            if not (v0 if g == 0 else v1): continue
+        for (nb0, nb1, shared) in items:
+            order = kv_order(nb0, nb1, shared)
+            u0 = u; u += len(order)
+            mine = [u0 + k for k, c in enumerate(order) if g in c]
+            if not mine: continue
             qs, qpar = qcnt & 1, (qcnt >> 1)
             qcnt += 1
-            rel2 = g == 0 and not v1
-            for j in range(nb):
-                uu = u0 + j; st = uu % S
+            rel2 = not shared
+            for j, uu in enumerate(mine):
+                st = uu % S
                 while npv + 2 <= b:
                     yield from issue_pv(npv); npv += 1
                 if early_pv and npv < b and u_last + S <= uu:
@@ -152,7 +169,7 @@ def run(items, mode, seed, rescale_p=0.2, early_pv=True):
                 if j == 0: yield W(("q_ready", g, qs), qpar)
                 yield W(("kv_ready", st), uu // S)
                 c = [("s_full", g, b & 1)]
-                if j == nb - 1: c.append(("q_empty", g, qs))
+                if j == len(mine) - 1: c.append(("q_empty", g, qs))
                 mmaq[g].append(c)
                 pend[b & 1] = (st, j > 0, rel2)
                 u_last = uu
@@ -169,16 +186,16 @@ def run(items, mode, seed, rescale_p=0.2, early_pv=True):
             while o_cons[0] <= upto:
                 yield W(("o_done", g, o_cons[0] & 1), o_cons[0] >> 1)
                 o_cons[0] += 1
-        for (any_, v0, v1, nb) in items:
-            ku0 = ku
-            if any_: ku += nb
-            if not (v0 if g == 0 else v1): continue
+        for (nb0, nb1, shared) in items:
+            order = kv_order(nb0, nb1, shared)
+            ku0 = ku; ku += len(order)
+            mine = [ku0 + k for k, c in enumerate(order) if g in c]
+            if not mine: continue
             qs = qu & 1
             yield W(("q_ready", g, qs), qu >> 1); qu += 1
             bars[("q_empty", g, qs)].arrive(4)
-            for j in range(nb):
+            for j, uu in enumerate(mine):
                 yield W(("s_full", g, blk & 1), blk >> 1)
-                uu = ku0 + j
                 if mode == 1: yield W(("kv_ready", uu % S), uu // S)
                 if blk >= 2: o_cons[0] = max(o_cons[0], blk - 1)  # implied by s_full(blk)
                 epi = j == 0 and pend
@@ -239,6 +256,7 @@ WORKLOADS = {  # B, H, W, heads, M, shift, mode
     "M24-no-shift-odd": (1, 100, 60, 5, 24, 0, 0),
     "M16-shift0": (2, 33, 33, 1, 16, 0, 2),
     "thin-M8": (1, 9, 200, 4, 8, 4, 1),
+    "M64-rows": (32, 70, 64, 3, 64, 0, 2),
 }
 
 
@@ -254,9 +272,12 @@ def test_protocol_no_deadlock_no_parity_alias(name):
 
 def test_model_catches_the_deadlock_it_guards_against():
     """Without the early PV issue (a pending PV whose K/V slot is a whole
-    ring behind the block being waited for) the model deadlocks on the M=16
-    workload, where most items have one query tile."""
-    items = items_for(64, 64, 64, 3, 16, 8, 0, 148)
+    ring behind the block being waited for) the model deadlocks: with M = 64
+    and a 6-row last rectangle row, an item that only warpgroup 0 works on
+    fills the ring while warpgroup 1's last PV waits behind its next item."""
+    items = items_for(32, 70, 64, 3, 64, 0, 5, 148)
     with pytest.raises(Deadlock):
         for seed in range(8):
-            run(items, 1, seed, early_pv=False)
+            run(items, 2, seed, early_pv=False)
+    for seed in range(4):
+        run(items, 2, seed)

@@ -85,10 +85,13 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
 
 struct TcParams {
   CUtensorMap tmap[3][3];  // [tensor q/k/v][x-class first/middle/last]
-  FastDiv div_pmax, div_nsx, div_nsy, div_B;
+  FastDiv div_ipb, div_B, div_mid_items, div_mid_tiles[3];
   int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
+  // per row class (first, middle, last row of rectangles): height, items,
+  // and per x-class the query tiles and K/V blocks of one rectangle
+  int row_ly[3], row_items[3], row_tiles[3][3], row_nb[3][3];
   void* out;
-  int B, H, W, heads, M, s, nsy, nsx, pmax;
+  int B, H, W, heads, M, s, nsy, nsx;
   int R2e;  // row stride of the bias slot (even, >= 2M - 1, chosen against bank conflicts)
   long long n_items;
   const float* tau;
@@ -139,45 +142,119 @@ struct Bars {
 };
 static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
 
+// One warpgroup's query tile: its rectangle (a column segment of the item's
+// row of rectangles) and the tile's index in it.
+struct Rect {
+  int cls, lx, R, Rk, x0, tile, nb;  // x-class, width, tile rows, K/V block rows, first column, tile, K/V blocks
+};
+
+// A work item: query tiles 2i and 2i + 1 of one row of rectangles of one
+// (head, image), the row's tiles listed rectangle by rectangle.  Warpgroup 0
+// takes the first; warpgroup 1 the second, if the row has it.  Two tiles of
+// one rectangle share its K/V blocks; tiles of two rectangles stream both
+// rectangles' blocks, alternating (A0, B0, A1, B1, ...), then the longer one's
+// remainder, each block used by one warpgroup.
 struct Task {
-  bool any;  // item has work (a query tile for warpgroup 0)
-  int b, h, cls, lx, R, Rk, y0, x0, ly, n, nb, pr, ntiles;
-  // warpgroup g's query tile: rectangle rows [tile(g) R, tile(g) R + R)
-  __device__ __forceinline__ int tile(int g) const { return 2 * pr + g; }
-  __device__ __forceinline__ bool valid(int g) const { return tile(g) < ntiles; }
+  int b, h, y0, ly;
+  bool v1;      // warpgroup 1 has a tile
+  bool shared;  // both tiles in one rectangle
+  int nbt;      // K/V blocks the item loads
+  Rect r0, r1;
+  __device__ __forceinline__ bool valid(int g) const { return g == 0 || v1; }
+  __device__ __forceinline__ Rect rect(int g) const { return g ? r1 : r0; }
   __device__ __forceinline__ int nq(int g) const {  // queries of warpgroup g's tile
-    const int rows = ly - tile(g) * R;
-    return valid(g) ? (rows < R ? rows : R) * lx : 0;
+    const Rect r = rect(g);
+    const int rows = ly - r.tile * r.R;
+    return (rows < r.R ? rows : r.R) * r.lx;
+  }
+  // position among the item's K/V loads of warpgroup g's block j
+  __device__ __forceinline__ int kv_index(int g, int j) const {
+    if (shared) return j;
+    const int mn = r0.nb < r1.nb ? r0.nb : r1.nb;
+    return j < mn ? 2 * j + g : mn + j;
+  }
+  // owner warpgroup (its rectangle) and block index of the item's K/V load jj
+  __device__ __forceinline__ Rect kv_rect(int jj, int& j) const {
+    const int mn = shared ? 0 : (r0.nb < r1.nb ? r0.nb : r1.nb);
+    if (jj < 2 * mn) {
+      j = jj >> 1;
+      return (jj & 1) ? r1 : r0;
+    }
+    j = jj - mn;
+    return (shared || r0.nb > r1.nb) ? r0 : r1;
   }
 };
 
 __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
   Task t;
   uint32_t i = (uint32_t)item;
-  uint32_t q = fdiv(i, p.div_pmax);
-  const int pr = (int)(i - q * p.div_pmax.d);
-  i = q;
-  q = fdiv(i, p.div_nsx);
-  const int sx = (int)(i - q * p.div_nsx.d);
-  i = q;
-  q = fdiv(i, p.div_nsy);
-  const int sy = (int)(i - q * p.div_nsy.d);
+  uint32_t q = fdiv(i, p.div_ipb);
+  uint32_t rem = i - q * p.div_ipb.d;  // item within (head, image)
   i = q;
   q = fdiv(i, p.div_B);
   t.b = (int)(i - q * p.div_B.d);
   t.h = (int)q;  // heads outermost: a CTA keeps one head's bias table for many items
-  t.cls = sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1);
-  t.lx = p.lx[t.cls];
-  t.R = p.R[t.cls];
-  t.Rk = p.Rk[t.cls];
+  // row of rectangles: row 0, the nsy - 2 middle rows, the last row
+  int rc, sy;
+  uint32_t ii;
+  if (rem < (uint32_t)p.row_items[0]) {
+    rc = 0;
+    sy = 0;
+    ii = rem;
+  } else {
+    rem -= (uint32_t)p.row_items[0];
+    const uint32_t mid = p.nsy > 2 ? (uint32_t)(p.nsy - 2) * (uint32_t)p.row_items[1] : 0u;
+    if (rem < mid) {
+      const uint32_t r = fdiv(rem, p.div_mid_items);
+      rc = 1;
+      sy = 1 + (int)r;
+      ii = rem - r * (uint32_t)p.row_items[1];
+    } else {
+      rc = 2;
+      sy = p.nsy - 1;
+      ii = rem - mid;
+    }
+  }
   t.y0 = swin_seg_start(sy, p.M, p.s);
-  t.ly = swin_seg_len(sy, p.H, p.M, p.s);
-  t.x0 = swin_seg_start(sx, p.M, p.s);
-  t.n = t.ly * t.lx;
-  t.nb = (t.ly + t.Rk - 1) / t.Rk;
-  t.pr = pr;
-  t.ntiles = (t.ly + t.R - 1) / t.R;
-  t.any = t.valid(0);
+  t.ly = p.row_ly[rc];
+  const int T = p.nsx == 1 ? p.row_tiles[rc][0]
+                           : p.row_tiles[rc][0] + (p.nsx - 2) * p.row_tiles[rc][1] + p.row_tiles[rc][2];
+  // tile k of the row -> (column segment, tile)
+  auto tile_at = [&](int k, Rect& r) -> int {
+    int sx = 0;
+    const int t0 = p.row_tiles[rc][0];
+    if (p.nsx > 1 && k >= t0) {
+      k -= t0;
+      const int mid = (p.nsx - 2) * p.row_tiles[rc][1];
+      if (k < mid) {
+        const int r2 = (int)fdiv((uint32_t)k, p.div_mid_tiles[rc]);
+        sx = 1 + r2;
+        k -= r2 * p.row_tiles[rc][1];
+      } else {
+        sx = p.nsx - 1;
+        k -= mid;
+      }
+    }
+    r.cls = sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1);
+    r.lx = p.lx[r.cls];
+    r.R = p.R[r.cls];
+    r.Rk = p.Rk[r.cls];
+    r.x0 = swin_seg_start(sx, p.M, p.s);
+    r.tile = k;
+    r.nb = p.row_nb[rc][r.cls];
+    return sx;
+  };
+  const int sx0 = tile_at(2 * (int)ii, t.r0);
+  t.v1 = 2 * (int)ii + 1 < T;
+  int sx1 = -1;
+  if (t.v1) {
+    sx1 = tile_at(2 * (int)ii + 1, t.r1);
+  } else {
+    t.r1 = t.r0;
+    t.r1.nb = 0;
+  }
+  t.shared = sx1 == sx0;
+  t.nbt = t.shared ? t.r0.nb : t.r0.nb + t.r1.nb;
   return t;
 }
 
@@ -414,27 +491,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         bool ok = true;
         for (long long it = first; it < p.n_items && ok; it += step) {
           const Task t = decode(p, it);
-          if (!t.any) continue;
-          const uint32_t qbytes = (uint32_t)(64 * t.lx * t.R), kbytes = (uint32_t)(64 * t.lx * t.Rk);
           for (int g = 0; g < 2 && ok; ++g) {
             if (!t.valid(g)) continue;
+            const Rect r = t.rect(g);
             const int qs = qu[g] & 1;
             if (qu[g] >= 2) ok = wait_bar(&bars->q_empty[g][qs], ((qu[g] >> 1) - 1) & 1, ctl);
             if (!ok) break;
-            ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], qbytes);
-            ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][t.cls], &bars->q_full[g][qs], 0, t.h,
-                             t.x0, t.y0 + t.tile(g) * t.R, t.b);
+            ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], (uint32_t)(64 * r.lx * r.R));
+            ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][r.cls], &bars->q_full[g][qs], 0, t.h,
+                             r.x0, t.y0 + r.tile * r.R, t.b);
             ++qu[g];
           }
-          for (int j = 0; j < t.nb && ok; ++j) {
+          for (int jj = 0; jj < t.nbt && ok; ++jj) {
+            int j;
+            const Rect r = t.kv_rect(jj, j);
             const int st = ku % kStages;
             if (ku >= (uint32_t)kStages) ok = wait_bar(&bars->kv_empty[st], ((ku / kStages) - 1) & 1, ctl);
             if (!ok) break;
             uint8_t* kb = kvbuf + st * 2 * kTileBytes;
-            ptx::mbar_arrive_expect_tx(&bars->kv_full[st], 2 * kbytes);
-            ptx::tma_load_5d(kb, &p.tmap[1][t.cls], &bars->kv_full[st], 0, t.h, t.x0, t.y0 + j * t.Rk, t.b);
-            ptx::tma_load_5d(kb + kTileBytes, &p.tmap[2][t.cls], &bars->kv_full[st], 0, t.h, t.x0,
-                             t.y0 + j * t.Rk, t.b);
+            ptx::mbar_arrive_expect_tx(&bars->kv_full[st], (uint32_t)(2 * 64 * r.lx * r.Rk));
+            ptx::tma_load_5d(kb, &p.tmap[1][r.cls], &bars->kv_full[st], 0, t.h, r.x0, t.y0 + j * r.Rk, t.b);
+            ptx::tma_load_5d(kb + kTileBytes, &p.tmap[2][r.cls], &bars->kv_full[st], 0, t.h, r.x0,
+                             t.y0 + j * r.Rk, t.b);
             ++ku;
           }
         }
@@ -497,16 +575,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         uint32_t u = 0, qcnt = 0, b = 0, npv = 0, u_last = 0;
         for (long long it = first; it < p.n_items && ok; it += step) {
           const Task t = decode(p, it);
-          if (!t.any) continue;
           const uint32_t u0 = u;
-          u += t.nb;
+          u += t.nbt;
           if (!t.valid(g)) continue;
           const uint32_t qs = qcnt & 1, qpar = (qcnt >> 1) & 1;
           ++qcnt;
           const uint64_t ad = qd0 + qs * kQBuf;
-          const uint32_t rel2 = (g == 0 && !t.valid(1)) ? 512u : 0u;
-          for (int j = 0; j < t.nb; ++j, ++b) {
-            const uint32_t uu = u0 + j, st = uu % kStages;
+          const int nb = t.rect(g).nb;
+          // a block used by this warpgroup alone takes both releases of its stage
+          const uint32_t rel2 = t.shared ? 0u : 512u;
+          for (int j = 0; j < nb; ++j, ++b) {
+            const uint32_t uu = u0 + t.kv_index(g, j), st = uu % kStages;
             // S(b) overwrites P(b - 2): PV(b - 2) first
             while (ok && npv + 2 <= b) ok = issue_pv(npv++);
             // A pending PV(b - 1) whose K/V use is a whole ring behind block
@@ -522,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ptx::mma_ss(dS, ad, bd, idS, 0);
             ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
             ptx::mma_commit(&bars->s_full[g][b & 1]);
-            if (j == t.nb - 1) ptx::mma_commit(&bars->q_empty[g][qs]);
+            if (j == nb - 1) ptx::mma_commit(&bars->q_empty[g][qs]);
             const uint32_t info = st | (j > 0 ? 256u : 0u) | rel2;
             if (b & 1) pend1 = info; else pend0 = info;
             u_last = uu;
@@ -545,15 +624,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
       for (long long it = first; it < p.n_items && ok; it += step) {
         const Task t = decode(p, it);
-        if (!t.any) continue;
-        const int qrows = t.lx * t.R, krows = t.lx * t.Rk;
-        const int* rp = rpos + t.cls * 128;
-        // window-local coordinates of the rectangle's first row and column
-        const int py0 = swin_local_coord(t.y0, M, s), px0 = swin_local_coord(t.x0, M, s);
+        // window-local coordinate of the row of rectangles' first row
+        const int py0 = swin_local_coord(t.y0, M, s);
         for (int g = 0; g < 2 && ok; ++g) {
           if (!t.valid(g)) continue;
+          const Rect rq = t.rect(g);
+          const int qrows = rq.lx * rq.R;
+          const int* rp = rpos + rq.cls * 128;
+          const int px0 = swin_local_coord(rq.x0, M, s);
           const int qs = qu[g] & 1;
-          ok = wait_bar(&bars->q_full[g][qs], (qu[g] >> 1) & 1, ctl);
+          // warp-uniform outcome (the shuffles below need every lane)
+          ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[g][qs], (qu[g] >> 1) & 1, ctl));
           ++qu[g];
           if (!ok) break;
           uint8_t* tile = qbuf + (g * 2 + qs) * kTileBytes;
@@ -574,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               } else {
                 if (act) {
                   const int pr = rp[r];
-                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + t.tile(g) * t.R + (pr & 0xFFFF), 63), rcos,
+                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + rq.tile * rq.R + (pr & 0xFFFF), 63), rcos,
                             rsin);
                 }
                 float m = half_absmax(v);
@@ -590,9 +671,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
           ptx::mbar_arrive(&bars->q_ready[g][qs]);
         }
-        for (int j = 0; j < t.nb && ok; ++j) {
+        for (int jj = 0; jj < t.nbt && ok; ++jj) {
+          int j;
+          const Rect rk = t.kv_rect(jj, j);
+          const int krows = rk.lx * rk.Rk;
+          const int* rp = rpos + rk.cls * 128;
+          const int px0 = swin_local_coord(rk.x0, M, s);
           const int st = ku % kStages;
-          ok = wait_bar(&bars->kv_full[st], (ku / kStages) & 1, ctl);
+          ok = __all_sync(0xffffffffu, wait_bar(&bars->kv_full[st], (ku / kStages) & 1, ctl));
           ++ku;
           if (!ok) break;
           uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
@@ -614,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               if (act && h == 0) kcol[st * 128 + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
             } else if (act) {
               const int pr = rp[r];
-              rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + j * t.Rk + (pr & 0xFFFF), 63), rcos, rsin);
+              rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + j * rk.Rk + (pr & 0xFFFF), 63), rcos, rsin);
               range_hit |= half_absmax(v) >= 65504.0f;
               store_half_f16(ktile, r, h, v, 1.0f);
             }
@@ -692,8 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (long long it = first; it < p.n_items && ok; it += step) {
       const Task tk = decode(p, it);
       const uint32_t ku0 = ku;
-      if (tk.any) ku += tk.nb;  // K/V block uses of this item (both warpgroups)
+      ku += tk.nbt;  // K/V loads of this item (both warpgroups)
       if (!tk.valid(g)) continue;
+      const Rect rg = tk.rect(g);
       if (has_table && tk.h != cur_h) {
         // new head: once all four warps are done with the old table, each
         // loads a quarter of the new one (times log2 e, zero padding column)
@@ -726,7 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
       const bool row_ok = t < tk.nq(g);
-      const int qy = tk.tile(g) * tk.R + t / tk.lx, qx = t % tk.lx;
+      const int qy = rg.tile * rg.R + t / rg.lx, qx = t % rg.lx;
       // Slot index of this row's bias for key (0, 0) of the rectangle; the
       // pair load for keys (2c, 2c+1) of a row starts one float earlier, in
       // copy 0 when that index is even, else in copy 1 (the parity is fixed
@@ -736,9 +823,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // most 95 rows of 2M floats before slot 0, inside shared memory.
       const int bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
       const float* pbase = slot + (((bbase - 1) & 1) ? kCopy1 - 1 : 0) + bbase - 1;
-      const int* kof = kofs + tk.cls * 128;
+      const int* kof = kofs + rg.cls * 128;
       float m_run = -INFINITY;
-      for (int j = 0; j < tk.nb; ++j, ++blk) {
+      for (int j = 0; j < rg.nb; ++j, ++blk) {
         SWIN_TC_MARK(0);
         ok = wait_bar(&bars->s_full[g][blk & 1], (blk >> 1) & 1, ctl);
         ok = __all_sync(0xffffffffu, ok);
@@ -761,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
         }
         SWIN_TC_MARK(2);
-        const uint32_t u = ku0 + j, ust = u % kStages;
+        const uint32_t u = ku0 + tk.kv_index(g, j), ust = u % kStages;
         if (MODE == 1) {
           // 1/|k| of the block's keys was written by prep before it released kv_ready
           ok = wait_bar(&bars->kv_ready[ust], (u / kStages) & 1, ctl);
@@ -770,8 +857,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
         SWIN_TC_MARK(11);
         const float ascale = alpha;
-        const int nk_all = tk.n - j * tk.Rk * tk.lx;
-        const int nk = nk_all < tk.Rk * tk.lx ? nk_all : tk.Rk * tk.lx;
+        const int nk_all = (tk.ly - j * rg.Rk) * rg.lx;
+        const int nk = nk_all < rg.Rk * rg.lx ? nk_all : rg.Rk * rg.lx;
         // x = log2-domain logits.  Mode 2: the scale is applied inside the
         // exponent below (max over raw scores, scale > 0).  Modes 0/1:
         // x = S * scale + bias in one rounding; the bias slot already holds
@@ -779,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (MODE != 2) {
           const float4* kc4 = reinterpret_cast<const float4*>(kcol + ust * 128);
           const int4* kof4 = reinterpret_cast<const int4*>(kof);
-          const int jo = j * tk.Rk * R2e;  // block j starts Rk rectangle rows further
+          const int jo = j * rg.Rk * R2e;  // block j starts Rk rectangle rows further
           if (!has_table) {
             const float2 a2 = make_float2(ascale, ascale);
 #pragma unroll
@@ -918,7 +1005,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       SWIN_TC_MARK(8);
       pend = true;
       pend_ok = row_ok;
-      pend_off = (((size_t)tk.b * p.H + (tk.y0 + qy)) * p.W + (tk.x0 + qx)) * (size_t)(p.heads * 32) +
+      pend_off = (((size_t)tk.b * p.H + (tk.y0 + qy)) * p.W + (rg.x0 + qx)) * (size_t)(p.heads * 32) +
                  (size_t)tk.h * 32;
       SWIN_TC_MARK(10);
     }
@@ -1010,18 +1097,32 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   const int lxs[3] = {swin_seg_len(0, a.W, a.M, a.shift),
                       p.nsx > 2 ? swin_seg_len(1, a.W, a.M, a.shift) : swin_seg_len(0, a.W, a.M, a.shift),
                       swin_seg_len(p.nsx - 1, a.W, a.M, a.shift)};
-  int tiles_max = 1;
   for (int c = 0; c < 3; ++c) {
     p.lx[c] = lxs[c];
     p.R[c] = 128 / lxs[c];    // query tile: whole rectangle rows, at most 128 queries
     p.Rk[c] = kBlk / lxs[c];  // K/V block: whole rectangle rows, at most 96 keys
-    const int tl = (a.M + p.R[c] - 1) / p.R[c];
-    if (tl > tiles_max) tiles_max = tl;
     if (!encode_map(&p.tmap[0][c], a.q, a, p.lx[c], p.R[c]) ||
         !encode_map(&p.tmap[1][c], a.k, a, p.lx[c], p.Rk[c]) ||
         !encode_map(&p.tmap[2][c], a.v, a, p.lx[c], p.Rk[c]))
       return fail(SWIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (lx=%d, R=%d)", p.lx[c], p.R[c]);
   }
+  // rows of rectangles by class: first, middle (if any), last
+  const int lys[3] = {swin_seg_len(0, a.H, a.M, a.shift),
+                      p.nsy > 2 ? swin_seg_len(1, a.H, a.M, a.shift) : swin_seg_len(0, a.H, a.M, a.shift),
+                      swin_seg_len(p.nsy - 1, a.H, a.M, a.shift)};
+  for (int rc = 0; rc < 3; ++rc) {
+    p.row_ly[rc] = lys[rc];
+    for (int c = 0; c < 3; ++c) {
+      p.row_tiles[rc][c] = (lys[rc] + p.R[c] - 1) / p.R[c];
+      p.row_nb[rc][c] = (lys[rc] + p.Rk[c] - 1) / p.Rk[c];
+    }
+    const int T = p.nsx == 1 ? p.row_tiles[rc][0]
+                             : p.row_tiles[rc][0] + (p.nsx - 2) * p.row_tiles[rc][1] + p.row_tiles[rc][2];
+    p.row_items[rc] = (T + 1) / 2;
+    p.div_mid_tiles[rc] = make_fastdiv((uint32_t)p.row_tiles[rc][1]);
+  }
+  const long long ipb = (long long)p.row_items[0] + (p.nsy > 2 ? (long long)(p.nsy - 2) * p.row_items[1] : 0) +
+                        (p.nsy > 1 ? p.row_items[2] : 0);
   // Bias-slot row stride: the even value in [2M, 2M + 14] (whose two copies fit
   // the slot) with the fewest shared-memory wavefronts for the paired bias
   // loads of this launch's rectangle widths.  A warp's 32 queries load 8
@@ -1055,12 +1156,10 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
       }
     }
   }
-  p.pmax = (tiles_max + 1) / 2;
-  p.n_items = (long long)a.B * a.heads * p.nsy * p.nsx * p.pmax;
+  p.n_items = (long long)a.B * a.heads * ipb;
   if (p.n_items >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "too many work items (%lld)", p.n_items);
-  p.div_pmax = make_fastdiv((uint32_t)p.pmax);
-  p.div_nsx = make_fastdiv((uint32_t)p.nsx);
-  p.div_nsy = make_fastdiv((uint32_t)p.nsy);
+  p.div_ipb = make_fastdiv((uint32_t)ipb);
+  p.div_mid_items = make_fastdiv((uint32_t)p.row_items[1]);
   p.div_B = make_fastdiv((uint32_t)a.B);
   p.out = a.out;
   p.tau = a.tau;
