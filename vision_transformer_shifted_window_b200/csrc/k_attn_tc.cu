@@ -9,9 +9,10 @@
 // — without ever storing a score matrix: FlashSwin's point is that the
 // per-window score matrix is the memory problem; here S lives only in TMEM.
 //
-// Work unit: a pair of query tiles of one rectangle (tile = floor(128 / lx)
-// whole rectangle rows), one per softmax warpgroup; both warpgroups stream
-// the same K/V blocks of floor(96 / lx) rectangle rows (at most 96 keys).
+// Work unit: two consecutive query tiles (tile = floor(128 / lx) whole
+// rectangle rows) of one row of rectangles, one per softmax warpgroup.  Tiles
+// of one rectangle share its K/V blocks of floor(96 / lx) rectangle rows (at
+// most 96 keys); tiles of two rectangles stream both rectangles' blocks.
 //
 // Warp roles (512 threads, one persistent CTA per SM):
 //   warp 0      TMA producer: Q tiles and K/V blocks, 5-D tensor maps over
