@@ -61,7 +61,8 @@ def call_fwd(L, **kw):
 
 @pytest.mark.parametrize("kw,why", [
     (dict(q=None), "NULL"), (dict(shift=4), "shift"), (dict(shift=-1), "shift"), (dict(M=0), "M"),
-    (dict(M=65, shift=0), "M"), (dict(B=0), ">= 1"), (dict(q=FAKE + 8), "aligned"),
+    (dict(M=65, shift=0), "M"), (dict(B=0), ">= 1"), (dict(H=0), ">= 1"), (dict(W=0), ">= 1"),
+    (dict(heads=0), ">= 1"), (dict(d=0), ">= 1"), (dict(q=FAKE + 8), "aligned"),
     (dict(out=FAKE * 2), "overlaps"), (dict(mode=1), "tau"), (dict(mode=2), "rope"),
     (dict(mode=2, rope=FAKE * 5, d=30), "d % 4"), (dict(mode=2, rope=FAKE * 5, table=FAKE * 6), "no bias"),
     (dict(mode=7), "mode"), (dict(dt=5), "dtype"), (dict(dt=0, odt=1), "output dtype"),
