@@ -183,6 +183,18 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+MUFU_EX2_PER_CLK_PER_SM = 16  # B200: exp2 throughput of the special-function unit
+
+
+def exp_bound(wk: dict, sms: int, clock_mhz: float, kernel_ms: float) -> dict:
+    """Time the exponentials alone need if every one ran on the MUFU (one per
+    attended pair), and the fraction of it the kernel achieves: at d = 32 this,
+    not the tensor pipe, is the ceiling of an all-MUFU softmax."""
+    t_ms = wk["exps"] / (MUFU_EX2_PER_CLK_PER_SM * sms * clock_mhz * 1e6) * 1e3
+    return {"ex2_per_clk_per_sm": MUFU_EX2_PER_CLK_PER_SM, "sms": sms, "clock_mhz": clock_mhz,
+            "bound_ms": round(t_ms, 5), "frac": round(t_ms / kernel_ms, 4)}
+
+
 def whole_job(wk: dict, world: int, ms_max: float) -> dict:
     """Whole-job rates of `world` replica ranks that each processed one
     workload `wk` (weak scaling), timed as the slowest rank's ms per step."""
@@ -276,7 +288,9 @@ def run_native(args, rank: int, world: int, local_rank: int):
                 "hbm_achieved_gbs": round(wk["bytes"] / (k_ms * 1e-3) / 1e9, 1),
                 "hbm_frac": round(wk["bytes"] / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                 "attainable_frac": round(achieved / min(peaks["bf16_tflops"],
-                                                        peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3), 4)}
+                                                        peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3), 4),
+                "exp_bound": exp_bound(wk, torch.cuda.get_device_properties(device).multi_processor_count,
+                                       float(clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965.0), k_ms)}
 
     # end to end through host buffers: H2D of q/k/v, the call, D2H of out
     hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
