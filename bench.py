@@ -277,8 +277,17 @@ def run_native(args, rank: int, world: int, local_rank: int):
             sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, stream=stream, **kw_k)
         timed_loop(kstep, 5)
         ktimes = timed_loop(kstep, max(10, min(args.steps, 200)))
+        # the CPB meta network alone, in both forms (eq. 3 / eq. 4 and the released code's)
+        cpb_us = {}
+        for name, form in (("paper", sa.SWIN_CPB_PAPER), ("code", sa.SWIN_CPB_CODE)):
+            def cstep(form=form):
+                sa.swin_cpb_eval_form(w.M, w.heads, *kw["cpb"], form, 0, out=table, stream=stream)
+            timed_loop(cstep, 5, flush_l2=False)
+            ct = timed_loop(cstep, 50, flush_l2=False)
+            cpb_us[name] = round(1e3 * sorted(ct)[len(ct) // 2], 2)
     else:
         ktimes = times
+        cpb_us = None
     k_ms = max_over_ranks(sum(ktimes) / len(ktimes), world, device)
     achieved = wk["flops_std"] / (k_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
@@ -320,6 +329,7 @@ def run_native(args, rank: int, world: int, local_rank: int):
                    "l2": "flushed before every timed step (256 MB write)"},
         "tflops": round(tflops, 2), "tflops_exact_pairs": round(job["tflops_exact"], 2),
         "roofline": roofline,
+        **({"cpb_us": cpb_us} if cpb_us else {}),
         "e2e": {"value": round(tokens / (e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
         "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
@@ -411,7 +421,8 @@ def main():
             others.append({"workload": l2["config"]["workload"], "tokens_per_s": l2["value"],
                            "tflops": l2["tflops"], "ms_per_step": l2["ms_per_step"],
                            "kernel_frac_of_tensor_peak": l2["roofline"]["frac"],
-                           "kernel_hbm_frac": l2["roofline"]["hbm_frac"]})
+                           "kernel_hbm_frac": l2["roofline"]["hbm_frac"],
+                           **({"cpb_us": l2["cpb_us"]} if "cpb_us" in l2 else {})})
         line["other_workloads"] = others
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = run_cpu_baseline(w, args.cpu_budget)

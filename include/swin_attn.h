@@ -93,6 +93,25 @@ typedef struct {
 swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* table_out,
                           swin_stream_t stream);
 
+/* Forms of G's input transform and output ("Swin Transformer V2" wiki card,
+ * "Paper vs code": the released code departs from eq. 3 / eq. 4). */
+typedef enum {
+  SWIN_CPB_PAPER = 0, /* eq. 4 on raw offsets: sign(d) ln(1 + |d|); B = G (as swin_cpb_eval) */
+  SWIN_CPB_CODE = 1   /* d' = 8 d / (Mp - 1), Mp the pretrained window (M if none);
+                         sign(d') log2(1 + |d'|) / log2(8); B = 16 sigmoid(G), in (0, 16) */
+} swin_cpb_form;
+
+/* swin_cpb_eval_form — swin_cpb_eval with a choice of form.  pretrained_M is
+ * the window G was trained at (0: M itself); a table for a larger test-time
+ * window M then extrapolates G beyond the trained coordinate range (§3.3:
+ * transfer across window sizes).  With Mp == 1 every coordinate is 0.
+ *   form          a swin_cpb_form
+ *   pretrained_M  0 or 1 <= pretrained_M <= 64 (SWIN_CPB_CODE only; must be 0
+ *                 for SWIN_CPB_PAPER, whose transform has no normaliser)
+ * Other arguments, layout and errors as swin_cpb_eval. */
+swin_status swin_cpb_eval_form(int M, int heads, const swin_cpb_weights* g, swin_cpb_form form,
+                               int pretrained_M, float* table_out, swin_stream_t stream);
+
 /* swin_window_attn_fwd — the shifted-window attention forward pass.
  *   q, k, v, out   device [B][H][W][heads][d]; q, k, v of dtype dt, out of
  *                  dtype out_dt (out_dt == dt, or SWIN_F32 output for SWIN_BF16

@@ -59,6 +59,10 @@ def _load():
         lib.oracle_log_coords.restype = None
         lib.oracle_cpb_table.argtypes = [ctypes.c_int] * 3 + [dp] * 5
         lib.oracle_cpb_table.restype = None
+        lib.oracle_log2_map.argtypes = [ctypes.c_double, ctypes.c_int]
+        lib.oracle_log2_map.restype = ctypes.c_double
+        lib.oracle_cpb_table_code.argtypes = [ctypes.c_int] * 4 + [dp] * 5
+        lib.oracle_cpb_table_code.restype = None
         lib.oracle_index_tables.argtypes = [ctypes.c_int] * 4 + [ip] * 4
         lib.oracle_index_tables.restype = None
         lib.oracle_window_attn.argtypes = (
@@ -116,6 +120,29 @@ def cpb_table(M: int, heads: int, w1, b1, w2, b2) -> np.ndarray:
     R = 2 * M - 1
     out = np.zeros((R * R, heads), dtype=np.float64)
     _load().oracle_cpb_table(M, heads, hidden, _dp(w1), _dp(b1), _dp(w2), _dp(b2), _dp(out))
+    return out
+
+
+def log2_map(delta: float, Mp: int) -> float:
+    """The released code's coordinate: sign(x) log2(1 + |x|) / log2(8) of
+    x = delta * 8 / (Mp - 1)."""
+    return float(_load().oracle_log2_map(float(delta), int(Mp)))
+
+
+def cpb_table_code(M: int, heads: int, w1, b1, w2, b2, pretrained_M: int = 0) -> np.ndarray:
+    """G in the released code's form (normalised log2 coordinates, output
+    16 sigmoid(G)) over every offset of an MxM window; pretrained_M = 0 means
+    M.  [(2M-1)^2, heads] float64."""
+    w1 = _f64(w1)
+    w2 = _f64(w2)
+    hidden = w1.shape[0]
+    assert w1.shape == (hidden, 2) and w2.shape == (heads, hidden)
+    b1 = _f64(b1)
+    b2 = _f64(b2)
+    R = 2 * M - 1
+    out = np.zeros((R * R, heads), dtype=np.float64)
+    _load().oracle_cpb_table_code(M, pretrained_M if pretrained_M > 0 else M, heads, hidden, _dp(w1), _dp(b1),
+                                  _dp(w2), _dp(b2), _dp(out))
     return out
 
 

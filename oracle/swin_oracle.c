@@ -20,6 +20,9 @@
  *        learnable 2D RoPE, no additive bias.
  *  [V2-pitfalls] Pitfalls, "Window divisibility": shift offsets with even or
  *        odd window sizes.
+ *  [V2-code] "Paper vs code": the released code's CPB coordinates (offset
+ *        scaled by 8 / (window - 1), sign(x) log2(1 + |x|) / log2(8)) and its
+ *        16 sigmoid bound on G's output.
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  R1  Shift mechanism (not spelled out; Swin V1 is cited only): along each
@@ -42,6 +45,9 @@
  *      inside each half rotate by p * omega[axis][t], t < d/4; the window-local
  *      coordinate is p = (y - s) mod M; RoPE touches q and k only; the score
  *      is scaled by 1/sqrt(d); no bias.
+ *  R11 The code form of G ([V2] "Paper vs code"): the normaliser is the
+ *      pretrained window Mp (the window itself when none is given); a window
+ *      of 1 (Mp - 1 = 0) has only offset 0, whose coordinate is 0.
  *
  * Parity pins live in tests/test_oracle_*.py.  The CPB meta-network beyond
  * its W2 = 0 special case and a float64 library Linear stack is arithmetic
@@ -103,6 +109,39 @@ void oracle_cpb_table(int M, int heads, int hidden,
     }
     free(hid);
     free(coords);
+}
+
+/* The released code's form of G ("Swin Transformer V2" wiki card, "Paper vs
+ * code"): each offset component is first scaled by 8 / (Mp - 1), Mp the
+ * window G was pretrained at (a window of 1 has only offset 0: coordinate 0),
+ * then mapped by sign(x) log2(1 + |x|) / log2(8); the MLP's output is bounded
+ * as 16 sigmoid(G). */
+double oracle_log2_map(double delta, int Mp) {
+    double x = Mp > 1 ? delta * 8.0 / (double)(Mp - 1) : 0.0;
+    double sgn = (x > 0.0) ? 1.0 : ((x < 0.0) ? -1.0 : 0.0);
+    return sgn * log2(1.0 + fabs(x)) / log2(8.0);
+}
+
+void oracle_cpb_table_code(int M, int Mp, int heads, int hidden,
+                           const double* w1, const double* b1,
+                           const double* w2, const double* b2, double* table) {
+    int R = 2 * M - 1;
+    double* hid = (double*)malloc(sizeof(double) * (size_t)hidden);
+    for (int dy = -(M - 1); dy <= M - 1; ++dy)
+        for (int dx = -(M - 1); dx <= M - 1; ++dx) {
+            size_t r = (size_t)(dy + M - 1) * R + (dx + M - 1);
+            double in0 = oracle_log2_map((double)dx, Mp), in1 = oracle_log2_map((double)dy, Mp);
+            for (int j = 0; j < hidden; ++j) {
+                double a = w1[j * 2 + 0] * in0 + w1[j * 2 + 1] * in1 + (b1 ? b1[j] : 0.0);
+                hid[j] = a > 0.0 ? a : 0.0;
+            }
+            for (int h = 0; h < heads; ++h) {
+                double z = b2 ? b2[h] : 0.0;
+                for (int j = 0; j < hidden; ++j) z += w2[(size_t)h * hidden + j] * hid[j];
+                table[r * heads + h] = 16.0 / (1.0 + exp(-z));
+            }
+        }
+    free(hid);
 }
 
 /* Swin-style bookkeeping tables, built by literally simulating the cyclic

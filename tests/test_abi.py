@@ -73,6 +73,16 @@ def test_rejects_bad_arguments(L, kw, why):
     assert why in L.swin_last_error().decode()
 
 
+def test_cpb_form_arguments_rejected_before_launch(L):
+    w = sa.swin_cpb_weights(8, FAKE, None, FAKE, None)
+    assert L.swin_cpb_eval_form(8, 3, ctypes.byref(w), 2, 0, FAKE, None) == sa.SWIN_ERR_INVALID_ARG
+    assert "form" in L.swin_last_error().decode()
+    assert L.swin_cpb_eval_form(8, 3, ctypes.byref(w), sa.SWIN_CPB_PAPER, 8, FAKE, None) == sa.SWIN_ERR_INVALID_ARG
+    assert "SWIN_CPB_CODE only" in L.swin_last_error().decode()
+    assert L.swin_cpb_eval_form(8, 3, ctypes.byref(w), sa.SWIN_CPB_CODE, 65, FAKE, None) == sa.SWIN_ERR_INVALID_ARG
+    assert "pretrained_M" in L.swin_last_error().decode()
+
+
 def test_cpu_entry_points_reject_before_launch(L):
     assert L.swin_index_tables(8, 8, 4, 4, None, None, None, None, None) == sa.SWIN_ERR_INVALID_ARG
     assert L.swin_cpb_eval(0, 3, None, FAKE, None) == sa.SWIN_ERR_INVALID_ARG

@@ -361,3 +361,73 @@ def test_rejects_bad_arguments():
         oracle.window_attn(q, q, q, 4, 4, 0)  # shift must be < M
     with pytest.raises(ValueError):
         oracle.window_attn(q, q, q, 4, 0, 1)  # cosine needs tau
+
+
+# ---- the released code's form of G ("Swin Transformer V2", "Paper vs code")
+
+def test_code_coordinates_endpoints_do_not_depend_on_the_window():
+    """Offsets are normalised by (window - 1) and scaled by 8 before the
+    log2 map, so the extreme offsets +-(M-1) land on +-log2(9)/log2(8) for
+    every window size (normalising by M, or a natural log, would not)."""
+    end = math.log2(9.0) / 3.0
+    for M in (2, 3, 7, 8, 12, 16, 24, 32):
+        assert oracle.log2_map(M - 1, M) == pytest.approx(end, abs=1e-15)
+        assert oracle.log2_map(-(M - 1), M) == pytest.approx(-end, abs=1e-15)
+        assert oracle.log2_map(0, M) == 0.0
+
+
+def test_code_coordinates_odd_and_increasing():
+    for M in (5, 16):
+        vals = [oracle.log2_map(d, M) for d in range(-(M - 1), M)]
+        assert all(b > a for a, b in zip(vals, vals[1:]))
+        for d in range(M):
+            assert oracle.log2_map(-d, M) == -oracle.log2_map(d, M)
+
+
+def test_code_window_of_one_has_coordinate_zero():
+    assert oracle.log2_map(0, 1) == 0.0
+    rng = np.random.default_rng(5)
+    w1, b1, w2, b2 = rng.normal(size=(6, 2)), rng.normal(size=6), rng.normal(size=(2, 6)), rng.normal(size=2)
+    t = oracle.cpb_table_code(1, 2, w1, b1, w2, b2)
+    z = w2 @ np.maximum(b1, 0.0) + b2
+    np.testing.assert_allclose(t[0], 16.0 / (1.0 + np.exp(-z)), rtol=1e-14)
+
+
+def test_code_table_bounded_and_half_scale_for_zero_output_layer():
+    rng = np.random.default_rng(6)
+    w1, b1 = rng.normal(size=(16, 2)), rng.normal(size=16)
+    t = oracle.cpb_table_code(8, 3, w1, b1, np.zeros((3, 16)), np.zeros(3))
+    assert np.all(t == 8.0)  # 16 sigmoid(0)
+    # outputs near +-8: strictly inside (0, 16) (far larger |G| rounds to the ends in double)
+    t = oracle.cpb_table_code(8, 2, w1, b1, 0.01 * rng.normal(size=(2, 16)), np.array([8.0, -8.0]))
+    assert np.all((t > 0.0) & (t < 16.0))
+    assert np.all(t[:, 0] > 15.9) and np.all(t[:, 1] < 0.1)
+
+
+def test_code_table_is_sigmoid_of_g_on_code_coordinates():
+    """One hidden unit reading dx only, identity output layer: the table is
+    16 sigmoid(relu(dx_hat)) row by row, with dx_hat the code coordinate."""
+    M = 6
+    t = oracle.cpb_table_code(M, 1, np.array([[1.0, 0.0]]), None, np.array([[1.0]]), None)
+    R = 2 * M - 1
+    for dy in range(-(M - 1), M):
+        for dx in range(-(M - 1), M):
+            x = max(oracle.log2_map(dx, M), 0.0)
+            assert t[(dy + M - 1) * R + dx + M - 1, 0] == pytest.approx(16.0 / (1.0 + math.exp(-x)), rel=1e-14)
+
+
+def test_code_table_transfer_to_a_larger_window_extends_the_pretrained_table():
+    """With the pretrained window Mp as normaliser, a table for a larger
+    test-time window agrees with the Mp table on every offset both have, and
+    pretrained_M = M is the same as giving none."""
+    rng = np.random.default_rng(7)
+    w1, b1, w2, b2 = rng.normal(size=(32, 2)), rng.normal(size=32), rng.normal(size=(2, 32)), rng.normal(size=2)
+    Mp, M = 8, 12
+    small = oracle.cpb_table_code(Mp, 2, w1, b1, w2, b2)
+    big = oracle.cpb_table_code(M, 2, w1, b1, w2, b2, pretrained_M=Mp)
+    Rs, Rb = 2 * Mp - 1, 2 * M - 1
+    for dy in range(-(Mp - 1), Mp):
+        for dx in range(-(Mp - 1), Mp):
+            np.testing.assert_array_equal(big[(dy + M - 1) * Rb + dx + M - 1], small[(dy + Mp - 1) * Rs + dx + Mp - 1])
+    np.testing.assert_array_equal(oracle.cpb_table_code(M, 2, w1, b1, w2, b2, pretrained_M=M),
+                                  oracle.cpb_table_code(M, 2, w1, b1, w2, b2))

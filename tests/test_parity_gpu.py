@@ -50,6 +50,34 @@ def test_cpb_eval(M, heads, hidden):
     assert rel_err(got, want) <= TOL_F32
 
 
+@pytest.mark.parametrize("M,pretrained_M,heads,hidden", [(8, 0, 2, 512), (16, 0, 3, 512), (24, 16, 16, 512),
+                                                       (12, 8, 4, 64), (1, 0, 1, 1), (5, 1, 2, 7)])
+def test_cpb_eval_code_form(M, pretrained_M, heads, hidden):
+    """The released code's form of G (normalised log2 coordinates, 16 sigmoid
+    output), also at a test-time window larger than the pretrained one."""
+    rng = np.random.default_rng(M * 100 + heads + 7)
+    w1 = rng.standard_normal((hidden, 2)).astype(np.float32)
+    b1 = rng.standard_normal(hidden).astype(np.float32)
+    w2 = (0.05 * rng.standard_normal((heads, hidden))).astype(np.float32)
+    b2 = rng.standard_normal(heads).astype(np.float32)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    got = sa.swin_cpb_eval_form(M, heads, dev(w1), dev(b1), dev(w2), dev(b2), sa.SWIN_CPB_CODE,
+                                pretrained_M).cpu().numpy()
+    want = oracle.cpb_table_code(M, heads, w1, b1, w2, b2, pretrained_M=pretrained_M)
+    assert rel_err(got, want) <= TOL_F32
+    assert np.all((got > 0.0) & (got < 16.0))
+
+
+def test_cpb_eval_form_paper_equals_cpb_eval():
+    rng = np.random.default_rng(3)
+    w1, b1 = rng.standard_normal((64, 2)).astype(np.float32), rng.standard_normal(64).astype(np.float32)
+    w2, b2 = rng.standard_normal((3, 64)).astype(np.float32), rng.standard_normal(3).astype(np.float32)
+    dev = lambda a: torch.from_numpy(a).cuda()
+    a = sa.swin_cpb_eval(9, 3, dev(w1), dev(b1), dev(w2), dev(b2))
+    b = sa.swin_cpb_eval_form(9, 3, dev(w1), dev(b1), dev(w2), dev(b2), sa.SWIN_CPB_PAPER)
+    assert torch.equal(a, b)
+
+
 # ---------------------------------------------------------------------------
 # fp32 workload (16x16, M=8, cosine + CPB), both shifts, full output
 # ---------------------------------------------------------------------------

@@ -62,6 +62,16 @@ int swin_version(void) { return 100; }
 
 swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* table_out,
                           swin_stream_t stream) {
+  return swin_cpb_eval_form(M, heads, g, SWIN_CPB_PAPER, 0, table_out, stream);
+}
+
+swin_status swin_cpb_eval_form(int M, int heads, const swin_cpb_weights* g, swin_cpb_form form,
+                               int pretrained_M, float* table_out, swin_stream_t stream) {
+  if (form != SWIN_CPB_PAPER && form != SWIN_CPB_CODE) return fail(SWIN_ERR_INVALID_ARG, "form=%d", (int)form);
+  if (pretrained_M < 0 || pretrained_M > 64)
+    return fail(SWIN_ERR_INVALID_ARG, "pretrained_M=%d outside [0, 64]", pretrained_M);
+  if (form == SWIN_CPB_PAPER && pretrained_M != 0)
+    return fail(SWIN_ERR_INVALID_ARG, "pretrained_M applies to SWIN_CPB_CODE only");
   if (M < 1 || M > 64) return fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
   if (heads < 1 || heads > 64) return fail(SWIN_ERR_INVALID_ARG, "heads=%d outside [1, 64]", heads);
   if (!g) return fail(SWIN_ERR_INVALID_ARG, "cpb weights struct is NULL");
@@ -69,7 +79,8 @@ swin_status swin_cpb_eval(int M, int heads, const swin_cpb_weights* g, float* ta
     return fail(SWIN_ERR_INVALID_ARG, "hidden=%d outside [1, 4096]", g->hidden);
   if (!g->w1 || !g->w2 || !table_out)
     return fail(SWIN_ERR_INVALID_ARG, "w1, w2 and table_out must be non-NULL");
-  return swin::launch_cpb_eval(M, heads, *g, table_out, reinterpret_cast<cudaStream_t>(stream));
+  return swin::launch_cpb_eval(M, heads, *g, table_out, reinterpret_cast<cudaStream_t>(stream), (int)form,
+                               pretrained_M);
 }
 
 size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int have_table) {

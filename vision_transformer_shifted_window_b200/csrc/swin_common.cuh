@@ -37,7 +37,7 @@ struct AttnArgs {
 
 // Launchers (one per translation unit).
 swin_status launch_cpb_eval(int M, int heads, const swin_cpb_weights& g, float* table,
-                            cudaStream_t stream);
+                            cudaStream_t stream, int form = SWIN_CPB_PAPER, int pretrained_M = 0);
 swin_status launch_index_tables(int H, int W, int M, int shift, int32_t* tw, int32_t* tr,
                                 int32_t* tl, int32_t* ri, cudaStream_t stream);
 swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream);

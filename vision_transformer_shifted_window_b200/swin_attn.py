@@ -28,9 +28,11 @@ SWIN_MODE_ROPE = 2
 
 SWIN_F32 = 0
 SWIN_BF16 = 1
+SWIN_CPB_PAPER = 0
+SWIN_CPB_CODE = 1
 
 #: every symbol include/swin_attn.h declares
-EXPORTED = ("swin_cpb_eval", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
+EXPORTED = ("swin_cpb_eval", "swin_cpb_eval_form", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
             "swin_window_attn_workspace_size",
             "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version",
             "swin_debug_set")
@@ -61,6 +63,8 @@ def lib():
         vp, i, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
         L.swin_cpb_eval.argtypes = [i, i, ctypes.POINTER(swin_cpb_weights), vp, st]
         L.swin_cpb_eval.restype = i
+        L.swin_cpb_eval_form.argtypes = [i, i, ctypes.POINTER(swin_cpb_weights), i, i, vp, st]
+        L.swin_cpb_eval_form.restype = i
         L.swin_window_attn_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp,
                                            ctypes.POINTER(swin_cpb_weights), vp, vp,
                                            ctypes.c_size_t, st]
@@ -146,6 +150,21 @@ def swin_cpb_eval(M: int, heads: int, w1, b1, w2, b2, out: Optional[torch.Tensor
         out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
     s, keep = _cpb_struct((w1, b1, w2, b2))
     _check(lib().swin_cpb_eval(M, heads, ctypes.byref(s), _ptr(out), _stream(stream)))
+    del keep
+    return out
+
+
+def swin_cpb_eval_form(M: int, heads: int, w1, b1, w2, b2, form: int, pretrained_M: int = 0,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """swin_cpb_eval with a choice of form (SWIN_CPB_PAPER or SWIN_CPB_CODE: the
+    released code's normalised log2 coordinates and 16 sigmoid bound); pretrained_M
+    is the window G was trained at (0: M)."""
+    R = 2 * M - 1
+    if out is None:
+        out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
+    s, keep = _cpb_struct((w1, b1, w2, b2))
+    _check(lib().swin_cpb_eval_form(M, heads, ctypes.byref(s), int(form), int(pretrained_M), _ptr(out),
+                                    _stream(stream)))
     del keep
     return out
 
