@@ -922,14 +922,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (2 * c + 1 >= nk) x[c].y = -INFINITY;
           }
         }
-        // block maximum: four independent 3-input max chains
+        // block maximum: four independent 3-input max chains, two pairs a step
+        static_assert(kBlk % 4 == 0, "pairs are taken two at a time");
         float mq[4] = {x[0].x, x[0].y, x[1].x, x[1].y};
 #pragma unroll
-        for (int c = 2; c < kBlk / 2; c += 4) {
-          mq[0] = ptx::max3(mq[0], x[c].x, x[c + 2].x);
-          mq[1] = ptx::max3(mq[1], x[c].y, x[c + 2].y);
-          mq[2] = ptx::max3(mq[2], x[c + 1].x, x[c + 3].x);
-          mq[3] = ptx::max3(mq[3], x[c + 1].y, x[c + 3].y);
+        for (int c = 2; c < kBlk / 2; c += 2) {
+          const int ch = 2 * ((c >> 1) & 1);
+          mq[ch] = ptx::max3(mq[ch], x[c].x, x[c + 1].x);
+          mq[ch + 1] = ptx::max3(mq[ch + 1], x[c].y, x[c + 1].y);
         }
         float mb = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
         if (MODE == 2) mb *= ascale;
