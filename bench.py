@@ -1,7 +1,7 @@
 #!/usr/bin/env python3
 """Benchmark of the shifted-window attention forward pass on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl native|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--others] [--impl native|reference]
 
 A step is one call of swin_window_attn_fwd (the whole hot path: CPB
 evaluation where the workload has one, then the attention kernel) over one
@@ -10,9 +10,16 @@ write) before every timed step; each step is timed with CUDA events on the
 library's stream.  For N > 1 (torchrun) every rank runs its own batch (weak
 scaling, no collective on the data path) and the time is the max over ranks.
 
-Prints one JSON line.  ``--impl reference`` times the CPU oracle (the
-project's plain double-precision statement of the method) on the host cores
-on a bounded sample of the same workload.
+Prints one JSON line: whole-job tokens/s, TFLOP/s, ``roofline`` (the
+attention kernel against the measured bf16 peak, DRAM traffic from the
+committed ncu summary of the same kernel source, and ``exp_bound``: the share
+of the all-MUFU exponential bound it reaches), ``e2e`` (host buffers, copies
+in the timed region), SM clocks sampled during the timed region, and
+``cpu_baseline`` (the oracle on the host cores).  ``--others`` adds the other
+bf16 workloads, with the CPB kernel's time in both forms where a workload has
+one.  ``--impl reference`` times the CPU oracle (the project's plain
+double-precision statement of the method) on the host cores on a bounded
+sample of the same workload.
 """
 from __future__ import annotations
 
