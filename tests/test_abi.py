@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from vision_transformer_shifted_window_b200 import build as swin_build
 from vision_transformer_shifted_window_b200 import swin_attn as sa
@@ -96,3 +97,33 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 4, 1, 32)
     with pytest.raises(ValueError):
         sa.swin_window_attn_fwd(x, x, x, 4, 0, 0)
+
+
+def _z(*shape):
+    return torch.zeros(*shape, dtype=torch.float32)
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(mode=1, tau=_z(3)), "tau"),
+    (dict(bias_table=_z(48, 2)), "bias_table"),
+    (dict(mode=2, rope_freqs=_z(2, 4)), "rope_freqs"),
+    (dict(mode=1, tau=_z(2), cpb=(_z(16, 2), None, _z(3, 16), None)), "cpb w2"),
+    (dict(mode=1, tau=_z(2), cpb=(_z(16, 2), _z(8), _z(2, 16), None)), "cpb b1"),
+])
+def test_binding_checks_parameter_shapes_before_the_call(kw, why):
+    """The C ABI sees bare pointers; the binding checks every parameter
+    tensor's shape against the sizes the call implies ((2M-1)^2 x heads
+    table, [heads] tau, [2, d/4] RoPE frequencies, G's weights)."""
+    q = _z(1, 8, 8, 2, 32)
+    args = dict(q=q, k=q, v=q, M=4, shift=2, mode=0)
+    args.update(kw)
+    with pytest.raises(ValueError, match=why):
+        sa.swin_window_attn_fwd(**args)
+
+
+def test_binding_checks_cpb_weight_shapes():
+    w1, w2 = _z(16, 2), _z(4, 16)
+    with pytest.raises(ValueError, match="cpb w2"):
+        sa.swin_cpb_eval(8, 3, w1, None, w2, None)
+    with pytest.raises(ValueError, match="cpb b2"):
+        sa.swin_cpb_eval_form(8, 4, w1, None, w2, _z(3), sa.SWIN_CPB_CODE)

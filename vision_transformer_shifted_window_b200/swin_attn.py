@@ -117,12 +117,31 @@ def _f32(t: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
     return t.contiguous()
 
 
-def _cpb_struct(cpb: Optional[Tuple[torch.Tensor, ...]]):
+def _shape(name: str, t: Optional[torch.Tensor], shape: Tuple[int, ...]) -> None:
+    """The C ABI takes bare pointers; sizes it cannot see are checked here."""
+    if t is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _cpb_struct(cpb: Optional[Tuple[torch.Tensor, ...]], heads: int):
     if cpb is None:
         return None, ()
     w1, b1, w2, b2 = (_f32(t) for t in cpb)
-    s = swin_cpb_weights(int(w1.shape[0]), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
+    if w1 is None or w2 is None or w1.dim() != 2:
+        raise ValueError("cpb needs w1 [hidden, 2] and w2 [heads, hidden]")
+    hidden = int(w1.shape[0])
+    _shape("cpb w1", w1, (hidden, 2))
+    _shape("cpb b1", b1, (hidden,))
+    _shape("cpb w2", w2, (heads, hidden))
+    _shape("cpb b2", b2, (heads,))
+    s = swin_cpb_weights(hidden, _ptr(w1), _ptr(b1), _ptr(w2), _ptr(b2))
     return s, (w1, b1, w2, b2)
+
+
+def _param_shapes(M: int, heads: int, d: int, tau, bias_table, rope_freqs) -> None:
+    _shape("tau", tau, (heads,))
+    _shape("bias_table", bias_table, ((2 * M - 1) ** 2, heads))
+    _shape("rope_freqs", rope_freqs, (2, d // 4))
 
 
 def swin_debug_set(flags: int, wait_limit_cycles: int = 0) -> None:
@@ -148,7 +167,7 @@ def swin_cpb_eval(M: int, heads: int, w1, b1, w2, b2, out: Optional[torch.Tensor
     R = 2 * M - 1
     if out is None:
         out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
-    s, keep = _cpb_struct((w1, b1, w2, b2))
+    s, keep = _cpb_struct((w1, b1, w2, b2), heads)
     _check(lib().swin_cpb_eval(M, heads, ctypes.byref(s), _ptr(out), _stream(stream)))
     del keep
     return out
@@ -162,7 +181,7 @@ def swin_cpb_eval_form(M: int, heads: int, w1, b1, w2, b2, form: int, pretrained
     R = 2 * M - 1
     if out is None:
         out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
-    s, keep = _cpb_struct((w1, b1, w2, b2))
+    s, keep = _cpb_struct((w1, b1, w2, b2), heads)
     _check(lib().swin_cpb_eval_form(M, heads, ctypes.byref(s), int(form), int(pretrained_M), _ptr(out),
                                     _stream(stream)))
     del keep
@@ -198,7 +217,8 @@ def swin_window_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: i
     if odt is None:
         raise ValueError("out must be float32 or bfloat16")
     tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
-    cs, keep = _cpb_struct(cpb)
+    _param_shapes(M, heads, d, tau, bias_table, rope_freqs)
+    cs, keep = _cpb_struct(cpb, heads)
     need = swin_window_attn_workspace_size(M, heads, mode, bias_table is not None) if cs else 0
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -232,7 +252,8 @@ def swin_window_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     if odt is None or out.shape != q.shape:
         raise ValueError("out must be float32 or bfloat16 with q's shape")
     tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
-    cs, keep = _cpb_struct(cpb)
+    _param_shapes(M, heads, d, tau, bias_table, rope_freqs)
+    cs, keep = _cpb_struct(cpb, heads)
     rc = lib().swin_window_attn_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
         _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
