@@ -39,6 +39,8 @@
  * that runs out records SWIN_ERR_TIMEOUT in a device status word, which
  * swin_stream_status reads (after synchronising the stream) and clears.
  * swin_last_error returns a message for the last failure on this host thread.
+ * The library caches device addresses of its own variables per device, so it
+ * must not be used across a cudaDeviceReset.
  */
 #ifndef SWIN_ATTN_H
 #define SWIN_ATTN_H
@@ -167,7 +169,8 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
  * held on every GPU that loads the library until exit) instead of caller
  * scratch; (2M-1)^2 * heads above 131072 returns SWIN_ERR_UNSUPPORTED.  The
  * first call on a device looks the array's address up (cudaGetSymbolAddress)
- * and should come before any stream capture.  All calls share the array, and
+ * and should come before any stream capture.  Argument errors return before
+ * anything is enqueued, leaving the array untouched.  All calls share the array, and
  * calls whose kernels overlap on the GPU race on it: serialise them.  Every
  * table entry is rewritten on each call; the array keeps the last call's
  * table.  Allocates nothing. */

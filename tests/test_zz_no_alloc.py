@@ -2,11 +2,15 @@
 
 swin_window_attn_fwd_noalloc keeps the cosine mode's CPB bias table in a fixed
 device array of the library instead of a caller workspace.  Called through the
-C ABI (ctypes, no Python wrapper), it must give the regular entry point's
-output, within the bf16/fp32 tolerances used everywhere else, on two calls in
-a row (the second call reuses the array the first one filled).  This file
-sorts last so that a run stopping at its first failure has run everything
-else already; it also passes when run alone in a fresh process.
+C ABI (ctypes, no Python wrapper), it runs the same kernels on the same inputs
+as the regular entry point, so its output must equal that entry point's bit for
+bit, on two calls in a row (the second call reuses the array the first one
+filled); the first call is also compared with the oracle at the tolerances
+used everywhere else.  A call with a bad argument must return its error before
+enqueueing anything (checked by capturing the stream: the captured graph must
+be empty).  This file sorts last so that a run stopping at its first failure
+has run everything else already; it also passes when run alone in a fresh
+process.
 """
 import ctypes
 
@@ -14,11 +18,28 @@ import numpy as np
 import pytest
 import torch
 
-from swin_testutil import TOL_BF16, TOL_F32, rel_err
+from swin_testutil import TOL_BF16, TOL_F32, oracle_run, rel_err
 from vision_transformer_shifted_window_b200 import swin_attn as sa
 from vision_transformer_shifted_window_b200 import synthetic as syn
 
 pytestmark = pytest.mark.gpu
+
+SHAPE = (2, 40, 36, 3, 32)  # B, H, W, heads, d
+M, SHIFT = 16, 8
+
+
+def _workload(dtype):
+    B, H, W, heads, d = SHAPE
+    return syn.Workload(95, "noalloc", "bf16" if dtype == torch.bfloat16 else "f32", B, H, W, heads, d, M,
+                        (SHIFT,), sa.SWIN_MODE_COSINE_CPB, tau=(0.05, 0.2), cpb_hidden=512)
+
+
+def _call_noalloc(L, q, k, v, out, dt, tau_ptr, g, stream, shift=SHIFT):
+    B, H, W, heads, d = SHAPE
+    return L.swin_window_attn_fwd_noalloc(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dt, sa.SWIN_F32, B, H, W, heads, d, M, shift,
+        sa.SWIN_MODE_COSINE_CPB, tau_ptr, None, ctypes.byref(g) if g is not None else None, None,
+        ctypes.c_void_p(stream.cuda_stream))
 
 
 @pytest.mark.parametrize("dtype,tol", [(torch.bfloat16, TOL_BF16), (torch.float32, TOL_F32)])
@@ -28,28 +49,75 @@ def test_noalloc_matches_workspace_entry_point(dtype, tol):
     L = sa.lib()
     outs = []
     for call, seed in enumerate((11, 12)):
-        w = syn.Workload(95, "noalloc", "bf16" if dtype == torch.bfloat16 else "f32", 2, 40, 36, 3, 32, 16,
-                         (8,), sa.SWIN_MODE_COSINE_CPB, tau=(0.05, 0.2), cpb_hidden=512)
+        w = _workload(dtype)
         inp = syn.make_inputs(w, seed=seed)
         dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
         q, k, v = (dev(inp[n]).to(dtype) for n in ("q", "k", "v"))
         tau = dev(inp["tau"])
         cpb = tuple(dev(inp[n]) for n in ("w1", "b1", "w2", "b2"))
-        ref = sa.swin_window_attn_fwd(q, k, v, 16, 8, sa.SWIN_MODE_COSINE_CPB, tau=tau, cpb=cpb,
+        ref = sa.swin_window_attn_fwd(q, k, v, M, SHIFT, sa.SWIN_MODE_COSINE_CPB, tau=tau, cpb=cpb,
                                       out_dtype=torch.float32)
         out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
         g = sa.swin_cpb_weights(512, cpb[0].data_ptr(), cpb[1].data_ptr(), cpb[2].data_ptr(), cpb[3].data_ptr())
         dt = sa.SWIN_BF16 if dtype == torch.bfloat16 else sa.SWIN_F32
-        rc = L.swin_window_attn_fwd_noalloc(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dt, sa.SWIN_F32, 2, 40, 36, 3, 32, 16, 8,
-            sa.SWIN_MODE_COSINE_CPB, tau.data_ptr(), None, ctypes.byref(g), None,
-            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        rc = _call_noalloc(L, q, k, v, out, dt, tau.data_ptr(), g, torch.cuda.current_stream())
         assert rc == sa.SWIN_OK, L.swin_last_error().decode()
         assert sa.swin_stream_status() == sa.SWIN_OK
-        err = rel_err(out.cpu().numpy(), ref.cpu().numpy())
-        assert err <= tol, (call, err)
+        # same kernels, same inputs: the same bits as the workspace entry point
+        assert torch.equal(out, ref), (call, rel_err(out.cpu().numpy(), ref.cpu().numpy()))
+        if call == 0:
+            want = oracle_run(inp, w, SHIFT)
+            assert rel_err(out.cpu().numpy(), want) <= tol
         outs.append(out)
     assert not torch.equal(outs[0], outs[1])  # the second call really recomputed
+
+
+def _captured_nodes(stream, fn):
+    """Run fn() while `stream` is being captured; return the captured node count."""
+    from cuda.bindings import runtime as cudart
+    h = stream.cuda_stream
+    (err,) = cudart.cudaStreamBeginCapture(h, cudart.cudaStreamCaptureMode.cudaStreamCaptureModeRelaxed)
+    assert err == cudart.cudaError_t.cudaSuccess
+    try:
+        rc = fn()
+    finally:
+        err, graph = cudart.cudaStreamEndCapture(h)
+    assert err == cudart.cudaError_t.cudaSuccess
+    err, _, n = cudart.cudaGraphGetNodes(graph, 0)
+    assert err == cudart.cudaError_t.cudaSuccess
+    cudart.cudaGraphDestroy(graph)
+    return rc, n
+
+
+def test_noalloc_argument_errors_enqueue_nothing():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L = sa.lib()
+    w = _workload(torch.bfloat16)
+    inp = syn.make_inputs(w, seed=13)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    q, k, v = (dev(inp[n]).to(torch.bfloat16) for n in ("q", "k", "v"))
+    tau = dev(inp["tau"])
+    cpb = tuple(dev(inp[n]) for n in ("w1", "b1", "w2", "b2"))
+    g = sa.swin_cpb_weights(512, cpb[0].data_ptr(), cpb[1].data_ptr(), cpb[2].data_ptr(), cpb[3].data_ptr())
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+    # one valid call first: the per-device set-up happens outside any capture
+    assert _call_noalloc(L, q, k, v, out, sa.SWIN_BF16, tau.data_ptr(), g, stream) == sa.SWIN_OK
+    torch.cuda.synchronize()
+    # a valid call under capture records work (the CPB and attention kernels) ...
+    rc, n = _captured_nodes(stream, lambda: _call_noalloc(L, q, k, v, out, sa.SWIN_BF16, tau.data_ptr(), g,
+                                                          stream))
+    assert rc == sa.SWIN_OK and n >= 2
+    # ... a rejected one records none
+    for bad in (dict(shift=M), dict(tau_ptr=None)):
+        kw = dict(tau_ptr=tau.data_ptr(), shift=SHIFT)
+        kw.update(bad)
+        rc, n = _captured_nodes(stream, lambda: _call_noalloc(L, q, k, v, out, sa.SWIN_BF16, kw["tau_ptr"], g,
+                                                              stream, shift=kw["shift"]))
+        assert rc == sa.SWIN_ERR_INVALID_ARG, bad
+        assert n == 0, (bad, n)
+    assert sa.swin_stream_status(stream) == sa.SWIN_OK
 
 
 def test_noalloc_rejects_oversized_table():

@@ -12,7 +12,9 @@ namespace swin {
 namespace {
 thread_local std::string g_last_error;
 
-// One status word per device; kernels OR error codes into it, never trap.
+// One status word per device; kernels OR error codes into it, never trap.  Its
+// address is cached per device ordinal for the life of the process: the
+// library must not be used across a cudaDeviceReset.
 __device__ int g_status_word;
 
 constexpr int kMaxDevices = 64;
@@ -53,6 +55,45 @@ static bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
   return a0 < b0 + bn && b0 < a0 + an;
 }
+
+namespace swin {
+
+swin_status check_fwd_args(const void* q, const void* k, const void* v, const void* out, swin_dtype dt,
+                           swin_dtype out_dt, int B, int H, int W, int heads, int d, int M, int shift,
+                           swin_mode mode, const float* tau, const float* bias_table,
+                           const swin_cpb_weights* cpb, const float* rope_freqs) {
+  if (!q || !k || !v || !out) return fail(SWIN_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
+  if (dt != SWIN_F32 && dt != SWIN_BF16) return fail(SWIN_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (out_dt != dt && !(dt == SWIN_BF16 && out_dt == SWIN_F32))
+    return fail(SWIN_ERR_INVALID_ARG, "output dtype %d not allowed for input dtype %d", (int)out_dt, (int)dt);
+  if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1)
+    return fail(SWIN_ERR_INVALID_ARG, "B, H, W, heads and d must be >= 1");
+  if (M < 1 || M > 64) return fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
+  if (shift < 0 || shift >= M) return fail(SWIN_ERR_INVALID_ARG, "shift=%d outside [0, M)", shift);
+  if (mode != SWIN_MODE_DOT_BIAS && mode != SWIN_MODE_COSINE_CPB && mode != SWIN_MODE_ROPE)
+    return fail(SWIN_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
+  const long long elems = (long long)B * H * W * heads * d;
+  if (elems >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "B*H*W*heads*d must be < 2^31");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(SWIN_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
+  const size_t bytes = (size_t)elems * (dt == SWIN_F32 ? 4 : 2);
+  const size_t obytes = (size_t)elems * (out_dt == SWIN_F32 ? 4 : 2);
+  if (overlaps(out, obytes, q, bytes) || overlaps(out, obytes, k, bytes) || overlaps(out, obytes, v, bytes))
+    return fail(SWIN_ERR_INVALID_ARG, "out overlaps q, k or v");
+  if (mode == SWIN_MODE_COSINE_CPB && !tau) return fail(SWIN_ERR_INVALID_ARG, "cosine mode needs tau");
+  if (mode == SWIN_MODE_ROPE) {
+    if (!rope_freqs) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode needs rope_freqs");
+    if (d % 4 != 0) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode needs d %% 4 == 0, got %d", d);
+    if (bias_table) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode takes no bias table");
+  }
+  if (cpb && (cpb->hidden < 1 || cpb->hidden > 4096 || !cpb->w1 || !cpb->w2))
+    return fail(SWIN_ERR_INVALID_ARG, "cpb weights incomplete or hidden outside [1, 4096]");
+  if (heads > 64 && mode == SWIN_MODE_COSINE_CPB && !bias_table && cpb)
+    return fail(SWIN_ERR_INVALID_ARG, "cpb evaluation supports heads <= 64");
+  return SWIN_OK;
+}
+
+}  // namespace swin
 
 extern "C" {
 
@@ -97,34 +138,9 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
                                  const float* rope_freqs, void* workspace,
                                  size_t workspace_bytes, swin_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (!q || !k || !v || !out) return fail(SWIN_ERR_INVALID_ARG, "q, k, v and out must be non-NULL");
-  if (dt != SWIN_F32 && dt != SWIN_BF16) return fail(SWIN_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
-  if (out_dt != dt && !(dt == SWIN_BF16 && out_dt == SWIN_F32))
-    return fail(SWIN_ERR_INVALID_ARG, "output dtype %d not allowed for input dtype %d", (int)out_dt, (int)dt);
-  if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1)
-    return fail(SWIN_ERR_INVALID_ARG, "B, H, W, heads and d must be >= 1");
-  if (M < 1 || M > 64) return fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
-  if (shift < 0 || shift >= M) return fail(SWIN_ERR_INVALID_ARG, "shift=%d outside [0, M)", shift);
-  if (mode != SWIN_MODE_DOT_BIAS && mode != SWIN_MODE_COSINE_CPB && mode != SWIN_MODE_ROPE)
-    return fail(SWIN_ERR_INVALID_ARG, "unknown mode %d", (int)mode);
-  const long long elems = (long long)B * H * W * heads * d;
-  if (elems >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "B*H*W*heads*d must be < 2^31");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return fail(SWIN_ERR_INVALID_ARG, "q, k, v and out must be 16-byte aligned");
-  const size_t bytes = (size_t)elems * (dt == SWIN_F32 ? 4 : 2);
-  const size_t obytes = (size_t)elems * (out_dt == SWIN_F32 ? 4 : 2);
-  if (overlaps(out, obytes, q, bytes) || overlaps(out, obytes, k, bytes) || overlaps(out, obytes, v, bytes))
-    return fail(SWIN_ERR_INVALID_ARG, "out overlaps q, k or v");
-  if (mode == SWIN_MODE_COSINE_CPB && !tau) return fail(SWIN_ERR_INVALID_ARG, "cosine mode needs tau");
-  if (mode == SWIN_MODE_ROPE) {
-    if (!rope_freqs) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode needs rope_freqs");
-    if (d % 4 != 0) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode needs d %% 4 == 0, got %d", d);
-    if (bias_table) return fail(SWIN_ERR_INVALID_ARG, "RoPE mode takes no bias table");
-  }
-  if (cpb && (cpb->hidden < 1 || cpb->hidden > 4096 || !cpb->w1 || !cpb->w2))
-    return fail(SWIN_ERR_INVALID_ARG, "cpb weights incomplete or hidden outside [1, 4096]");
-  if (heads > 64 && mode == SWIN_MODE_COSINE_CPB && !bias_table && cpb)
-    return fail(SWIN_ERR_INVALID_ARG, "cpb evaluation supports heads <= 64");
+  swin_status vs = swin::check_fwd_args(q, k, v, out, dt, out_dt, B, H, W, heads, d, M, shift, mode, tau,
+                                        bias_table, cpb, rope_freqs);
+  if (vs != SWIN_OK) return vs;
 
   const float* table = bias_table;
   if (mode == SWIN_MODE_COSINE_CPB && !bias_table && cpb) {
@@ -180,7 +196,7 @@ swin_status swin_stream_status(swin_stream_t stream) {
     return fail(SWIN_ERR_CUDA, "reading the device status word failed");
   if (val & SWIN_ERR_TIMEOUT) return fail(SWIN_ERR_TIMEOUT, "a kernel's bounded wait ran out");
   if (val & SWIN_ERR_UNSUPPORTED)
-    return fail(SWIN_ERR_UNSUPPORTED, "a V entry of magnitude >= 2^22 was saturated on the tensor-core path");
+    return fail(SWIN_ERR_UNSUPPORTED, "an operand left the fp16 range on the tensor-core path (a RoPE-rotated k or a V entry of magnitude >= 65504)");
   if (val != 0) return fail(SWIN_ERR_CUDA, "unknown device status %d", val);
   return SWIN_OK;
 }

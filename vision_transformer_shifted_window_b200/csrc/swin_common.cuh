@@ -18,6 +18,13 @@ swin_status fail(swin_status st, const char* fmt, ...);
 // Device address of this device's status word (set up once per device).
 int* status_word();
 
+// Every argument check of swin_window_attn_fwd that does not depend on the
+// workspace; SWIN_OK or the failure (message recorded), nothing launched.
+swin_status check_fwd_args(const void* q, const void* k, const void* v, const void* out, swin_dtype dt,
+                           swin_dtype out_dt, int B, int H, int W, int heads, int d, int M, int shift,
+                           swin_mode mode, const float* tau, const float* bias_table,
+                           const swin_cpb_weights* cpb, const float* rope_freqs);
+
 // fp32 RoPE tables are built in the kernels from the caller's frequencies.
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kTauMin = 0.01f;

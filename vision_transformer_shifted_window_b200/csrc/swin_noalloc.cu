@@ -19,8 +19,11 @@
 // Host code may not use the array's name as a device address (it is a host
 // stand-in).  The first call on each device looks the address up with
 // cudaGetSymbolAddress while that device is current; make that first call
-// before any stream capture.  No cudaMalloc, cudaFree or allocating library
-// routine is called here.
+// before any stream capture.  The address is cached per device ordinal for the
+// life of the process, so the library must not be used across a
+// cudaDeviceReset (which unloads the module and invalidates it).  No
+// cudaMalloc, cudaFree or allocating library routine is called here, and an
+// argument error returns before anything is enqueued.
 #include <mutex>
 
 #include "swin_common.cuh"
@@ -63,15 +66,15 @@ extern "C" swin_status swin_window_attn_fwd_noalloc(
     int H, int W, int heads, int d, int M, int shift, swin_mode mode, const float* tau,
     const float* bias_table, const swin_cpb_weights* cpb, const float* rope_freqs,
     swin_stream_t stream) {
+  // every argument check first, so that a rejected call launches nothing and
+  // leaves the shared table as it was
+  swin_status st = swin::check_fwd_args(q, k, v, out, dt, out_dt, B, H, W, heads, d, M, shift, mode, tau,
+                                        bias_table, cpb, rope_freqs);
+  if (st != SWIN_OK) return st;
   const bool needs_table = mode == SWIN_MODE_COSINE_CPB && !bias_table && cpb;
   if (!needs_table)
     return swin_window_attn_fwd(q, k, v, out, dt, out_dt, B, H, W, heads, d, M, shift, mode, tau,
                                 bias_table, cpb, rope_freqs, nullptr, 0, stream);
-  if (M < 1 || M > 64) return swin::fail(SWIN_ERR_INVALID_ARG, "M=%d outside [1, 64]", M);
-  if (heads < 1 || heads > 64)
-    return swin::fail(SWIN_ERR_INVALID_ARG, "heads=%d outside [1, 64]", heads);
-  if (cpb->hidden < 1 || cpb->hidden > 4096 || !cpb->w1 || !cpb->w2)
-    return swin::fail(SWIN_ERR_INVALID_ARG, "cpb weights incomplete or hidden outside [1, 4096]");
   const size_t need = (size_t)(2 * M - 1) * (2 * M - 1) * heads;
   if (need > swin::kNoallocTableFloats)
     return swin::fail(SWIN_ERR_UNSUPPORTED,
@@ -79,7 +82,7 @@ extern "C" swin_status swin_window_attn_fwd_noalloc(
                       "%zu floats; use swin_window_attn_fwd with a workspace",
                       need, swin::kNoallocTableFloats);
   float* table = nullptr;
-  swin_status st = swin::noalloc_table(&table);
+  st = swin::noalloc_table(&table);
   if (st != SWIN_OK) return st;
   st = swin::launch_cpb_eval(M, heads, *cpb, table, reinterpret_cast<cudaStream_t>(stream));
   if (st != SWIN_OK) return st;

@@ -7,6 +7,7 @@ shared library is missing or a call fails, a RuntimeError is raised.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional, Tuple
@@ -109,6 +110,13 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _on(stream):
+    """Allocate temporaries and copies on the stream the kernels run on, so the
+    caching allocator never hands their memory to other work while those
+    kernels may still read it."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _f32(t: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
     if t is None:
         return None
@@ -165,11 +173,12 @@ def swin_cpb_eval(M: int, heads: int, w1, b1, w2, b2, out: Optional[torch.Tensor
                   stream=None) -> torch.Tensor:
     """Evaluate the Log-CPB MLP for every offset -> fp32 [(2M-1)^2, heads]."""
     R = 2 * M - 1
-    if out is None:
-        out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
-    s, keep = _cpb_struct((w1, b1, w2, b2), heads)
-    _check(lib().swin_cpb_eval(M, heads, ctypes.byref(s), _ptr(out), _stream(stream)))
-    del keep
+    with _on(stream):
+        if out is None:
+            out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
+        s, keep = _cpb_struct((w1, b1, w2, b2), heads)
+        _check(lib().swin_cpb_eval(M, heads, ctypes.byref(s), _ptr(out), _stream(stream)))
+        del keep
     return out
 
 
@@ -179,12 +188,13 @@ def swin_cpb_eval_form(M: int, heads: int, w1, b1, w2, b2, form: int, pretrained
     released code's normalised log2 coordinates and 16 sigmoid bound); pretrained_M
     is the window G was trained at (0: M)."""
     R = 2 * M - 1
-    if out is None:
-        out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
-    s, keep = _cpb_struct((w1, b1, w2, b2), heads)
-    _check(lib().swin_cpb_eval_form(M, heads, ctypes.byref(s), int(form), int(pretrained_M), _ptr(out),
-                                    _stream(stream)))
-    del keep
+    with _on(stream):
+        if out is None:
+            out = torch.empty((R * R, heads), dtype=torch.float32, device=w1.device)
+        s, keep = _cpb_struct((w1, b1, w2, b2), heads)
+        _check(lib().swin_cpb_eval_form(M, heads, ctypes.byref(s), int(form), int(pretrained_M), _ptr(out),
+                                        _stream(stream)))
+        del keep
     return out
 
 
@@ -209,6 +219,13 @@ def swin_window_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: i
     if q.dim() != 5:
         raise ValueError("q, k, v must be [B, H, W, heads, d]")
     B, H, W, heads, d = q.shape
+    with _on(stream):
+        return _fwd_on_stream(q, k, v, M, shift, mode, dt, B, H, W, heads, d, tau, bias_table, cpb, rope_freqs,
+                              out, workspace, stream, out_dtype)
+
+
+def _fwd_on_stream(q, k, v, M, shift, mode, dt, B, H, W, heads, d, tau, bias_table, cpb, rope_freqs, out,
+                   workspace, stream, out_dtype):
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if out.shape != q.shape:
@@ -246,20 +263,21 @@ def swin_window_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
     if dt is None or k.dtype != q.dtype or v.dtype != q.dtype or k.shape != q.shape or v.shape != q.shape:
         raise ValueError("q, k, v must share a float32/bfloat16 dtype and shape")
     B, H, W, heads, d = q.shape
-    if out is None:
-        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
-    odt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(out.dtype)
-    if odt is None or out.shape != q.shape:
-        raise ValueError("out must be float32 or bfloat16 with q's shape")
-    tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
-    _param_shapes(M, heads, d, tau, bias_table, rope_freqs)
-    cs, keep = _cpb_struct(cpb, heads)
-    rc = lib().swin_window_attn_fwd_noalloc(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
-        _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
-        _ptr(rope_freqs), _stream(stream))
-    _check(rc)
-    del keep
+    with _on(stream):
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+        odt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(out.dtype)
+        if odt is None or out.shape != q.shape:
+            raise ValueError("out must be float32 or bfloat16 with q's shape")
+        tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
+        _param_shapes(M, heads, d, tau, bias_table, rope_freqs)
+        cs, keep = _cpb_struct(cpb, heads)
+        rc = lib().swin_window_attn_fwd_noalloc(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
+            _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
+            _ptr(rope_freqs), _stream(stream))
+        _check(rc)
+        del keep
     return out
 
 
