@@ -1,57 +1,63 @@
-// Shifted-window attention on the CUDA cores, in fp32 arithmetic.
+// Shifted-window attention on the CUDA cores, for fp32 tensors (and for bf16
+// tensors the tensor-core path does not cover: d != 32, or a bias table with
+// M > 32).  Inputs and outputs keep their dtype; the arithmetic inside is
+// double precision — normalisation or rotation of q and k, logits, the
+// exponentials and the running sums — so that the fp32 result stays within
+// 1e-5 of the exact one (max error over the output's RMS) even for the
+// sharpest softmax the pages' settings give (tau = 0.05, i.e. logits scaled by
+// 20): in fp32, the logit roundings and the running-sum roundings each came to
+// a few 1e-6 on a 16 x 16 window.
 //
-// This is the path for fp32 tensors (and for bf16 tensors with d != 32),
-// where the tensor cores' bf16/tf32 inputs would not meet fp32 accuracy.
-// Scores follow "Swin Transformer V2" eq. 1 (mode 0) and eq. 2 (mode 1,
-// tau clamped at 0.01, §3.2), or FlashSwin's window-local 2-D RoPE
-// (mode 2); the softmax is the exact online form FlashSwin relies on: a
-// running maximum and rescaled running sums, so no score row is stored.
+// Scores follow "Swin Transformer V2" eq. 1 (mode 0) and eq. 2 (mode 1, tau
+// clamped at 0.01, §3.2), or FlashSwin's window-local 2-D RoPE (mode 2); the
+// softmax is the exact online form FlashSwin relies on: a running maximum and
+// rescaled running sums, so no score row is stored.
 //
 // Decomposition: one CTA of 128 threads per (image, head, rectangle, block of
 // 128 queries); a rectangle is one segment per axis of the shifted partition
 // (see swin_index.cuh), i.e. one independent attention problem of up to M*M
 // tokens.  Each thread owns one query row; keys and values stream through
-// shared memory 32 at a time (normalised or rotated once per key), and
-// every thread reads them as broadcasts.
+// shared memory 16 at a time (normalised or rotated once per key), and every
+// thread reads them as broadcasts.
 #include "swin_common.cuh"
 
 namespace swin {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kKeyTile = 32;
+constexpr int kKeyTile = 16;
 constexpr int kMaxM = 64;
 
 template <typename T>
-__device__ __forceinline__ float load_elem(const T* p);
+__device__ __forceinline__ double load_elem(const T* p);
 template <>
-__device__ __forceinline__ float load_elem<float>(const float* p) {
-  return __ldg(p);
+__device__ __forceinline__ double load_elem<float>(const float* p) {
+  return (double)__ldg(p);
 }
 template <>
-__device__ __forceinline__ float load_elem<__nv_bfloat16>(const __nv_bfloat16* p) {
-  return __bfloat162float(*p);
+__device__ __forceinline__ double load_elem<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return (double)__bfloat162float(*p);
 }
 template <typename T>
-__device__ __forceinline__ T store_conv(float x);
+__device__ __forceinline__ T store_conv(double x);
 template <>
-__device__ __forceinline__ float store_conv<float>(float x) {
-  return x;
+__device__ __forceinline__ float store_conv<float>(double x) {
+  return (float)x;
 }
 template <>
-__device__ __forceinline__ __nv_bfloat16 store_conv<__nv_bfloat16>(float x) {
-  return __float2bfloat16_rn(x);
+__device__ __forceinline__ __nv_bfloat16 store_conv<__nv_bfloat16>(double x) {
+  // round once, from the fp32 result: a bf16 output is the fp32 output rounded
+  return __float2bfloat16_rn((float)x);
 }
 
 // Rotate channel pairs of one half (row or column axis) by position p.
 template <int D>
-__device__ __forceinline__ void rope_rotate(float* x, int half, int p, const float* cs,
-                                            const float* sn) {
+__device__ __forceinline__ void rope_rotate(double* x, int half, int p, const double* cs, const double* sn) {
   constexpr int Q = D / 4;
 #pragma unroll
   for (int t = 0; t < Q; ++t) {
-    float c = cs[p * Q + t], s = sn[p * Q + t];
-    float a = x[half * (D / 2) + 2 * t], b = x[half * (D / 2) + 2 * t + 1];
+    const double c = cs[p * Q + t], s = sn[p * Q + t];
+    const double a = x[half * (D / 2) + 2 * t], b = x[half * (D / 2) + 2 * t + 1];
     x[half * (D / 2) + 2 * t] = a * c - b * s;
     x[half * (D / 2) + 2 * t + 1] = a * s + b * c;
   }
@@ -59,11 +65,11 @@ __device__ __forceinline__ void rope_rotate(float* x, int half, int p, const flo
 
 template <typename T, typename TO, int D, int MODE>
 __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx, int chunks) {
-  __shared__ float ks[kKeyTile][D];
-  __shared__ float vs[kKeyTile][D];
+  __shared__ double ks[kKeyTile][D];
+  __shared__ float vs[kKeyTile][D];  // V entries are fp32 or bf16 values: exact in fp32
   // RoPE tables: [axis][p][t] for p < M, t < D/4
-  __shared__ float rcos[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
-  __shared__ float rsin[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
+  __shared__ double rcos[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
+  __shared__ double rsin[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
 
   const int M = a.M, s = a.shift;
   const int rect = blockIdx.x / chunks, chunk = blockIdx.x % chunks;
@@ -82,9 +88,9 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
   if (MODE == 2) {
     constexpr int Qd = D / 4;
     for (int i = threadIdx.x; i < 2 * M * Qd; i += kThreads) {
-      int axis = i / (M * Qd), p = (i / Qd) % M, t = i % Qd;
-      float sv, cv;
-      sincosf((float)p * a.rope[axis * Qd + t], &sv, &cv);
+      const int axis = i / (M * Qd), p = (i / Qd) % M, t = i % Qd;
+      double sv, cv;
+      sincos((double)p * (double)a.rope[axis * Qd + t], &sv, &cv);
       rcos[axis * kMaxM * Qd + p * Qd + t] = cv;
       rsin[axis * kMaxM * Qd + p * Qd + t] = sv;
     }
@@ -94,51 +100,49 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
   const int qi = chunk * kThreads + threadIdx.x;
   const bool active = qi < n;
   const int yq = y0 + (active ? qi / lx : 0), xq = x0 + (active ? qi % lx : 0);
-  float q[D], o[D];
-  float inv_tau = 0.0f;
+  double q[D], o[D];
   {
     const T* src = Q + (((size_t)b * a.H + yq) * a.W + xq) * C + (size_t)h * D;
 #pragma unroll
-    for (int e = 0; e < D; ++e) q[e] = active ? load_elem(src + e) : 0.0f;
+    for (int e = 0; e < D; ++e) q[e] = active ? load_elem(src + e) : 0.0;
   }
+  // logit = (q . k) * scale (+ bias): mode 1 scale = 1 / (|q| max(tau, 0.01)),
+  // k unit-normalised; modes 0 and 2 scale = 1 / sqrt(d)
+  double scale = 1.0 / sqrt((double)D);
   if (MODE == 1) {
-    float ss = 0.0f;
+    double ss = 0.0;
 #pragma unroll
-    for (int e = 0; e < D; ++e) ss = fmaf(q[e], q[e], ss);
-    float nrm = fmaxf(sqrtf(ss), kNormEps);
-#pragma unroll
-    for (int e = 0; e < D; ++e) q[e] = q[e] / nrm;
-    inv_tau = 1.0f / fmaxf(__ldg(a.tau + h), kTauMin);
+    for (int e = 0; e < D; ++e) ss = fma(q[e], q[e], ss);
+    scale = 1.0 / (fmax(sqrt(ss), (double)kNormEps) * fmax((double)__ldg(a.tau + h), (double)kTauMin));
   }
   if (MODE == 2) {
     rope_rotate<D>(q, 0, swin_local_coord(yq, M, s), rcos, rsin);
     rope_rotate<D>(q, 1, swin_local_coord(xq, M, s), rcos + kMaxM * (D / 4), rsin + kMaxM * (D / 4));
   }
-  const float rsd = rsqrtf((float)D);
 #pragma unroll
-  for (int e = 0; e < D; ++e) o[e] = 0.0f;
-  float m = -INFINITY, l = 0.0f;
+  for (int e = 0; e < D; ++e) o[e] = 0.0;
+  double m = -INFINITY, l = 0.0;
 
   for (int j0 = 0; j0 < n; j0 += kKeyTile) {
     const int nk = min(kKeyTile, n - j0);
     __syncthreads();
     for (int i = threadIdx.x; i < nk * D; i += kThreads) {
-      int j = i / D, e = i % D, kk = j0 + j;
-      size_t off = (((size_t)b * a.H + y0 + kk / lx) * a.W + x0 + kk % lx) * C + (size_t)h * D + e;
+      const int j = i / D, e = i % D, kk = j0 + j;
+      const size_t off = (((size_t)b * a.H + y0 + kk / lx) * a.W + x0 + kk % lx) * C + (size_t)h * D + e;
       ks[j][e] = load_elem(K + off);
-      vs[j][e] = load_elem(V + off);
+      vs[j][e] = (float)load_elem(V + off);
     }
     __syncthreads();
     if (MODE != 0 && threadIdx.x < nk) {
-      float* kr = ks[threadIdx.x];
+      double* kr = ks[threadIdx.x];
       if (MODE == 1) {
-        float ss = 0.0f;
-        for (int e = 0; e < D; ++e) ss = fmaf(kr[e], kr[e], ss);
-        float nrm = fmaxf(sqrtf(ss), kNormEps);
-        for (int e = 0; e < D; ++e) kr[e] = kr[e] / nrm;
+        double ss = 0.0;
+        for (int e = 0; e < D; ++e) ss = fma(kr[e], kr[e], ss);
+        const double inv = 1.0 / fmax(sqrt(ss), (double)kNormEps);
+        for (int e = 0; e < D; ++e) kr[e] *= inv;
       } else {
-        int kk = j0 + threadIdx.x;
-        float tmp[D];
+        const int kk = j0 + threadIdx.x;
+        double tmp[D];
         for (int e = 0; e < D; ++e) tmp[e] = kr[e];
         rope_rotate<D>(tmp, 0, swin_local_coord(y0 + kk / lx, M, s), rcos, rsin);
         rope_rotate<D>(tmp, 1, swin_local_coord(x0 + kk % lx, M, s), rcos + kMaxM * (D / 4),
@@ -149,35 +153,31 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
     __syncthreads();
     if (!active) continue;
     for (int j = 0; j < nk; ++j) {
-      float dot = 0.0f;
+      double dot = 0.0;
 #pragma unroll
-      for (int e = 0; e < D; ++e) dot = fmaf(q[e], ks[j][e], dot);
-      float lg;
-      if (MODE == 1)
-        lg = dot * inv_tau;
-      else
-        lg = dot * rsd;
+      for (int e = 0; e < D; ++e) dot = fma(q[e], ks[j][e], dot);
+      double lg = dot * scale;
       if (MODE != 2 && a.table) {
-        int kk = j0 + j;
-        int r = swin_rel_row(yq - (y0 + kk / lx), xq - (x0 + kk % lx), M);
-        lg += __ldg(a.table + (size_t)r * a.heads + h);
+        const int kk = j0 + j;
+        const int r = swin_rel_row(yq - (y0 + kk / lx), xq - (x0 + kk % lx), M);
+        lg += (double)__ldg(a.table + (size_t)r * a.heads + h);
       }
       if (lg > m) {
-        float c = expf(m - lg);
-        l = fmaf(l, c, 1.0f);
+        const double c = exp(m - lg);
+        l = fma(l, c, 1.0);
 #pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = fmaf(o[e], c, vs[j][e]);
+        for (int e = 0; e < D; ++e) o[e] = fma(o[e], c, (double)vs[j][e]);
         m = lg;
       } else {
-        float p = expf(lg - m);
+        const double p = exp(lg - m);
         l += p;
 #pragma unroll
-        for (int e = 0; e < D; ++e) o[e] = fmaf(p, vs[j][e], o[e]);
+        for (int e = 0; e < D; ++e) o[e] = fma(p, (double)vs[j][e], o[e]);
       }
     }
   }
   if (active) {
-    float inv = 1.0f / l;
+    const double inv = 1.0 / l;
     TO* dst = O + (((size_t)b * a.H + yq) * a.W + xq) * C + (size_t)h * D;
 #pragma unroll
     for (int e = 0; e < D; ++e) dst[e] = store_conv<TO>(o[e] * inv);
