@@ -1,23 +1,27 @@
 #!/usr/bin/env python3
 """Benchmark of the shifted-window attention forward pass on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--others] [--impl native|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--only] [--impl native|reference]
 
 A step is one call of swin_window_attn_fwd (the whole hot path: CPB
 evaluation where the workload has one, then the attention kernel) over one
 batch of the workload, inputs resident in HBM.  L2 is flushed (a 256 MB
 write) before every timed step; each step is timed with CUDA events on the
-library's stream.  For N > 1 (torchrun) every rank runs its own batch (weak
-scaling, no collective on the data path) and the time is the max over ranks.
+library's stream and the median step is reported.  For N > 1 (torchrun)
+every rank runs its own batch (weak scaling, no collective on the data path)
+and the time is the max over ranks.
 
-Prints one JSON line: whole-job tokens/s, TFLOP/s, ``roofline`` (the
-attention kernel against the measured bf16 peak, DRAM traffic from the
-committed ncu summary of the same kernel source, and ``exp_bound``: the share
-of the all-MUFU exponential bound it reaches), ``e2e`` (host buffers, copies
-in the timed region), SM clocks sampled during the timed region, and
-``cpu_baseline`` (the oracle on the host cores).  ``--others`` adds the other
-bf16 workloads, with the CPB kernel's time in both forms where a workload has
-one.  ``--impl reference`` times the CPU oracle (the project's plain
+Prints one JSON line.  The headline workload (FlashSwin-T dense tokens, M=32,
+unless --workload) gives ``value`` (whole-job tokens/s), ``tflops``,
+``roofline`` (the attention kernel against the measured bf16 peak, DRAM
+traffic from the committed ncu summary of the same kernel source, and
+``exp_bound``: the share of the all-MUFU exponential bound it reaches) and
+``e2e`` (host buffers, copies in the timed region).  ``workloads`` repeats
+those figures for every bf16 workload (headline first; --only skips the
+others), with the CPB kernel's time in both forms where a workload has one.
+Also: SM clocks sampled during the timed loops, the number of this library's
+kernel launches timed, and ``cpu_baseline`` (the oracle on the host cores and
+on one core).  ``--impl reference`` times the CPU oracle (the project's plain
 double-precision statement of the method) on the host cores on a bounded
 sample of the same workload.
 """
@@ -211,143 +215,200 @@ def whole_job(wk: dict, world: int, ms_max: float) -> dict:
             "tflops_exact": wk["flops_exact"] * world / sec / 1e12}
 
 
-def run_native(args, rank: int, world: int, local_rank: int):
-    import torch
-    import torch.distributed as dist
-    from vision_transformer_shifted_window_b200 import swin_attn as sa
-    from vision_transformer_shifted_window_b200 import build as swin_build
+def config_of(w: syn.Workload, world: int) -> dict:
+    """The workload as both arms name it (same keys and values)."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d, "M": w.M,
+            "shift": w.shifts[0], "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode],
+            "global_batch": w.B * world, "parallelism": "replicas x%d" % world,
+            "l2": "flushed before every timed step (256 MB write)", "timing": "median of per-step CUDA events"}
 
-    swin_build.build()
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    w = syn.WORKLOADS[args.workload]
+
+def _median(xs):
+    return float(np.median(np.asarray(xs, dtype=np.float64)))
+
+
+class Timer:
+    """Per-step CUDA-event timing on the library's stream, with an L2 flush
+    (a write larger than L2) before every timed step."""
+
+    def __init__(self, device, stream):
+        import torch
+        self.torch, self.device, self.stream = torch, device, stream
+        self.flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def loop(self, fn, n, flush_l2=True):
+        torch = self.torch
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        with torch.cuda.stream(self.stream):
+            for i in range(n):
+                if flush_l2:
+                    self.flush.fill_(i & 0xFF)
+                evs[i][0].record(self.stream)
+                fn()
+                evs[i][1].record(self.stream)
+        torch.cuda.synchronize(self.device)
+        return [a.elapsed_time(b) for a, b in evs]
+
+
+def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: dict, sms: int, clock_mhz: float,
+                  with_e2e: bool):
+    """One workload: the whole call (CPB + attention) per step, the attention
+    kernel alone, and, for the headline, the end-to-end call through host
+    buffers.  Returns (entry, launches of this library's kernels timed)."""
+    import torch
+    from vision_transformer_shifted_window_b200 import swin_attn as sa
+    device, stream = timer.device, timer.stream
     s = w.shifts[0]
     q, k, v, kw = make_device_inputs(w, device, rank)
     out = torch.empty_like(q)
     ws_bytes = sa.swin_window_attn_workspace_size(w.M, w.heads, w.mode, "bias_table" in kw)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=device)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    stream = torch.cuda.Stream(device)
     launches_per_step = 2 if "cpb" in kw else 1
 
     def step():
         sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, workspace=ws, stream=stream, **kw)
 
-    def timed_loop(fn, n, flush_l2=True):
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-        with torch.cuda.stream(stream):
-            for i in range(n):
-                if flush_l2:
-                    flush.fill_(i & 0xFF)
-                evs[i][0].record(stream)
-                fn()
-                evs[i][1].record(stream)
-        torch.cuda.synchronize(device)
-        return [a.elapsed_time(b) for a, b in evs]
-
-    # warm-up (untimed)
-    timed_loop(step, max(args.warmup, 3))
-    assert sa.swin_stream_status(stream) == 0
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
-    sampler.start()
+    timer.loop(step, max(args.warmup, 3))
+    if sa.swin_stream_status(stream) != 0:
+        raise RuntimeError("device status after warm-up of %s" % w.name)
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize(device)
-    times = timed_loop(step, args.steps)
-    torch.cuda.synchronize(device)
-    if world > 1:
-        dist.barrier()
-    # keep the GPU busy a little longer for the clock record when the timed loop was short
-    t_soak = time.time()
-    while sum(times) < 1500.0 and time.time() - t_soak < 2.0:
-        timed_loop(step, 20)
-    clocks = sampler.stop()
-    st = sa.swin_stream_status(stream)
-    if st != 0:
-        raise RuntimeError("device status %d after timed loop" % st)
-
-    ms = max_over_ranks(sum(times) / len(times), world, device)
+    times = timer.loop(step, args.steps)
+    launches = launches_per_step * args.steps
+    ms = max_over_ranks(_median(times), world, device)
     wk = work(w)
-    tokens = wk["tokens"] * world
     job = whole_job(wk, world, ms)
-    value, tflops = job["tokens_per_s"], job["tflops"]
-    peaks = read_peaks()
 
-    # dominant kernel alone: the attention kernel with the bias table given
+    # the attention kernel alone (the bias table given, no CPB evaluation)
+    cpb_us = None
     if "cpb" in kw:
-        table = sa.swin_cpb_eval(w.M, w.heads, *kw["cpb"])
+        table = sa.swin_cpb_eval(w.M, w.heads, *kw["cpb"], stream=stream)
         kw_k = {kk: vv for kk, vv in kw.items() if kk != "cpb"}
         kw_k["bias_table"] = table
 
         def kstep():
             sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, stream=stream, **kw_k)
-        timed_loop(kstep, 5)
-        ktimes = timed_loop(kstep, max(10, min(args.steps, 200)))
-        # the CPB meta network alone, in both forms (eq. 3 / eq. 4 and the released code's)
+        timer.loop(kstep, 3)
+        ktimes = timer.loop(kstep, args.steps)
+        launches += args.steps
         cpb_us = {}
         for name, form in (("paper", sa.SWIN_CPB_PAPER), ("code", sa.SWIN_CPB_CODE)):
             def cstep(form=form):
                 sa.swin_cpb_eval_form(w.M, w.heads, *kw["cpb"], form, 0, out=table, stream=stream)
-            timed_loop(cstep, 5, flush_l2=False)
-            ct = timed_loop(cstep, 50, flush_l2=False)
-            cpb_us[name] = round(1e3 * sorted(ct)[len(ct) // 2], 2)
+            timer.loop(cstep, 3, flush_l2=False)
+            ct = timer.loop(cstep, 20, flush_l2=False)
+            launches += 20
+            cpb_us[name] = round(1e3 * _median(ct), 2)
     else:
         ktimes = times
-        cpb_us = None
-    k_ms = max_over_ranks(sum(ktimes) / len(ktimes), world, device)
+    k_ms = max_over_ranks(_median(ktimes), world, device)
     achieved = wk["flops_std"] / (k_ms * 1e-3) / 1e12
+    hbm = wk["bytes"] / (k_ms * 1e-3) / 1e9
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
                 "traffic": read_traffic("attn_tc", w), "peak_source": peaks["source"] + " (burst)",
-                "kernel_ms": round(k_ms, 5),
-                "hbm_achieved_gbs": round(wk["bytes"] / (k_ms * 1e-3) / 1e9, 1),
-                "hbm_frac": round(wk["bytes"] / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "kernel_ms": round(k_ms, 5), "algorithmic_bytes": wk["bytes"],
+                "hbm_achieved_gbs": round(hbm, 1), "hbm_frac": round(hbm / peaks["hbm_gbs"], 4),
                 "attainable_frac": round(achieved / min(peaks["bf16_tflops"],
                                                         peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3), 4),
-                "exp_bound": exp_bound(wk, torch.cuda.get_device_properties(device).multi_processor_count,
-                                       float(clocks["sm_mhz"] or clocks["sm_max_mhz"] or 1965.0), k_ms)}
+                "exp_bound": exp_bound(wk, sms, clock_mhz, k_ms)}
+    entry = {"workload": w.name, "config": {"B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d, "M": w.M,
+                                            "shift": s, "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode]},
+             "ms_per_step": round(ms, 5), "tokens_per_s": round(job["tokens_per_s"], 1),
+             "tflops": round(job["tflops"], 2), "tflops_exact_pairs": round(job["tflops_exact"], 2),
+             "roofline": roofline}
+    if cpb_us:
+        entry["cpb_us"] = cpb_us
+    if with_e2e:
+        # end to end through host buffers: H2D of q/k/v, the call, D2H of out
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
 
-    # end to end through host buffers: H2D of q/k/v, the call, D2H of out
-    hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
-    hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            hout.copy_(out, non_blocking=True)
+        timer.loop(e2e_step, 3, flush_l2=False)
+        n_e2e = max(3, min(args.steps, 20))
+        etimes = timer.loop(e2e_step, n_e2e, flush_l2=False)
+        launches += launches_per_step * n_e2e
+        e_ms = max_over_ranks(_median(etimes), world, device)
+        entry["e2e"] = {"value": round(wk["tokens"] * world / (e_ms * 1e-3), 1), "unit": "tokens/s",
+                        "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                        "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": round(e_ms, 4)}
+    if sa.swin_stream_status(stream) != 0:
+        raise RuntimeError("device status after the timed loops of %s" % w.name)
+    del q, k, v, out, ws
+    torch.cuda.empty_cache()
+    return entry, launches
 
-    def e2e_step():
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        step()
-        hout.copy_(out, non_blocking=True)
-    timed_loop(e2e_step, 3, flush_l2=False)
-    n_e2e = max(3, min(args.steps, 20))
-    etimes = timed_loop(e2e_step, n_e2e, flush_l2=False)
-    e_ms = max_over_ranks(sum(etimes) / len(etimes), world, device)
-    h2d = 3 * q.numel() * q.element_size()
-    d2h = out.numel() * out.element_size()
 
+def run_native(args, rank: int, world: int, local_rank: int):
+    import torch
+    from vision_transformer_shifted_window_b200 import build as swin_build
+
+    swin_build.build()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.Stream(device)
+    timer = Timer(device, stream)
+    peaks = read_peaks()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    headline = syn.WORKLOADS[args.workload]
+    others = [] if args.only else [i for i in sorted(syn.WORKLOADS)
+                                   if i != args.workload and syn.WORKLOADS[i].dtype == "bf16"]
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    sampler.start()
+    # clocks are sampled over the timed loops; the exponential bound uses the
+    # SM clock the box advertises (the sampled median is reported beside it)
+    clock_guess = 1965.0
+    entry, launches = time_workload(headline, args, timer, rank, world, peaks, sms, clock_guess, with_e2e=True)
+    other_entries = []
+    for idx in others:
+        e, n = time_workload(syn.WORKLOADS[idx], args, timer, rank, world, peaks, sms, clock_guess, False)
+        other_entries.append(e)
+        launches += n
+    clocks = sampler.stop()
+    sm_mhz = float(clocks["sm_mhz"] or clocks["sm_max_mhz"] or clock_guess)
+    wk = work(headline)
+    for e, w in [(entry, headline)] + [(o, syn.WORKLOADS[i]) for o, i in zip(other_entries, others)]:
+        e["roofline"]["exp_bound"] = exp_bound(work(w), sms, sm_mhz, e["roofline"]["kernel_ms"])
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "metric": METRIC, "value": entry["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": entry["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d,
-                   "M": w.M, "shift": s, "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode],
-                   "global_batch": w.B * world, "parallelism": "replicas x%d" % world,
-                   "l2": "flushed before every timed step (256 MB write)"},
-        "tflops": round(tflops, 2), "tflops_exact_pairs": round(job["tflops_exact"], 2),
-        "roofline": roofline,
-        **({"cpb_us": cpb_us} if cpb_us else {}),
-        "e2e": {"value": round(tokens / (e_ms * 1e-3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 4)},
-        "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+        "dtype": "bf16" if headline.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": config_of(headline, world),
+        "tflops": entry["tflops"], "tflops_exact_pairs": entry["tflops_exact_pairs"],
+        "roofline": entry["roofline"],
+        "e2e": entry["e2e"],
+        "clocks": clocks, "gpu_launches": launches,
+        "workloads": [{k: v for k, v in entry.items() if k != "e2e"}] + other_entries,
     }
-    return line, w
+    return line, headline
+
+
+def cpu_model() -> str:
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.lower().startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
 
 
 def run_cpu_baseline(w: syn.Workload, budget_s: float):
-    """Time the oracle on a bounded, seeded sample of the workload's queries."""
+    """Time the oracle on a bounded, seeded sample of the workload's queries
+    (drawn without replacement from every image of the batch), on all host
+    cores and on one core."""
     import oracle
-    inp = syn.make_inputs(w, B=1)
+    inp = syn.make_inputs(w)
     s = w.shifts[0]
     table = None
     if "table" in inp:
@@ -355,36 +416,42 @@ def run_cpu_baseline(w: syn.Workload, budget_s: float):
     elif "w1" in inp:
         table = oracle.cpb_table(w.M, w.heads, inp["w1"], inp["b1"], inp["w2"], inp["b2"])
     rng = np.random.default_rng(99)
+    n_all = w.B * w.H * w.W
 
-    def run(nq):
-        ids = rng.integers(0, w.H * w.W, nq)
+    def run(nq, nthreads=0):
+        ids = np.sort(rng.choice(n_all, size=min(nq, n_all), replace=False))
         t0 = time.perf_counter()
         oracle.window_attn(inp["q"], inp["k"], inp["v"], w.M, s, w.mode, tau=inp.get("tau"), table=table,
-                           rope_freqs=inp.get("rope_freqs"), queries=ids)
-        return time.perf_counter() - t0
+                           rope_freqs=inp.get("rope_freqs"), queries=ids, nthreads=nthreads)
+        return len(ids), time.perf_counter() - t0
 
-    nq = 64
-    t = run(nq)
-    while t < 0.5 and nq < w.H * w.W:
-        nq *= 4
-        t = run(nq)
-    nq = int(min(w.H * w.W * w.B, max(nq, nq * budget_s / max(t, 1e-6))))
-    t = run(nq)
-    return {"value": round(nq / t, 2), "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d query tokens drawn with replacement from one %dx%d image (all %d heads), %.1f s" % (nq, w.H, w.W, w.heads, t),
+    def sized(budget, nthreads):
+        nq, t = run(64, nthreads)
+        while t < 0.3 and nq < n_all:
+            nq, t = run(nq * 4, nthreads)
+        return run(int(min(n_all, max(nq, nq * budget / max(t, 1e-6)))), nthreads)
+
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    nq, t = sized(budget_s, cores)
+    nq1, t1 = sized(max(1.0, budget_s / 4), 1)
+    return {"value": round(nq / t, 2), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "single_core_tokens_per_s": round(nq1 / t1, 2),
+            "sample": "%d query tokens drawn without replacement from all %d images of %s (all %d heads), %.1f s "
+                      "on %d threads; %d tokens on 1 thread, %.1f s" % (nq, w.B, w.name, w.heads, t,
+                                                                       cores, nq1, t1),
             "seconds": round(t, 2)}
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(syn.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=("native", "reference"))
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work to time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--others", action="store_true", help="also time the other bf16 workloads")
+    ap.add_argument("--only", action="store_true", help="time the headline workload alone")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -400,8 +467,7 @@ def main():
         line = {"metric": METRIC, "impl": "reference", "value": cb["value"], "unit": "tokens/s", "n_gpus": 1,
                 "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d,
-                           "M": w.M, "shift": w.shifts[0]},
+                "config": config_of(w, world),
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -416,21 +482,6 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     line, w = run_native(args, rank, world, local_rank)
-    if args.others and rank == 0:
-        others = []
-        for idx in sorted(syn.WORKLOADS):
-            if idx == args.workload or syn.WORKLOADS[idx].dtype != "bf16":
-                continue
-            a2 = argparse.Namespace(**vars(args))
-            a2.workload = idx
-            a2.steps = min(args.steps, 100)
-            l2, _ = run_native(a2, 0, 1, local_rank)
-            others.append({"workload": l2["config"]["workload"], "tokens_per_s": l2["value"],
-                           "tflops": l2["tflops"], "ms_per_step": l2["ms_per_step"],
-                           "kernel_frac_of_tensor_peak": l2["roofline"]["frac"],
-                           "kernel_hbm_frac": l2["roofline"]["hbm_frac"],
-                           **({"cpb_us": l2["cpb_us"]} if "cpb_us" in l2 else {})})
-        line["other_workloads"] = others
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = run_cpu_baseline(w, args.cpu_budget)
     if world > 1:
