@@ -218,29 +218,60 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
             yield from issue_pv(k)
 
     def softmax_warp(g, wq):
-        b = qcnt = base = pv_done = 0
+        """One softmax warp, in the kernel's order: S(b + 1) is copied out
+        (prefetched) at the top of block b, P(b - 1)'s p_full arrival is
+        deferred to the top of block b, and O is touched at the end of a block."""
+        steps = []  # (tile id, unit row, tile index k, block j, ring position)
+        base = 0
+        for t, n, u in ps:
+            nb, k0 = int(u[11]), int(u[12])
+            for i in range(n):
+                if wg_of(t + i) == g:
+                    steps += [(t + i, u, k0 + i, j, base + j) for j in range(nb)]
+            base += nb
+        nblk = len(steps)
+        pv_done = 0
         pend, pend_tile = False, None
         last_tile = None
+        active = False
+        p_pending = False
 
         def wait_pv(upto):
             nonlocal pv_done
             while pv_done <= upto:
                 yield W(("p_free", g, pv_done & 1), pv_done >> 1)
                 pv_done += 1
-        for t, n, u in ps:
-            nb, k0 = int(u[11]), int(u[12])
-            for i in range(n):
-                if wg_of(t + i) != g:
-                    continue
-                tid = t + i
-                rows, nq, loff = tile_geom(u, k0 + i, g)
+
+        def read_s(b):
+            check(Sb[(g, b & 1)]["b"] == b, "softmax read S(%d) but the buffer holds S(%s)" % (b, Sb[(g, b & 1)]["b"]))
+            Sb[(g, b & 1)]["reads"] += 1
+
+        def release_p(b):  # P(b) written by this warp (store landed), then p_full(b)
+            Pb[(g, b & 1)]["writers"] = Pb[(g, b & 1)]["writers"] + 1 if Pb[(g, b & 1)].get("for") == b else 1
+            Pb[(g, b & 1)]["for"] = b
+            bars[("p_full", g, b & 1)].arrive()
+
+        qcnt = 0
+        if nblk:
+            yield W(("s_full", g, 0), 0)
+            read_s(0)
+            bars[("s_free", g, 0)].arrive()
+        for b, (tid, u, k, j, pos) in enumerate(steps):
+            nb = int(u[11])
+            slot, rnd = pos % nst, pos // nst
+            has_next = b + 1 < nblk
+            if has_next:
+                yield W(("s_full", g, (b + 1) & 1), (b + 1) >> 1)
+                read_s(b + 1)  # the copy is issued here and lands before s_free(b + 1)
+            if p_pending:
+                release_p(b - 1)
+                p_pending = False
+            if j == 0:
+                rows, nq, loff = tile_geom(u, k, g)
                 active = wq * 32 + 31 >= loff and wq * 32 < loff + nq
                 prev_tile[(g, tid)] = last_tile
                 last_tile = tid
-                if active:
-                    o_epi.setdefault((g, tid), [0, 0])[0] += 1
-                else:
-                    o_epi.setdefault((g, tid), [0, 0])
+                o_epi.setdefault((g, tid), [0, 0])[0] += 1 if active else 0
                 qslot, qrnd = qcnt % nqb, qcnt // nqb
                 if mode != 0:
                     yield W(("q_ready", g, qslot), qrnd)
@@ -250,41 +281,31 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
                 sm_reads[tid] = sm_reads.get(tid, 0) + 1
                 bars[("q_empty", g, qslot)].arrive()
                 qcnt += 1
-                for j in range(nb):
-                    pos = base + j
-                    slot, rnd = pos % nst, pos // nst
-                    yield W(("s_full", g, b & 1), b >> 1)
-                    if active:
-                        check(Sb[(g, b & 1)]["b"] == b, "softmax read S(%d) but the buffer holds S(%s)" %
-                              (b, Sb[(g, b & 1)]["b"]))
-                    Sb[(g, b & 1)]["reads"] += 1
-                    bars[("s_free", g, b & 1)].arrive()
-                    if active and mode == 1:
-                        yield W(("kv_ready", slot), rnd)
-                        check(kv[slot]["pos"] == pos and kv[slot]["prepped"], "1/|k| of a stale stage")
-                    epi = j == 0 and pend
-                    resc = j > 0 and active and rng.random() < rescale_p
-                    if epi or resc:
-                        yield from wait_pv(b - 1)
-                        check(pv_exec[g] == b, "O read with %d PVs executed at block %d" % (pv_exec[g], b))
-                        if epi:
-                            o_epi[(g, pend_tile)][1] += 1
-                    if b >= 2 and bug != "p_without_pv_wait":
-                        yield from wait_pv(b - 2)
-                    if active:
-                        check(pv_exec[g] >= b - 1, "P(%d) written before PV(%d) executed" % (b, b - 2))
-                    Pb[(g, b & 1)]["b"] = b
-                    Pb[(g, b & 1)]["writers"] = Pb[(g, b & 1)]["writers"] + 1 if Pb[(g, b & 1)].get("for") == b else 1
-                    Pb[(g, b & 1)]["for"] = b
-                    bars[("p_full", g, b & 1)].arrive()
-                    if epi:
-                        pend = False
-                    b += 1
+            if active and mode == 1:
+                yield W(("kv_ready", slot), rnd)
+                check(kv[slot]["pos"] == pos and kv[slot]["prepped"], "1/|k| of a stale stage")
+            if b >= 2 and bug != "p_without_pv_wait":
+                yield from wait_pv(b - 2)
+            if active:
+                check(pv_exec[g] >= b - 1, "P(%d) written before PV(%d) executed" % (b, b - 2))
+            p_pending = True
+            epi = j == 0 and pend
+            resc = j > 0 and active and rng.random() < rescale_p
+            if epi or resc:
+                yield from wait_pv(b - 1)
+                check(pv_exec[g] == b, "O read with %d PVs executed at block %d" % (pv_exec[g], b))
+                if epi:
+                    o_epi[(g, pend_tile)][1] += 1
+                    pend = False
+            if has_next:
+                bars[("s_free", g, (b + 1) & 1)].arrive()
+            if j == nb - 1:
                 pend, pend_tile = active, tid
-            base += nb
+        if p_pending:
+            release_p(nblk - 1)
         if pend:
-            yield from wait_pv(b - 1)
-            check(pv_exec[g] == b, "final O read early")
+            yield from wait_pv(nblk - 1)
+            check(pv_exec[g] == nblk, "final O read early")
             o_epi[(g, pend_tile)][1] += 1
 
     def execute(entry):

@@ -32,18 +32,18 @@
 //   warps 1, 2   tcgen05.mma issuers, one thread each: warp 1 + g issues the
 //                MMAs of softmax warpgroup g; warp 1 owns TMEM
 //   warps 12-13  Q prep: 1/(tau |q|) per row (mode 1), RoPE of q (mode 2)
-//   warps 14-15  K prep: 1/|k| per key (mode 1), RoPE of k (mode 2)
+//   warps 14-15  K prep: 1/|k| per key (mode 1), RoPE of k (mode 2), V to fp16
 //   warps 4-7    softmax of warpgroup 0 (one TMEM lane = one query row)
 //   warps 8-11   softmax of warpgroup 1
 //
 // TMEM per softmax warpgroup g (128 lanes, columns from 256 g): score buffers
-// S0, S1 (64 fp32 columns each), probability buffers P0, P1 (64 bf16 keys =
+// S0, S1 (64 fp32 columns each), probability buffers P0, P1 (64 fp16 keys =
 // 32 columns each) and O (48 columns: 32 outputs and, in column 32, the row
 // sum of P).  Block b's S = Q K^T lands in S[b % 2]; the softmax copies it to
 // registers and frees the buffer at once, so the issuer computes S(b + 2)
 // while the softmax works on block b.  P(b) goes to P[b % 2], and
 // O += P(b) [V | c] reads it there (c = the constant column 1: the same MMAs
-// accumulate the row sum of exactly the bf16 probabilities that weight V).
+// accumulate the row sum of exactly the fp16 probabilities that weight V).
 // The softmax waits for the tensor core only where a buffer comes back two
 // blocks later (PV(b - 2) done before P(b) is written), where it rescales O,
 // and where it reads a finished O.  Each issuer runs its warpgroup's blocks in
@@ -56,17 +56,19 @@
 // the tile follow the barrier protocol but skip the arithmetic.
 //
 // Softmax: online, with the running maximum kept until a block exceeds it by
-// more than 8 (log2 units), so O is rescaled rarely; P in bf16 (values up to
-// 2^8).  Exponentials of the first keys of each block go through a
-// polynomial on the FMA pipe and the rest through the MUFU, in a ratio set by
+// more than 8 (log2 units), so O is rescaled rarely; P in fp16 (values up to
+// 2^8): fp16 keeps 3 more mantissa bits than bf16, which the output needs
+// (rounding P to bf16 gave about 9 times the output error of fp16).
+// Exponentials of the first keys of each block go through a polynomial on
+// the FMA pipe and the rest through the MUFU, in a ratio set by
 // the measured pipe rates (MUFU 16 exp2 per clock per SM, FMA pipe 128 lanes).
 //
 // Precision of the score operands: modes 0 and 1 multiply the bf16 inputs as
 // they are (mode 1 applies 1/|q|, 1/|k| and 1/tau in fp32 afterwards, so the
 // cosine is not rounded); mode 2 rotates q and k in fp32 and stores them as
 // fp16 (q scaled by a per-row power of two so that no finite input
-// overflows; a rotated k entry at or beyond 65504 saturates and records
-// SWIN_ERR_UNSUPPORTED).  V is used as given (bf16).
+// overflows).  V is carried in fp16, the type of P.  A rotated k entry or a V
+// entry at or beyond 65504 saturates and records SWIN_ERR_UNSUPPORTED.
 //
 // Every wait is bounded: on time-out the kernel records SWIN_ERR_TIMEOUT in
 // the status word, every role leaves its loop, in-flight copies and MMAs are
@@ -296,6 +298,53 @@ __device__ __forceinline__ Ring ring_adv(Ring r, uint32_t k, uint32_t n) {
   return r;
 }
 
+// A softmax warpgroup's walk over its blocks: passes in order, the
+// warpgroup's tiles of each pass, the blocks of each tile.
+struct Walk {
+  uint32_t t;  // first tile of the current pass
+  Pass ps;
+  int i, j;    // tile of the pass, block of the tile
+  Ring base;   // ring position of the pass's block 0
+  bool valid;
+};
+
+// Move to the first tile of warpgroup g at or after tile i of the current pass.
+__device__ __forceinline__ void walk_seek(Walk& w, const TcParams& p, uint32_t t_begin, uint32_t t_end, int g,
+                                          uint32_t nst) {
+  while (true) {
+    while (w.i < w.ps.n && (int)((w.t + w.i - t_begin) & 1u) != g) ++w.i;
+    if (w.i < w.ps.n) return;
+    w.base = ring_adv(w.base, w.ps.u.nb, nst);
+    w.t += w.ps.n;
+    if (w.t >= t_end) {
+      w.valid = false;
+      return;
+    }
+    w.ps = pass_at(p, w.t, t_end);
+    w.i = 0;
+  }
+}
+
+__device__ __forceinline__ void walk_init(Walk& w, const TcParams& p, uint32_t t_begin, uint32_t t_end, int g,
+                                          uint32_t nst) {
+  w.t = t_begin;
+  w.base = Ring{0, 0};
+  w.i = w.j = 0;
+  w.valid = t_begin < t_end;
+  if (w.valid) {
+    w.ps = pass_at(p, t_begin, t_end);
+    walk_seek(w, p, t_begin, t_end, g, nst);
+  }
+}
+
+__device__ __forceinline__ void walk_next(Walk& w, const TcParams& p, uint32_t t_begin, uint32_t t_end, int g,
+                                          uint32_t nst) {
+  if (++w.j < w.ps.u.nb) return;
+  w.j = 0;
+  ++w.i;
+  walk_seek(w, p, t_begin, t_end, g, nst);
+}
+
 struct Ctl {
   volatile int* abort;
   const TcParams* p;
@@ -324,6 +373,18 @@ __device__ __forceinline__ uint32_t swz64(int row, int chunk) {
 
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Registers written by an asynchronous tcgen05.ld are only valid after
+// tcgen05.wait::ld; this empty asm "rewrites" them after the wait, so that no
+// use can be scheduled before it.
+__device__ __forceinline__ void reg_fence32(uint32_t* r) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
+}
 
 // ------------------------------------------------------------------ prep
 // Mode 2 feeds the score MMA fp16 operands (both Q and K, one type): fp16
@@ -400,7 +461,7 @@ __device__ __forceinline__ float pow2_scale(float m) {
 // MUFU: e = j + f with j = rint(e) read from the low mantissa bits of
 // e + 1.5 * 2^23 and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by
 // the Remez exchange algorithm for minimax relative error on [-1/2, 1/2]
-// (7.5e-5, well below half a bf16 ulp), and j is added to its exponent field.
+// (7.5e-5, below half an fp16 ulp), and j is added to its exponent field.
 // Arguments below -125 are clamped (the result is then at most 2^-125).
 __device__ __forceinline__ float2 exp2_poly2(float2 e) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
@@ -511,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   for (int i = threadIdx.x; i < (nst * kStageBytes + 1024) / 16; i += kThreads)
     reinterpret_cast<uint4*>(kvbuf)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  // the constant column: bf16 1.0 in the first column of 16 rows
-  if (threadIdx.x < 16) *reinterpret_cast<uint16_t*>(ones + swz64(threadIdx.x, 0)) = 0x3F80;
+  // the constant column: fp16 1.0 in the first column of 16 rows
+  if (threadIdx.x < 16) *reinterpret_cast<uint16_t*>(ones + swz64(threadIdx.x, 0)) = 0x3C00;
   if (warp == 1) {
     ptx::tmem_alloc(tmem_holder, 512);
     ptx::tmem_relinquish();
@@ -600,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
         constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
         constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlkKeys, 128);
-        constexpr uint32_t idPV = ptx::idesc_f16(1, 1, 0, 1, 48, 128);  // bf16 P (TMEM) x bf16 [V | c]
+        constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
         // Operand descriptors (64-byte swizzle) of this warpgroup's Q buffer 0
         // and of K/V stage 0; the others differ only in the start-address field
         // (16-byte units) and, for [V | c], in the leading byte offset to the
@@ -739,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       const int pk = (int)threadIdx.x - 448;
       Ring w{0, 0};
       bool ok = true;
-      bool range_hit = false;  // a rotated K entry saturated the fp16 range
+      bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
       for (uint32_t t = t_begin; t < t_end && ok;) {
         const Pass ps = pass_at(p, t, t_end);
         const Unit& u = ps.u;
@@ -747,27 +808,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         for (int j = 0; j < u.nb && ok; ++j, ring_next(w, nst)) {
           ok = __all_sync(0xffffffffu, wait_bar(&bars->kv_full[w.slot], w.ph, ctl));
           if (!ok) break;
-          if (MODE != 0) {
+          {
             const int nk = block_rows(u, j) * u.lx;
             uint8_t* ktile = kvbuf + w.slot * kStageBytes;
+            uint8_t* vtile = ktile + kHalfStage;
+            // units: half h of K row r and half h of V row r (r < nk <= 64);
+            // fp16 with saturation, a saturated entry is reported after the
+            // loop.  Trip counts are uniform per warp (the shuffle needs all lanes).
 #pragma unroll 1
             for (int un = pk; un < 2 * kBlkKeys; un += kPrepThreads) {
               const int r = un >> 1, h = un & 1;
               const bool act = r < nk;
-              float v[16];
-              if (act) load_half_bf16(ktile, r, h, v);
-              else for (int e = 0; e < 16; ++e) v[e] = 0.f;
-              if (MODE == 1) {
-                float ss = half_sumsq(v);
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if (act && h == 0) kcol[w.slot * kBlkKeys + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
-              } else if (act) {
-                const int pr = kp[r];
-                const int pos = h ? swin_local_coord(u.x0 + (pr >> 16), M, s)
-                                  : swin_local_coord(u.y0 + j * u.Rk + (pr & 0xFFFF), M, s);
-                rope_half(v, h, pos, rcos, rsin);
+              if (MODE != 0) {
+                float v[16];
+                if (act) load_half_bf16(ktile, r, h, v);
+                else for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                if (MODE == 1) {
+                  float ss = half_sumsq(v);
+                  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                  if (act && h == 0) kcol[w.slot * kBlkKeys + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
+                } else if (act) {
+                  const int pr = kp[r];
+                  const int pos = h ? swin_local_coord(u.x0 + (pr >> 16), M, s)
+                                    : swin_local_coord(u.y0 + j * u.Rk + (pr & 0xFFFF), M, s);
+                  rope_half(v, h, pos, rcos, rsin);
+                  range_hit |= half_absmax(v) >= 65504.0f;
+                  store_half_f16(ktile, r, h, v, 1.0f);
+                }
+              }
+              if (act) {
+                float v[16];
+                load_half_bf16(vtile, r, h, v);
                 range_hit |= half_absmax(v) >= 65504.0f;
-                store_half_f16(ktile, r, h, v, 1.0f);
+                store_half_f16(vtile, r, h, v, 1.0f);
               }
             }
             ptx::fence_proxy_async_smem();
@@ -781,6 +854,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
     // ================================================================ softmax
+    // Software-pipelined over this warpgroup's blocks: while block b is
+    // computed from registers, S(b + 1) is already being copied out of TMEM
+    // into the other register set, and P(b)'s store lands while the next
+    // block starts (its p_full arrival is deferred to the top of block b + 1).
+    // O is touched (rescale, deferred epilogue) at the end of a block, after
+    // P(b) is stored, which leaves PV(b - 1) the most time to complete.  The
+    // loop body alternates the two register sets.
     const int g = (warp - 4) >> 2;  // warpgroup 0 or 1
     const int wq = warp & 3;        // TMEM lanes 32 wq .. 32 wq + 31
     const uint32_t tX = tmem_base + g * 256 + ((uint32_t)(wq * 32) << 16);
@@ -790,15 +870,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     const int R2e = p.R2e, copy1 = p.copy1;
     int cur_h = -1;
     uint32_t tabn = 0;  // table loads of this warpgroup
-    Ring qr{0, 0}, base{0, 0};
-    uint32_t b = 0;  // blocks of this warpgroup
+    Ring qr{0, 0};
     bool ok = true;
     bool pend = false, pend_ok = false;  // a tile's O still waiting in TMEM (this warp's rows)
     size_t pend_off = 0;
     // O / l of one row to global memory (32 values; column 32 holds l)
     auto store_rows = [&](const uint32_t (&o)[32], uint32_t l, size_t off, bool row_valid) {
       if (!row_valid) return;
-      const float inv = 1.0f / __uint_as_float(l);  // row sum of the bf16 P
+      const float inv = 1.0f / __uint_as_float(l);  // row sum of the fp16 P
       if (OUT_F32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
 #pragma unroll
@@ -832,164 +911,196 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       ptx::tc_fence_after();
       return r;
     };
-    for (uint32_t t = t_begin; t < t_end && ok;) {
+    // tile state
+    bool active = false, row_ok = false;
+    int qy = 0, qx = 0, bbase = 0;
+    float alpha = 0.f, m_run = -INFINITY;
+    const float* pbase = slot;
+    uint32_t b = 0;            // blocks of this warpgroup
+    bool p_pending = false;    // P(b - 1) stored; its p_full arrival not made yet
+    Walk wk;
+    walk_init(wk, p, t_begin, t_end, g, nst);
+    uint32_t n_blocks = 0;  // blocks of this warpgroup in the CTA's range
+    for (uint32_t t = t_begin; t < t_end;) {
       const Pass ps = pass_at(p, t, t_end);
-      const Unit& u = ps.u;
-      const bool mine = ps.n > 1 || (int)((t - t_begin) & 1u) == g;  // a tile of this warpgroup in the pass
-      if (has_table && mine && u.h != cur_h) {
-        // new head: once all four warps are done with the old table, each
-        // loads a quarter of the new one (times log2 e, zero padding columns)
+      int mine = 0;
+      for (int i = 0; i < ps.n; ++i) mine += (int)((t + i - t_begin) & 1u) == g;
+      n_blocks += (uint32_t)(mine * ps.u.nb);
+      t += ps.n;
+    }
+    uint32_t xs[2][kBlkKeys];  // two register sets of scores (this block, the next)
+
+    auto arrive_p = [&]() {  // the deferred p_full of block b - 1
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->p_full[g][(b - 1) & 1]);
+      p_pending = false;
+    };
+
+    if (wk.valid) {
+      // prologue: S(0) into registers
+      ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[g][0], 0, ctl));
+      if (ok) {
+        ptx::tc_fence_after();
+        ptx::tmem_ld32(tX, *reinterpret_cast<uint32_t(*)[32]>(&xs[0][0]));
+        ptx::tmem_ld32(tX + 32, *reinterpret_cast<uint32_t(*)[32]>(&xs[0][32]));
+        ptx::tmem_wait_ld();
+        reg_fence32(&xs[0][0]);
+        reg_fence32(&xs[0][32]);
+        ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->tab_free[g]);
-        ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_free[g], tabn & 1, ctl));
-        if (!ok) break;
-        const int n = (2 * M - 1) * R2e;
-        for (int i = wq * 32 + lane; i < n; i += 128) {
-          const int dy = i / R2e, c = i - dy * R2e;
-          const float v =
-              c < 2 * M - 1 ? __ldg(p.table + (size_t)(dy * (2 * M - 1) + c) * p.heads + u.h) * kLog2eF : 0.f;
-          slot[i] = v;
-          if (i > 0) slot[copy1 + i - 1] = v;
-        }
-        if (wq == 0 && lane == 0) slot[copy1 + n - 1] = 0.f;
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->tab_ready[g]);
-        ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_ready[g], tabn & 1, ctl));
-        ++tabn;
-        if (!ok) break;
-        cur_h = u.h;
+        if (lane == 0) ptx::mbar_arrive(&bars->s_free[g][0]);
       }
-      const int* qp = qpos + u.cls * 128;
-      const int4* kof4 = reinterpret_cast<const int4*>(kofs + u.cls * kBlkKeys);
-      for (int i = 0; i < ps.n && ok; ++i) {
-        if ((int)((t + i - t_begin) & 1u) != g) continue;
-        const int k = ps.k0 + i;
-        const bool half = tile_half(u, k);
-        const int loff = half ? 64 * g : 0, nq = tile_rows(u, k) * u.lx;
-        const bool active = wq * 32 + 31 >= loff && wq * 32 < loff + nq;  // warp-uniform
-        const int r = wq * 32 + lane - loff;                                // query row in the tile
-        const bool row_ok = r >= 0 && r < nq;
-        const int rr = min(max(r, 0), 127);
-        const int qy = k * u.R + (qp[rr] & 0xFFFF), qx = qp[rr] >> 16;  // position in the rectangle
-        const uint32_t qs = qr.slot;
-        if (MODE != 0) {
-          ok = __all_sync(0xffffffffu, wait_bar(&bars->q_ready[g][qs], qr.ph, ctl));
-          if (!ok) break;
-        }
-        // per-row score scale: mode 1 log2e / (tau |q|), mode 2 log2e / (sqrt(d) 2^e)
-        const float alpha = MODE == 0 ? cscale : qscale[(g * kMaxQBuf + qs) * 128 + wq * 32 + lane];
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
-        ring_next(qr, nqb);
-        // Slot index of this row's bias for key (0, 0) of the rectangle; the
-        // pair load for keys (2c, 2c+1) of a row starts one float earlier, in
-        // copy 0 when that index is even, else in copy 1 (the parity is fixed
-        // per query: row stride and even key offsets do not change it).
-        // Bias loads are unconditional: rows past the tile use row M - 1, and
-        // keys past the block (masked below) read other slot entries, at
-        // most 64 rows of R2e floats before slot 0, inside shared memory.
-        const int bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
-        const float* pbase = slot + (((bbase - 1) & 1) ? copy1 - 1 : 0) + bbase - 1;
-        float m_run = -INFINITY;
-        Ring w = base;
-        for (int j = 0; j < u.nb; ++j, ++b, ring_next(w, nst)) {
-          ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[g][b & 1], (b >> 1) & 1, ctl));
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const int nk = block_rows(u, j) * u.lx;
-          const int nch = (nk + 15) >> 4;
-          const uint32_t tS = tX + (b & 1) * 64, tP = tX + 128 + (b & 1) * 32;
-          float2 x[kBlkKeys / 2];  // scores as packed pairs (keys 2c, 2c+1)
-          if (active) {
-            uint32_t r0[32], r1[32];
-            ptx::tmem_ld32(tS, r0);
-            ptx::tmem_ld32(tS + 32, r1);
-            ptx::tmem_wait_ld();
+    }
+#pragma unroll 1
+    while (ok && wk.valid) {
+      // two blocks per trip, so that the register sets alternate statically
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              x[e] = make_float2(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
-              x[16 + e] = make_float2(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+      for (int pp = 0; pp < 2; ++pp) {
+        if (ok && wk.valid) {
+          uint32_t* xc = xs[pp];
+          uint32_t* xn = xs[pp ^ 1];
+          const bool has_next = b + 1 < n_blocks;
+          if (has_next) {
+            // S(b + 1) was issued while block b - 1 was computed
+            ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[g][(b + 1) & 1], ((b + 1) >> 1) & 1, ctl));
+            if (ok) {
+              ptx::tc_fence_after();
+              const uint32_t tSn = tX + ((b + 1) & 1) * 64;
+              ptx::tmem_ld32(tSn, *reinterpret_cast<uint32_t(*)[32]>(xn));
+              ptx::tmem_ld32(tSn + 32, *reinterpret_cast<uint32_t(*)[32]>(xn + 32));
             }
           }
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->s_free[g][b & 1]);  // S[b % 2] may take S(b + 2)
-          uint32_t pr[kBlkKeys / 2];
+          // the previous block's P store has had a block boundary to land:
+          // release it to the issuer
+          if (ok && p_pending) arrive_p();
+          const Unit& u = wk.ps.u;
+          const int j = wk.j;
+          if (ok && j == 0) {
+            // ---- new tile: bias table of its head, row scale, row position
+            if (has_table && u.h != cur_h) {
+              // new head: once all four warps are done with the old table,
+              // each loads a quarter of the new one (times log2 e, zero
+              // padding columns)
+              __syncwarp();
+              if (lane == 0) ptx::mbar_arrive(&bars->tab_free[g]);
+              ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_free[g], tabn & 1, ctl));
+              if (ok) {
+                const int n = (2 * M - 1) * R2e;
+                for (int i = wq * 32 + lane; i < n; i += 128) {
+                  const int dy = i / R2e, c = i - dy * R2e;
+                  const float v = c < 2 * M - 1
+                                      ? __ldg(p.table + (size_t)(dy * (2 * M - 1) + c) * p.heads + u.h) * kLog2eF
+                                      : 0.f;
+                  slot[i] = v;
+                  if (i > 0) slot[copy1 + i - 1] = v;
+                }
+                if (wq == 0 && lane == 0) slot[copy1 + n - 1] = 0.f;
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&bars->tab_ready[g]);
+                ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_ready[g], tabn & 1, ctl));
+                ++tabn;
+                cur_h = u.h;
+              }
+            }
+            const int k = wk.ps.k0 + wk.i;
+            const int loff = tile_half(u, k) ? 64 * g : 0, nq = tile_rows(u, k) * u.lx;
+            active = wq * 32 + 31 >= loff && wq * 32 < loff + nq;  // warp-uniform
+            const int r = wq * 32 + lane - loff;                    // query row in the tile
+            row_ok = r >= 0 && r < nq;
+            const int rr = min(max(r, 0), 127);
+            const int* qp = qpos + u.cls * 128;
+            qy = k * u.R + (qp[rr] & 0xFFFF);  // position in the rectangle
+            qx = qp[rr] >> 16;
+            const uint32_t qs = qr.slot;
+            if (ok && MODE != 0) ok = __all_sync(0xffffffffu, wait_bar(&bars->q_ready[g][qs], qr.ph, ctl));
+            // per-row score scale: mode 1 log2e / (tau |q|), mode 2 log2e / (sqrt(d) 2^e)
+            alpha = MODE == 0 ? cscale : qscale[(g * kMaxQBuf + qs) * 128 + wq * 32 + lane];
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
+            ring_next(qr, nqb);
+            // Slot index of this row's bias for key (0, 0) of the rectangle;
+            // the pair load for keys (2c, 2c+1) of a row starts one float
+            // earlier, in copy 0 when that index is even, else in copy 1 (the
+            // parity is fixed per query: row stride and even key offsets do
+            // not change it).  Bias loads are unconditional: rows past the
+            // tile use row M - 1, and keys past the block (masked below) read
+            // other slot entries, at most 64 rows of R2e floats before slot 0,
+            // inside shared memory.
+            bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
+            pbase = slot + (((bbase - 1) & 1) ? copy1 - 1 : 0) + bbase - 1;
+            m_run = -INFINITY;
+          }
+          const int nk = block_rows(u, j) * u.lx;
+          const int nch = (nk + 15) >> 4;
+          const uint32_t tP = tX + 128 + (b & 1) * 32;
           float factor = 1.f;
           bool rescale = false;
-          if (active) {
+          constexpr bool scale_in_exp = MODE == 2 || (MODE == 0 && !has_table);
+          const float ea = scale_in_exp ? alpha : 1.0f;
+          if (ok && active) {
+            const Ring w = ring_adv(wk.base, (uint32_t)j, nst);
             if (MODE == 1) {
               // 1/|k| of the block's keys was written by the K prep before kv_ready
               ok = __all_sync(0xffffffffu, wait_bar(&bars->kv_ready[w.slot], w.ph, ctl));
-              if (!ok) break;
             }
             // x = log2-domain logits.  Mode 2 (and mode 0 without a table):
             // the scale is applied inside the exponent below (max over raw
             // scores, scale > 0).  Otherwise x = S * scale + bias in one
             // rounding; the bias slot holds T * log2(e), and mode 1's scale
             // is log2e / (tau |q| |k|).
-            constexpr bool scale_in_exp = MODE == 2 || (MODE == 0 && !has_table);
             if (!scale_in_exp) {
               const float4* kc4 = reinterpret_cast<const float4*>(kcol + w.slot * kBlkKeys);
+              const int4* kof4 = reinterpret_cast<const int4*>(kofs + u.cls * kBlkKeys);
               const int jo = j * u.Rk * R2e;  // block j starts Rk rectangle rows further
-              if (!has_table) {
 #pragma unroll
-                for (int c4 = 0; c4 < kBlkKeys / 4; ++c4) {
+              for (int c4 = 0; c4 < kBlkKeys / 4; ++c4) {
+                float2 s0 = make_float2(alpha, alpha), s1 = s0;
+                if (MODE == 1) {
                   const float4 kc = kc4[c4];  // same address in every lane: broadcast
-                  x[2 * c4] = __fmul2_rn(x[2 * c4], __fmul2_rn(make_float2(kc.x, kc.y), make_float2(alpha, alpha)));
-                  x[2 * c4 + 1] =
-                      __fmul2_rn(x[2 * c4 + 1], __fmul2_rn(make_float2(kc.z, kc.w), make_float2(alpha, alpha)));
+                  s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
+                  s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
                 }
-              } else if (BIAS == kBiasPairs) {
-                const float* pb = pbase - jo;
-#pragma unroll
-                for (int c4 = 0; c4 < kBlkKeys / 4; ++c4) {
-                  float2 s0 = make_float2(alpha, alpha), s1 = s0;
-                  if (MODE == 1) {
-                    const float4 kc = kc4[c4];
-                    s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
-                    s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
-                  }
+                float2 b0 = make_float2(0.f, 0.f), b1 = b0;
+                if (BIAS == kBiasPairs) {
                   const int4 ko = kof4[c4];  // broadcast; keys 4 c4 .. 4 c4 + 3 share a row pairwise
-                  const float2 b0 = *reinterpret_cast<const float2*>(pb - ko.x);  // (bias key+1, bias key)
-                  const float2 b1 = *reinterpret_cast<const float2*>(pb - ko.z);
-                  x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(b0.y, b0.x));
-                  x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(b1.y, b1.x));
-                }
-              } else {
-                // odd rectangle widths: one load per key
-                const float* hb = slot + bbase - jo;
-#pragma unroll
-                for (int c4 = 0; c4 < kBlkKeys / 4; ++c4) {
-                  float2 s0 = make_float2(alpha, alpha), s1 = s0;
-                  if (MODE == 1) {
-                    const float4 kc = kc4[c4];
-                    s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
-                    s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
-                  }
+                  const float2 v0 = *reinterpret_cast<const float2*>(pbase - jo - ko.x);  // (bias key+1, key)
+                  const float2 v1 = *reinterpret_cast<const float2*>(pbase - jo - ko.z);
+                  b0 = make_float2(v0.y, v0.x);
+                  b1 = make_float2(v1.y, v1.x);
+                } else if (BIAS == kBiasKeys) {
+                  // odd rectangle widths: one load per key
                   const int4 ko = kof4[c4];
-                  x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(hb[-ko.x], hb[-ko.y]));
-                  x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(hb[-ko.z], hb[-ko.w]));
+                  const float* hb = slot + bbase - jo;
+                  b0 = make_float2(hb[-ko.x], hb[-ko.y]);
+                  b1 = make_float2(hb[-ko.z], hb[-ko.w]);
                 }
+                const float2 x0 = make_float2(__uint_as_float(xc[4 * c4]), __uint_as_float(xc[4 * c4 + 1]));
+                const float2 x1 = make_float2(__uint_as_float(xc[4 * c4 + 2]), __uint_as_float(xc[4 * c4 + 3]));
+                const float2 y0 = has_table ? __ffma2_rn(x0, s0, b0) : __fmul2_rn(x0, s0);
+                const float2 y1 = has_table ? __ffma2_rn(x1, s1, b1) : __fmul2_rn(x1, s1);
+                xc[4 * c4] = __float_as_uint(y0.x);
+                xc[4 * c4 + 1] = __float_as_uint(y0.y);
+                xc[4 * c4 + 2] = __float_as_uint(y1.x);
+                xc[4 * c4 + 3] = __float_as_uint(y1.y);
               }
             }
             if (nk < kBlkKeys) {  // partial block (uniform across the warpgroup): mask the tail keys
 #pragma unroll
-              for (int c = 0; c < kBlkKeys / 2; ++c) {
-                if (2 * c >= nk) x[c].x = -INFINITY;
-                if (2 * c + 1 >= nk) x[c].y = -INFINITY;
-              }
+              for (int c = 0; c < kBlkKeys; ++c)
+                if (c >= nk) xc[c] = __float_as_uint(-INFINITY);
             }
-            // block maximum: four independent 3-input max chains, two pairs a step
-            float mq[4] = {x[0].x, x[0].y, x[1].x, x[1].y};
+            // block maximum: four independent 3-input max chains
+            float mq[4] = {__uint_as_float(xc[0]), __uint_as_float(xc[1]), __uint_as_float(xc[2]),
+                           __uint_as_float(xc[3])};
 #pragma unroll
-            for (int c = 2; c < kBlkKeys / 2; c += 2) {
-              const int ch = 2 * ((c >> 1) & 1);
-              mq[ch] = ptx::max3(mq[ch], x[c].x, x[c + 1].x);
-              mq[ch + 1] = ptx::max3(mq[ch + 1], x[c].y, x[c + 1].y);
+            for (int c = 4; c < kBlkKeys; c += 4) {
+              const int chn = 2 * ((c >> 2) & 1);
+              mq[chn] = ptx::max3(mq[chn], __uint_as_float(xc[c]), __uint_as_float(xc[c + 2]));
+              mq[chn + 1] = ptx::max3(mq[chn + 1], __uint_as_float(xc[c + 1]), __uint_as_float(xc[c + 3]));
             }
             float mb = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-            const float ea = scale_in_exp ? alpha : 1.0f;
             if (scale_in_exp) mb *= ea;
             // running maximum, kept unless this block exceeds it by more than 8
             if (j == 0) {
@@ -999,75 +1110,93 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
               m_run = mb;
               rescale = true;
             }
-            // probabilities, bf16: exponent argument x * ea - m
+          }
+          // P[b % 2] is free once PV(b - 2) has read it
+          if (ok && b >= 2) ok = wait_pv(b - 2);
+          if (ok && active) {
+            // probabilities, fp16, 16 keys (8 columns) at a time: exponent
+            // argument x * ea - m
             const float eb = -m_run;
             constexpr int kPoly = ExpSplit<MODE>::kPoly;
 #pragma unroll
-            for (int c = 0; c < kBlkKeys / 2; ++c) {
-              if (c >= 8 && (c >> 3) >= nch) {  // a chunk of 16 keys past the block
-                pr[c] = 0u;
-                continue;
-              }
-              const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
-              if (2 * c < kPoly) {
-                const float2 pe = exp2_poly2(e);
-                pr[c] = ptx::pack_bf16x2(pe.x, pe.y);
-              } else {
-                pr[c] = ptx::pack_bf16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+            for (int ch = 0; ch < kBlkKeys / 16; ++ch) {
+              if (ch == 0 || ch < nch) {  // chunks past the block: PV never reads them
+                uint32_t pr[8];
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) {
+                  const int c = ch * 16 + 2 * e2;
+                  const float2 e = __ffma2_rn(make_float2(__uint_as_float(xc[c]), __uint_as_float(xc[c + 1])),
+                                              make_float2(ea, ea), make_float2(eb, eb));
+                  if (c < kPoly) {
+                    const float2 pe = exp2_poly2(e);
+                    pr[e2] = ptx::pack_f16x2(pe.x, pe.y);
+                  } else {
+                    pr[e2] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+                  }
+                }
+                ptx::tmem_st8(tP + ch * 8, pr);
               }
             }
           }
+          p_pending = true;
           // O (32 columns) and its row sum (column 32): rescaled to the new
           // maximum, or, in a tile's first block, the previous tile's result
-          // read for the deferred store.  Both need PV(b - 1) complete.
-          uint32_t po[32], pl = 0;
+          // read for the deferred store.  Both need PV(b - 1) complete, and
+          // both come before PV(b) (issued once p_full(b) is arrived, at the
+          // top of the next block).
           const bool epi = j == 0 && pend;
           const bool resc = j > 0 && __any_sync(0xffffffffu, rescale);
-          if (epi || resc) {
+          if (ok && (epi || resc)) {
             ok = wait_pv(b - 1);
-            if (!ok) break;
-            ptx::tmem_ld32(tO, po);
-            pl = ptx::tmem_ld1(tO + 32);
-            ptx::tmem_wait_ld();
-            if (resc) {
+            if (ok) {
+              uint32_t po[32];
+              ptx::tmem_ld32(tO, po);
+              uint32_t pl = ptx::tmem_ld1(tO + 32);
+              ptx::tmem_wait_ld();
+              reg_fence32(po);
+              asm volatile("" : "+r"(pl));
+              if (resc) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) po[e] = __float_as_uint(__uint_as_float(po[e]) * factor);
-              ptx::tmem_st32(tO, po);
-              ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
+                for (int e = 0; e < 32; ++e) po[e] = __float_as_uint(__uint_as_float(po[e]) * factor);
+                ptx::tmem_st32(tO, po);
+                ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
+              } else {
+                store_rows(po, pl, pend_off, pend_ok);
+                pend = false;
+              }
             }
           }
-          // P[b % 2] is free once PV(b - 2) has read it
-          if (b >= 2) {
-            ok = wait_pv(b - 2);
-            if (!ok) break;
+          if (ok && has_next) {
+            // S(b + 1) is in registers: S[(b + 1) % 2] may take S(b + 3)
+            ptx::tmem_wait_ld();
+            reg_fence32(xn);
+            reg_fence32(xn + 32);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&bars->s_free[g][(b + 1) & 1]);
           }
-          if (active) ptx::tmem_st32(tP, pr);
-          ptx::tmem_wait_st();
-          ptx::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&bars->p_full[g][b & 1]);
-          if (epi) {
-            store_rows(po, pl, pend_off, pend_ok);
-            pend = false;
+          if (j == u.nb - 1) {
+            // this tile's O is read in the next tile's first block (or after the loop)
+            pend = active;
+            pend_ok = row_ok;
+            pend_off = (((size_t)u.b * p.H + (u.y0 + qy)) * p.W + (u.x0 + qx)) * (size_t)(p.heads * 32) +
+                       (size_t)u.h * 32;
           }
+          ++b;
+          walk_next(wk, p, t_begin, t_end, g, nst);
         }
-        if (!ok) break;
-        // this tile's O is read in the next tile's first block (or after the loop)
-        pend = active;
-        pend_ok = row_ok;
-        pend_off = (((size_t)u.b * p.H + (u.y0 + qy)) * p.W + (u.x0 + qx)) * (size_t)(p.heads * 32) +
-                   (size_t)u.h * 32;
       }
-      base = ring_adv(base, u.nb, nst);
-      t += ps.n;
     }
+    if (ok && p_pending) arrive_p();
     if (ok && pend && b > 0) {
       ok = wait_pv(b - 1);
       if (ok) {
         uint32_t po[32];
         ptx::tmem_ld32(tO, po);
-        const uint32_t pl = ptx::tmem_ld1(tO + 32);
+        uint32_t pl = ptx::tmem_ld1(tO + 32);
         ptx::tmem_wait_ld();
+        reg_fence32(po);
+        asm volatile("" : "+r"(pl));
         store_rows(po, pl, pend_off, pend_ok);
       }
     }
