@@ -62,11 +62,12 @@ def _kernel_consts():
         expr = re.search(r"constexpr int %s = ([^;]+);" % name, src).group(1)
         env[name] = eval(expr.split("//")[0], {}, env)
     # struct Bars: q_full/q_ready/q_empty [2][kMaxQBuf], kv_* [kMaxStages], s/p full/free [2][2],
-    # tab_free/tab_ready [2], never, drain[2]
+    # tab_free/tab_ready [2], never, drain[n]
     body = src[src.index("struct Bars {"):]
     body = body[:body.index("};")]
     assert body.count("uint64_t") == 5, body
-    env["kNumBars"] = 3 * 2 * env["kMaxQBuf"] + 3 * env["kMaxStages"] + 4 * 4 + 4 + 3
+    n_drain = int(re.search(r"drain\[(\d+)\]", body).group(1))
+    env["kNumBars"] = 3 * 2 * env["kMaxQBuf"] + 3 * env["kMaxStages"] + 4 * 4 + 4 + 1 + n_drain
     return env
 
 

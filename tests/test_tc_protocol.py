@@ -2,9 +2,9 @@
 
 Every role of attn_tc_kernel is a program of mbarrier arrivals and waits in
 the kernel's order: the K/V and Q producers (TMA loads), the K and Q prep, one
-MMA issuer per softmax warpgroup, and each of the eight softmax warps.  TMA
-copies complete in any order; each issuer's MMAs and commits execute in issue
-order.  Random interleavings run over real per-CTA tile sequences (the
+S-MMA and one PV-MMA issuer per softmax warpgroup, and each of the eight
+softmax warps.  TMA copies complete in any order; each issuer thread's MMAs
+and commits execute in its issue order, with no order between threads.  Random interleavings run over real per-CTA tile sequences (the
 kernel's own host plan, `swin_debug_tc_plan`, decoded tile by tile).
 
 Beyond deadlock freedom and unambiguous parity waits (no wait may see a phase
@@ -109,11 +109,9 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
     Pb = {(g, x): {"b": None, "writers": 0} for g in range(2) for x in range(2)}
     pv_exec = [0, 0]           # PVs executed per warpgroup (in order)
     o_epi = {}                 # (g, tile) -> [warps that must read, warps that read]
-    tile_of_pv = {}            # (g, b) -> tile id
-    first_pv_of_tile = {}      # (g, tile) -> b
     prev_tile = {}             # (g, tile) -> previous tile of the warpgroup
     tma = []                   # pending TMA completions
-    mmaq = {0: [], 1: []}
+    mmaq = {("S", 0): [], ("S", 1): [], ("PV", 0): [], ("PV", 1): []}
 
     def wg_of(t):
         return (t - t0) & 1
@@ -175,23 +173,12 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
                 bars[("q_ready", g, slot)].arrive()
                 qn[g] += 1
 
-    def issuer(g):
+    def s_issuer(g):
+        """S MMAs of warpgroup g (their own thread)."""
         b = qcnt = base = 0
-        pv = {}
-
-        def issue_pv(k):
-            if bug != "pv_without_p_full":
-                yield W(("p_full", g, k & 1), k >> 1)
-            slot, pos, acc, rel, tile = pv[k]
-            c = [("PV", g, k, slot, pos, acc, tile), ("bar", ("p_free", g, k & 1))]
-            c += [("bar", ("kv_empty", slot))] * rel
-            mmaq[g].append(c)
         for t, n, u in ps:
             nb = int(u[11])
-            mine = [i for i in range(n) if wg_of(t + i) == g]
-            last_i = mine[-1] if mine else -1
-            for i in mine:
-                rel = (2 if n == 1 else 1) if i == last_i else 0
+            for i in [i for i in range(n) if wg_of(t + i) == g]:
                 qslot, qrnd = qcnt % nqb, qcnt // nqb
                 for j in range(nb):
                     pos = base + j
@@ -205,17 +192,29 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
                     if j == nb - 1:
                         c.append(("bar", ("q_empty", g, qslot)))
                         qcnt += 1
-                    mmaq[g].append(c)
-                    pv[b] = (slot, pos, j > 0, rel, t + i)
-                    tile_of_pv[(g, b)] = t + i
-                    if j == 0:
-                        first_pv_of_tile[(g, t + i)] = b
-                    if b >= 2:
-                        yield from issue_pv(b - 2)
+                    mmaq[("S", g)].append(c)
                     b += 1
             base += nb
-        for k in range(max(b - 2, 0), b):
-            yield from issue_pv(k)
+
+    def pv_issuer(g):
+        """PV MMAs of warpgroup g (their own thread)."""
+        b = base = 0
+        for t, n, u in ps:
+            nb = int(u[11])
+            mine = [i for i in range(n) if wg_of(t + i) == g]
+            last_i = mine[-1] if mine else -1
+            for i in mine:
+                rel = (2 if n == 1 else 1) if i == last_i else 0
+                for j in range(nb):
+                    pos = base + j
+                    slot = pos % nst
+                    if bug != "pv_without_p_full":
+                        yield W(("p_full", g, b & 1), b >> 1)
+                    c = [("PV", g, b, slot, pos, j > 0, t + i), ("bar", ("p_free", g, b & 1))]
+                    c += [("bar", ("kv_empty", slot))] * rel
+                    mmaq[("PV", g)].append(c)
+                    b += 1
+            base += nb
 
     def softmax_warp(g, wq):
         """One softmax warp, in the kernel's order: S(b + 1) is copied out
@@ -326,7 +325,7 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
             _, g, k, slot, pos, acc, tile = entry
             check(kv[slot]["pos"] == pos, "PV(%d) read V of a stale stage" % k)
             kv[slot]["reads"] += 1
-            check(Pb[(g, k & 1)]["for"] == k and Pb[(g, k & 1)]["writers"] == 4,
+            check(Pb[(g, k & 1)].get("for") == k and Pb[(g, k & 1)]["writers"] == 4,
                   "PV(%d) read P before all warps wrote it" % k)
             if not acc:
                 prev = prev_tile.get((g, tile))
@@ -337,7 +336,7 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
             pv_exec[g] += 1
 
     roles = {"kvp": kv_producer(), "qp": q_producer(), "kprep": k_prep(), "qprep": q_prep(),
-             "iss0": issuer(0), "iss1": issuer(1)}
+             "s0": s_issuer(0), "s1": s_issuer(1), "pv0": pv_issuer(0), "pv1": pv_issuer(1)}
     for g in range(2):
         for wq in range(4):
             roles["sm%d_%d" % (g, wq)] = softmax_warp(g, wq)
@@ -351,14 +350,14 @@ def run(tiles, plan, t0, t1, mode, seed, rescale_p=0.2, bug=None, nst=None, max_
             raise AssertionError("parity alias on %s: waiting for completion %d, %d done" % (name, k, c))
         return c >= k + 1
     steps = 0
-    while alive or tma or mmaq[0] or mmaq[1]:
+    while alive or tma or any(mmaq.values()):
         steps += 1
         cands = [("role", r) for r in alive if waiting[r] is None or ready(waiting[r])]
         if tma:
             cands.append(("tma", None))
-        for g in (0, 1):
-            if mmaq[g]:
-                cands.append(("mma", g))
+        for key, q in mmaq.items():
+            if q:
+                cands.append(("mma", key))
         if not cands:
             raise Deadlock({r: waiting[r] for r in alive})
         kind, x = rng.choice(cands)

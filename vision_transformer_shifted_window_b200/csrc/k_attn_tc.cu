@@ -29,10 +29,12 @@
 //                (64-byte swizzle, no multicast) into the ring
 //   warp 3       Q producer: one TMA load per query tile into that tile's
 //                warpgroup's buffers (4, or 2 for long tiles)
-//   warps 1, 2   tcgen05.mma issuers, one thread each: warp 1 + g issues the
-//                MMAs of softmax warpgroup g; warp 1 owns TMEM
-//   warps 12-13  Q prep: 1/(tau |q|) per row (mode 1), RoPE of q (mode 2)
-//   warps 14-15  K prep: 1/|k| per key (mode 1), RoPE of k (mode 2), V to fp16
+//   warps 1, 2   tcgen05.mma S issuers, one thread each: warp 1 + g issues
+//                the S = Q K^T MMAs of softmax warpgroup g; warp 1 owns TMEM
+//   warps 13, 15 tcgen05.mma PV issuers: warp 13 + 2g issues the O += P V
+//                MMAs of softmax warpgroup g
+//   warp 12      Q prep: 1/(tau |q|) per row (mode 1), RoPE of q (mode 2)
+//   warp 14      K prep: 1/|k| per key (mode 1), RoPE of k (mode 2), V to fp16
 //   warps 4-7    softmax of warpgroup 0 (one TMEM lane = one query row)
 //   warps 8-11   softmax of warpgroup 1
 //
@@ -46,9 +48,8 @@
 // accumulate the row sum of exactly the fp16 probabilities that weight V).
 // The softmax waits for the tensor core only where a buffer comes back two
 // blocks later (PV(b - 2) done before P(b) is written), where it rescales O,
-// and where it reads a finished O.  Each issuer runs its warpgroup's blocks in
-// the order S(0), S(1), S(2), PV(0), S(3), PV(1), ...; a thread's MMAs execute
-// in issue order.
+// and where it reads a finished O.  S and PV MMAs of a warpgroup come from two
+// threads, so an S never queues behind a PV that waits for its probabilities.
 //
 // A query tile of at most 64 rows is placed in TMEM lanes 64-127 when it
 // belongs to warpgroup 1 (lanes 0-63 for warpgroup 0), so that small windows
@@ -120,7 +121,7 @@ constexpr int kTileBytes = 128 * 64;          // Q tile: 128 rows x 32 16-bit va
 constexpr int kHalfStage = 64 * 64;           // K or V block: 64 rows x 32 16-bit values
 constexpr int kStageBytes = 2 * kHalfStage;   // K then V
 constexpr int kBlkKeys = 64;                  // keys per K/V block (TMEM: 2 x 64 + 2 x 32 + 48 columns)
-constexpr int kPrepThreads = 64;              // Q prep: warps 12-13; K prep: warps 14-15
+constexpr int kPrepThreads = 32;              // Q prep: warp 12; K prep: warp 14
 constexpr int kSmemMax = 227 * 1024;
 constexpr int kSmemSlack = 1024;              // for the 1024-byte alignment of the base
 constexpr int kRopeBytes = 2 * 2 * 64 * 8 * 4;  // cos, sin [2 axes][64 positions][8]
@@ -133,7 +134,7 @@ struct Bars {
   // has not taken yet, so parity waits never alias (see the softmax)
   uint64_t s_full[2][2], s_free[2][2], p_full[2][2], p_free[2][2];
   uint64_t tab_free[2], tab_ready[2];  // bias-table slot handshake of each softmax warpgroup (4 warps)
-  uint64_t never, drain[2];
+  uint64_t never, drain[4];
 };
 constexpr int kNumBars = sizeof(Bars) / 8;
 
@@ -544,8 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       ptx::mbar_init(&bars->tab_ready[g], 4);
     }
     ptx::mbar_init(&bars->never, 1);
-    ptx::mbar_init(&bars->drain[0], 1);
-    ptx::mbar_init(&bars->drain[1], 1);
+    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars->drain[i], 1);
     *abort_flag = 0;
     tmem_holder[2] = 0;  // abort flag of the drain waits (never set by a role)
     ptx::fence_mbar_init();
@@ -654,97 +654,115 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           for (uint32_t i = 0; i < m; ++i, ring_next(d, nqb)) wait_bar(&bars->q_full[g][d.slot], d.ph, drain);
         }
       }
-    } else if (warp == 1 || warp == 2) {
+    } else if (warp == 1 || warp == 2 || warp == 13 || warp == 15) {
       // ============================================================ MMA issuers
+      // Two issuer threads per softmax warpgroup g: warp 1 + g issues its S
+      // MMAs, warp 13 + 2g its PV MMAs.  S and PV never touch the same TMEM
+      // columns, and every dependence between them goes through the softmax
+      // (S(b) -> softmax -> P(b) -> PV(b)), so they need no common order: an
+      // S MMA never waits behind a PV whose probabilities are not written yet.
       if (lane == 0) {
-        const int g = warp - 1;
-        // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
-        constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
-        constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlkKeys, 128);
-        constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
-        // Operand descriptors (64-byte swizzle) of this warpgroup's Q buffer 0
-        // and of K/V stage 0; the others differ only in the start-address field
-        // (16-byte units) and, for [V | c], in the leading byte offset to the
-        // constant column block, which sits after the ring (N columns 32-47).
-        const uint64_t qd0 =
-            ptx::smem_desc(ptx::smem_addr(qbuf + g * nqb * kTileBytes), 16, 512, ptx::kSwizzle64B);
-        const uint64_t kd0 = ptx::smem_desc(ptx::smem_addr(kvbuf), 16, 512, ptx::kSwizzle64B);
-        const uint32_t va0 = ptx::smem_addr(kvbuf + kHalfStage), oa0 = ptx::smem_addr(ones);
-        const uint64_t vd0 = ptx::smem_desc(va0, oa0 - va0, 512, ptx::kSwizzle64B);
-        constexpr uint64_t kQBuf = kTileBytes >> 4;
-        constexpr uint64_t kStageK = kStageBytes >> 4;
-        constexpr uint64_t kStageV = kStageK - (kStageK << 16);
-        // k-step kk of PV: V rows 16 kk.. (+1024 bytes), constant block unchanged
-        constexpr uint64_t kStepV = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
+        const bool s_role = warp < 4;
+        const int g = s_role ? warp - 1 : (warp - 13) >> 1;
         const uint32_t tg = tmem_base + g * 256;
         bool ok = true;
-        if (g == 0 && (p.debug_flags & 1)) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
-        // PV of block b: stage, accumulate, K/V releases, k-steps (by b % 3)
-        uint32_t pv_stage[3] = {0, 0, 0}, pv_acc[3] = {0, 0, 0}, pv_rel[3] = {0, 0, 0}, pv_nch[3] = {0, 0, 0};
-        auto issue_pv = [&](uint32_t k) -> bool {
-          if (!wait_bar(&bars->p_full[g][k & 1], (k >> 1) & 1, ctl)) return false;
-          ptx::tc_fence_after();
-          const uint32_t e = k % 3;
-          const uint64_t vd = vd0 + pv_stage[e] * kStageV;
-          const uint32_t aP = tg + 128 + (k & 1) * 32;
-          for (uint32_t kk = 0; kk < pv_nch[e]; ++kk)
-            ptx::mma_ts(tg + 192, aP + kk * 8, vd + kk * kStepV, idPV, (kk > 0 || pv_acc[e]) ? 1u : 0u);
-          ptx::mma_commit(&bars->p_free[g][k & 1]);
-          for (uint32_t r = 0; r < pv_rel[e]; ++r) ptx::mma_commit(&bars->kv_empty[pv_stage[e]]);
-          return true;
-        };
-        Ring qr{0, 0}, base{0, 0};
-        uint32_t b = 0;
-        for (uint32_t t = t_begin; t < t_end && ok;) {
-          const Pass ps = pass_at(p, t, t_end);
-          const Unit& u = ps.u;
-          int last_i = -1;  // this warpgroup's last tile in the pass
-          for (int i = 0; i < ps.n; ++i)
-            if ((int)((t + i - t_begin) & 1u) == g) last_i = i;
-          for (int i = 0; i < ps.n && ok; ++i) {
-            if ((int)((t + i - t_begin) & 1u) != g) continue;
-            const uint32_t rel = i == last_i ? (ps.n == 1 ? 2u : 1u) : 0u;
-            Ring w = base;
-            for (int j = 0; j < u.nb; ++j, ++b, ring_next(w, nst)) {
-              // S(b) into S[b % 2]: the softmax has copied S(b - 2) out
-              if (b >= 2) ok = wait_bar(&bars->s_free[g][b & 1], ((b - 2) >> 1) & 1, ctl);
-              ok = ok && (j > 0 || wait_bar(&bars->q_ready[g][qr.slot], qr.ph, ctl)) &&
-                   wait_bar(&bars->kv_ready[w.slot], w.ph, ctl);
-              if (!ok) break;
-              ptx::tc_fence_after();
-              const uint64_t ad = qd0 + qr.slot * kQBuf, bd = kd0 + w.slot * kStageK;
-              const uint32_t dS = tg + (b & 1) * 64;
-              ptx::mma_ss(dS, ad, bd, idS, 0);
-              ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
-              ptx::mma_commit(&bars->s_full[g][b & 1]);
-              if (j == u.nb - 1) {
-                ptx::mma_commit(&bars->q_empty[g][qr.slot]);
-                ring_next(qr, nqb);
+        if (s_role) {
+          // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
+          constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
+          constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlkKeys, 128);
+          // Operand descriptors (64-byte swizzle) of this warpgroup's Q buffer
+          // 0 and of K stage 0; the others differ only in the start-address
+          // field (16-byte units).
+          const uint64_t qd0 =
+              ptx::smem_desc(ptx::smem_addr(qbuf + g * nqb * kTileBytes), 16, 512, ptx::kSwizzle64B);
+          const uint64_t kd0 = ptx::smem_desc(ptx::smem_addr(kvbuf), 16, 512, ptx::kSwizzle64B);
+          constexpr uint64_t kQBuf = kTileBytes >> 4;
+          constexpr uint64_t kStageK = kStageBytes >> 4;
+          if (g == 0 && (p.debug_flags & 1)) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
+          Ring qr{0, 0}, base{0, 0};
+          uint32_t b = 0;
+          for (uint32_t t = t_begin; t < t_end && ok;) {
+            const Pass ps = pass_at(p, t, t_end);
+            const Unit& u = ps.u;
+            for (int i = 0; i < ps.n && ok; ++i) {
+              if ((int)((t + i - t_begin) & 1u) != g) continue;
+              Ring w = base;
+              for (int j = 0; j < u.nb; ++j, ++b, ring_next(w, nst)) {
+                // S(b) into S[b % 2]: the softmax has copied S(b - 2) out
+                if (b >= 2) ok = wait_bar(&bars->s_free[g][b & 1], ((b - 2) >> 1) & 1, ctl);
+                ok = ok && (j > 0 || wait_bar(&bars->q_ready[g][qr.slot], qr.ph, ctl)) &&
+                     wait_bar(&bars->kv_ready[w.slot], w.ph, ctl);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint64_t ad = qd0 + qr.slot * kQBuf, bd = kd0 + w.slot * kStageK;
+                const uint32_t dS = tg + (b & 1) * 64;
+                ptx::mma_ss(dS, ad, bd, idS, 0);
+                ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
+                ptx::mma_commit(&bars->s_full[g][b & 1]);
+                if (j == u.nb - 1) {
+                  ptx::mma_commit(&bars->q_empty[g][qr.slot]);
+                  ring_next(qr, nqb);
+                }
               }
-              const uint32_t e = b % 3;
-              pv_stage[e] = w.slot;
-              pv_acc[e] = j > 0 ? 1u : 0u;
-              pv_rel[e] = rel;
-              pv_nch[e] = (uint32_t)(block_rows(u, j) * u.lx + 15) >> 4;
-              // PV(b - 2): its P is written once the softmax of block b - 2 ends
-              if (b >= 2) ok = issue_pv(b - 2);
-              if (!ok) break;
             }
+            base = ring_adv(base, u.nb, nst);
+            t += ps.n;
           }
-          base = ring_adv(base, u.nb, nst);
-          t += ps.n;
+        } else {
+          constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
+          // [V | c] of V stage 0: the constant column block sits after the
+          // ring (N columns 32-47), at the leading byte offset; other stages
+          // and k-steps move the start address and shorten that offset.
+          const uint32_t va0 = ptx::smem_addr(kvbuf + kHalfStage), oa0 = ptx::smem_addr(ones);
+          const uint64_t vd0 = ptx::smem_desc(va0, oa0 - va0, 512, ptx::kSwizzle64B);
+          constexpr uint64_t kStageK = kStageBytes >> 4;
+          constexpr uint64_t kStageV = kStageK - (kStageK << 16);
+          // k-step kk of PV: V rows 16 kk.. (+1024 bytes), constant block unchanged
+          constexpr uint64_t kStepV = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
+          Ring base{0, 0};
+          uint32_t b = 0;
+          for (uint32_t t = t_begin; t < t_end && ok;) {
+            const Pass ps = pass_at(p, t, t_end);
+            const Unit& u = ps.u;
+            int last_i = -1;  // this warpgroup's last tile in the pass
+            for (int i = 0; i < ps.n; ++i)
+              if ((int)((t + i - t_begin) & 1u) == g) last_i = i;
+            for (int i = 0; i < ps.n && ok; ++i) {
+              if ((int)((t + i - t_begin) & 1u) != g) continue;
+              // a block used by this warpgroup's last tile of the pass is
+              // released after its PV; by both releases when the other
+              // warpgroup has no tile in the pass
+              const uint32_t rel = i == last_i ? (ps.n == 1 ? 2u : 1u) : 0u;
+              Ring w = base;
+              for (int j = 0; j < u.nb; ++j, ++b, ring_next(w, nst)) {
+                // PV(b): its P is written once the softmax has released it
+                ok = wait_bar(&bars->p_full[g][b & 1], (b >> 1) & 1, ctl);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint64_t vd = vd0 + w.slot * kStageV;
+                const uint32_t aP = tg + 128 + (b & 1) * 32;
+                const uint32_t nch = (uint32_t)(block_rows(u, j) * u.lx + 15) >> 4;
+                for (uint32_t kk = 0; kk < nch; ++kk)
+                  ptx::mma_ts(tg + 192, aP + kk * 8, vd + kk * kStepV, idPV, (kk > 0 || j > 0) ? 1u : 0u);
+                ptx::mma_commit(&bars->p_free[g][b & 1]);
+                for (uint32_t r = 0; r < rel; ++r) ptx::mma_commit(&bars->kv_empty[w.slot]);
+              }
+            }
+            base = ring_adv(base, u.nb, nst);
+            t += ps.n;
+          }
         }
-        for (uint32_t k = b >= 2 ? b - 2 : 0; ok && k < b; ++k) ok = issue_pv(k);
         // drain: every MMA this thread issued has completed before TMEM is freed
-        ptx::mma_commit(&bars->drain[g]);
-        wait_bar(&bars->drain[g], 0, drain);
+        const int di = s_role ? g : 2 + g;
+        ptx::mma_commit(&bars->drain[di]);
+        wait_bar(&bars->drain[di], 0, drain);
       }
-    } else if (warp == 12 || warp == 13) {
+    } else if (warp == 12) {
       // ============================================================ Q prep
-      // 64 threads; work in half rows (16 channels): the two halves of a row
+      // 32 threads; work in half rows (16 channels): the two halves of a row
       // sit in adjacent lanes, and each half of a RoPE row rotates along one
       // axis only.  Trip counts are uniform per warp (shuffles need all lanes).
-      const int pt = (int)threadIdx.x - 384;
+      const int pt = lane;
       Ring qr[2] = {{0, 0}, {0, 0}};
       bool ok = true;
       for (uint32_t t = t_begin; t < t_end && ok;) {
@@ -797,7 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       }
     } else {
       // ============================================================ K prep
-      const int pk = (int)threadIdx.x - 448;
+      const int pk = lane;
       Ring w{0, 0};
       bool ok = true;
       bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
