@@ -217,20 +217,6 @@ const char* swin_last_error(void);
  * normal operation.  Process-wide; not thread-safe against concurrent calls. */
 swin_status swin_debug_set(int flags, long long wait_limit_cycles);
 
-/* Test hook (no counterpart in the pages): the tensor-core kernel's launch
- * plan, computed on the host alone, so that host tests can replay the kernel's
- * barrier protocol over the real per-CTA work.  Arguments as
- * swin_window_attn_fwd (have_table: a bias table is used), sms = the number of
- * SMs to plan for.  plan (host int32, at least 10 + 257 entries) receives
- * nst (K/V ring stages), nqb (Q buffers per softmax warpgroup),
- * max_pass_tiles, n_ctas, shared-memory bytes, number of query tiles, R2e,
- * copy1, slot_floats, 0, then cta_start[0..n_ctas].  tiles (host int32, may
- * be NULL) receives per query tile t < max_tiles: head, image, x-class, y0,
- * ly, x0, lx, R, Rh, Rk, tiles of the rectangle, K/V blocks, tile index k.
- * Returns the plan's own errors (e.g. SWIN_ERR_UNSUPPORTED). */
-swin_status swin_debug_tc_plan(int B, int H, int W, int heads, int M, int shift, int mode, int have_table, int sms,
-                               int32_t* plan, int32_t* tiles, long long max_tiles);
-
 /* Library version, major * 10000 + minor * 100 + patch. */
 int swin_version(void);
 

@@ -57,39 +57,12 @@ def test_exp2_poly_exact_at_integers_within_bound_and_tiny_below_range():
 def _kernel_consts():
     src = open(SRC).read()
     env = {}
-    for name in ["kMaxStages", "kMaxQBuf", "kTileBytes", "kHalfStage", "kStageBytes", "kBlkKeys", "kSmemMax",
-                 "kSmemSlack", "kRopeBytes"]:
+    for name in ["kStages", "kTileBytes", "kBlk", "kQOff", "kKVOff", "kOnesOff", "kScaleOff", "kRopeOff",
+                 "kKofsOff", "kRposOff", "kKcolOff", "kSlotFloats", "kBiasOff", "kBarOff", "kNumBars",
+                 "kSmemBytes", "kCopy1"]:
         expr = re.search(r"constexpr int %s = ([^;]+);" % name, src).group(1)
         env[name] = eval(expr.split("//")[0], {}, env)
-    # struct Bars: q_full/q_ready/q_empty [2][kMaxQBuf], kv_* [kMaxStages], s/p full/free [2][2],
-    # tab_free/tab_ready [2], never, drain[n]
-    body = src[src.index("struct Bars {"):]
-    body = body[:body.index("};")]
-    assert body.count("uint64_t") == 5, body
-    n_drain = int(re.search(r"drain\[(\d+)\]", body).group(1))
-    env["kNumBars"] = 3 * 2 * env["kMaxQBuf"] + 3 * env["kMaxStages"] + 4 * 4 + 4 + 1 + n_drain
     return env
-
-
-def _layout(c, nqb, nst, rope, slot_floats):
-    """The kernel's tc_layout, replayed: byte offsets of the bias slots and the total."""
-    o = 2 * nqb * c["kTileBytes"] + nst * c["kStageBytes"] + 1024 + (c["kRopeBytes"] if rope else 0)
-    o += 2 * c["kMaxQBuf"] * 128 * 4 + nst * c["kBlkKeys"] * 4 + 3 * c["kBlkKeys"] * 4 * 2 + 3 * 128 * 4
-    bias = o
-    o += 2 * slot_floats * 4
-    bars = (o + 7) & ~7
-    total = bars + c["kNumBars"] * 8 + 16
-    return bias, total
-
-
-def test_layout_replay_matches_source():
-    """The replayed layout follows the source's field order (a change there must change this test)."""
-    src = open(SRC).read()
-    body = src[src.index("inline Layout tc_layout("):]
-    body = body[:body.index("return L;")]
-    order = re.findall(r"L\.(\w+) = ", body)
-    assert order == ["q", "kv", "ones", "rope", "qscale", "kcol", "kofs", "kpos", "qpos", "bias", "bars",
-                     "holder", "total"], order
 
 
 def _seg_len(k, L, M, s):
@@ -108,46 +81,41 @@ def test_bias_slot_reads_stay_inside_shared_memory():
     """The bias loads of the tensor-core softmax are unconditional (rows past
     the tile use row M-1; keys past the block read whatever sits there and are
     masked afterwards).  Replay their slot indices for every rectangle width,
-    tile, lane placement, block, lane and key of the workloads and test shapes,
-    for every row stride the host may choose, in both warpgroups' slots, with
-    the fewest ring stages the launch can get: each read must fall inside the
-    kernel's shared memory, and each paired load must be 8-byte aligned."""
+    tile, block, query lane and key of the workloads and test shapes, for every
+    row stride the host may choose, in both warpgroups' slots: each read must
+    fall inside the kernel's shared memory, and each paired load must be 8-byte
+    aligned."""
     c = _kernel_consts()
+    lo_lim = -c["kBiasOff"] // 4
+    hi_lim = (c["kSmemBytes"] - c["kBiasOff"]) // 4
     shapes = [(56, 56, 7, 3), (64, 64, 16, 8), (112, 112, 32, 16), (384, 384, 24, 12), (16, 16, 8, 4),
               (20, 13, 7, 3), (40, 36, 16, 8), (33, 70, 24, 12), (64, 64, 32, 16), (50, 45, 32, 5),
               (5, 130, 3, 1), (6, 7, 1, 0), (24, 24, 12, 6), (17, 23, 11, 10), (32, 32, 8, 4), (35, 30, 7, 3),
               (48, 40, 24, 12), (9, 200, 8, 4), (3, 3, 2, 1), (70, 64, 32, 0)]
-    lane = np.arange(128)[:, None, None]
-    col = np.arange(c["kBlkKeys"])[None, None, :]
+    t = np.arange(128)[:, None, None]
+    col = np.arange(96)[None, None, :]
     for H, W, M, s in shapes:
         lxs = {_seg_len(k, W, M, s) for k in range(_nseg(W, M, s))}
         lys = {_seg_len(k, H, M, s) for k in range(_nseg(H, M, s))}
         for R2e in range(2 * M, 2 * M + 15, 2):
-            copy1 = (2 * M - 1) * R2e + 16
-            slot_floats = copy1 + (2 * M - 1) * R2e
-            nst = 3  # fewest stages: the least shared memory before the slots
-            bias_off, total = _layout(c, 4, nst, False, slot_floats)
-            lo_lim, hi_lim = -bias_off // 4, (total - bias_off) // 4
+            if (2 * M - 1) * R2e > c["kSlotFloats"] - c["kCopy1"]:
+                break  # the host never picks it
             for lx in lxs:
-                R, Rh, Rk = 128 // lx, 64 // lx, c["kBlkKeys"] // lx
+                R, Rk = 128 // lx, 96 // lx
                 kofs = (col // lx) * R2e + col % lx
-                qpos_y, qpos_x = np.arange(128) // lx, np.arange(128) % lx
                 for ly in lys:
                     nb = (ly + Rk - 1) // Rk
                     j = np.arange(nb)[None, :, None]
                     for tile in range((ly + R - 1) // R):
-                        rows = min(R, ly - tile * R)
+                        qy, qx = tile * R + t // lx, t % lx
+                        bbase = (np.minimum(qy, M - 1) + M - 1) * R2e + qx + M - 1
+                        if lx % 2 == 0:
+                            e = bbase - 1 - j * Rk * R2e - kofs[:, :, 0::2]
+                            idx = np.where((bbase - 1) % 2 == 0, e, c["kCopy1"] + e - 1)
+                            assert np.all(idx % 2 == 0)
+                            idx = np.concatenate([idx, idx + 1], axis=2)
+                        else:
+                            idx = bbase - j * Rk * R2e - kofs
                         for g in (0, 1):
-                            loff = 64 * g if rows <= Rh else 0
-                            rr = np.clip(lane - loff, 0, 127)
-                            qy, qx = tile * R + qpos_y[rr], qpos_x[rr]
-                            bbase = (np.minimum(qy, M - 1) + M - 1) * R2e + qx + M - 1
-                            if lx % 2 == 0:
-                                e = bbase - 1 - j * Rk * R2e - kofs[:, :, 0::2]
-                                idx = np.where((bbase - 1) % 2 == 0, e, copy1 + e - 1)
-                                assert np.all(idx % 2 == 0)
-                                idx = np.concatenate([idx, idx + 1], axis=2)
-                            else:
-                                idx = bbase - j * Rk * R2e - kofs
-                            a = g * slot_floats + idx
-                            assert a.min() >= lo_lim and a.max() < hi_lim, (H, W, M, s, R2e, lx, ly, tile, g)
+                            a = g * c["kSlotFloats"] + idx
+                            assert a.min() >= lo_lim and a.max() < hi_lim, (H, W, M, s, R2e, lx, ly, tile)

@@ -7,69 +7,44 @@
 //   mode 1  cos(q,k)/max(tau,0.01) + T   same page, eq. 2 (§3.2, §3.3)
 //   mode 2  RoPE(q).RoPE(k)/sqrt(d)      FlashSwin abstract (window-local 2-D RoPE)
 // — without ever storing a score matrix: FlashSwin's point is that the
-// per-window score matrix is the memory problem; here S and P live only in
-// TMEM and O in TMEM until it is normalised and stored to its own token.
+// per-window score matrix is the memory problem; here S lives only in TMEM.
 //
-// Work.  One rectangle of one (image, head) is a unit.  Its queries are cut
-// into tiles of R = floor(128 / lx) whole rows (<= 128 queries, one TMEM lane
-// each), its keys into blocks of Rk = floor(64 / lx) whole rows (<= 64 keys).
-// The tiles of all units are listed heads outermost, then images, rows and
-// columns of rectangles; each persistent CTA takes a contiguous range of the
-// list (cut on the host so that the ranges carry equal work) and hands its
-// tiles alternately to its two softmax warpgroups.  Consecutive tiles of one
-// unit in a CTA's range form a pass: the unit's K/V blocks are loaded once per
-// pass into a ring of shared-memory stages, and every tile of the pass reads
-// them there.  When the ring holds all of a unit's blocks plus three, a pass
-// is every tile of the unit (the window's K/V stays resident while all its
-// query tiles go by); otherwise a pass is at most two tiles, one per
-// warpgroup, that stream the blocks together.
+// Work unit: two consecutive query tiles (tile = floor(128 / lx) whole
+// rectangle rows) of one row of rectangles, one per softmax warpgroup.  Tiles
+// of one rectangle share its K/V blocks of floor(96 / lx) rectangle rows (at
+// most 96 keys); tiles of two rectangles stream both rectangles' blocks.
 //
 // Warp roles (512 threads, one persistent CTA per SM):
-//   warp 0       K/V producer: TMA 5-D tile loads over [B][H][W][heads][d]
-//                (64-byte swizzle, no multicast) into the ring
-//   warp 3       Q producer: one TMA load per query tile into that tile's
-//                warpgroup's buffers (4, or 2 for long tiles)
-//   warps 1, 2   tcgen05.mma S issuers, one thread each: warp 1 + g issues
-//                the S = Q K^T MMAs of softmax warpgroup g; warp 1 owns TMEM
-//   warps 13, 15 tcgen05.mma PV issuers: warp 13 + 2g issues the O += P V
-//                MMAs of softmax warpgroup g
-//   warp 12      Q prep: 1/(tau |q|) per row (mode 1), RoPE of q (mode 2)
-//   warp 14      K prep: 1/|k| per key (mode 1), RoPE of k (mode 2), V to fp16
-//   warps 4-7    softmax of warpgroup 0 (one TMEM lane = one query row)
-//   warps 8-11   softmax of warpgroup 1
-//
-// TMEM per softmax warpgroup g (128 lanes, columns from 256 g): score buffers
-// S0, S1 (64 fp32 columns each), probability buffers P0, P1 (64 fp16 keys =
-// 32 columns each) and O (48 columns: 32 outputs and, in column 32, the row
-// sum of P).  Block b's S = Q K^T lands in S[b % 2]; the softmax copies it to
-// registers and frees the buffer at once, so the issuer computes S(b + 2)
-// while the softmax works on block b.  P(b) goes to P[b % 2], and
-// O += P(b) [V | c] reads it there (c = the constant column 1: the same MMAs
-// accumulate the row sum of exactly the fp16 probabilities that weight V).
-// The softmax waits for the tensor core only where a buffer comes back two
-// blocks later (PV(b - 2) done before P(b) is written), where it rescales O,
-// and where it reads a finished O.  S and PV MMAs of a warpgroup come from two
-// threads, so an S never queues behind a PV that waits for its probabilities.
-//
-// A query tile of at most 64 rows is placed in TMEM lanes 64-127 when it
-// belongs to warpgroup 1 (lanes 0-63 for warpgroup 0), so that small windows
-// keep all four SM sub-partitions busy; warps of a warpgroup without rows in
-// the tile follow the barrier protocol but skip the arithmetic.
+//   warp 0      TMA producer: Q tiles and K/V blocks, 5-D tensor maps over
+//               [B][H][W][heads][d] with 64-byte swizzle, no multicast
+//   warps 1, 2  tcgen05.mma issuers, one thread each: warp 1 + g issues the
+//               MMAs of softmax warpgroup g; warp 1 owns TMEM
+//   warps 3, 12-15  operand prep in shared memory: K unit-normalisation
+//               (mode 1), RoPE rotation of Q and K (mode 2), per-row
+//               1/(tau |q|) (mode 1), V to fp16
+//   warps 4-7   softmax of warpgroup 0 (one TMEM lane = one query row)
+//   warps 8-11  softmax of warpgroup 1
+// TMEM per softmax warpgroup g (128 lanes): two score buffers X0, X1 of 96
+// fp32 columns and O (48 columns: 32 outputs and, in column 32, the row sum
+// of P).  Block b's scores S = Q K^T land in X[b % 2]; the softmax turns them
+// into fp16 probabilities P written over the same columns, and O += P [V | c]
+// (6 MMAs, N = 48, A from TMEM) reads them there.  With two buffers the
+// softmax never waits for the previous block's PV; a thread's MMAs execute
+// in issue order, so S(b+2) cannot overwrite P(b) before PV(b) has read it.
 //
 // Softmax: online, with the running maximum kept until a block exceeds it by
 // more than 8 (log2 units), so O is rescaled rarely; P in fp16 (values up to
-// 2^8): fp16 keeps 3 more mantissa bits than bf16, which the output needs
-// (rounding P to bf16 gave about 9 times the output error of fp16).
-// Exponentials of the first keys of each block go through a polynomial on
-// the FMA pipe and the rest through the MUFU, in a ratio set by
-// the measured pipe rates (MUFU 16 exp2 per clock per SM, FMA pipe 128 lanes).
+// 2^8) keeps that accurate.  V is converted to fp16 by the prep warps; the
+// constant column c = 1 of [V | c] makes the same MMAs accumulate the row sum
+// of the fp16 P, so O / l uses exactly the probabilities that weighted V.
+// V entries of magnitude 65504 or more saturate and record
+// SWIN_ERR_UNSUPPORTED in the status word.
 //
-// Precision of the score operands: modes 0 and 1 multiply the bf16 inputs as
-// they are (mode 1 applies 1/|q|, 1/|k| and 1/tau in fp32 afterwards, so the
-// cosine is not rounded); mode 2 rotates q and k in fp32 and stores them as
-// fp16 (q scaled by a per-row power of two so that no finite input
-// overflows).  V is carried in fp16, the type of P.  A rotated k entry or a V
-// entry at or beyond 65504 saturates and records SWIN_ERR_UNSUPPORTED.
+// Precision of the score operands: mode 0 multiplies the bf16 inputs as they
+// are; mode 1 also multiplies the raw inputs and applies 1/|q| (per row),
+// 1/|k| (per column) and 1/tau in fp32 afterwards, so the cosine is not
+// rounded; mode 2 rotates q and k in fp32 and stores them as fp16 (scaled by
+// powers of two so that no finite input overflows), the largest error term.
 //
 // Every wait is bounded: on time-out the kernel records SWIN_ERR_TIMEOUT in
 // the status word, every role leaves its loop, in-flight copies and MMAs are
@@ -77,12 +52,15 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 
-#include <algorithm>
 #include <cstring>
-#include <vector>
 
 #include "sm100_ptx.cuh"
 #include "swin_common.cuh"
+
+// Phase markers for external timing builds; they compile to nothing here.
+#ifndef SWIN_TC_MARK
+#define SWIN_TC_MARK(k)
+#endif
 
 namespace swin {
 
@@ -95,7 +73,6 @@ struct FastDiv {
 
 inline FastDiv make_fastdiv(uint32_t d) {
   FastDiv f;
-  if (d == 0) d = 1;
   f.d = d;
   f.l = 0;
   while ((1ull << f.l) < d) ++f.l;
@@ -103,95 +80,21 @@ inline FastDiv make_fastdiv(uint32_t d) {
   return f;
 }
 
-__host__ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
-#ifdef __CUDA_ARCH__
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
   return (__umulhi(f.m, n) + n) >> f.l;
-#else
-  return (uint32_t)((((uint64_t)f.m * n) >> 32) + n) >> f.l;
-#endif
 }
-
-namespace {
-
-constexpr int kThreads = 512;
-constexpr int kMaxCtas = 256;
-constexpr int kMaxStages = 32;
-constexpr int kMaxQBuf = 4;
-constexpr int kTileBytes = 128 * 64;          // Q tile: 128 rows x 32 16-bit values
-constexpr int kHalfStage = 64 * 64;           // K or V block: 64 rows x 32 16-bit values
-constexpr int kStageBytes = 2 * kHalfStage;   // K then V
-constexpr int kBlkKeys = 64;                  // keys per K/V block (TMEM: 2 x 64 + 2 x 32 + 48 columns)
-constexpr int kPrepThreads = 32;              // Q prep: warp 12; K prep: warp 14
-constexpr int kSmemMax = 227 * 1024;
-constexpr int kSmemSlack = 1024;              // for the 1024-byte alignment of the base
-constexpr int kRopeBytes = 2 * 2 * 64 * 8 * 4;  // cos, sin [2 axes][64 positions][8]
-constexpr float kLog2eF = 1.4426950408889634f;
-
-struct Bars {
-  uint64_t q_full[2][kMaxQBuf], q_ready[2][kMaxQBuf], q_empty[2][kMaxQBuf];
-  uint64_t kv_full[kMaxStages], kv_ready[kMaxStages], kv_empty[kMaxStages];
-  // per warpgroup and buffer; a barrier's next phase needs a step its waiter
-  // has not taken yet, so parity waits never alias (see the softmax)
-  uint64_t s_full[2][2], s_free[2][2], p_full[2][2], p_free[2][2];
-  uint64_t tab_free[2], tab_ready[2];  // bias-table slot handshake of each softmax warpgroup (4 warps)
-  uint64_t never, drain[4];
-};
-constexpr int kNumBars = sizeof(Bars) / 8;
-
-// Shared-memory layout (byte offsets from the 1024-byte aligned base); the
-// same function sizes the launch on the host.
-struct Layout {
-  uint32_t q, kv, ones, rope, qscale, kcol, kofs, kpos, qpos, bias, bars, holder, total;
-};
-
-__host__ __device__ inline Layout tc_layout(int nqb, int nst, bool rope, int slot_floats) {
-  Layout L;
-  uint32_t o = 0;
-  L.q = o;
-  o += 2u * nqb * kTileBytes;
-  L.kv = o;
-  o += (uint32_t)nst * kStageBytes;
-  L.ones = o;  // 16 rows of [1, 0, ...]: the constant column block of [V | c]
-  o += 1024;
-  L.rope = o;
-  o += rope ? kRopeBytes : 0;
-  L.qscale = o;  // [2 warpgroups][kMaxQBuf][128] f32
-  o += 2 * kMaxQBuf * 128 * 4;
-  L.kcol = o;  // [stage][64] f32: 1/|k| (mode 1)
-  o += (uint32_t)nst * kBlkKeys * 4;
-  L.kofs = o;  // [3 classes][64] int: bias-slot offset of key c of a block
-  o += 3 * kBlkKeys * 4;
-  L.kpos = o;  // [3][64] int: (c / lx) | (c % lx) << 16
-  o += 3 * kBlkKeys * 4;
-  L.qpos = o;  // [3][128] int: (r / lx) | (r % lx) << 16
-  o += 3 * 128 * 4;
-  // Bias slots come after at least three ring stages: the unconditional bias
-  // loads of masked keys may read up to 64 slot rows before slot 0.
-  L.bias = o;
-  o += 2u * (uint32_t)slot_floats * 4;
-  L.bars = (o + 7) & ~7u;
-  o = L.bars + kNumBars * 8;
-  L.holder = o;  // TMEM base, abort flag, drain flag
-  o += 16;
-  L.total = o;
-  return L;
-}
-
-}  // namespace
 
 struct TcParams {
-  CUtensorMap tmq[3], tmqh[3], tmk[3], tmv[3];  // per x-class: Q (R rows), Q (Rh rows), K, V (Rk rows)
-  FastDiv div_img, div_B, div_rowmid, div_colmid[3];
-  int lx[3], R[3], Rh[3], Rk[3];    // per x-class: width, rows per Q tile / half tile / K-V block
-  int row_ly[3], row_tiles[3];      // per row class: height, tiles in one row of rectangles
-  int rect_tiles[3][3], rect_nb[3][3];
-  int nsy, nsx;
-  int B, H, W, heads, M, s;
-  int R2e, copy1, slot_floats;      // bias slot: row stride, offset of the shifted copy, floats per slot
-  int nst, nqb, max_pass_tiles;     // ring stages, Q buffers per warpgroup, tiles per pass
-  int n_ctas;
-  int cta_start[kMaxCtas + 1];      // CTA c takes tiles [cta_start[c], cta_start[c + 1])
+  CUtensorMap tmap[3][3];  // [tensor q/k/v][x-class first/middle/last]
+  FastDiv div_ipb, div_B, div_mid_items, div_mid_tiles[3];
+  int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
+  // per row class (first, middle, last row of rectangles): height, items,
+  // and per x-class the query tiles and K/V blocks of one rectangle
+  int row_ly[3], row_items[3], row_tiles[3][3], row_nb[3][3];
   void* out;
+  int B, H, W, heads, M, s, nsy, nsx;
+  int R2e;  // row stride of the bias slot (even, >= 2M - 1, chosen against bank conflicts)
+  long long n_items;
   const float* tau;
   const float* table;
   const float* rope;
@@ -202,148 +105,158 @@ struct TcParams {
 
 namespace {
 
-// One unit (rectangle of one (image, head)) and a pass over it.
-struct Unit {
-  int h, b, cls, y0, ly, x0, lx, R, Rh, Rk, ntile, nb;
+constexpr int kThreads = 512;
+constexpr int kPrepThreads = 160;  // warps 3 and 12-15
+constexpr int kStages = 6;                  // K/V ring
+constexpr int kTileBytes = 128 * 64;        // 128 rows x 32 16-bit values
+constexpr int kBlk = 96;                    // keys per K/V block (TMEM: 2 x 96 + 48 columns per warpgroup)
+constexpr int kQOff = 0;                    // [2 wg][2 buf] Q tiles
+constexpr int kKVOff = kQOff + 4 * kTileBytes;
+constexpr int kOnesOff = kKVOff + kStages * 2 * kTileBytes;   // per stage: 16 rows of [c, 0...] (1 KB)
+constexpr int kScaleOff = kOnesOff + kStages * 1024;         // [2][2][128] f32
+constexpr int kRopeOff = kScaleOff + 2 * 2 * 128 * 4;        // cos,sin [2][64][8] f32
+constexpr int kKofsOff = kRopeOff + 2 * 2 * 64 * 8 * 4;      // [3][128] int
+constexpr int kRposOff = kKofsOff + 3 * 128 * 4;             // [3][128] int: (r / lx) | (r % lx) << 16
+constexpr int kKcolOff = kRposOff + 3 * 128 * 4;             // [kStages][128] f32, 1/|k| (mode 1)
+// Relative-bias table of the current head, one slot per softmax warpgroup:
+// rows dy padded to an even stride 2M, stored twice (the second copy one
+// float ahead) so that every pair of adjacent keys is one aligned 8-byte load.
+constexpr int kSlotFloats = 8192;                            // two copies of (2M-1) rows fit for M <= 32
+constexpr int kCopy1 = kSlotFloats / 2 + 16;
+constexpr int kBiasOff = kKcolOff + kStages * 128 * 4;
+constexpr int kBarOff = kBiasOff + 2 * kSlotFloats * 4;
+constexpr int kNumBars = 12 + 3 * kStages + 12 + 3 + 4;
+constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 64;
+constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+
+constexpr float kLog2eF = 1.4426950408889634f;
+
+struct Bars {
+  uint64_t q_full[2][2], q_ready[2][2], q_empty[2][2];
+  uint64_t kv_full[kStages], kv_ready[kStages], kv_empty[kStages];
+  // per warpgroup and score buffer: a barrier's next phase (block b + 2) can
+  // only start after its current one was consumed, so parity tests never alias
+  uint64_t s_full[2][2], p_full[2][2], o_done[2][2];
+  uint64_t never, drain[2];
+  uint64_t tab_free[2], tab_ready[2];  // bias-table slot handshake of each softmax warpgroup (4 warps)
+};
+static_assert(sizeof(Bars) == kNumBars * 8, "barrier block size");
+
+// One warpgroup's query tile: its rectangle (a column segment of the item's
+// row of rectangles) and the tile's index in it.
+struct Rect {
+  int cls, lx, R, Rk, x0, tile, nb;  // x-class, width, tile rows, K/V block rows, first column, tile, K/V blocks
 };
 
-struct Pass {
-  Unit u;
-  int k0, n;  // tiles k0 .. k0 + n - 1 of the unit
+// A work item: query tiles 2i and 2i + 1 of one row of rectangles of one
+// (head, image), the row's tiles listed rectangle by rectangle.  Warpgroup 0
+// takes the first; warpgroup 1 the second, if the row has it.  Two tiles of
+// one rectangle share its K/V blocks; tiles of two rectangles stream both
+// rectangles' blocks, alternating (A0, B0, A1, B1, ...), then the longer one's
+// remainder, each block used by one warpgroup.
+struct Task {
+  int b, h, y0, ly;
+  bool v1;      // warpgroup 1 has a tile
+  bool shared;  // both tiles in one rectangle
+  int nbt;      // K/V blocks the item loads
+  Rect r0, r1;
+  __device__ __forceinline__ bool valid(int g) const { return g == 0 || v1; }
+  __device__ __forceinline__ Rect rect(int g) const { return g ? r1 : r0; }
+  __device__ __forceinline__ int nq(int g) const {  // queries of warpgroup g's tile
+    const Rect r = rect(g);
+    const int rows = ly - r.tile * r.R;
+    return (rows < r.R ? rows : r.R) * r.lx;
+  }
+  // position among the item's K/V loads of warpgroup g's block j
+  __device__ __forceinline__ int kv_index(int g, int j) const {
+    if (shared) return j;
+    const int mn = r0.nb < r1.nb ? r0.nb : r1.nb;
+    return j < mn ? 2 * j + g : mn + j;
+  }
+  // owner warpgroup (its rectangle) and block index of the item's K/V load jj
+  __device__ __forceinline__ Rect kv_rect(int jj, int& j) const {
+    const int mn = shared ? 0 : (r0.nb < r1.nb ? r0.nb : r1.nb);
+    if (jj < 2 * mn) {
+      j = jj >> 1;
+      return (jj & 1) ? r1 : r0;
+    }
+    j = jj - mn;
+    return (shared || r0.nb > r1.nb) ? r0 : r1;
+  }
 };
 
-__host__ __device__ __forceinline__ Unit decode_tile(const TcParams& p, uint32_t t, int& k) {
-  Unit u;
-  const uint32_t ih = fdiv(t, p.div_img);  // h * B + b
-  uint32_t rem = t - ih * p.div_img.d;
-  const uint32_t hq = fdiv(ih, p.div_B);
-  u.h = (int)hq;
-  u.b = (int)(ih - hq * p.div_B.d);
-  int sy, rc;
-  if (rem < (uint32_t)p.row_tiles[0]) {
-    sy = 0;
+__device__ __forceinline__ Task decode(const TcParams& p, long long item) {
+  Task t;
+  uint32_t i = (uint32_t)item;
+  uint32_t q = fdiv(i, p.div_ipb);
+  uint32_t rem = i - q * p.div_ipb.d;  // item within (head, image)
+  i = q;
+  q = fdiv(i, p.div_B);
+  t.b = (int)(i - q * p.div_B.d);
+  t.h = (int)q;  // heads outermost: a CTA keeps one head's bias table for many items
+  // row of rectangles: row 0, the nsy - 2 middle rows, the last row
+  int rc, sy;
+  uint32_t ii;
+  if (rem < (uint32_t)p.row_items[0]) {
     rc = 0;
+    sy = 0;
+    ii = rem;
   } else {
-    rem -= (uint32_t)p.row_tiles[0];
-    const uint32_t mid = p.nsy > 2 ? (uint32_t)(p.nsy - 2) * (uint32_t)p.row_tiles[1] : 0u;
+    rem -= (uint32_t)p.row_items[0];
+    const uint32_t mid = p.nsy > 2 ? (uint32_t)(p.nsy - 2) * (uint32_t)p.row_items[1] : 0u;
     if (rem < mid) {
-      const uint32_t r = fdiv(rem, p.div_rowmid);
-      sy = 1 + (int)r;
+      const uint32_t r = fdiv(rem, p.div_mid_items);
       rc = 1;
-      rem -= r * (uint32_t)p.row_tiles[1];
+      sy = 1 + (int)r;
+      ii = rem - r * (uint32_t)p.row_items[1];
     } else {
-      sy = p.nsy - 1;
       rc = 2;
-      rem -= mid;
+      sy = p.nsy - 1;
+      ii = rem - mid;
     }
   }
-  int sx, cls;
-  if (p.nsx == 1 || rem < (uint32_t)p.rect_tiles[rc][0]) {
-    sx = 0;
-    cls = 0;
+  t.y0 = swin_seg_start(sy, p.M, p.s);
+  t.ly = p.row_ly[rc];
+  const int T = p.nsx == 1 ? p.row_tiles[rc][0]
+                           : p.row_tiles[rc][0] + (p.nsx - 2) * p.row_tiles[rc][1] + p.row_tiles[rc][2];
+  // tile k of the row -> (column segment, tile)
+  auto tile_at = [&](int k, Rect& r) -> int {
+    int sx = 0;
+    const int t0 = p.row_tiles[rc][0];
+    if (p.nsx > 1 && k >= t0) {
+      k -= t0;
+      const int mid = (p.nsx - 2) * p.row_tiles[rc][1];
+      if (k < mid) {
+        const int r2 = (int)fdiv((uint32_t)k, p.div_mid_tiles[rc]);
+        sx = 1 + r2;
+        k -= r2 * p.row_tiles[rc][1];
+      } else {
+        sx = p.nsx - 1;
+        k -= mid;
+      }
+    }
+    r.cls = sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1);
+    r.lx = p.lx[r.cls];
+    r.R = p.R[r.cls];
+    r.Rk = p.Rk[r.cls];
+    r.x0 = swin_seg_start(sx, p.M, p.s);
+    r.tile = k;
+    r.nb = p.row_nb[rc][r.cls];
+    return sx;
+  };
+  const int sx0 = tile_at(2 * (int)ii, t.r0);
+  t.v1 = 2 * (int)ii + 1 < T;
+  int sx1 = -1;
+  if (t.v1) {
+    sx1 = tile_at(2 * (int)ii + 1, t.r1);
   } else {
-    rem -= (uint32_t)p.rect_tiles[rc][0];
-    const uint32_t mid = p.nsx > 2 ? (uint32_t)(p.nsx - 2) * (uint32_t)p.rect_tiles[rc][1] : 0u;
-    if (rem < mid) {
-      const uint32_t r = fdiv(rem, p.div_colmid[rc]);
-      sx = 1 + (int)r;
-      cls = 1;
-      rem -= r * (uint32_t)p.rect_tiles[rc][1];
-    } else {
-      sx = p.nsx - 1;
-      cls = 2;
-      rem -= mid;
-    }
+    t.r1 = t.r0;
+    t.r1.nb = 0;
   }
-  k = (int)rem;
-  u.cls = cls;
-  u.y0 = swin_seg_start(sy, p.M, p.s);
-  u.ly = p.row_ly[rc];
-  u.x0 = swin_seg_start(sx, p.M, p.s);
-  u.lx = p.lx[cls];
-  u.R = p.R[cls];
-  u.Rh = p.Rh[cls];
-  u.Rk = p.Rk[cls];
-  u.ntile = p.rect_tiles[rc][cls];
-  u.nb = p.rect_nb[rc][cls];
-  return u;
-}
-
-__device__ __forceinline__ Pass pass_at(const TcParams& p, uint32_t t, uint32_t t_end) {
-  Pass ps;
-  ps.u = decode_tile(p, t, ps.k0);
-  int n = ps.u.ntile - ps.k0;
-  n = min(n, (int)(t_end - t));
-  ps.n = min(n, p.max_pass_tiles);
-  return ps;
-}
-
-__device__ __forceinline__ int tile_rows(const Unit& u, int k) { return min(u.R, u.ly - k * u.R); }
-__device__ __forceinline__ bool tile_half(const Unit& u, int k) { return tile_rows(u, k) <= u.Rh; }
-__device__ __forceinline__ int block_rows(const Unit& u, int j) { return min(u.Rk, u.ly - j * u.Rk); }
-
-// Position in a ring of n slots: slot and the parity of the round.
-struct Ring {
-  uint32_t slot, ph;
-};
-__device__ __forceinline__ void ring_next(Ring& r, uint32_t n) {
-  if (++r.slot == n) {
-    r.slot = 0;
-    r.ph ^= 1u;
-  }
-}
-__device__ __forceinline__ Ring ring_adv(Ring r, uint32_t k, uint32_t n) {
-  const uint32_t s = r.slot + k, q = s / n;
-  r.slot = s - q * n;
-  r.ph ^= q & 1u;
-  return r;
-}
-
-// A softmax warpgroup's walk over its blocks: passes in order, the
-// warpgroup's tiles of each pass, the blocks of each tile.
-struct Walk {
-  uint32_t t;  // first tile of the current pass
-  Pass ps;
-  int i, j;    // tile of the pass, block of the tile
-  Ring base;   // ring position of the pass's block 0
-  bool valid;
-};
-
-// Move to the first tile of warpgroup g at or after tile i of the current pass.
-__device__ __forceinline__ void walk_seek(Walk& w, const TcParams& p, uint32_t t_begin, uint32_t t_end, int g,
-                                          uint32_t nst) {
-  while (true) {
-    while (w.i < w.ps.n && (int)((w.t + w.i - t_begin) & 1u) != g) ++w.i;
-    if (w.i < w.ps.n) return;
-    w.base = ring_adv(w.base, w.ps.u.nb, nst);
-    w.t += w.ps.n;
-    if (w.t >= t_end) {
-      w.valid = false;
-      return;
-    }
-    w.ps = pass_at(p, w.t, t_end);
-    w.i = 0;
-  }
-}
-
-__device__ __forceinline__ void walk_init(Walk& w, const TcParams& p, uint32_t t_begin, uint32_t t_end, int g,
-                                          uint32_t nst) {
-  w.t = t_begin;
-  w.base = Ring{0, 0};
-  w.i = w.j = 0;
-  w.valid = t_begin < t_end;
-  if (w.valid) {
-    w.ps = pass_at(p, t_begin, t_end);
-    walk_seek(w, p, t_begin, t_end, g, nst);
-  }
-}
-
-__device__ __forceinline__ void walk_next(Walk& w, const TcParams& p, uint32_t t_begin, uint32_t t_end, int g,
-                                          uint32_t nst) {
-  if (++w.j < w.ps.u.nb) return;
-  w.j = 0;
-  ++w.i;
-  walk_seek(w, p, t_begin, t_end, g, nst);
+  t.shared = sx1 == sx0;
+  t.nbt = t.shared ? t.r0.nb : t.r0.nb + t.r1.nb;
+  return t;
 }
 
 struct Ctl {
@@ -375,25 +288,13 @@ __device__ __forceinline__ uint32_t swz64(int row, int chunk) {
 __device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
-// Registers written by an asynchronous tcgen05.ld are only valid after
-// tcgen05.wait::ld; this empty asm "rewrites" them after the wait, so that no
-// use can be scheduled before it.
-__device__ __forceinline__ void reg_fence32(uint32_t* r) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
-                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31]));
-}
-
 // ------------------------------------------------------------------ prep
-// Mode 2 feeds the score MMA fp16 operands (both Q and K, one type): fp16
-// keeps 3 more mantissa bits than bf16, and rounding the rotated operands is
-// the largest error term of that mode.  A rotated Q row is first scaled by an
-// exact power of two that brings it below 2^15 (divided out in the softmax);
-// rotated K rows are converted with saturation, and an entry at or beyond the
-// fp16 range is reported as unsupported.
+// Score-prep operands go to the tensor core as fp16 (both Q and K, so the MMA
+// sees one type): fp16 keeps 3 more mantissa bits than bf16, and rounding the
+// rotated operands is the largest error term of the path.  A rotated Q row is
+// first scaled by an exact power of two that brings it below 2^15 (divided
+// out in the softmax); rotated K rows and V are converted with saturation,
+// and an entry at or beyond the fp16 range is reported as unsupported.
 
 // Half rows: channels [16 h, 16 h + 16) = 16-byte chunks 2h and 2h + 1.
 __device__ __forceinline__ void load_half_bf16(const uint8_t* tile, int row, int h, float (&v)[16]) {
@@ -436,34 +337,12 @@ __device__ __forceinline__ void rope_half(float (&v)[16], int h, int pos, const 
   }
 }
 
-__device__ __forceinline__ float half_absmax(const float (&v)[16]) {
-  float m = 0.f;
-#pragma unroll
-  for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
-  return m;
-}
-
-__device__ __forceinline__ float half_sumsq(const float (&v)[16]) {
-  float ss = 0.f;
-#pragma unroll
-  for (int e = 0; e < 16; ++e) ss = fmaf(v[e], v[e], ss);
-  return ss;
-}
-
-// Power of two that brings a row maximum m below 2^15 (fp16 max is 65504).
-__device__ __forceinline__ float pow2_scale(float m) {
-  if (!(m > 0.f)) return 1.f;
-  int e;
-  frexpf(m, &e);  // m < 2^e
-  return ldexpf(1.0f, 15 - e);
-}
-
 // 2^e for a pair on the FMA pipe, so that part of the exponentials leave the
 // MUFU: e = j + f with j = rint(e) read from the low mantissa bits of
 // e + 1.5 * 2^23 and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted by
 // the Remez exchange algorithm for minimax relative error on [-1/2, 1/2]
 // (7.5e-5, below half an fp16 ulp), and j is added to its exponent field.
-// Arguments below -125 are clamped (the result is then at most 2^-125).
+// Arguments below -125 are clamped (the result then rounds to 0 in fp16).
 __device__ __forceinline__ float2 exp2_poly2(float2 e) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   e.x = fmaxf(e.x, -125.0f);
@@ -478,19 +357,33 @@ __device__ __forceinline__ float2 exp2_poly2(float2 e) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
+__device__ __forceinline__ float half_absmax(const float (&v)[16]) {
+  float m = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m = fmaxf(m, fabsf(v[e]));
+  return m;
+}
+
+__device__ __forceinline__ float half_sumsq(const float (&v)[16]) {
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) ss = fmaf(v[e], v[e], ss);
+  return ss;
+}
+
+
+// Power of two that brings a row maximum m below 2^15 (fp16 max is 65504).
+__device__ __forceinline__ float pow2_scale(float m) {
+  if (!(m > 0.f)) return 1.f;
+  int e;
+  frexpf(m, &e);  // m < 2^e
+  return ldexpf(1.0f, 15 - e);
+}
+
 // How a launch adds the relative bias (a template argument, so that each
 // kernel carries only the code it runs): no table; pair loads (every
 // rectangle width of the launch even); one load per key (some width odd).
 enum BiasKind { kBiasNone = 0, kBiasPairs = 1, kBiasKeys = 2 };
-
-// Keys of a 64-key block whose exponentials go through the FMA-pipe
-// polynomial (the first ones; the rest, including any masked tail keys,
-// through the MUFU).  Mode 2 has no per-element bias work, so the FMA pipe
-// can take a larger share.
-template <int MODE>
-struct ExpSplit {
-  static constexpr int kPoly = MODE == 2 ? 24 : 16;
-};
 
 // ------------------------------------------------------------------ kernel
 template <int MODE, bool OUT_F32, int BIAS>
@@ -499,37 +392,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
   // 1024-byte alignment by pointer arithmetic on the shared array itself, so
   // that every access below stays a shared-space load or store
   uint8_t* smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
-  const int nst = p.nst, nqb = p.nqb;
-  constexpr bool has_table = MODE != 2 && BIAS != kBiasNone;
-  const Layout L = tc_layout(nqb, nst, MODE == 2, has_table ? p.slot_floats : 0);
-  uint8_t* qbuf = smem + L.q;
-  uint8_t* kvbuf = smem + L.kv;
-  uint8_t* ones = smem + L.ones;
-  float* rcos = reinterpret_cast<float*>(smem + L.rope);
+  uint8_t* qbuf = smem + kQOff;
+  uint8_t* kvbuf = smem + kKVOff;
+  uint8_t* ones = smem + kOnesOff;
+  float* qscale = reinterpret_cast<float*>(smem + kScaleOff);
+  float* rcos = reinterpret_cast<float*>(smem + kRopeOff);
   float* rsin = rcos + 2 * 64 * 8;
-  float* qscale = reinterpret_cast<float*>(smem + L.qscale);
-  float* kcol = reinterpret_cast<float*>(smem + L.kcol);
-  int* kofs = reinterpret_cast<int*>(smem + L.kofs);
-  int* kpos = reinterpret_cast<int*>(smem + L.kpos);
-  int* qpos = reinterpret_cast<int*>(smem + L.qpos);
-  float* sbias = reinterpret_cast<float*>(smem + L.bias);  // [2 warpgroups][slot_floats]
-  Bars* bars = reinterpret_cast<Bars*>(smem + L.bars);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L.holder);
+  int* kofs = reinterpret_cast<int*>(smem + kKofsOff);
+  int* rpos = reinterpret_cast<int*>(smem + kRposOff);
+  float* kcol = reinterpret_cast<float*>(smem + kKcolOff);
+  float* sbias = reinterpret_cast<float*>(smem + kBiasOff);  // [2 warpgroups][kSlotFloats]
+  Bars* bars = reinterpret_cast<Bars*>(smem + kBarOff);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + kBarOff + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int M = p.M, s = p.s;
-  const uint32_t t_begin = (uint32_t)p.cta_start[blockIdx.x], t_end = (uint32_t)p.cta_start[blockIdx.x + 1];
 
-  // ---- set-up: barriers, RoPE tables, index tables, constant column, TMEM
+  // ---- set-up: barriers, RoPE tables, bias tables and column offsets, TMEM
   if (threadIdx.x == 0) {
     for (int g = 0; g < 2; ++g)
-      for (int b = 0; b < kMaxQBuf; ++b) {
+      for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(&bars->q_full[g][b], 1);
         ptx::mbar_init(&bars->q_ready[g][b], kPrepThreads);
-        ptx::mbar_init(&bars->q_empty[g][b], 1 + 4);  // last S MMA of the tile + 4 softmax warps
+        ptx::mbar_init(&bars->q_empty[g][b], 1 + 4);
       }
-    for (int i = 0; i < kMaxStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       ptx::mbar_init(&bars->kv_full[i], 1);
       ptx::mbar_init(&bars->kv_ready[i], kPrepThreads);
       ptx::mbar_init(&bars->kv_empty[i], 2);  // one release per softmax warpgroup
@@ -537,20 +425,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     for (int g = 0; g < 2; ++g) {
       for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(&bars->s_full[g][b], 1);
-        ptx::mbar_init(&bars->s_free[g][b], 4);
-        ptx::mbar_init(&bars->p_full[g][b], 4);
-        ptx::mbar_init(&bars->p_free[g][b], 1);
+        ptx::mbar_init(&bars->p_full[g][b], 128);
+        ptx::mbar_init(&bars->o_done[g][b], 1);
       }
+    }
+    ptx::mbar_init(&bars->never, 1);
+    ptx::mbar_init(&bars->drain[0], 1);
+    ptx::mbar_init(&bars->drain[1], 1);
+    for (int g = 0; g < 2; ++g) {
       ptx::mbar_init(&bars->tab_free[g], 4);
       ptx::mbar_init(&bars->tab_ready[g], 4);
     }
-    ptx::mbar_init(&bars->never, 1);
-    for (int i = 0; i < 4; ++i) ptx::mbar_init(&bars->drain[i], 1);
     *abort_flag = 0;
     tmem_holder[2] = 0;  // abort flag of the drain waits (never set by a role)
     ptx::fence_mbar_init();
   }
   if (MODE == 2) {
+    // all 64 positions (rows past a rectangle's end, which are masked, read up to 63)
     for (int i = threadIdx.x; i < 2 * 64 * 8; i += kThreads) {
       const int axis = i / (64 * 8), pos = (i / 8) % 64, t = i % 8;
       float sv = 0.f, cv = 1.f;
@@ -559,251 +450,221 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       rsin[(axis * 64 + pos) * 8 + t] = sv;
     }
   }
+  const int R2e = p.R2e;
+  constexpr bool has_table = MODE != 2 && BIAS != kBiasNone;
   for (int i = threadIdx.x; i < 3 * 128; i += kThreads) {
-    const int c = i / 128, r = i % 128, lx = p.lx[c];
-    qpos[i] = (r / lx) | ((r % lx) << 16);
-    if (r < kBlkKeys) {
-      kofs[c * kBlkKeys + r] = (r / lx) * p.R2e + (r % lx);
-      kpos[c * kBlkKeys + r] = (r / lx) | ((r % lx) << 16);
-    }
+    const int c = i / 128, col = i % 128, lx = p.lx[c];
+    kofs[i] = (col / lx) * R2e + (col % lx);  // slot offset of key col
+    rpos[i] = (col / lx) | ((col % lx) << 16);
   }
-  // zero the K/V ring and the constant block once, so rows a block never
-  // writes hold finite values
-  for (int i = threadIdx.x; i < (nst * kStageBytes + 1024) / 16; i += kThreads)
+  // zero the K/V ring and the ones blocks once, so rows a tile never writes
+  // hold finite values
+  for (int i = threadIdx.x; i < (kStages * 2 * kTileBytes + kStages * 1024) / 16; i += kThreads)
     reinterpret_cast<uint4*>(kvbuf)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  // the constant column: fp16 1.0 in the first column of 16 rows
-  if (threadIdx.x < 16) *reinterpret_cast<uint16_t*>(ones + swz64(threadIdx.x, 0)) = 0x3C00;
+  // the constant column block of every stage: fp16 1.0 in the first column of 16 rows
+  if (threadIdx.x < 16 * kStages)
+    *reinterpret_cast<uint16_t*>(ones + (threadIdx.x / 16) * 1024 + swz64(threadIdx.x % 16, 0)) = 0x3C00;
   if (warp == 1) {
     ptx::tmem_alloc(tmem_holder, 512);
     ptx::tmem_relinquish();
   }
   if (warp == 0 && lane == 0)
-    for (int c = 0; c < 3; ++c) {
-      ptx::prefetch_tmap(&p.tmq[c]);
-      ptx::prefetch_tmap(&p.tmqh[c]);
-      ptx::prefetch_tmap(&p.tmk[c]);
-      ptx::prefetch_tmap(&p.tmv[c]);
-    }
+    for (int t = 0; t < 3; ++t)
+      for (int c = 0; c < 3; ++c) ptx::prefetch_tmap(&p.tmap[t][c]);
   ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   Ctl ctl{abort_flag, &p};
-  Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
+  const long long first = blockIdx.x, step = gridDim.x;
 
-  // Register split: warpgroups 0 (producers, issuers) and 3 (prep) give
+  // Register split: warpgroups 0 (producer, MMA, prep) and 3 (prep) give
   // registers to the two softmax warpgroups: 512 x 128 = 256 x 64 + 256 x 192.
   if (warp < 4 || warp >= 12) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
     if (warp == 0) {
-      // ============================================================ K/V producer
+      // ============================================================== producer
       if (lane == 0) {
-        Ring w{0, 0};
-        uint32_t loads = 0;
+        uint32_t qu[2] = {0, 0};
+        uint32_t ku = 0;
         bool ok = true;
-        for (uint32_t t = t_begin; t < t_end && ok;) {
-          const Pass ps = pass_at(p, t, t_end);
-          const Unit& u = ps.u;
-          for (int j = 0; j < u.nb && ok; ++j) {
-            if (loads >= (uint32_t)nst) ok = wait_bar(&bars->kv_empty[w.slot], w.ph ^ 1u, ctl);
+        for (long long it = first; it < p.n_items && ok; it += step) {
+          const Task t = decode(p, it);
+          for (int g = 0; g < 2 && ok; ++g) {
+            if (!t.valid(g)) continue;
+            const Rect r = t.rect(g);
+            const int qs = qu[g] & 1;
+            if (qu[g] >= 2) ok = wait_bar(&bars->q_empty[g][qs], ((qu[g] >> 1) - 1) & 1, ctl);
             if (!ok) break;
-            uint8_t* dst = kvbuf + w.slot * kStageBytes;
-            ptx::mbar_arrive_expect_tx(&bars->kv_full[w.slot], (uint32_t)(2 * 64 * u.lx * u.Rk));
-            ptx::tma_load_5d(dst, &p.tmk[u.cls], &bars->kv_full[w.slot], 0, u.h, u.x0, u.y0 + j * u.Rk, u.b);
-            ptx::tma_load_5d(dst + kHalfStage, &p.tmv[u.cls], &bars->kv_full[w.slot], 0, u.h, u.x0,
-                             u.y0 + j * u.Rk, u.b);
-            ring_next(w, nst);
-            ++loads;
+            ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], (uint32_t)(64 * r.lx * r.R));
+            ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][r.cls], &bars->q_full[g][qs], 0, t.h,
+                             r.x0, t.y0 + r.tile * r.R, t.b);
+            ++qu[g];
           }
-          t += ps.n;
-        }
-        // copies still landing in shared memory (after an abort; in a normal
-        // exit every one of them has been waited for by the K prep)
-        const uint32_t m = loads < (uint32_t)nst ? loads : (uint32_t)nst;
-        Ring d = ring_adv(Ring{0, 0}, loads - m, nst);
-        for (uint32_t i = 0; i < m; ++i, ring_next(d, nst)) wait_bar(&bars->kv_full[d.slot], d.ph, drain);
-      }
-    } else if (warp == 3) {
-      // ============================================================ Q producer
-      if (lane == 0) {
-        Ring qr[2] = {{0, 0}, {0, 0}};
-        uint32_t qn[2] = {0, 0};
-        bool ok = true;
-        for (uint32_t t = t_begin; t < t_end && ok;) {
-          const Pass ps = pass_at(p, t, t_end);
-          const Unit& u = ps.u;
-          for (int i = 0; i < ps.n && ok; ++i) {
-            const int g = (int)((t + i - t_begin) & 1u), k = ps.k0 + i;
-            if (qn[g] >= (uint32_t)nqb) ok = wait_bar(&bars->q_empty[g][qr[g].slot], qr[g].ph ^ 1u, ctl);
+          for (int jj = 0; jj < t.nbt && ok; ++jj) {
+            int j;
+            const Rect r = t.kv_rect(jj, j);
+            const int st = ku % kStages;
+            if (ku >= (uint32_t)kStages) ok = wait_bar(&bars->kv_empty[st], ((ku / kStages) - 1) & 1, ctl);
             if (!ok) break;
-            const bool half = tile_half(u, k);
-            uint8_t* dst = qbuf + (g * nqb + qr[g].slot) * kTileBytes + (half ? g * 4096 : 0);
-            ptx::mbar_arrive_expect_tx(&bars->q_full[g][qr[g].slot], (uint32_t)(64 * u.lx * (half ? u.Rh : u.R)));
-            ptx::tma_load_5d(dst, half ? &p.tmqh[u.cls] : &p.tmq[u.cls], &bars->q_full[g][qr[g].slot], 0, u.h,
-                             u.x0, u.y0 + k * u.R, u.b);
-            ring_next(qr[g], nqb);
-            ++qn[g];
+            uint8_t* kb = kvbuf + st * 2 * kTileBytes;
+            ptx::mbar_arrive_expect_tx(&bars->kv_full[st], (uint32_t)(2 * 64 * r.lx * r.Rk));
+            ptx::tma_load_5d(kb, &p.tmap[1][r.cls], &bars->kv_full[st], 0, t.h, r.x0, t.y0 + j * r.Rk, t.b);
+            ptx::tma_load_5d(kb + kTileBytes, &p.tmap[2][r.cls], &bars->kv_full[st], 0, t.h, r.x0,
+                             t.y0 + j * r.Rk, t.b);
+            ++ku;
           }
-          t += ps.n;
         }
-        for (int g = 0; g < 2; ++g) {
-          const uint32_t m = qn[g] < (uint32_t)nqb ? qn[g] : (uint32_t)nqb;
-          Ring d = ring_adv(Ring{0, 0}, qn[g] - m, nqb);
-          for (uint32_t i = 0; i < m; ++i, ring_next(d, nqb)) wait_bar(&bars->q_full[g][d.slot], d.ph, drain);
-        }
+        // drain copies that may still be landing in shared memory (after an
+        // abort; in a normal exit every phase waited here has completed)
+        Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
+        for (uint32_t u = (ku > (uint32_t)kStages ? ku - kStages : 0); u < ku; ++u)
+          wait_bar(&bars->kv_full[u % kStages], (u / kStages) & 1, drain);
+        for (int g = 0; g < 2; ++g)
+          for (uint32_t u = (qu[g] > 2 ? qu[g] - 2 : 0); u < qu[g]; ++u)
+            wait_bar(&bars->q_full[g][u & 1], (u >> 1) & 1, drain);
       }
-    } else if (warp == 1 || warp == 2 || warp == 13 || warp == 15) {
-      // ============================================================ MMA issuers
-      // Two issuer threads per softmax warpgroup g: warp 1 + g issues its S
-      // MMAs, warp 13 + 2g its PV MMAs.  S and PV never touch the same TMEM
-      // columns, and every dependence between them goes through the softmax
-      // (S(b) -> softmax -> P(b) -> PV(b)), so they need no common order: an
-      // S MMA never waits behind a PV whose probabilities are not written yet.
+    } else if (warp == 1 || warp == 2) {
+      // ============================================================== MMA issuers
+      // One thread per softmax warpgroup g (warp 1 + g) issues that group's
+      // MMAs in program order: S(0), S(1), then for every later block b first
+      // PV(b - 2), as soon as P(b - 2) is in TMEM, and then S(b).  A thread's
+      // MMAs execute in issue order, so S(b) cannot overwrite P(b - 2) before
+      // PV(b - 2) has read it.
       if (lane == 0) {
-        const bool s_role = warp < 4;
-        const int g = s_role ? warp - 1 : (warp - 13) >> 1;
+        const int g = warp - 1;
+        // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
+        constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
+        constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlk, 128);
+        constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
+        // Operand descriptors (64-byte swizzle) of Q buffer 0 and K/V stage 0;
+        // the others differ only in the start-address field (16-byte units)
+        // and, for [V | c], in the leading byte offset to the stage's constant
+        // column block, which sits outside the ring (N columns 32-47).
+        const uint64_t qd0 = ptx::smem_desc(ptx::smem_addr(qbuf + g * 2 * kTileBytes), 16, 512, ptx::kSwizzle64B);
+        const uint64_t kd0 = ptx::smem_desc(ptx::smem_addr(kvbuf), 16, 512, ptx::kSwizzle64B);
+        const uint32_t va0 = ptx::smem_addr(kvbuf + kTileBytes), oa0 = ptx::smem_addr(ones);
+        const uint64_t vd0 = ptx::smem_desc(va0, oa0 - va0, 512, ptx::kSwizzle64B);
+        constexpr uint64_t kQBuf = kTileBytes >> 4;
+        constexpr uint64_t kStageK = (2 * kTileBytes) >> 4;
+        constexpr uint64_t kStageV = kStageK - ((uint64_t)((2 * kTileBytes - 1024) >> 4) << 16);
+        // k-step kk of PV: V rows 16 kk.. (+1024 bytes), constant block unchanged
+        constexpr uint64_t kStepV = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
         const uint32_t tg = tmem_base + g * 256;
         bool ok = true;
-        if (s_role) {
-          // mode 2 feeds fp16 score operands (see prep), modes 0 and 1 the bf16 inputs
-          constexpr uint32_t fmtS = MODE == 2 ? 0u : 1u;
-          constexpr uint32_t idS = ptx::idesc_f16(fmtS, fmtS, 0, 0, kBlkKeys, 128);
-          // Operand descriptors (64-byte swizzle) of this warpgroup's Q buffer
-          // 0 and of K stage 0; the others differ only in the start-address
-          // field (16-byte units).
-          const uint64_t qd0 =
-              ptx::smem_desc(ptx::smem_addr(qbuf + g * nqb * kTileBytes), 16, 512, ptx::kSwizzle64B);
-          const uint64_t kd0 = ptx::smem_desc(ptx::smem_addr(kvbuf), 16, 512, ptx::kSwizzle64B);
-          constexpr uint64_t kQBuf = kTileBytes >> 4;
-          constexpr uint64_t kStageK = kStageBytes >> 4;
-          if (g == 0 && (p.debug_flags & 1)) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
-          Ring qr{0, 0}, base{0, 0};
-          uint32_t b = 0;
-          for (uint32_t t = t_begin; t < t_end && ok;) {
-            const Pass ps = pass_at(p, t, t_end);
-            const Unit& u = ps.u;
-            for (int i = 0; i < ps.n && ok; ++i) {
-              if ((int)((t + i - t_begin) & 1u) != g) continue;
-              Ring w = base;
-              for (int j = 0; j < u.nb; ++j, ++b, ring_next(w, nst)) {
-                // S(b) into S[b % 2]: the softmax has copied S(b - 2) out
-                if (b >= 2) ok = wait_bar(&bars->s_free[g][b & 1], ((b - 2) >> 1) & 1, ctl);
-                ok = ok && (j > 0 || wait_bar(&bars->q_ready[g][qr.slot], qr.ph, ctl)) &&
-                     wait_bar(&bars->kv_ready[w.slot], w.ph, ctl);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint64_t ad = qd0 + qr.slot * kQBuf, bd = kd0 + w.slot * kStageK;
-                const uint32_t dS = tg + (b & 1) * 64;
-                ptx::mma_ss(dS, ad, bd, idS, 0);
-                ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
-                ptx::mma_commit(&bars->s_full[g][b & 1]);
-                if (j == u.nb - 1) {
-                  ptx::mma_commit(&bars->q_empty[g][qr.slot]);
-                  ring_next(qr, nqb);
-                }
-              }
-            }
-            base = ring_adv(base, u.nb, nst);
-            t += ps.n;
-          }
-        } else {
-          constexpr uint32_t idPV = ptx::idesc_f16(0, 0, 0, 1, 48, 128);  // fp16 P (TMEM) x fp16 [V | c]
-          // [V | c] of V stage 0: the constant column block sits after the
-          // ring (N columns 32-47), at the leading byte offset; other stages
-          // and k-steps move the start address and shorten that offset.
-          const uint32_t va0 = ptx::smem_addr(kvbuf + kHalfStage), oa0 = ptx::smem_addr(ones);
-          const uint64_t vd0 = ptx::smem_desc(va0, oa0 - va0, 512, ptx::kSwizzle64B);
-          constexpr uint64_t kStageK = kStageBytes >> 4;
-          constexpr uint64_t kStageV = kStageK - (kStageK << 16);
-          // k-step kk of PV: V rows 16 kk.. (+1024 bytes), constant block unchanged
-          constexpr uint64_t kStepV = (uint64_t)(1024 >> 4) - ((uint64_t)(1024 >> 4) << 16);
-          Ring base{0, 0};
-          uint32_t b = 0;
-          for (uint32_t t = t_begin; t < t_end && ok;) {
-            const Pass ps = pass_at(p, t, t_end);
-            const Unit& u = ps.u;
-            int last_i = -1;  // this warpgroup's last tile in the pass
-            for (int i = 0; i < ps.n; ++i)
-              if ((int)((t + i - t_begin) & 1u) == g) last_i = i;
-            for (int i = 0; i < ps.n && ok; ++i) {
-              if ((int)((t + i - t_begin) & 1u) != g) continue;
-              // a block used by this warpgroup's last tile of the pass is
-              // released after its PV; by both releases when the other
-              // warpgroup has no tile in the pass
-              const uint32_t rel = i == last_i ? (ps.n == 1 ? 2u : 1u) : 0u;
-              Ring w = base;
-              for (int j = 0; j < u.nb; ++j, ++b, ring_next(w, nst)) {
-                // PV(b): its P is written once the softmax has released it
-                ok = wait_bar(&bars->p_full[g][b & 1], (b >> 1) & 1, ctl);
-                if (!ok) break;
-                ptx::tc_fence_after();
-                const uint64_t vd = vd0 + w.slot * kStageV;
-                const uint32_t aP = tg + 128 + (b & 1) * 32;
-                const uint32_t nch = (uint32_t)(block_rows(u, j) * u.lx + 15) >> 4;
-                for (uint32_t kk = 0; kk < nch; ++kk)
-                  ptx::mma_ts(tg + 192, aP + kk * 8, vd + kk * kStepV, idPV, (kk > 0 || j > 0) ? 1u : 0u);
-                ptx::mma_commit(&bars->p_free[g][b & 1]);
-                for (uint32_t r = 0; r < rel; ++r) ptx::mma_commit(&bars->kv_empty[w.slot]);
-              }
-            }
-            base = ring_adv(base, u.nb, nst);
-            t += ps.n;
+        if (p.debug_flags & 1) ok = wait_bar(&bars->never, 0, ctl);  // forced time-out
+        // blocks whose PV is still to be issued, by b & 1: stage | accumulate << 8 | second release << 9
+        uint32_t pend0 = 0, pend1 = 0;
+        auto issue_pv = [&](uint32_t k) -> bool {
+          if (!wait_bar(&bars->p_full[g][k & 1], (k >> 1) & 1, ctl)) return false;
+          ptx::tc_fence_after();
+          const uint32_t info = (k & 1) ? pend1 : pend0;
+          const uint32_t st = info & 0xffu;
+          const uint64_t vd = vd0 + st * kStageV;
+          const uint32_t aP = tg + (k & 1) * kBlk;
+          ptx::mma_ts(tg + 2 * kBlk, aP, vd, idPV, (info >> 8) & 1u);
+#pragma unroll
+          for (int kk = 1; kk < kBlk / 16; ++kk) ptx::mma_ts(tg + 2 * kBlk, aP + kk * 8, vd + kk * kStepV, idPV, 1u);
+          ptx::mma_commit(&bars->o_done[g][k & 1]);
+          ptx::mma_commit(&bars->kv_empty[st]);
+          if (info >> 9) ptx::mma_commit(&bars->kv_empty[st]);  // the other warpgroup has no tile here
+          return true;
+        };
+        // K/V uses (all items), Q tiles, S and PV issued by this group, K/V use of S(b - 1)
+        uint32_t u = 0, qcnt = 0, b = 0, npv = 0, u_last = 0;
+        for (long long it = first; it < p.n_items && ok; it += step) {
+          const Task t = decode(p, it);
+          const uint32_t u0 = u;
+          u += t.nbt;
+          if (!t.valid(g)) continue;
+          const uint32_t qs = qcnt & 1, qpar = (qcnt >> 1) & 1;
+          ++qcnt;
+          const uint64_t ad = qd0 + qs * kQBuf;
+          const int nb = t.rect(g).nb;
+          // a block used by this warpgroup alone takes both releases of its stage
+          const uint32_t rel2 = t.shared ? 0u : 512u;
+          for (int j = 0; j < nb; ++j, ++b) {
+            const uint32_t uu = u0 + t.kv_index(g, j), st = uu % kStages;
+            // S(b) overwrites P(b - 2): PV(b - 2) first
+            while (ok && npv + 2 <= b) ok = issue_pv(npv++);
+            // A pending PV(b - 1) whose K/V use is a whole ring behind block
+            // uu holds a slot the producer needs before it can load uu (or
+            // the next Q tile): issue it before waiting for either.
+            if (ok && npv < b && u_last + kStages <= uu) ok = issue_pv(npv++);
+            ok = ok && (j > 0 || wait_bar(&bars->q_ready[g][qs], qpar, ctl)) &&
+                 wait_bar(&bars->kv_ready[st], (uu / kStages) & 1, ctl);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const uint64_t bd = kd0 + st * kStageK;
+            const uint32_t dS = tg + (b & 1) * kBlk;
+            ptx::mma_ss(dS, ad, bd, idS, 0);
+            ptx::mma_ss(dS, ad + 2, bd + 2, idS, 1);  // second 16-wide K step: +32 bytes
+            ptx::mma_commit(&bars->s_full[g][b & 1]);
+            if (j == nb - 1) ptx::mma_commit(&bars->q_empty[g][qs]);
+            const uint32_t info = st | (j > 0 ? 256u : 0u) | rel2;
+            if (b & 1) pend1 = info; else pend0 = info;
+            u_last = uu;
           }
         }
+        while (ok && npv < b) ok = issue_pv(npv++);
         // drain: every MMA this thread issued has completed before TMEM is freed
-        const int di = s_role ? g : 2 + g;
-        ptx::mma_commit(&bars->drain[di]);
-        wait_bar(&bars->drain[di], 0, drain);
+        ptx::mma_commit(&bars->drain[g]);
+        Ctl drain{reinterpret_cast<volatile int*>(tmem_holder + 2), &p};
+        wait_bar(&bars->drain[g], 0, drain);
       }
-    } else if (warp == 12) {
-      // ============================================================ Q prep
-      // 32 threads; work in half rows (16 channels): the two halves of a row
-      // sit in adjacent lanes, and each half of a RoPE row rotates along one
-      // axis only.  Trip counts are uniform per warp (shuffles need all lanes).
-      const int pt = lane;
-      Ring qr[2] = {{0, 0}, {0, 0}};
+    } else {
+      // ============================================================== prep
+      // 160 threads (warps 3 and 12-15); work in half rows (16 channels):
+      // the two halves of a row sit in adjacent lanes, and each half of a
+      // RoPE row rotates along one axis only.
+      const int pt = warp < 4 ? (int)threadIdx.x - 96 : (int)threadIdx.x - 384 + 32;  // 0..159
+      uint32_t qu[2] = {0, 0}, ku = 0;
       bool ok = true;
-      for (uint32_t t = t_begin; t < t_end && ok;) {
-        const Pass ps = pass_at(p, t, t_end);
-        const Unit& u = ps.u;
-        const float te = MODE == 1 ? fmaxf(__ldg(p.tau + u.h), kTauMin) : 1.f;
-        const int* qp = qpos + u.cls * 128;
-        for (int i = 0; i < ps.n && ok; ++i) {
-          const int g = (int)((t + i - t_begin) & 1u), k = ps.k0 + i;
-          const uint32_t qs = qr[g].slot;
-          ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[g][qs], qr[g].ph, ctl));
-          ring_next(qr[g], nqb);
+      bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
+      for (long long it = first; it < p.n_items && ok; it += step) {
+        const Task t = decode(p, it);
+        // window-local coordinate of the row of rectangles' first row
+        const int py0 = swin_local_coord(t.y0, M, s);
+        for (int g = 0; g < 2 && ok; ++g) {
+          if (!t.valid(g)) continue;
+          const Rect rq = t.rect(g);
+          const int qrows = rq.lx * rq.R;
+          const int* rp = rpos + rq.cls * 128;
+          const int px0 = swin_local_coord(rq.x0, M, s);
+          const int qs = qu[g] & 1;
+          // warp-uniform outcome (the shuffles below need every lane)
+          ok = __all_sync(0xffffffffu, wait_bar(&bars->q_full[g][qs], (qu[g] >> 1) & 1, ctl));
+          ++qu[g];
           if (!ok) break;
+          uint8_t* tile = qbuf + (g * 2 + qs) * kTileBytes;
+          const float te = MODE == 1 ? fmaxf(__ldg(p.tau + t.h), kTauMin) : 1.f;
           if (MODE != 0) {
-            const int loff = tile_half(u, k) ? 64 * g : 0, nq = tile_rows(u, k) * u.lx;
-            uint8_t* tile = qbuf + (g * nqb + qs) * kTileBytes;
-            float* qsc = qscale + (g * kMaxQBuf + qs) * 128;
 #pragma unroll 1
-            for (int un = pt; un < 2 * 128; un += kPrepThreads) {
-              const int r = un >> 1, h = un & 1, row = loff + r;
-              const bool act = r < nq;
+            for (int u = pt; u < 2 * 128; u += kPrepThreads) {  // uniform trip count per lane pair
+              const int r = u >> 1, h = u & 1;
+              const bool act = r < qrows;
               float v[16];
-              if (act) load_half_bf16(tile, row, h, v);
+              if (act) load_half_bf16(tile, r, h, v);
               else for (int e = 0; e < 16; ++e) v[e] = 0.f;
               if (MODE == 1) {
                 float ss = half_sumsq(v);
                 ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if (act && h == 0) qsc[row] = kLog2eF / (fmaxf(sqrtf(ss), kNormEps) * te);
+                if (act && h == 0)
+                  qscale[(g * 2 + qs) * 128 + r] = kLog2eF / (fmaxf(sqrtf(ss), kNormEps) * te);
               } else {
                 if (act) {
-                  const int pr = qp[r];
-                  const int pos = h ? swin_local_coord(u.x0 + (pr >> 16), M, s)
-                                    : swin_local_coord(u.y0 + k * u.R + (pr & 0xFFFF), M, s);
-                  rope_half(v, h, pos, rcos, rsin);
+                  const int pr = rp[r];
+                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + rq.tile * rq.R + (pr & 0xFFFF), 63), rcos,
+                            rsin);
                 }
-                float mx = half_absmax(v);
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                const float sc = pow2_scale(mx);  // exact per-row scale, undone in the softmax
+                float m = half_absmax(v);
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                const float sc = pow2_scale(m);  // exact per-row scale, undone in the softmax
                 if (act) {
-                  store_half_f16(tile, row, h, v, sc);
-                  if (h == 0) qsc[row] = kLog2eF * rsqrtf(32.0f) / sc;
+                  store_half_f16(tile, r, h, v, sc);
+                  if (h == 0) qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
                 }
               }
             }
@@ -811,86 +672,69 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           }
           ptx::mbar_arrive(&bars->q_ready[g][qs]);
         }
-        t += ps.n;
-      }
-    } else {
-      // ============================================================ K prep
-      const int pk = lane;
-      Ring w{0, 0};
-      bool ok = true;
-      bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
-      for (uint32_t t = t_begin; t < t_end && ok;) {
-        const Pass ps = pass_at(p, t, t_end);
-        const Unit& u = ps.u;
-        const int* kp = kpos + u.cls * kBlkKeys;
-        for (int j = 0; j < u.nb && ok; ++j, ring_next(w, nst)) {
-          ok = __all_sync(0xffffffffu, wait_bar(&bars->kv_full[w.slot], w.ph, ctl));
+        for (int jj = 0; jj < t.nbt && ok; ++jj) {
+          int j;
+          const Rect rk = t.kv_rect(jj, j);
+          const int krows = rk.lx * rk.Rk;
+          const int* rp = rpos + rk.cls * 128;
+          const int px0 = swin_local_coord(rk.x0, M, s);
+          const int st = ku % kStages;
+          ok = __all_sync(0xffffffffu, wait_bar(&bars->kv_full[st], (ku / kStages) & 1, ctl));
+          ++ku;
           if (!ok) break;
-          {
-            const int nk = block_rows(u, j) * u.lx;
-            uint8_t* ktile = kvbuf + w.slot * kStageBytes;
-            uint8_t* vtile = ktile + kHalfStage;
-            // units: half h of K row r and half h of V row r (r < nk <= 64);
-            // fp16 with saturation, a saturated entry is reported after the
-            // loop.  Trip counts are uniform per warp (the shuffle needs all lanes).
+          uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
+          uint8_t* vtile = ktile + kTileBytes;
+          // units: half h of K row r and half h of V row r (r < krows <= 96);
+          // fp16 with saturation, a saturated entry is reported after the loop.
+          // Trip counts are uniform per warp (the shuffle below needs all lanes).
 #pragma unroll 1
-            for (int un = pk; un < 2 * kBlkKeys; un += kPrepThreads) {
-              const int r = un >> 1, h = un & 1;
-              const bool act = r < nk;
-              if (MODE != 0) {
-                float v[16];
-                if (act) load_half_bf16(ktile, r, h, v);
-                else for (int e = 0; e < 16; ++e) v[e] = 0.f;
-                if (MODE == 1) {
-                  float ss = half_sumsq(v);
-                  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                  if (act && h == 0) kcol[w.slot * kBlkKeys + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
-                } else if (act) {
-                  const int pr = kp[r];
-                  const int pos = h ? swin_local_coord(u.x0 + (pr >> 16), M, s)
-                                    : swin_local_coord(u.y0 + j * u.Rk + (pr & 0xFFFF), M, s);
-                  rope_half(v, h, pos, rcos, rsin);
-                  range_hit |= half_absmax(v) >= 65504.0f;
-                  store_half_f16(ktile, r, h, v, 1.0f);
-                }
-              }
-              if (act) {
-                float v[16];
-                load_half_bf16(vtile, r, h, v);
-                range_hit |= half_absmax(v) >= 65504.0f;
-                store_half_f16(vtile, r, h, v, 1.0f);
-              }
+          for (int un = pt; un < 2 * kBlk; un += kPrepThreads) {
+          const int r = un >> 1, h = un & 1;
+          const bool act = r < krows;
+          if (MODE != 0) {
+            float v[16];
+            if (act) load_half_bf16(ktile, r, h, v);
+            else for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            if (MODE == 1) {
+              float ss = half_sumsq(v);
+              ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+              if (act && h == 0) kcol[st * 128 + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
+            } else if (act) {
+              const int pr = rp[r];
+              rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + j * rk.Rk + (pr & 0xFFFF), 63), rcos, rsin);
+              range_hit |= half_absmax(v) >= 65504.0f;
+              store_half_f16(ktile, r, h, v, 1.0f);
             }
-            ptx::fence_proxy_async_smem();
           }
-          ptx::mbar_arrive(&bars->kv_ready[w.slot]);
+          if (act) {
+            float v[16];
+            load_half_bf16(vtile, r, h, v);
+            range_hit |= half_absmax(v) >= 65504.0f;
+            store_half_f16(vtile, r, h, v, 1.0f);
+          }
+          }
+          ptx::fence_proxy_async_smem();
+          ptx::mbar_arrive(&bars->kv_ready[st]);
         }
-        t += ps.n;
       }
       if (range_hit) atomicOr(p.status, (int)SWIN_ERR_UNSUPPORTED);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
     // ================================================================ softmax
-    // Software-pipelined over this warpgroup's blocks: while block b is
-    // computed from registers, S(b + 1) is already being copied out of TMEM
-    // into the other register set, and P(b)'s store lands while the next
-    // block starts (its p_full arrival is deferred to the top of block b + 1).
-    // O is touched (rescale, deferred epilogue) at the end of a block, after
-    // P(b) is stored, which leaves PV(b - 1) the most time to complete.  The
-    // loop body alternates the two register sets.
-    const int g = (warp - 4) >> 2;  // warpgroup 0 or 1
-    const int wq = warp & 3;        // TMEM lanes 32 wq .. 32 wq + 31
-    const uint32_t tX = tmem_base + g * 256 + ((uint32_t)(wq * 32) << 16);
-    const uint32_t tO = tX + 192;
+    const int g = (warp - 4) >> 2;              // warpgroup 0 or 1
+    const int t = threadIdx.x - 128 - g * 128;  // row of the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tX = tmem_base + g * 256 + lane_off;  // X0; X1 = tX + kBlk
+    const uint32_t tO = tX + 2 * kBlk;
     const float cscale = kLog2eF * rsqrtf(32.0f);
-    float* slot = sbias + g * p.slot_floats;
-    const int R2e = p.R2e, copy1 = p.copy1;
+    float* slot = sbias + g * kSlotFloats;
+    // second copy: slot[kCopy1 + i] = slot[i + 1], 16 banks away from the first
     int cur_h = -1;
     uint32_t tabn = 0;  // table loads of this warpgroup
-    Ring qr{0, 0};
+    uint32_t qu = 0, ku = 0, blk = 0;  // Q tiles, K/V uses, blocks of this warpgroup
     bool ok = true;
-    bool pend = false, pend_ok = false;  // a tile's O still waiting in TMEM (this warp's rows)
+    bool pend = false, pend_ok = false;  // an item's O still waiting in TMEM
     size_t pend_off = 0;
     // O / l of one row to global memory (32 values; column 32 holds l)
     auto store_rows = [&](const uint32_t (&o)[32], uint32_t l, size_t off, bool row_valid) {
@@ -915,306 +759,264 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         }
       }
     };
-    // PV completions: p_free[x] completes once per PV of a block b with
-    // b % 2 == x.  A wait for PV(k), k < the current block, cannot alias a
-    // later phase: PV(k + 2) needs P(k + 2), which this warp has not released.
-    uint32_t pv_done = 0;  // PVs of this warpgroup known complete
-    auto wait_pv = [&](uint32_t upto) -> bool {  // PV(0..upto) complete
+    // PV completion: o_done[parity] completes once per PV of that parity.
+    // The softmax waits on it only where O is read (rescale, deferred
+    // epilogue); every other completion is inferred: S(b)'s commit follows
+    // PV(b - 2)'s MMAs in the issuing thread, so s_full(b) implies that
+    // PV(0..b-2) are complete.  A parity wait for PV(k) cannot alias:
+    // PV(k + 2) needs P(k + 2), which this warpgroup has not written yet.
+    uint32_t o_cons = 0;  // PVs of this warpgroup known complete
+    auto consume_pv = [&](uint32_t upto) -> bool {  // PV(0..upto) complete
       bool r = true;
-      while (r && pv_done <= upto) {
-        r = wait_bar(&bars->p_free[g][pv_done & 1], (pv_done >> 1) & 1, ctl);
+      while (r && o_cons <= upto) {
+        r = wait_bar(&bars->o_done[g][o_cons & 1], (o_cons >> 1) & 1, ctl);
         r = __all_sync(0xffffffffu, r);
-        ++pv_done;
+        ++o_cons;
       }
       ptx::tc_fence_after();
       return r;
     };
-    // tile state
-    bool active = false, row_ok = false;
-    int qy = 0, qx = 0, bbase = 0;
-    float alpha = 0.f, m_run = -INFINITY;
-    const float* pbase = slot;
-    uint32_t b = 0;            // blocks of this warpgroup
-    bool p_pending = false;    // P(b - 1) stored; its p_full arrival not made yet
-    Walk wk;
-    walk_init(wk, p, t_begin, t_end, g, nst);
-    uint32_t n_blocks = 0;  // blocks of this warpgroup in the CTA's range
-    for (uint32_t t = t_begin; t < t_end;) {
-      const Pass ps = pass_at(p, t, t_end);
-      int mine = 0;
-      for (int i = 0; i < ps.n; ++i) mine += (int)((t + i - t_begin) & 1u) == g;
-      n_blocks += (uint32_t)(mine * ps.u.nb);
-      t += ps.n;
-    }
-    uint32_t xs[2][kBlkKeys];  // two register sets of scores (this block, the next)
-
-    auto arrive_p = [&]() {  // the deferred p_full of block b - 1
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&bars->p_full[g][(b - 1) & 1]);
-      p_pending = false;
-    };
-
-    if (wk.valid) {
-      // prologue: S(0) into registers
-      ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[g][0], 0, ctl));
-      if (ok) {
-        ptx::tc_fence_after();
-        ptx::tmem_ld32(tX, *reinterpret_cast<uint32_t(*)[32]>(&xs[0][0]));
-        ptx::tmem_ld32(tX + 32, *reinterpret_cast<uint32_t(*)[32]>(&xs[0][32]));
-        ptx::tmem_wait_ld();
-        reg_fence32(&xs[0][0]);
-        reg_fence32(&xs[0][32]);
-        ptx::tc_fence_before();
+    for (long long it = first; it < p.n_items && ok; it += step) {
+      const Task tk = decode(p, it);
+      const uint32_t ku0 = ku;
+      ku += tk.nbt;  // K/V loads of this item (both warpgroups)
+      if (!tk.valid(g)) continue;
+      const Rect rg = tk.rect(g);
+      if (has_table && tk.h != cur_h) {
+        // new head: once all four warps are done with the old table, each
+        // loads a quarter of the new one (times log2 e, zero padding column)
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->s_free[g][0]);
-      }
-    }
-#pragma unroll 1
-    while (ok && wk.valid) {
-      // two blocks per trip, so that the register sets alternate statically
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        if (ok && wk.valid) {
-          uint32_t* xc = xs[pp];
-          uint32_t* xn = xs[pp ^ 1];
-          const bool has_next = b + 1 < n_blocks;
-          if (has_next) {
-            // S(b + 1) was issued while block b - 1 was computed
-            ok = __all_sync(0xffffffffu, wait_bar(&bars->s_full[g][(b + 1) & 1], ((b + 1) >> 1) & 1, ctl));
-            if (ok) {
-              ptx::tc_fence_after();
-              const uint32_t tSn = tX + ((b + 1) & 1) * 64;
-              ptx::tmem_ld32(tSn, *reinterpret_cast<uint32_t(*)[32]>(xn));
-              ptx::tmem_ld32(tSn + 32, *reinterpret_cast<uint32_t(*)[32]>(xn + 32));
-            }
-          }
-          // the previous block's P store has had a block boundary to land:
-          // release it to the issuer
-          if (ok && p_pending) arrive_p();
-          const Unit& u = wk.ps.u;
-          const int j = wk.j;
-          if (ok && j == 0) {
-            // ---- new tile: bias table of its head, row scale, row position
-            if (has_table && u.h != cur_h) {
-              // new head: once all four warps are done with the old table,
-              // each loads a quarter of the new one (times log2 e, zero
-              // padding columns)
-              __syncwarp();
-              if (lane == 0) ptx::mbar_arrive(&bars->tab_free[g]);
-              ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_free[g], tabn & 1, ctl));
-              if (ok) {
-                const int n = (2 * M - 1) * R2e;
-                for (int i = wq * 32 + lane; i < n; i += 128) {
-                  const int dy = i / R2e, c = i - dy * R2e;
-                  const float v = c < 2 * M - 1
-                                      ? __ldg(p.table + (size_t)(dy * (2 * M - 1) + c) * p.heads + u.h) * kLog2eF
-                                      : 0.f;
-                  slot[i] = v;
-                  if (i > 0) slot[copy1 + i - 1] = v;
-                }
-                if (wq == 0 && lane == 0) slot[copy1 + n - 1] = 0.f;
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&bars->tab_ready[g]);
-                ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_ready[g], tabn & 1, ctl));
-                ++tabn;
-                cur_h = u.h;
-              }
-            }
-            const int k = wk.ps.k0 + wk.i;
-            const int loff = tile_half(u, k) ? 64 * g : 0, nq = tile_rows(u, k) * u.lx;
-            active = wq * 32 + 31 >= loff && wq * 32 < loff + nq;  // warp-uniform
-            const int r = wq * 32 + lane - loff;                    // query row in the tile
-            row_ok = r >= 0 && r < nq;
-            const int rr = min(max(r, 0), 127);
-            const int* qp = qpos + u.cls * 128;
-            qy = k * u.R + (qp[rr] & 0xFFFF);  // position in the rectangle
-            qx = qp[rr] >> 16;
-            const uint32_t qs = qr.slot;
-            if (ok && MODE != 0) ok = __all_sync(0xffffffffu, wait_bar(&bars->q_ready[g][qs], qr.ph, ctl));
-            // per-row score scale: mode 1 log2e / (tau |q|), mode 2 log2e / (sqrt(d) 2^e)
-            alpha = MODE == 0 ? cscale : qscale[(g * kMaxQBuf + qs) * 128 + wq * 32 + lane];
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
-            ring_next(qr, nqb);
-            // Slot index of this row's bias for key (0, 0) of the rectangle;
-            // the pair load for keys (2c, 2c+1) of a row starts one float
-            // earlier, in copy 0 when that index is even, else in copy 1 (the
-            // parity is fixed per query: row stride and even key offsets do
-            // not change it).  Bias loads are unconditional: rows past the
-            // tile use row M - 1, and keys past the block (masked below) read
-            // other slot entries, at most 64 rows of R2e floats before slot 0,
-            // inside shared memory.
-            bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
-            pbase = slot + (((bbase - 1) & 1) ? copy1 - 1 : 0) + bbase - 1;
-            m_run = -INFINITY;
-          }
-          const int nk = block_rows(u, j) * u.lx;
-          const int nch = (nk + 15) >> 4;
-          const uint32_t tP = tX + 128 + (b & 1) * 32;
-          float factor = 1.f;
-          bool rescale = false;
-          constexpr bool scale_in_exp = MODE == 2 || (MODE == 0 && !has_table);
-          const float ea = scale_in_exp ? alpha : 1.0f;
-          if (ok && active) {
-            const Ring w = ring_adv(wk.base, (uint32_t)j, nst);
-            if (MODE == 1) {
-              // 1/|k| of the block's keys was written by the K prep before kv_ready
-              ok = __all_sync(0xffffffffu, wait_bar(&bars->kv_ready[w.slot], w.ph, ctl));
-            }
-            // x = log2-domain logits.  Mode 2 (and mode 0 without a table):
-            // the scale is applied inside the exponent below (max over raw
-            // scores, scale > 0).  Otherwise x = S * scale + bias in one
-            // rounding; the bias slot holds T * log2(e), and mode 1's scale
-            // is log2e / (tau |q| |k|).
-            if (!scale_in_exp) {
-              const float4* kc4 = reinterpret_cast<const float4*>(kcol + w.slot * kBlkKeys);
-              const int4* kof4 = reinterpret_cast<const int4*>(kofs + u.cls * kBlkKeys);
-              const int jo = j * u.Rk * R2e;  // block j starts Rk rectangle rows further
-#pragma unroll
-              for (int c4 = 0; c4 < kBlkKeys / 4; ++c4) {
-                float2 s0 = make_float2(alpha, alpha), s1 = s0;
-                if (MODE == 1) {
-                  const float4 kc = kc4[c4];  // same address in every lane: broadcast
-                  s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
-                  s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
-                }
-                float2 b0 = make_float2(0.f, 0.f), b1 = b0;
-                if (BIAS == kBiasPairs) {
-                  const int4 ko = kof4[c4];  // broadcast; keys 4 c4 .. 4 c4 + 3 share a row pairwise
-                  const float2 v0 = *reinterpret_cast<const float2*>(pbase - jo - ko.x);  // (bias key+1, key)
-                  const float2 v1 = *reinterpret_cast<const float2*>(pbase - jo - ko.z);
-                  b0 = make_float2(v0.y, v0.x);
-                  b1 = make_float2(v1.y, v1.x);
-                } else if (BIAS == kBiasKeys) {
-                  // odd rectangle widths: one load per key
-                  const int4 ko = kof4[c4];
-                  const float* hb = slot + bbase - jo;
-                  b0 = make_float2(hb[-ko.x], hb[-ko.y]);
-                  b1 = make_float2(hb[-ko.z], hb[-ko.w]);
-                }
-                const float2 x0 = make_float2(__uint_as_float(xc[4 * c4]), __uint_as_float(xc[4 * c4 + 1]));
-                const float2 x1 = make_float2(__uint_as_float(xc[4 * c4 + 2]), __uint_as_float(xc[4 * c4 + 3]));
-                const float2 y0 = has_table ? __ffma2_rn(x0, s0, b0) : __fmul2_rn(x0, s0);
-                const float2 y1 = has_table ? __ffma2_rn(x1, s1, b1) : __fmul2_rn(x1, s1);
-                xc[4 * c4] = __float_as_uint(y0.x);
-                xc[4 * c4 + 1] = __float_as_uint(y0.y);
-                xc[4 * c4 + 2] = __float_as_uint(y1.x);
-                xc[4 * c4 + 3] = __float_as_uint(y1.y);
-              }
-            }
-            if (nk < kBlkKeys) {  // partial block (uniform across the warpgroup): mask the tail keys
-#pragma unroll
-              for (int c = 0; c < kBlkKeys; ++c)
-                if (c >= nk) xc[c] = __float_as_uint(-INFINITY);
-            }
-            // block maximum: four independent 3-input max chains
-            float mq[4] = {__uint_as_float(xc[0]), __uint_as_float(xc[1]), __uint_as_float(xc[2]),
-                           __uint_as_float(xc[3])};
-#pragma unroll
-            for (int c = 4; c < kBlkKeys; c += 4) {
-              const int chn = 2 * ((c >> 2) & 1);
-              mq[chn] = ptx::max3(mq[chn], __uint_as_float(xc[c]), __uint_as_float(xc[c + 2]));
-              mq[chn + 1] = ptx::max3(mq[chn + 1], __uint_as_float(xc[c + 1]), __uint_as_float(xc[c + 3]));
-            }
-            float mb = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-            if (scale_in_exp) mb *= ea;
-            // running maximum, kept unless this block exceeds it by more than 8
-            if (j == 0) {
-              m_run = mb;
-            } else if (mb > m_run + 8.0f) {
-              factor = ptx::ex2_approx(m_run - mb);
-              m_run = mb;
-              rescale = true;
-            }
-          }
-          // P[b % 2] is free once PV(b - 2) has read it
-          if (ok && b >= 2) ok = wait_pv(b - 2);
-          if (ok && active) {
-            // probabilities, fp16, 16 keys (8 columns) at a time: exponent
-            // argument x * ea - m
-            const float eb = -m_run;
-            constexpr int kPoly = ExpSplit<MODE>::kPoly;
-#pragma unroll
-            for (int ch = 0; ch < kBlkKeys / 16; ++ch) {
-              if (ch == 0 || ch < nch) {  // chunks past the block: PV never reads them
-                uint32_t pr[8];
-#pragma unroll
-                for (int e2 = 0; e2 < 8; ++e2) {
-                  const int c = ch * 16 + 2 * e2;
-                  const float2 e = __ffma2_rn(make_float2(__uint_as_float(xc[c]), __uint_as_float(xc[c + 1])),
-                                              make_float2(ea, ea), make_float2(eb, eb));
-                  if (c < kPoly) {
-                    const float2 pe = exp2_poly2(e);
-                    pr[e2] = ptx::pack_f16x2(pe.x, pe.y);
-                  } else {
-                    pr[e2] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
-                  }
-                }
-                ptx::tmem_st8(tP + ch * 8, pr);
-              }
-            }
-          }
-          p_pending = true;
-          // O (32 columns) and its row sum (column 32): rescaled to the new
-          // maximum, or, in a tile's first block, the previous tile's result
-          // read for the deferred store.  Both need PV(b - 1) complete, and
-          // both come before PV(b) (issued once p_full(b) is arrived, at the
-          // top of the next block).
-          const bool epi = j == 0 && pend;
-          const bool resc = j > 0 && __any_sync(0xffffffffu, rescale);
-          if (ok && (epi || resc)) {
-            ok = wait_pv(b - 1);
-            if (ok) {
-              uint32_t po[32];
-              ptx::tmem_ld32(tO, po);
-              uint32_t pl = ptx::tmem_ld1(tO + 32);
-              ptx::tmem_wait_ld();
-              reg_fence32(po);
-              asm volatile("" : "+r"(pl));
-              if (resc) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) po[e] = __float_as_uint(__uint_as_float(po[e]) * factor);
-                ptx::tmem_st32(tO, po);
-                ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
-              } else {
-                store_rows(po, pl, pend_off, pend_ok);
-                pend = false;
-              }
-            }
-          }
-          if (ok && has_next) {
-            // S(b + 1) is in registers: S[(b + 1) % 2] may take S(b + 3)
-            ptx::tmem_wait_ld();
-            reg_fence32(xn);
-            reg_fence32(xn + 32);
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&bars->s_free[g][(b + 1) & 1]);
-          }
-          if (j == u.nb - 1) {
-            // this tile's O is read in the next tile's first block (or after the loop)
-            pend = active;
-            pend_ok = row_ok;
-            pend_off = (((size_t)u.b * p.H + (u.y0 + qy)) * p.W + (u.x0 + qx)) * (size_t)(p.heads * 32) +
-                       (size_t)u.h * 32;
-          }
-          ++b;
-          walk_next(wk, p, t_begin, t_end, g, nst);
+        if (lane == 0) ptx::mbar_arrive(&bars->tab_free[g]);
+        ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_free[g], tabn & 1, ctl));
+        if (!ok) break;
+        const int n = (2 * M - 1) * R2e;
+        for (int i = (warp & 3) * 32 + lane; i < n; i += 128) {
+          const int dy = i / R2e, c = i - dy * R2e;
+          const float v = c < 2 * M - 1 ? __ldg(p.table + (size_t)(dy * (2 * M - 1) + c) * p.heads + tk.h) * kLog2eF : 0.f;
+          slot[i] = v;
+          if (i > 0) slot[kCopy1 + i - 1] = v;
         }
+        if (warp == 4 + 4 * g && lane == 0) slot[kCopy1 + n - 1] = 0.f;
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->tab_ready[g]);
+        ok = __all_sync(0xffffffffu, wait_bar(&bars->tab_ready[g], tabn & 1, ctl));
+        ++tabn;
+        if (!ok) break;
+        cur_h = tk.h;
       }
+      const int qs = qu & 1;
+      ok = wait_bar(&bars->q_ready[g][qs], (qu >> 1) & 1, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      ++qu;
+      if (!ok) break;
+      // per-row score scale: mode 1 log2e / (tau |q|), mode 2 log2e / (sqrt(d) 2^e)
+      const float alpha = MODE == 0 ? cscale : qscale[(g * 2 + qs) * 128 + t];
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&bars->q_empty[g][qs]);
+      const bool row_ok = t < tk.nq(g);
+      const int qy = rg.tile * rg.R + t / rg.lx, qx = t % rg.lx;
+      // Slot index of this row's bias for key (0, 0) of the rectangle; the
+      // pair load for keys (2c, 2c+1) of a row starts one float earlier, in
+      // copy 0 when that index is even, else in copy 1 (the parity is fixed
+      // per query: row stride and even key offsets do not change it).
+      // Bias loads are unconditional: rows past the tile use row M - 1, and
+      // keys past the block (masked below) read other slot entries, at
+      // most 95 rows of 2M floats before slot 0, inside shared memory.
+      const int bbase = (min(qy, M - 1) + M - 1) * R2e + (qx + M - 1);
+      const float* pbase = slot + (((bbase - 1) & 1) ? kCopy1 - 1 : 0) + bbase - 1;
+      const int* kof = kofs + rg.cls * 128;
+      float m_run = -INFINITY;
+      for (int j = 0; j < rg.nb; ++j, ++blk) {
+        SWIN_TC_MARK(0);
+        ok = wait_bar(&bars->s_full[g][blk & 1], (blk >> 1) & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        SWIN_TC_MARK(1);
+        ptx::tc_fence_after();
+        const uint32_t tS = tX + (blk & 1) * kBlk;
+        float2 x[kBlk / 2];  // scores as packed pairs (keys 2c, 2c+1)
+        {
+          uint32_t r0[32], r1[32], r2[32];
+          ptx::tmem_ld32(tS, r0);
+          ptx::tmem_ld32(tS + 32, r1);
+          ptx::tmem_ld32(tS + 64, r2);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            x[e] = make_float2(__uint_as_float(r0[2 * e]), __uint_as_float(r0[2 * e + 1]));
+            x[16 + e] = make_float2(__uint_as_float(r1[2 * e]), __uint_as_float(r1[2 * e + 1]));
+            x[32 + e] = make_float2(__uint_as_float(r2[2 * e]), __uint_as_float(r2[2 * e + 1]));
+          }
+        }
+        SWIN_TC_MARK(2);
+        const uint32_t u = ku0 + tk.kv_index(g, j), ust = u % kStages;
+        if (MODE == 1) {
+          // 1/|k| of the block's keys was written by prep before it released kv_ready
+          ok = wait_bar(&bars->kv_ready[ust], (u / kStages) & 1, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+        }
+        SWIN_TC_MARK(11);
+        const float ascale = alpha;
+        const int nk_all = (tk.ly - j * rg.Rk) * rg.lx;
+        const int nk = nk_all < rg.Rk * rg.lx ? nk_all : rg.Rk * rg.lx;
+        // x = log2-domain logits.  Mode 2: the scale is applied inside the
+        // exponent below (max over raw scores, scale > 0).  Modes 0/1:
+        // x = S * scale + bias in one rounding; the bias slot already holds
+        // T * log2(e), and mode 1's scale is log2e / (tau |q| |k|).
+        if (MODE != 2) {
+          const float4* kc4 = reinterpret_cast<const float4*>(kcol + ust * 128);
+          const int4* kof4 = reinterpret_cast<const int4*>(kof);
+          const int jo = j * rg.Rk * R2e;  // block j starts Rk rectangle rows further
+          if (!has_table) {
+            const float2 a2 = make_float2(ascale, ascale);
+#pragma unroll
+            for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+              float2 s0 = a2, s1 = a2;
+              if (MODE == 1) {
+                const float4 kc = kc4[c4];
+                s0 = __fmul2_rn(make_float2(kc.x, kc.y), a2);
+                s1 = __fmul2_rn(make_float2(kc.z, kc.w), a2);
+              }
+              x[2 * c4] = __fmul2_rn(x[2 * c4], s0);
+              x[2 * c4 + 1] = __fmul2_rn(x[2 * c4 + 1], s1);
+            }
+          } else if (BIAS == kBiasPairs) {
+            const float* pb = pbase - jo;
+#pragma unroll
+            for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+              float2 s0 = make_float2(ascale, ascale), s1 = s0;
+              if (MODE == 1) {
+                const float4 kc = kc4[c4];  // same address in every lane: broadcast
+                s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
+                s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
+              }
+              const int4 ko = kof4[c4];  // broadcast; keys 4 c4 .. 4 c4 + 3 share a row pairwise
+              const float2 b0 = *reinterpret_cast<const float2*>(pb - ko.x);  // (bias key+1, bias key)
+              const float2 b1 = *reinterpret_cast<const float2*>(pb - ko.z);
+              x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(b0.y, b0.x));
+              x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(b1.y, b1.x));
+            }
+          } else {
+            // odd rectangle widths: one load per key
+            const float* hb = slot + bbase - jo;
+#pragma unroll
+            for (int c4 = 0; c4 < kBlk / 4; ++c4) {
+              float2 s0 = make_float2(ascale, ascale), s1 = s0;
+              if (MODE == 1) {
+                const float4 kc = kc4[c4];
+                s0 = __fmul2_rn(make_float2(kc.x, kc.y), s0);
+                s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
+              }
+              const int4 ko = kof4[c4];
+              x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(hb[-ko.x], hb[-ko.y]));
+              x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(hb[-ko.z], hb[-ko.w]));
+            }
+          }
+        }
+        SWIN_TC_MARK(12);
+        if (nk < kBlk) {  // partial block (uniform across the warpgroup): mask the tail keys
+#pragma unroll
+          for (int c = 0; c < kBlk / 2; ++c) {
+            if (2 * c >= nk) x[c].x = -INFINITY;
+            if (2 * c + 1 >= nk) x[c].y = -INFINITY;
+          }
+        }
+        // block maximum: four independent 3-input max chains, two pairs a step
+        static_assert(kBlk % 4 == 0, "pairs are taken two at a time");
+        float mq[4] = {x[0].x, x[0].y, x[1].x, x[1].y};
+#pragma unroll
+        for (int c = 2; c < kBlk / 2; c += 2) {
+          const int ch = 2 * ((c >> 1) & 1);
+          mq[ch] = ptx::max3(mq[ch], x[c].x, x[c + 1].x);
+          mq[ch + 1] = ptx::max3(mq[ch + 1], x[c].y, x[c + 1].y);
+        }
+        float mb = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        if (MODE == 2) mb *= ascale;
+        SWIN_TC_MARK(3);
+        // running maximum, kept unless this block exceeds it by more than 8
+        float factor = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_run = mb;
+        } else if (mb > m_run + 8.0f) {
+          factor = ptx::ex2_approx(m_run - mb);
+          m_run = mb;
+          rescale = true;
+        }
+        if (blk >= 2 && o_cons < blk - 1) o_cons = blk - 1;  // PV(0..blk-2) done: s_full(blk) seen
+        SWIN_TC_MARK(4);
+        // probabilities, fp16; written over the scores after O is brought up to
+        // date, so the scores' registers are free by then.
+        // exponent argument: mode 2  x * ascale - m,  modes 0/1  x - m
+        const float ea = MODE == 2 ? ascale : 1.0f, eb = -m_run;
+        // keys 0-63 on the MUFU, stored to TMEM while keys 64-95 are done;
+        // mode 2 (no bias work, MUFU-bound) takes those through the
+        // polynomial on the FMA pipe
+        uint32_t pa[32], pb[16];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
+          pa[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+        }
+        ptx::tmem_st32(tS, pa);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float2 e = __ffma2_rn(x[32 + c], make_float2(ea, ea), make_float2(eb, eb));
+          if (MODE == 2) {
+            const float2 pe = exp2_poly2(e);
+            pb[c] = ptx::pack_f16x2(pe.x, pe.y);
+          } else {
+            pb[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
+          }
+        }
+        SWIN_TC_MARK(5);
+        // O (32 columns) and its row sum (column 32): rescaled to the new
+        // maximum, or, in an item's first block, the previous item's result
+        // read for the deferred store.  Both need PV(blk - 1) complete.
+        uint32_t po[32], pl = 0;
+        const bool epi = j == 0 && pend;
+        const bool resc = j > 0 && __any_sync(0xffffffffu, rescale);
+        if (epi || resc) {
+          ok = consume_pv(blk - 1);
+          if (!ok) break;
+          ptx::tmem_ld32(tO, po);
+          pl = ptx::tmem_ld1(tO + 32);
+          ptx::tmem_wait_ld();
+          if (resc) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) po[e] = __float_as_uint(__uint_as_float(po[e]) * factor);
+            ptx::tmem_st32(tO, po);
+            ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
+          }
+        }
+        ptx::tmem_st16(tS + 32, pb);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_full[g][blk & 1]);
+        SWIN_TC_MARK(6);
+        if (epi) {
+          store_rows(po, pl, pend_off, pend_ok);
+          pend = false;
+        }
+        SWIN_TC_MARK(7);
+      }
+      if (!ok) break;
+      // this item's O is read in the next item's first block (or after the loop)
+      SWIN_TC_MARK(8);
+      pend = true;
+      pend_ok = row_ok;
+      pend_off = (((size_t)tk.b * p.H + (tk.y0 + qy)) * p.W + (rg.x0 + qx)) * (size_t)(p.heads * 32) +
+                 (size_t)tk.h * 32;
+      SWIN_TC_MARK(10);
     }
-    if (ok && p_pending) arrive_p();
-    if (ok && pend && b > 0) {
-      ok = wait_pv(b - 1);
+    if (ok && pend) {
+      ok = consume_pv(blk - 1);
       if (ok) {
         uint32_t po[32];
         ptx::tmem_ld32(tO, po);
-        uint32_t pl = ptx::tmem_ld1(tO + 32);
+        const uint32_t pl = ptx::tmem_ld1(tO + 32);
         ptx::tmem_wait_ld();
-        reg_fence32(po);
-        asm volatile("" : "+r"(pl));
         store_rows(po, pl, pend_off, pend_ok);
       }
     }
@@ -1248,30 +1050,26 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Box of lx tokens x rows rectangle rows of one head (32 channels, 64 bytes).
-// A head's 64-byte chunks of neighbouring tokens are heads * 64 bytes apart,
-// so no L2 promotion: a wider fetch would bring in other heads' channels that
-// are used much later.
-bool encode_map(CUtensorMap* m, const void* base, const AttnArgs& a, int lx, int rows) {
+bool encode_map(CUtensorMap* m, const void* base, const AttnArgs& a, int lx, int R) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[5] = {32, (cuuint64_t)a.heads, (cuuint64_t)a.W, (cuuint64_t)a.H, (cuuint64_t)a.B};
   const cuuint64_t row = 64;  // bytes of one head
   const cuuint64_t strides[4] = {row, row * a.heads, row * a.heads * a.W, row * a.heads * a.W * a.H};
-  const cuuint32_t box[5] = {32, 1, (cuuint32_t)lx, (cuuint32_t)rows, 1};
+  const cuuint32_t box[5] = {32, 1, (cuuint32_t)lx, (cuuint32_t)R, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 template <int MODE, bool F32, int BIAS>
-swin_status launch_mode(const TcParams& p, int smem, cudaStream_t stream) {
+swin_status launch_mode(const TcParams& p, int grid, cudaStream_t stream) {
   auto k = attn_tc_kernel<MODE, F32, BIAS>;
-  cudaError_t ea = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t ea = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
   if (ea != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_tc smem attribute: %s", cudaGetErrorString(ea));
-  k<<<p.n_ctas, kThreads, smem, stream>>>(p);
+  k<<<grid, kThreads, kSmemAlloc, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_tc launch: %s", cudaGetErrorString(e));
   return SWIN_OK;
@@ -1287,68 +1085,55 @@ void tc_set_debug(int flags, long long wait_limit) {
   g_tc_wait_limit = wait_limit > 0 ? wait_limit : 4000000000ll;
 }
 
-// Everything about a launch that does not need the device: geometry, tile
-// list, ring and buffer counts, bias-slot layout, per-CTA ranges, shared
-// memory.  Tensor maps and pointers are filled in by launch_attn_tc.
-swin_status tc_plan(int B, int H, int W, int heads, int M, int shift, int mode, bool table, int sms, TcParams& p,
-                    int& smem, long long& n_tiles) {
-  if (M > 64) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs M <= 64");
-  if (table && M > 32) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path keeps a bias table only for M <= 32");
+swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream) {
+  if (a.d != 32) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs d == 32, got %d", a.d);
+  if (a.M > 64) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs M <= 64");
+  if (a.mode != 2 && a.table && (2 * a.M - 1) * (2 * a.M) > kSlotFloats - kCopy1)
+    return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path keeps a bias table only for M <= 32");
+  TcParams p;
   memset(&p, 0, sizeof(p));
-  p.B = B; p.H = H; p.W = W; p.heads = heads; p.M = M; p.s = shift;
-  p.nsy = swin_nseg(H, M, shift);
-  p.nsx = swin_nseg(W, M, shift);
-  // column classes: first, middle (if any), last segment
-  const int lxs[3] = {swin_seg_len(0, W, M, shift),
-                      p.nsx > 2 ? swin_seg_len(1, W, M, shift) : swin_seg_len(0, W, M, shift),
-                      swin_seg_len(p.nsx - 1, W, M, shift)};
+  p.B = a.B; p.H = a.H; p.W = a.W; p.heads = a.heads; p.M = a.M; p.s = a.shift;
+  p.nsy = swin_nseg(a.H, a.M, a.shift);
+  p.nsx = swin_nseg(a.W, a.M, a.shift);
+  const int lxs[3] = {swin_seg_len(0, a.W, a.M, a.shift),
+                      p.nsx > 2 ? swin_seg_len(1, a.W, a.M, a.shift) : swin_seg_len(0, a.W, a.M, a.shift),
+                      swin_seg_len(p.nsx - 1, a.W, a.M, a.shift)};
   for (int c = 0; c < 3; ++c) {
     p.lx[c] = lxs[c];
-    p.R[c] = 128 / lxs[c];         // query tile: whole rectangle rows, at most 128 queries
-    p.Rh[c] = 64 / lxs[c];         // a tile of at most 64 rows: the half-height box
-    p.Rk[c] = kBlkKeys / lxs[c];   // K/V block: whole rectangle rows, at most 64 keys
+    p.R[c] = 128 / lxs[c];    // query tile: whole rectangle rows, at most 128 queries
+    p.Rk[c] = kBlk / lxs[c];  // K/V block: whole rectangle rows, at most 96 keys
+    if (!encode_map(&p.tmap[0][c], a.q, a, p.lx[c], p.R[c]) ||
+        !encode_map(&p.tmap[1][c], a.k, a, p.lx[c], p.Rk[c]) ||
+        !encode_map(&p.tmap[2][c], a.v, a, p.lx[c], p.Rk[c]))
+      return fail(SWIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (lx=%d, R=%d)", p.lx[c], p.R[c]);
   }
-  // row classes: first, middle (if any), last row of rectangles
-  const int lys[3] = {swin_seg_len(0, H, M, shift),
-                      p.nsy > 2 ? swin_seg_len(1, H, M, shift) : swin_seg_len(0, H, M, shift),
-                      swin_seg_len(p.nsy - 1, H, M, shift)};
+  // rows of rectangles by class: first, middle (if any), last
+  const int lys[3] = {swin_seg_len(0, a.H, a.M, a.shift),
+                      p.nsy > 2 ? swin_seg_len(1, a.H, a.M, a.shift) : swin_seg_len(0, a.H, a.M, a.shift),
+                      swin_seg_len(p.nsy - 1, a.H, a.M, a.shift)};
   for (int rc = 0; rc < 3; ++rc) {
     p.row_ly[rc] = lys[rc];
     for (int c = 0; c < 3; ++c) {
-      p.rect_tiles[rc][c] = (lys[rc] + p.R[c] - 1) / p.R[c];
-      p.rect_nb[rc][c] = (lys[rc] + p.Rk[c] - 1) / p.Rk[c];
+      p.row_tiles[rc][c] = (lys[rc] + p.R[c] - 1) / p.R[c];
+      p.row_nb[rc][c] = (lys[rc] + p.Rk[c] - 1) / p.Rk[c];
     }
-    p.row_tiles[rc] = p.nsx == 1 ? p.rect_tiles[rc][0]
-                                 : p.rect_tiles[rc][0] + (p.nsx - 2) * p.rect_tiles[rc][1] + p.rect_tiles[rc][2];
+    const int T = p.nsx == 1 ? p.row_tiles[rc][0]
+                             : p.row_tiles[rc][0] + (p.nsx - 2) * p.row_tiles[rc][1] + p.row_tiles[rc][2];
+    p.row_items[rc] = (T + 1) / 2;
+    p.div_mid_tiles[rc] = make_fastdiv((uint32_t)p.row_tiles[rc][1]);
   }
-  auto row_cls = [&](int sy) { return sy == 0 ? 0 : (sy == p.nsy - 1 ? 2 : 1); };
-  auto col_cls = [&](int sx) { return sx == 0 ? 0 : (sx == p.nsx - 1 ? 2 : 1); };
-  // one representative segment of each class present: first, a middle one, last
-  const int rep_y[3] = {0, p.nsy > 2 ? 1 : 0, p.nsy - 1}, rep_x[3] = {0, p.nsx > 2 ? 1 : 0, p.nsx - 1};
-  int nb_max = 0;
-  for (int i = 0; i < 3; ++i)
-    for (int j = 0; j < 3; ++j) nb_max = std::max(nb_max, p.rect_nb[row_cls(rep_y[i])][col_cls(rep_x[j])]);
-  const long long t_img = (long long)p.row_tiles[0] + (p.nsy > 2 ? (long long)(p.nsy - 2) * p.row_tiles[1] : 0) +
-                          (p.nsy > 1 ? p.row_tiles[2] : 0);
-  n_tiles = t_img * B * heads;
-  if (n_tiles >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "too many query tiles (%lld)", n_tiles);
-  p.div_img = make_fastdiv((uint32_t)t_img);
-  p.div_B = make_fastdiv((uint32_t)B);
-  p.div_rowmid = make_fastdiv((uint32_t)p.row_tiles[1]);
-  for (int rc = 0; rc < 3; ++rc) p.div_colmid[rc] = make_fastdiv((uint32_t)p.rect_tiles[rc][1]);
-
-  // Bias slot: rows dy with an even stride R2e in [2M, 2M + 14], stored twice
-  // (the second copy one float ahead, copy1 floats further), so that the two
-  // keys of an even-width row pair are one aligned 8-byte load.  R2e is the
-  // candidate with the fewest shared-memory wavefronts for the paired loads
-  // of this launch's rectangle widths: a warp's 32 queries load 8 bytes each
-  // in two 16-lane phases; query (qy, qx) of a width-lx rectangle reads
-  // floats qy R2e + qx - 1 (+ copy1 - 1 when that is odd) and on.
-  p.R2e = 2 * M;
-  if (table) {
+  const long long ipb = (long long)p.row_items[0] + (p.nsy > 2 ? (long long)(p.nsy - 2) * p.row_items[1] : 0) +
+                        (p.nsy > 1 ? p.row_items[2] : 0);
+  // Bias-slot row stride: the even value in [2M, 2M + 14] (whose two copies fit
+  // the slot) with the fewest shared-memory wavefronts for the paired bias
+  // loads of this launch's rectangle widths.  A warp's 32 queries load 8
+  // bytes each in two 16-lane phases; query (qy, qx) of a width-lx rectangle
+  // reads floats qy R2e + qx - 1 (+ kCopy1 - 1 when that is odd) and on.
+  p.R2e = 2 * a.M;
+  if (a.mode != 2 && a.table) {
     long best = -1;
-    for (int r2 = 2 * M; r2 <= 2 * M + 14; r2 += 2) {
-      const int cp1 = (2 * M - 1) * r2 + 16;
+    for (int r2 = 2 * a.M; r2 <= 2 * a.M + 14; r2 += 2) {
+      if ((2 * a.M - 1) * r2 > kSlotFloats - kCopy1) break;
       long cost = 0;
       for (int c = 0; c < 3; ++c) {
         const int lx = p.lx[c];
@@ -1358,8 +1143,8 @@ swin_status tc_plan(int B, int H, int W, int heads, int M, int shift, int mode, 
             int hits[16] = {0}, mx = 0;
             for (int l = 0; l < 16; ++l) {
               const int t = w0 + 16 * ph + l, qy = t / lx, qx = t % lx;
-              int idx = qy * r2 + qx + M - 2;  // parity as in the kernel's bbase - 1
-              if (idx & 1) idx += cp1 - 1;
+              int idx = qy * r2 + qx + a.M - 2;  // parity as in the kernel's bbase - 1
+              if (idx & 1) idx += kCopy1 - 1;
               const int bank2 = (idx >> 1) & 15;
               mx = ++hits[bank2] > mx ? hits[bank2] : mx;
             }
@@ -1371,81 +1156,12 @@ swin_status tc_plan(int B, int H, int W, int heads, int M, int shift, int mode, 
         p.R2e = r2;
       }
     }
-    p.copy1 = (2 * M - 1) * p.R2e + 16;
-    p.slot_floats = p.copy1 + (2 * M - 1) * p.R2e;
   }
-
-  // Ring stages from the shared-memory budget; Q buffers: 4 per warpgroup
-  // for short tiles (few blocks), where loads must run further ahead.
-  p.nqb = nb_max <= 4 ? 4 : 2;
-  const int slot_f = table ? p.slot_floats : 0;
-  int nst = kMaxStages;
-  while (nst > 3 && tc_layout(p.nqb, nst, mode == 2, slot_f).total + kSmemSlack > (uint32_t)kSmemMax) --nst;
-  if (tc_layout(p.nqb, nst, mode == 2, slot_f).total + kSmemSlack > (uint32_t)kSmemMax)
-    return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path: shared memory does not fit (M=%d)", M);
-  p.nst = nst;
-  // a whole window resident per pass when the ring holds its blocks plus three
-  p.max_pass_tiles = nst >= nb_max + 3 ? (1 << 30) : 2;
-  smem = (int)tc_layout(p.nqb, nst, mode == 2, slot_f).total + kSmemSlack;
-
-  // Per-CTA tile ranges of equal work.  Work of a tile ~ its K/V blocks x the
-  // 16-key chunks the softmax evaluates x the warps with rows, plus a fixed
-  // cost per block and per tile; the list repeats per (head, image).
-  std::vector<double> pre(1, 0.0);
-  pre.reserve((size_t)t_img + 1);
-  for (int sy = 0; sy < p.nsy; ++sy) {
-    const int rc = row_cls(sy), ly = p.row_ly[rc];
-    for (int sx = 0; sx < p.nsx; ++sx) {
-      const int c = col_cls(sx), lx = p.lx[c];
-      for (int k = 0; k < p.rect_tiles[rc][c]; ++k) {
-        const int rows = std::min(p.R[c], ly - k * p.R[c]), nq = rows * lx;
-        double w = 60.0;
-        for (int j = 0; j < p.rect_nb[rc][c]; ++j) {
-          const int nk = std::min(p.Rk[c], ly - j * p.Rk[c]) * lx;
-          w += 16.0 * ((nk + 15) / 16) * ((nq + 31) / 32) + 40.0;
-        }
-        pre.push_back(pre.back() + w);
-      }
-    }
-  }
-  const int G = (int)std::min<long long>(std::min(sms, kMaxCtas), n_tiles);
-  const long long n_ih = (long long)B * heads;
-  const double w_img = pre.back(), total = w_img * (double)n_ih;
-  p.n_ctas = G;
-  p.cta_start[0] = 0;
-  for (int c = 1; c < G; ++c) {
-    const double target = total * c / G;
-    long long ih = (long long)(target / w_img);
-    double rem = target - (double)ih * w_img;
-    if (ih >= n_ih) {
-      ih = n_ih - 1;
-      rem = w_img;
-    }
-    const long long idx = std::lower_bound(pre.begin(), pre.end(), rem) - pre.begin();
-    long long start = ih * t_img + std::min<long long>(idx, t_img);
-    start = std::max<long long>(start, (long long)p.cta_start[c - 1] + 1);  // every CTA gets a tile
-    start = std::min<long long>(start, n_tiles - (G - c));
-    p.cta_start[c] = (int)start;
-  }
-  p.cta_start[G] = (int)n_tiles;
-  return SWIN_OK;
-}
-
-swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream) {
-  if (a.d != 32) return fail(SWIN_ERR_UNSUPPORTED, "tensor-core path needs d == 32, got %d", a.d);
-  const bool table = a.mode != 2 && a.table != nullptr;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  TcParams p;
-  int smem = 0;
-  long long n_tiles = 0;
-  swin_status st = tc_plan(a.B, a.H, a.W, a.heads, a.M, a.shift, a.mode, table, sms, p, smem, n_tiles);
-  if (st != SWIN_OK) return st;
-  for (int c = 0; c < 3; ++c)
-    if (!encode_map(&p.tmq[c], a.q, a, p.lx[c], p.R[c]) || !encode_map(&p.tmqh[c], a.q, a, p.lx[c], p.Rh[c]) ||
-        !encode_map(&p.tmk[c], a.k, a, p.lx[c], p.Rk[c]) || !encode_map(&p.tmv[c], a.v, a, p.lx[c], p.Rk[c]))
-      return fail(SWIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (lx=%d)", p.lx[c]);
+  p.n_items = (long long)a.B * a.heads * ipb;
+  if (p.n_items >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "too many work items (%lld)", p.n_items);
+  p.div_ipb = make_fastdiv((uint32_t)ipb);
+  p.div_mid_items = make_fastdiv((uint32_t)p.row_items[1]);
+  p.div_B = make_fastdiv((uint32_t)a.B);
   p.out = a.out;
   p.tau = a.tau;
   p.table = a.table;
@@ -1453,62 +1169,34 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   p.status = a.status;
   p.wait_limit = g_tc_wait_limit;
   p.debug_flags = g_tc_debug_flags;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)(p.n_items < sms ? p.n_items : sms);
   switch (a.mode) {
     case 0:
     case 1: {
       const bool all_even = !(p.lx[0] & 1) && !(p.lx[1] & 1) && !(p.lx[2] & 1);
-      const int kind = !table ? kBiasNone : (all_even ? kBiasPairs : kBiasKeys);
+      const int kind = !a.table ? kBiasNone : (all_even ? kBiasPairs : kBiasKeys);
 #define SWIN_TC_LAUNCH(MD)                                                                               \
   switch (kind) {                                                                                       \
     case kBiasNone:                                                                                     \
-      return f32_out ? launch_mode<MD, true, kBiasNone>(p, smem, stream)                                \
-                     : launch_mode<MD, false, kBiasNone>(p, smem, stream);                              \
+      return f32_out ? launch_mode<MD, true, kBiasNone>(p, grid, stream)                                \
+                     : launch_mode<MD, false, kBiasNone>(p, grid, stream);                              \
     case kBiasPairs:                                                                                    \
-      return f32_out ? launch_mode<MD, true, kBiasPairs>(p, smem, stream)                               \
-                     : launch_mode<MD, false, kBiasPairs>(p, smem, stream);                             \
+      return f32_out ? launch_mode<MD, true, kBiasPairs>(p, grid, stream)                               \
+                     : launch_mode<MD, false, kBiasPairs>(p, grid, stream);                             \
     default:                                                                                            \
-      return f32_out ? launch_mode<MD, true, kBiasKeys>(p, smem, stream)                                \
-                     : launch_mode<MD, false, kBiasKeys>(p, smem, stream);                              \
+      return f32_out ? launch_mode<MD, true, kBiasKeys>(p, grid, stream)                                \
+                     : launch_mode<MD, false, kBiasKeys>(p, grid, stream);                              \
   }
       if (a.mode == 0) SWIN_TC_LAUNCH(0)
       SWIN_TC_LAUNCH(1)
 #undef SWIN_TC_LAUNCH
     }
     default:
-      return f32_out ? launch_mode<2, true, kBiasNone>(p, smem, stream)
-                     : launch_mode<2, false, kBiasNone>(p, smem, stream);
+      return f32_out ? launch_mode<2, true, kBiasNone>(p, grid, stream) : launch_mode<2, false, kBiasNone>(p, grid, stream);
   }
 }
 
 }  // namespace swin
-
-// Test hook: the launch plan of the tensor-core kernel, computed on the host
-// only (no device needed).  plan[0..9] = nst, nqb, max_pass_tiles, n_ctas,
-// smem bytes, tiles, R2e, copy1, slot_floats, 0; plan[10..10+n_ctas] =
-// cta_start.  tiles (may be NULL) receives, per tile t < max_tiles, the
-// decoded unit: h, b, cls, y0, ly, x0, lx, R, Rh, Rk, ntile, nb, k.
-extern "C" swin_status swin_debug_tc_plan(int B, int H, int W, int heads, int M, int shift, int mode, int have_table,
-                                          int sms, int32_t* plan, int32_t* tiles, long long max_tiles) {
-  using namespace swin;
-  if (!plan || B < 1 || H < 1 || W < 1 || heads < 1 || M < 1 || shift < 0 || shift >= M || sms < 1 || mode < 0 ||
-      mode > 2)
-    return fail(SWIN_ERR_INVALID_ARG, "swin_debug_tc_plan: bad arguments");
-  TcParams p;
-  int smem = 0;
-  long long n_tiles = 0;
-  swin_status st = tc_plan(B, H, W, heads, M, shift, mode, mode != 2 && have_table, sms, p, smem, n_tiles);
-  if (st != SWIN_OK) return st;
-  const int32_t head[10] = {p.nst, p.nqb, p.max_pass_tiles, p.n_ctas, smem, (int32_t)n_tiles, p.R2e, p.copy1,
-                            p.slot_floats, 0};
-  memcpy(plan, head, sizeof(head));
-  for (int c = 0; c <= p.n_ctas; ++c) plan[10 + c] = p.cta_start[c];
-  if (tiles)
-    for (long long t = 0; t < n_tiles && t < max_tiles; ++t) {
-      int k = 0;
-      const Unit u = decode_tile(p, (uint32_t)t, k);
-      const int32_t row[13] = {u.h, u.b, u.cls, u.y0, u.ly, u.x0, u.lx, u.R, u.Rh, u.Rk, u.ntile, u.nb, k};
-      memcpy(tiles + 13 * t, row, sizeof(row));
-    }
-  return SWIN_OK;
-}
-

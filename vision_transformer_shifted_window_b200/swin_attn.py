@@ -36,7 +36,7 @@ SWIN_CPB_CODE = 1
 EXPORTED = ("swin_cpb_eval", "swin_cpb_eval_form", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
             "swin_window_attn_workspace_size",
             "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version",
-            "swin_debug_set", "swin_debug_tc_plan")
+            "swin_debug_set")
 
 
 class SwinError(RuntimeError):
@@ -83,8 +83,6 @@ def lib():
         L.swin_last_error.restype = ctypes.c_char_p
         L.swin_debug_set.argtypes = [i, ctypes.c_longlong]
         L.swin_debug_set.restype = i
-        L.swin_debug_tc_plan.argtypes = [i] * 9 + [vp, vp, ctypes.c_longlong]
-        L.swin_debug_tc_plan.restype = i
         L.swin_version.argtypes = []
         L.swin_version.restype = i
         _lib = L
@@ -157,27 +155,6 @@ def _param_shapes(M: int, heads: int, d: int, tau, bias_table, rope_freqs) -> No
 def swin_debug_set(flags: int, wait_limit_cycles: int = 0) -> None:
     """Failure-path test hook (see include/swin_attn.h)."""
     _check(lib().swin_debug_set(int(flags), int(wait_limit_cycles)))
-
-
-def swin_debug_tc_plan(B: int, H: int, W: int, heads: int, M: int, shift: int, mode: int, have_table: bool,
-                       sms: int = 148, with_tiles: bool = True):
-    """Host-only launch plan of the tensor-core kernel (test hook, see
-    include/swin_attn.h): (dict of plan values, int32 [n_tiles, 13] tile table or None)."""
-    import numpy as np
-    plan = np.zeros(10 + 257, dtype=np.int32)
-    _check(lib().swin_debug_tc_plan(B, H, W, heads, M, shift, mode, int(bool(have_table)), sms,
-                                    plan.ctypes.data_as(ctypes.c_void_p), None, 0))
-    n_ctas, n_tiles = int(plan[3]), int(plan[5])
-    tiles = None
-    if with_tiles:
-        tiles = np.zeros((n_tiles, 13), dtype=np.int32)
-        _check(lib().swin_debug_tc_plan(B, H, W, heads, M, shift, mode, int(bool(have_table)), sms,
-                                        plan.ctypes.data_as(ctypes.c_void_p), tiles.ctypes.data_as(ctypes.c_void_p),
-                                        n_tiles))
-    keys = ("nst", "nqb", "max_pass_tiles", "n_ctas", "smem", "n_tiles", "R2e", "copy1", "slot_floats")
-    d = {k: int(plan[i]) for i, k in enumerate(keys)}
-    d["cta_start"] = [int(v) for v in plan[10:10 + n_ctas + 1]]
-    return d, tiles
 
 
 def swin_version() -> int:
