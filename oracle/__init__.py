@@ -14,6 +14,8 @@ Every function states the passage it follows:
 * ``cpb_table`` / ``log_coords`` — "Swin Transformer V2", Method §3.3, eq. 3 and
   eq. 4, ``continuous_bias`` pseudocode; hidden width 512 from the
   hyperparameter table's note on the code.
+* ``window_attn_bwd`` — the gradients of ``window_attn`` (chain rule through
+  the same definition; see the C source for the formulas).
 * ``index_tables`` — the Swin bookkeeping (window, band, local index, relative
   index) built by literally rolling a padded grid.
 """
@@ -69,6 +71,8 @@ def _load():
             [dp] * 4 + [ctypes.c_int] * 8 + [dp] * 3 + [lp, ctypes.c_int64, ctypes.c_int]
         )
         lib.oracle_window_attn.restype = ctypes.c_int
+        lib.oracle_window_attn_bwd.argtypes = ([dp] * 10 + [ctypes.c_int] * 8 + [dp] * 3 + [ctypes.c_int])
+        lib.oracle_window_attn_bwd.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -196,4 +200,33 @@ def window_attn(q, k, v, M: int, shift: int, mode: int, tau=None, table=None,
     )
     if rc != 0:
         raise ValueError("oracle_window_attn rejected its arguments")
+    return out
+
+
+def window_attn_bwd(q, k, v, dout, M: int, shift: int, mode: int, tau=None, table=None, rope_freqs=None,
+                    nthreads: int = 0) -> dict:
+    """Gradients of L = sum(dout * window_attn(...)) in float64: dq, dk, dv
+    ([B, H, W, heads, d]), dtable ([(2M-1)^2, heads], modes 0 and 1), dtau
+    ([heads], mode 1), drope ([2, d/4], mode 2)."""
+    q, k, v, dout = (_f64(a) for a in (q, k, v, dout))
+    B, H, W, heads, d = q.shape
+    assert k.shape == q.shape and v.shape == q.shape and dout.shape == q.shape
+    tau, table, rope_freqs = _f64(tau), _f64(table), _f64(rope_freqs)
+    R = 2 * M - 1
+    dq, dk, dv = (np.zeros_like(q) for _ in range(3))
+    dtable = np.zeros((R * R, heads)) if mode != 2 else None
+    dtau = np.zeros(heads) if mode == 1 else None
+    drope = np.zeros((2, d // 4)) if mode == 2 else None
+    rc = _load().oracle_window_attn_bwd(
+        _dp(q), _dp(k), _dp(v), _dp(dout), _dp(dq), _dp(dk), _dp(dv), _dp(dtable), _dp(dtau), _dp(drope),
+        B, H, W, heads, d, M, shift, mode, _dp(tau), _dp(table), _dp(rope_freqs), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_window_attn_bwd rejected its arguments")
+    out = {"dq": dq, "dk": dk, "dv": dv}
+    if dtable is not None:
+        out["dtable"] = dtable
+    if dtau is not None:
+        out["dtau"] = dtau
+    if drope is not None:
+        out["drope"] = drope
     return out

@@ -45,9 +45,13 @@
  *      inside each half rotate by p * omega[axis][t], t < d/4; the window-local
  *      coordinate is p = (y - s) mod M; RoPE touches q and k only; the score
  *      is scaled by 1/sqrt(d); no bias.
- *  R11 The code form of G ([V2] "Paper vs code"): the normaliser is the
+ *  R15 The code form of G ([V2] "Paper vs code"): the normaliser is the
  *      pretrained window Mp (the window itself when none is given); a window
  *      of 1 (Mp - 1 = 0) has only offset 0, whose coordinate is 0.
+ *  R16 Gradients (the pages train the model but state no backward): the
+ *      chain rule through the definitions above; the tau clamp passes the
+ *      gradient for tau >= 0.01 and none below; a norm held at its 1e-12
+ *      floor is a constant.
  *
  * Parity pins live in tests/test_oracle_*.py.  The CPB meta-network beyond
  * its W2 = 0 special case and a float64 library Linear stack is arithmetic
@@ -317,6 +321,228 @@ int oracle_window_attn(const double* q, const double* k, const double* v, double
             }
         }
         free(ky); free(kx); free(logit); free(qi); free(kj);
+    }
+    return 0;
+}
+
+/* Gradients of the shifted-window attention (the chain rule through the
+ * forward above, written out; the softmax is recomputed, nothing is stored
+ * between passes).  With L = sum(dout . out), P the softmax weights of query
+ * i over its key set, g_i = dout_i:
+ *   dv_j   = sum_i P_ij g_i
+ *   dP_ij  = g_i . v_j,   D_i = sum_j P_ij dP_ij,   dl_ij = P_ij (dP_ij - D_i)
+ * and dl_ij flows into the score:
+ *   mode 0  l = q.k/sqrt(d) + T[r]:  dq_i += dl k_j/sqrt(d), dk_j += dl q_i/sqrt(d), dT[r] += dl
+ *   mode 1  l = c/t + T[r], c = q.k/(|q||k|), t = max(tau, 0.01):
+ *           dc/dq = k/(|q||k|) - c q/|q|^2 (the second term absent when |q| is
+ *           clamped at 1e-12, R9), the same with q and k swapped;
+ *           dtau += -dl c/t^2 when tau >= 0.01 (reading R16: the clamp passes
+ *           the gradient from 0.01 up), else nothing
+ *   mode 2  l = (R_i q_i).(R_j k_j)/sqrt(d): the rotated vectors take the
+ *           mode-0 gradients, which rotate back by R^T; a pair rotated by
+ *           theta = p omega_t has d(Rx)/dtheta = (-(Rx)_1, (Rx)_0), so
+ *           domega_t += p (dRx . d(Rx)/dtheta) over every query and key.
+ * Outputs are overwritten (zeroed first).  dtable [(2M-1)^2][heads], dtau
+ * [heads] and drope [2][d/4] may be NULL.  Returns 0, or -1 as the forward. */
+int oracle_window_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
+                           double* dq, double* dk, double* dv, double* dtable, double* dtau, double* drope,
+                           int B, int H, int W, int heads, int d, int M, int s, int mode,
+                           const double* tau, const double* table, const double* rope_freqs, int nthreads) {
+    if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || M < 1 || s < 0 || s >= M) return -1;
+    if (mode == 2 && (d % 4 != 0 || !rope_freqs)) return -1;
+    if (mode == 1 && !tau) return -1;
+    if (mode < 0 || mode > 2) return -1;
+    const int R = 2 * M - 1;
+    const size_t C = (size_t)heads * d, ntok = (size_t)B * H * W;
+    const double rsd = 1.0 / sqrt((double)d);
+    memset(dq, 0, sizeof(double) * ntok * C);
+    memset(dk, 0, sizeof(double) * ntok * C);
+    memset(dv, 0, sizeof(double) * ntok * C);
+    if (dtable) memset(dtable, 0, sizeof(double) * (size_t)R * R * heads);
+    if (dtau) memset(dtau, 0, sizeof(double) * (size_t)heads);
+    if (drope) memset(drope, 0, sizeof(double) * 2 * (size_t)(d / 4));
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel
+    {
+        const size_t HW = (size_t)H * W;
+        int* ky = (int*)malloc(sizeof(int) * HW);
+        int* kx = (int*)malloc(sizeof(int) * HW);
+        double* pw = (double*)malloc(sizeof(double) * HW);     /* softmax weights of one query */
+        double* cw = (double*)malloc(sizeof(double) * HW);     /* mode 1: cosines of one query */
+        double* kr = (double*)malloc(sizeof(double) * HW * d); /* keys of the image-head, rotated in mode 2 */
+        double* qr = (double*)malloc(sizeof(double) * HW * d); /* queries, rotated in mode 2 */
+        double* dkr = (double*)malloc(sizeof(double) * HW * d);
+        double* nrm = (double*)malloc(sizeof(double) * HW);    /* mode 1: clamped norms */
+        unsigned char* clamped = (unsigned char*)malloc(HW);
+        double* gq = (double*)malloc(sizeof(double) * (size_t)d);
+        double* my_dtable = dtable ? (double*)calloc((size_t)R * R * heads, sizeof(double)) : NULL;
+        double* my_dtau = dtau ? (double*)calloc((size_t)heads, sizeof(double)) : NULL;
+        double* my_drope = drope ? (double*)calloc(2 * (size_t)(d / 4), sizeof(double)) : NULL;
+#pragma omp for schedule(dynamic, 1)
+        for (int bh = 0; bh < B * heads; ++bh) {
+            const int b = bh / heads, h = bh % heads;
+            /* this image-head's queries and keys, rotated in mode 2 */
+            for (size_t t = 0; t < HW; ++t) {
+                const size_t tok = (size_t)b * HW + t;
+                const int y = (int)(t / W), x = (int)(t % W);
+                for (int e = 0; e < d; ++e) {
+                    qr[t * d + e] = q[tok * C + (size_t)h * d + e];
+                    kr[t * d + e] = k[tok * C + (size_t)h * d + e];
+                    dkr[t * d + e] = 0.0;
+                }
+                if (mode == 1) {
+                    double ss = 0.0;
+                    for (int e = 0; e < d; ++e) ss += kr[t * d + e] * kr[t * d + e];
+                    nrm[t] = sqrt(ss) > 1e-12 ? sqrt(ss) : 1e-12;
+                    clamped[t] = !(sqrt(ss) > 1e-12);
+                }
+                if (mode == 2) {
+                    const int py = ((y - s) % M + M) % M, px = ((x - s) % M + M) % M;
+                    rope_half(qr + t * d, d, 0, py, rope_freqs);
+                    rope_half(qr + t * d, d, d / 2, px, rope_freqs + d / 4);
+                    rope_half(kr + t * d, d, 0, py, rope_freqs);
+                    rope_half(kr + t * d, d, d / 2, px, rope_freqs + d / 4);
+                }
+            }
+            const double tt = mode == 1 ? (tau[h] > 0.01 ? tau[h] : 0.01) : 1.0;
+            for (size_t ti = 0; ti < HW; ++ti) {
+                const size_t tok = (size_t)b * HW + ti;
+                const int yi = (int)(ti / W), xi = (int)(ti % W);
+                const int sy = oracle_segment_of(M, s, yi), sx = oracle_segment_of(M, s, xi);
+                int nk = 0;
+                for (int y = 0; y < H; ++y) {
+                    if (oracle_segment_of(M, s, y) != sy) continue;
+                    for (int x = 0; x < W; ++x) {
+                        if (oracle_segment_of(M, s, x) != sx) continue;
+                        ky[nk] = y; kx[nk] = x; ++nk;
+                    }
+                }
+                const double* qi = qr + ti * d;
+                double qn = 1.0;
+                int qclamped = 0;
+                if (mode == 1) {
+                    double qss = 0.0;
+                    for (int e = 0; e < d; ++e) qss += qi[e] * qi[e];
+                    qclamped = !(sqrt(qss) > 1e-12);
+                    qn = qclamped ? 1e-12 : sqrt(qss);
+                }
+                /* forward: logits, softmax, output */
+                double mx = -INFINITY;
+                for (int j = 0; j < nk; ++j) {
+                    const size_t tj = (size_t)ky[j] * W + kx[j];
+                    const double* kj = kr + tj * d;
+                    double dot = 0.0;
+                    for (int e = 0; e < d; ++e) dot += qi[e] * kj[e];
+                    double lg;
+                    if (mode == 1) {
+                        cw[j] = dot / (qn * nrm[tj]);
+                        lg = cw[j] / tt;
+                    } else {
+                        lg = dot * rsd;
+                    }
+                    if (mode != 2 && table)
+                        lg += table[(size_t)((yi - ky[j] + M - 1) * R + (xi - kx[j] + M - 1)) * heads + h];
+                    pw[j] = lg;
+                    if (lg > mx) mx = lg;
+                }
+                double den = 0.0;
+                for (int j = 0; j < nk; ++j) { pw[j] = exp(pw[j] - mx); den += pw[j]; }
+                for (int j = 0; j < nk; ++j) pw[j] /= den;
+                const double* g = dout + tok * C + (size_t)h * d;
+                /* D_i = sum_j P_ij (g . v_j) */
+                double Dsum = 0.0;
+                for (int j = 0; j < nk; ++j) {
+                    const size_t tj = ((size_t)b * H + ky[j]) * W + kx[j];
+                    const double* vj = v + tj * C + (size_t)h * d;
+                    double dp = 0.0;
+                    for (int e = 0; e < d; ++e) dp += g[e] * vj[e];
+                    Dsum += pw[j] * dp;
+                }
+                for (int e = 0; e < d; ++e) gq[e] = 0.0;
+                for (int j = 0; j < nk; ++j) {
+                    const size_t tj = (size_t)ky[j] * W + kx[j];
+                    const size_t gtj = (size_t)b * HW + tj;
+                    const double* vj = v + gtj * C + (size_t)h * d;
+                    double* dvj = dv + gtj * C + (size_t)h * d;
+                    double dp = 0.0;
+                    for (int e = 0; e < d; ++e) {
+                        dp += g[e] * vj[e];
+                        dvj[e] += pw[j] * g[e];
+                    }
+                    const double dl = pw[j] * (dp - Dsum);
+                    const double* kj = kr + tj * d;
+                    double* dkj = dkr + tj * d;
+                    if (mode == 1) {
+                        const double c = cw[j], kn = nrm[tj], a = dl / tt;
+                        for (int e = 0; e < d; ++e) {
+                            gq[e] += a * (kj[e] / (qn * kn) - (qclamped ? 0.0 : c * qi[e] / (qn * qn)));
+                            dkj[e] += a * (qi[e] / (qn * kn) - (clamped[tj] ? 0.0 : c * kj[e] / (kn * kn)));
+                        }
+                        if (my_dtau && tau[h] >= 0.01) my_dtau[h] += -dl * c / (tt * tt);
+                    } else {
+                        for (int e = 0; e < d; ++e) {
+                            gq[e] += dl * kj[e] * rsd;
+                            dkj[e] += dl * qi[e] * rsd;
+                        }
+                    }
+                    if (mode != 2 && my_dtable)
+                        my_dtable[(size_t)((yi - ky[j] + M - 1) * R + (xi - kx[j] + M - 1)) * heads + h] += dl;
+                }
+                /* gq is the gradient of the (rotated, in mode 2) query */
+                double* dqi = dq + tok * C + (size_t)h * d;
+                if (mode == 2) {
+                    const int pos[2] = {((yi - s) % M + M) % M, ((xi - s) % M + M) % M};
+                    for (int half = 0; half < 2; ++half)
+                        for (int t = 0; t < d / 4; ++t) {
+                            const int e0 = half * (d / 2) + 2 * t;
+                            const double th = (double)pos[half] * rope_freqs[half * (d / 4) + t];
+                            const double c = cos(th), sn = sin(th);
+                            /* R^T applied to the gradient pair */
+                            dqi[e0] = gq[e0] * c + gq[e0 + 1] * sn;
+                            dqi[e0 + 1] = -gq[e0] * sn + gq[e0 + 1] * c;
+                            if (my_drope) my_drope[half * (d / 4) + t] +=
+                                (double)pos[half] * (gq[e0] * -qi[e0 + 1] + gq[e0 + 1] * qi[e0]);
+                        }
+                } else {
+                    for (int e = 0; e < d; ++e) dqi[e] = gq[e];
+                }
+            }
+            /* keys: rotate the accumulated gradients back (mode 2) */
+            for (size_t tj = 0; tj < HW; ++tj) {
+                const size_t gtj = (size_t)b * HW + tj;
+                double* dkj = dk + gtj * C + (size_t)h * d;
+                const double* g2 = dkr + tj * d;
+                if (mode == 2) {
+                    const int y = (int)(tj / W), x = (int)(tj % W);
+                    const int pos[2] = {((y - s) % M + M) % M, ((x - s) % M + M) % M};
+                    const double* kj = kr + tj * d;
+                    for (int half = 0; half < 2; ++half)
+                        for (int t = 0; t < d / 4; ++t) {
+                            const int e0 = half * (d / 2) + 2 * t;
+                            const double th = (double)pos[half] * rope_freqs[half * (d / 4) + t];
+                            const double c = cos(th), sn = sin(th);
+                            dkj[e0] = g2[e0] * c + g2[e0 + 1] * sn;
+                            dkj[e0 + 1] = -g2[e0] * sn + g2[e0 + 1] * c;
+                            if (my_drope) my_drope[half * (d / 4) + t] +=
+                                (double)pos[half] * (g2[e0] * -kj[e0 + 1] + g2[e0 + 1] * kj[e0]);
+                        }
+                } else {
+                    for (int e = 0; e < d; ++e) dkj[e] = g2[e];
+                }
+            }
+        }
+#pragma omp critical
+        {
+            if (my_dtable) for (size_t i = 0; i < (size_t)R * R * heads; ++i) dtable[i] += my_dtable[i];
+            if (my_dtau) for (int i = 0; i < heads; ++i) dtau[i] += my_dtau[i];
+            if (my_drope) for (int i = 0; i < 2 * (d / 4); ++i) drope[i] += my_drope[i];
+        }
+        free(ky); free(kx); free(pw); free(cw); free(kr); free(qr); free(dkr); free(nrm); free(clamped); free(gq);
+        free(my_dtable); free(my_dtau); free(my_drope);
     }
     return 0;
 }
