@@ -1,6 +1,7 @@
 /*
  * swin_attn.h — C ABI of libswinattn.so: shifted-window multi-head
- * self-attention (forward) on a 2-D token grid, for NVIDIA B200 (sm_100a).
+ * self-attention (forward and gradients) on a 2-D token grid, for NVIDIA
+ * B200 (sm_100a).
  *
  * What is computed.  For an image b, head h and query token i at grid
  * position (y_i, x_i), the attended keys are the tokens j that share i's
@@ -184,6 +185,54 @@ swin_status swin_window_attn_fwd_noalloc(const void* q, const void* k, const voi
 /* Bytes of workspace swin_window_attn_fwd needs for these arguments
  * (have_table: whether bias_table is non-NULL).  0 when none is needed. */
 size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int have_table);
+
+/* swin_window_attn_bwd — gradients of swin_window_attn_fwd's output with
+ * respect to its inputs and parameters, for training (the pages train every
+ * model they describe; FlashSwin's abstract rests its training-memory claim
+ * on attention that keeps no score matrix, and neither does this pass).  For
+ * L = sum over all elements of dout * out, it writes dq, dk, dv = dL/dq,
+ * dL/dk, dL/dv and, when asked, dtable = dL/dT, dtau = dL/dtau and
+ * drope = dL/dw.  The softmax is recomputed from q, k, v; nothing from the
+ * forward pass is needed.  Conventions:
+ *   - tau below 0.01 is clamped, so its gradient is 0 there; at and above
+ *     0.01 (compared as real numbers: the fp32 value nearest 0.01 lies just
+ *     below it) the gradient passes ("Swin Transformer V2" §3.2);
+ *   - a q or k row of norm at most 1e-12 (mode 1) has its norm held at
+ *     1e-12, a constant;
+ *   - the gradient of the CPB meta network's weights is not formed: in mode
+ *     1, pass the table swin_cpb_eval produced and back-propagate dtable
+ *     through G.
+ *   q, k, v, dout    device [B][H][W][heads][d] of dtype dt (SWIN_F32 or
+ *                    SWIN_BF16)
+ *   dq, dk, dv       device [B][H][W][heads][d] of dtype grad_dt (== dt, or
+ *                    SWIN_F32 for SWIN_BF16 inputs; a bf16 gradient is the
+ *                    fp32 one rounded to nearest even); written, not added to;
+ *                    must not overlap each other or the inputs
+ *   B, H, W, heads, d, M, shift, mode, tau, rope_freqs
+ *                    as swin_window_attn_fwd, except that d may be 8, 16, 32
+ *                    or 64 for both dtypes
+ *   bias_table       device fp32 [(2M-1)^2][heads] or NULL, modes 0 and 1
+ *                    (mode 1 takes the table, not the CPB weights)
+ *   dtable           device fp32 [(2M-1)^2][heads] or NULL; needs bias_table
+ *   dtau             device fp32 [heads] or NULL; mode 1 only
+ *   drope            device fp32 [2][d/4] or NULL; mode 2 only
+ *   workspace        device scratch of swin_window_attn_bwd_workspace_size
+ *                    bytes, 256-byte aligned
+ * Arithmetic: double for SWIN_F32 tensors, fp32 for SWIN_BF16 tensors, on
+ * the CUDA cores; parameter gradients are summed in double and rounded once.
+ * Errors as swin_window_attn_fwd: argument errors return before anything is
+ * enqueued. */
+swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
+                                 void* dq, void* dk, void* dv, swin_dtype dt, swin_dtype grad_dt,
+                                 int B, int H, int W, int heads, int d, int M, int shift,
+                                 swin_mode mode, const float* tau, const float* bias_table,
+                                 const float* rope_freqs, float* dtable, float* dtau, float* drope,
+                                 void* workspace, size_t workspace_bytes, swin_stream_t stream);
+
+/* Bytes of workspace swin_window_attn_bwd needs: 16 per query row and head
+ * (its log-sum-exp and D = dout . out, in double) plus the double
+ * accumulators of the parameter gradients, rounded up to 256. */
+size_t swin_window_attn_bwd_workspace_size(int B, int H, int W, int heads, int d, int M);
 
 /* swin_index_tables — Swin's bookkeeping for an HxW grid in the rolled frame
  * (pad to Hp = ceil(H/M)*M, Wp likewise; roll by -shift; cut MxM windows), as

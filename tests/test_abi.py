@@ -127,3 +127,37 @@ def test_binding_checks_cpb_weight_shapes():
         sa.swin_cpb_eval(8, 3, w1, None, w2, None)
     with pytest.raises(ValueError, match="cpb b2"):
         sa.swin_cpb_eval_form(8, 4, w1, None, w2, _z(3), sa.SWIN_CPB_CODE)
+
+
+def test_bwd_workspace_size(L):
+    acc = ((31 * 31 * 3 + 3 + 2 * 8) * 8 + 255) // 256 * 256
+    stats = (8 * 2 * 2 * 64 * 64 * 3 + 255) // 256 * 256  # (lse, D) doubles per row and head, B = 2
+    assert sa.swin_window_attn_bwd_workspace_size(2, 64, 64, 3, 32, 16) == acc + stats
+    assert sa.swin_window_attn_bwd_workspace_size(0, 64, 64, 3, 32, 16) == 0
+    assert sa.swin_window_attn_bwd_workspace_size(1, 8, 8, 1, 32, 65) == 0
+
+
+def call_bwd(L, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, dout=FAKE * 4, dq=FAKE * 64, dk=FAKE * 65, dv=FAKE * 66,
+             dt=sa.SWIN_F32, gdt=None, B=1, H=8, W=8, heads=1, d=32, M=4, shift=2, mode=sa.SWIN_MODE_DOT_BIAS,
+             tau=None, table=None, rope=None, dtable=None, dtau=None, drope=None, ws=FAKE * 128, wsb=1 << 20)
+    a.update(kw)
+    return L.swin_window_attn_bwd(a["q"], a["k"], a["v"], a["dout"], a["dq"], a["dk"], a["dv"], a["dt"],
+                                  a["dt"] if a["gdt"] is None else a["gdt"], a["B"], a["H"], a["W"], a["heads"],
+                                  a["d"], a["M"], a["shift"], a["mode"], a["tau"], a["table"], a["rope"],
+                                  a["dtable"], a["dtau"], a["drope"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status,why", [
+    (dict(q=None), 1, "NULL"), (dict(dout=None), 1, "NULL"), (dict(dv=None), 1, "NULL"),
+    (dict(shift=4), 1, "shift"), (dict(M=65, shift=0), 1, "M"), (dict(heads=0), 1, ">= 1"),
+    (dict(dout=FAKE * 4 + 8), 1, "aligned"), (dict(dk=FAKE * 3), 1, "overlap"),
+    (dict(dk=FAKE * 64 + 16), 1, "overlap"), (dict(dq=FAKE), 1, "overlaps"),
+    (dict(mode=1), 1, "tau"), (dict(mode=2), 1, "rope"), (dict(dtable=FAKE * 7), 1, "dtable needs"),
+    (dict(dtau=FAKE * 7), 1, "dtau"), (dict(drope=FAKE * 7), 1, "drope"),
+    (dict(dt=0, gdt=1), 1, "output dtype"), (dict(d=24), 2, "d in"), (dict(ws=None), 1, "workspace"),
+    (dict(wsb=256), 1, "workspace"), (dict(ws=FAKE * 128 + 16), 1, "256-byte"),
+])
+def test_bwd_rejects_bad_arguments(L, kw, status, why):
+    assert call_bwd(L, **kw) == status
+    assert why in L.swin_last_error().decode()

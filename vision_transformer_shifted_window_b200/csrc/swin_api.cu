@@ -168,6 +168,69 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
   return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
 }
 
+static size_t bwd_acc_doubles(int heads, int d, int M) {
+  return (size_t)(2 * M - 1) * (2 * M - 1) * heads + (size_t)heads + 2 * (size_t)(d / 4);
+}
+
+size_t swin_window_attn_bwd_workspace_size(int B, int H, int W, int heads, int d, int M) {
+  if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || M < 1 || M > 64) return 0;
+  const size_t acc = (sizeof(double) * bwd_acc_doubles(heads, d, M) + 255) & ~size_t(255);
+  const size_t stats = sizeof(double) * 2 * (size_t)B * H * W * heads;
+  return acc + ((stats + 255) & ~size_t(255));
+}
+
+swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
+                                 void* dk, void* dv, swin_dtype dt, swin_dtype grad_dt, int B, int H, int W,
+                                 int heads, int d, int M, int shift, swin_mode mode, const float* tau,
+                                 const float* bias_table, const float* rope_freqs, float* dtable, float* dtau,
+                                 float* drope, void* workspace, size_t workspace_bytes, swin_stream_t stream) {
+  // the forward's checks with dq standing for out (dtype, shape, alignment,
+  // mode parameters, dq against q, k, v)
+  swin_status vs = swin::check_fwd_args(q, k, v, dq, dt, grad_dt, B, H, W, heads, d, M, shift, mode, tau,
+                                        bias_table, nullptr, rope_freqs);
+  if (vs != SWIN_OK) return vs;
+  if (!dout || !dk || !dv) return fail(SWIN_ERR_INVALID_ARG, "dout, dk and dv must be non-NULL");
+  if (!aligned16(dout) || !aligned16(dk) || !aligned16(dv))
+    return fail(SWIN_ERR_INVALID_ARG, "dout, dk and dv must be 16-byte aligned");
+  if (d != 8 && d != 16 && d != 32 && d != 64)
+    return fail(SWIN_ERR_UNSUPPORTED, "backward supports d in {8,16,32,64}, got %d", d);
+  const size_t elems = (size_t)B * H * W * heads * d;
+  const size_t ib = elems * (dt == SWIN_F32 ? 4 : 2), gb = elems * (grad_dt == SWIN_F32 ? 4 : 2);
+  const void* ins[4] = {q, k, v, dout};
+  void* outs[3] = {dq, dk, dv};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 4; ++i)
+      if (overlaps(outs[o], gb, ins[i], ib)) return fail(SWIN_ERR_INVALID_ARG, "dq, dk and dv must not overlap the inputs");
+    for (int p = o + 1; p < 3; ++p)
+      if (overlaps(outs[o], gb, outs[p], gb)) return fail(SWIN_ERR_INVALID_ARG, "dq, dk and dv must not overlap");
+  }
+  if (dtable && !bias_table) return fail(SWIN_ERR_INVALID_ARG, "dtable needs bias_table");
+  if (dtau && mode != SWIN_MODE_COSINE_CPB) return fail(SWIN_ERR_INVALID_ARG, "dtau applies to the cosine mode only");
+  if (drope && mode != SWIN_MODE_ROPE) return fail(SWIN_ERR_INVALID_ARG, "drope applies to the RoPE mode only");
+  const size_t need = swin_window_attn_bwd_workspace_size(B, H, W, heads, d, M);
+  if (!workspace || workspace_bytes < need)
+    return fail(SWIN_ERR_INVALID_ARG, "workspace of %zu bytes needed, got %zu", need, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(SWIN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+
+  double* acc = static_cast<double*>(workspace);
+  const size_t acc_bytes = (sizeof(double) * bwd_acc_doubles(heads, d, M) + 255) & ~size_t(255);
+  swin::BwdArgs a;
+  a.q = q; a.k = k; a.v = v; a.dout = dout; a.dq = dq; a.dk = dk; a.dv = dv;
+  a.B = B; a.H = H; a.W = W; a.heads = heads; a.d = d; a.M = M; a.shift = shift; a.mode = (int)mode;
+  a.tau = tau; a.table = mode == SWIN_MODE_ROPE ? nullptr : bias_table; a.rope = rope_freqs;
+  size_t slot = 0;
+  a.acc_base = acc;
+  a.acc_table = dtable ? acc + slot : nullptr;
+  slot += dtable ? (size_t)(2 * M - 1) * (2 * M - 1) * heads : 0;
+  a.acc_tau = dtau ? acc + slot : nullptr;
+  slot += dtau ? (size_t)heads : 0;
+  a.acc_rope = drope ? acc + slot : nullptr;
+  a.stats = reinterpret_cast<double2*>(static_cast<char*>(workspace) + acc_bytes);
+  return swin::launch_attn_bwd(a, dt == SWIN_BF16, grad_dt == SWIN_F32, dtable, dtau, drope,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
 swin_status swin_index_tables(int H, int W, int M, int shift, int32_t* tok_window,
                               int32_t* tok_region, int32_t* tok_local, int32_t* rel_index,
                               swin_stream_t stream) {

@@ -42,6 +42,28 @@ struct AttnArgs {
   int* status;
 };
 
+// Arguments of the backward kernels.  The double accumulators of the
+// parameter gradients lie contiguously at acc_base: table, then tau, then
+// rope; a gradient not asked for has a NULL pointer and no slot.
+struct BwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  int B, H, W, heads, d, M, shift, mode;
+  const float* tau;
+  const float* table;  // [(2M-1)^2][heads] or nullptr
+  const float* rope;   // [2][d/4] or nullptr
+  double* acc_base;
+  double* acc_table;
+  double* acc_tau;
+  double* acc_rope;
+  double2* stats;  // [B][H][W][heads]: (log-sum-exp, D) of each query row
+};
+
 // Launchers (one per translation unit).
 swin_status launch_cpb_eval(int M, int heads, const swin_cpb_weights& g, float* table,
                             cudaStream_t stream, int form = SWIN_CPB_PAPER, int pretrained_M = 0);
@@ -50,5 +72,7 @@ swin_status launch_index_tables(int H, int W, int M, int shift, int32_t* tw, int
 swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream);
 void tc_set_debug(int flags, long long wait_limit);
 swin_status launch_attn_simt(const AttnArgs& a, bool bf16_in, bool f32_out, cudaStream_t stream);
+swin_status launch_attn_bwd(const BwdArgs& a, bool bf16_in, bool f32_grad, float* dtable, float* dtau,
+                            float* drope, cudaStream_t stream);
 
 }  // namespace swin

@@ -34,7 +34,7 @@ SWIN_CPB_CODE = 1
 
 #: every symbol include/swin_attn.h declares
 EXPORTED = ("swin_cpb_eval", "swin_cpb_eval_form", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
-            "swin_window_attn_workspace_size",
+            "swin_window_attn_workspace_size", "swin_window_attn_bwd", "swin_window_attn_bwd_workspace_size",
             "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version",
             "swin_debug_set")
 
@@ -75,6 +75,11 @@ def lib():
         L.swin_window_attn_fwd_noalloc.restype = i
         L.swin_window_attn_workspace_size.argtypes = [i, i, i, i]
         L.swin_window_attn_workspace_size.restype = ctypes.c_size_t
+        L.swin_window_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp,
+                                           vp, vp, vp, vp, vp, ctypes.c_size_t, st]
+        L.swin_window_attn_bwd.restype = i
+        L.swin_window_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.swin_window_attn_bwd_workspace_size.restype = ctypes.c_size_t
         L.swin_index_tables.argtypes = [i, i, i, i, vp, vp, vp, vp, st]
         L.swin_index_tables.restype = i
         L.swin_stream_status.argtypes = [st]
@@ -279,6 +284,53 @@ def swin_window_attn_fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tens
         _check(rc)
         del keep
     return out
+
+
+def swin_window_attn_bwd_workspace_size(B: int, H: int, W: int, heads: int, d: int, M: int) -> int:
+    return int(lib().swin_window_attn_bwd_workspace_size(B, H, W, heads, d, M))
+
+
+def swin_window_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout: torch.Tensor, M: int,
+                         shift: int, mode: int, tau: Optional[torch.Tensor] = None,
+                         bias_table: Optional[torch.Tensor] = None,
+                         rope_freqs: Optional[torch.Tensor] = None, param_grads: bool = True,
+                         grad_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
+                         stream=None) -> dict:
+    """Gradients of sum(dout * swin_window_attn_fwd(...)): a dict with dq, dk, dv
+    ([B, H, W, heads, d], dtype ``grad_dtype`` or q's) and, when ``param_grads``,
+    dtable (with a bias table), dtau (mode 1) and drope (mode 2), fp32."""
+    dt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(q.dtype)
+    if dt is None or any(t.dtype != q.dtype or t.shape != q.shape for t in (k, v, dout)):
+        raise ValueError("q, k, v, dout must share a float32/bfloat16 dtype and shape")
+    if q.dim() != 5:
+        raise ValueError("q, k, v, dout must be [B, H, W, heads, d]")
+    B, H, W, heads, d = q.shape
+    gdt = grad_dtype or q.dtype
+    gcode = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(gdt)
+    if gcode is None:
+        raise ValueError("grad_dtype must be float32 or bfloat16")
+    with _on(stream):
+        tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
+        _param_shapes(M, heads, d, tau, bias_table, rope_freqs)
+        mk = lambda: torch.empty(q.shape, dtype=gdt, device=q.device)
+        g = {"dq": mk(), "dk": mk(), "dv": mk()}
+        f32 = lambda *s: torch.empty(s, dtype=torch.float32, device=q.device)
+        if param_grads and bias_table is not None and mode != SWIN_MODE_ROPE:
+            g["dtable"] = f32((2 * M - 1) ** 2, heads)
+        if param_grads and mode == SWIN_MODE_COSINE_CPB:
+            g["dtau"] = f32(heads)
+        if param_grads and mode == SWIN_MODE_ROPE:
+            g["drope"] = f32(2, d // 4)
+        need = swin_window_attn_bwd_workspace_size(B, H, W, heads, d, M)
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        rc = lib().swin_window_attn_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), dt, gcode,
+            B, H, W, heads, d, M, shift, mode, _ptr(tau), _ptr(bias_table), _ptr(rope_freqs),
+            _ptr(g.get("dtable")), _ptr(g.get("dtau")), _ptr(g.get("drope")), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+        _check(rc)
+    return g
 
 
 def swin_index_tables(H: int, W: int, M: int, shift: int, device="cuda", stream=None):

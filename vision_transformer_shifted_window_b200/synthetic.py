@@ -106,3 +106,16 @@ def make_inputs(w: Workload, B: Optional[int] = None, H: Optional[int] = None,
         f = (w.rope_base ** (-t / q4)).astype(np.float32)
         out["rope_freqs"] = np.stack([f, f]).astype(np.float32)  # [2][d/4]: row axis, col axis
     return out
+
+
+def make_dout(w: Workload, B: Optional[int] = None, H: Optional[int] = None, W: Optional[int] = None,
+              seed: Optional[int] = None) -> np.ndarray:
+    """An output gradient for the backward pass: N(0, 1) of q's shape (its own
+    stream, SeedSequence(5000 + index) unless ``seed`` is given), rounded to
+    bf16 for bf16 workloads."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    W = w.W if W is None else W
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(5000 + w.index if seed is None else seed)))
+    x = g.standard_normal((B, H, W, w.heads, w.d), dtype=np.float32)
+    return round_to_bf16(x) if w.dtype == "bf16" else x
