@@ -219,7 +219,9 @@ size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int hav
  *   workspace        device scratch of swin_window_attn_bwd_workspace_size
  *                    bytes, 256-byte aligned
  * Arithmetic: double for SWIN_F32 tensors, fp32 for SWIN_BF16 tensors, on
- * the CUDA cores; parameter gradients are summed in double and rounded once.
+ * the CUDA cores.  dq, dk, dv are deterministic.  Parameter gradients are
+ * summed by double atomic additions and rounded once to fp32; the order of
+ * the additions varies, so between calls they may differ in the last bit.
  * Errors as swin_window_attn_fwd: argument errors return before anything is
  * enqueued. */
 swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, const void* dout,

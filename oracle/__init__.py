@@ -68,10 +68,10 @@ def _load():
         lib.oracle_index_tables.argtypes = [ctypes.c_int] * 4 + [ip] * 4
         lib.oracle_index_tables.restype = None
         lib.oracle_window_attn.argtypes = (
-            [dp] * 4 + [ctypes.c_int] * 8 + [dp] * 3 + [lp, ctypes.c_int64, ctypes.c_int]
+            [dp] * 4 + [ctypes.c_int] * 9 + [dp] * 3 + [lp, ctypes.c_int64, ctypes.c_int]
         )
         lib.oracle_window_attn.restype = ctypes.c_int
-        lib.oracle_window_attn_bwd.argtypes = ([dp] * 10 + [ctypes.c_int] * 8 + [dp] * 3 + [ctypes.c_int])
+        lib.oracle_window_attn_bwd.argtypes = ([dp] * 10 + [ctypes.c_int] * 9 + [dp] * 3 + [ctypes.c_int])
         lib.oracle_window_attn_bwd.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
@@ -168,10 +168,14 @@ MODE_DOT_BIAS = 0
 MODE_COSINE_CPB = 1
 MODE_ROPE = 2
 
+PARTITION_SHIFTED = 0
+PARTITION_INTERLEAVED = 1
+
 
 def window_attn(q, k, v, M: int, shift: int, mode: int, tau=None, table=None,
-                rope_freqs=None, queries=None, nthreads: int = 0) -> np.ndarray:
-    """Shifted-window attention in float64.
+                rope_freqs=None, queries=None, nthreads: int = 0, partition: int = PARTITION_SHIFTED) -> np.ndarray:
+    """Shifted-window attention in float64 (or, with ``partition`` =
+    PARTITION_INTERLEAVED and shift 0, attention in Iwin's interleaved windows).
 
     q, k, v: [B, H, W, heads, d] (any float dtype; read as float64).
     Returns [B, H, W, heads, d] float64, or [len(queries), heads, d] when
@@ -195,7 +199,7 @@ def window_attn(q, k, v, M: int, shift: int, mode: int, tau=None, table=None,
         out = np.zeros((nq, heads, d), dtype=np.float64)
         qp = qarr.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))
     rc = _load().oracle_window_attn(
-        _dp(q), _dp(k), _dp(v), _dp(out), B, H, W, heads, d, M, shift, mode,
+        _dp(q), _dp(k), _dp(v), _dp(out), B, H, W, heads, d, M, shift, int(partition), mode,
         _dp(tau), _dp(table), _dp(rope_freqs), qp, nq, int(nthreads),
     )
     if rc != 0:
@@ -204,7 +208,7 @@ def window_attn(q, k, v, M: int, shift: int, mode: int, tau=None, table=None,
 
 
 def window_attn_bwd(q, k, v, dout, M: int, shift: int, mode: int, tau=None, table=None, rope_freqs=None,
-                    nthreads: int = 0) -> dict:
+                    nthreads: int = 0, partition: int = PARTITION_SHIFTED) -> dict:
     """Gradients of L = sum(dout * window_attn(...)) in float64: dq, dk, dv
     ([B, H, W, heads, d]), dtable ([(2M-1)^2, heads], modes 0 and 1), dtau
     ([heads], mode 1), drope ([2, d/4], mode 2)."""
@@ -219,7 +223,7 @@ def window_attn_bwd(q, k, v, dout, M: int, shift: int, mode: int, tau=None, tabl
     drope = np.zeros((2, d // 4)) if mode == 2 else None
     rc = _load().oracle_window_attn_bwd(
         _dp(q), _dp(k), _dp(v), _dp(dout), _dp(dq), _dp(dk), _dp(dv), _dp(dtable), _dp(dtau), _dp(drope),
-        B, H, W, heads, d, M, shift, mode, _dp(tau), _dp(table), _dp(rope_freqs), int(nthreads))
+        B, H, W, heads, d, M, shift, int(partition), mode, _dp(tau), _dp(table), _dp(rope_freqs), int(nthreads))
     if rc != 0:
         raise ValueError("oracle_window_attn_bwd rejected its arguments")
     out = {"dq": dq, "dk": dk, "dv": dv}

@@ -45,6 +45,9 @@
  *      inside each half rotate by p * omega[axis][t], t < d/4; the window-local
  *      coordinate is p = (y - s) mod M; RoPE touches q and k only; the score
  *      is scaled by 1/sqrt(d); no bias.
+ *  R17 Interleaved windows ("Iwin Transformer", abstract only): the strided
+ *      partition described at win_of below; the same three scores, with
+ *      window-local coordinates in place of the shifted ones; no shift.
  *  R15 The code form of G ([V2] "Paper vs code"): the normaliser is the
  *      pretrained window Mp (the window itself when none is given); a window
  *      of 1 (Mp - 1 = 0) has only offset 0, whose coordinate is 0.
@@ -69,6 +72,29 @@
  * s + kM.  Shifting the axis by (M - s) mod M turns them into multiples of M. */
 int oracle_segment_of(int M, int s, int y) {
     return (y + (M - s) % M) / M;
+}
+
+/* The two partitions of an axis of length L into windows of M tokens:
+ *   part 0, shifted (R1): the window is the segment under boundaries s + kM;
+ *     the window-local coordinate is (y - s) mod M; the offset of two tokens
+ *     of one window is the difference of their coordinates.
+ *   part 1, interleaved ("Iwin Transformer" abstract, reading R17): with
+ *     G = ceil(L / M) windows per axis, window a holds the tokens a + G i,
+ *     i < M, that lie inside the axis, i.e. the window is y mod G and the
+ *     window-local coordinate is i = y div G; offsets are differences of i. */
+static int win_of(int part, int L, int M, int s, int y) {
+    if (part == 0) return oracle_segment_of(M, s, y);
+    return y % ((L + M - 1) / M);
+}
+
+static int loc_of(int part, int L, int M, int s, int y) {
+    if (part == 0) return ((y - s) % M + M) % M;
+    return y / ((L + M - 1) / M);
+}
+
+static int off_of(int part, int L, int M, int s, int yq, int yk) {
+    if (part == 0) return yq - yk;
+    return loc_of(part, L, M, s, yq) - loc_of(part, L, M, s, yk);
 }
 
 /* eq. 4: signed natural-log map of one offset component (reading R6). */
@@ -219,6 +245,7 @@ static double norm_clamped(const double* x, int d) {
 /* Shifted-window multi-head attention, one query token (all heads) at a time.
  *
  *  q, k, v  [B][H][W][heads][d]
+ *  part     0: shifted windows (shift s); 1: interleaved windows (s must be 0)
  *  mode 0   eq. 1: q.k/sqrt(d) + table[rel][h]
  *  mode 1   eq. 2: cos(q,k)/max(tau_h, 0.01) + table[rel][h]
  *  mode 2   FlashSwin: (R(p_i) q).(R(p_j) k)/sqrt(d), rope_freqs [2][d/4]
@@ -227,10 +254,11 @@ static double norm_clamped(const double* x, int d) {
  *  out      [nq][heads][d]
  * Returns 0, or -1 on an argument the definition does not cover. */
 int oracle_window_attn(const double* q, const double* k, const double* v, double* out,
-                       int B, int H, int W, int heads, int d, int M, int s, int mode,
+                       int B, int H, int W, int heads, int d, int M, int s, int part, int mode,
                        const double* tau, const double* table, const double* rope_freqs,
                        const int64_t* queries, int64_t nq, int nthreads) {
     if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || M < 1 || s < 0 || s >= M) return -1;
+    if (part < 0 || part > 1 || (part == 1 && s != 0)) return -1;
     if (mode == 2 && (d % 4 != 0 || !rope_freqs)) return -1;
     if (mode == 1 && !tau) return -1;
     if (mode < 0 || mode > 2) return -1;
@@ -258,13 +286,13 @@ int oracle_window_attn(const double* q, const double* k, const double* v, double
             int64_t tok = queries ? queries[n] : n;
             int b = (int)(tok / ((int64_t)H * W));
             int yi = (int)((tok / W) % H), xi = (int)(tok % W);
-            /* R1: key set = same segment on both axes */
-            int sy = oracle_segment_of(M, s, yi), sx = oracle_segment_of(M, s, xi);
+            /* R1 / R17: key set = same window on both axes */
+            int sy = win_of(part, H, M, s, yi), sx = win_of(part, W, M, s, xi);
             int nk = 0;
             for (int y = 0; y < H; ++y) {
-                if (oracle_segment_of(M, s, y) != sy) continue;
+                if (win_of(part, H, M, s, y) != sy) continue;
                 for (int x = 0; x < W; ++x) {
-                    if (oracle_segment_of(M, s, x) != sx) continue;
+                    if (win_of(part, W, M, s, x) != sx) continue;
                     ky[nk] = y; kx[nk] = x; ++nk;
                 }
             }
@@ -274,7 +302,7 @@ int oracle_window_attn(const double* q, const double* k, const double* v, double
                 double qn = 1.0;
                 if (mode == 1) qn = norm_clamped(qi, d);
                 if (mode == 2) {
-                    int py = ((yi - s) % M + M) % M, px = ((xi - s) % M + M) % M;
+                    int py = loc_of(part, H, M, s, yi), px = loc_of(part, W, M, s, xi);
                     rope_half(qi, d, 0, py, rope_freqs);
                     rope_half(qi, d, d / 2, px, rope_freqs + d / 4);
                 }
@@ -285,7 +313,7 @@ int oracle_window_attn(const double* q, const double* k, const double* v, double
                     for (int e = 0; e < d; ++e) kj[e] = ksrc[e];
                     double lg;
                     if (mode == 2) {
-                        int py = ((ky[j] - s) % M + M) % M, px = ((kx[j] - s) % M + M) % M;
+                        int py = loc_of(part, H, M, s, ky[j]), px = loc_of(part, W, M, s, kx[j]);
                         rope_half(kj, d, 0, py, rope_freqs);
                         rope_half(kj, d, d / 2, px, rope_freqs + d / 4);
                     }
@@ -301,7 +329,7 @@ int oracle_window_attn(const double* q, const double* k, const double* v, double
                         lg = dot * rsd;
                     }
                     if (mode != 2 && table) {
-                        int dy = yi - ky[j], dx = xi - kx[j];
+                        int dy = off_of(part, H, M, s, yi, ky[j]), dx = off_of(part, W, M, s, xi, kx[j]);
                         lg += table[(size_t)((dy + M - 1) * R + (dx + M - 1)) * heads + h];
                     }
                     logit[j] = lg;
@@ -346,9 +374,10 @@ int oracle_window_attn(const double* q, const double* k, const double* v, double
  * [heads] and drope [2][d/4] may be NULL.  Returns 0, or -1 as the forward. */
 int oracle_window_attn_bwd(const double* q, const double* k, const double* v, const double* dout,
                            double* dq, double* dk, double* dv, double* dtable, double* dtau, double* drope,
-                           int B, int H, int W, int heads, int d, int M, int s, int mode,
+                           int B, int H, int W, int heads, int d, int M, int s, int part, int mode,
                            const double* tau, const double* table, const double* rope_freqs, int nthreads) {
     if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1 || M < 1 || s < 0 || s >= M) return -1;
+    if (part < 0 || part > 1 || (part == 1 && s != 0)) return -1;
     if (mode == 2 && (d % 4 != 0 || !rope_freqs)) return -1;
     if (mode == 1 && !tau) return -1;
     if (mode < 0 || mode > 2) return -1;
@@ -401,7 +430,7 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v, co
                     clamped[t] = !(sqrt(ss) > 1e-12);
                 }
                 if (mode == 2) {
-                    const int py = ((y - s) % M + M) % M, px = ((x - s) % M + M) % M;
+                    const int py = loc_of(part, H, M, s, y), px = loc_of(part, W, M, s, x);
                     rope_half(qr + t * d, d, 0, py, rope_freqs);
                     rope_half(qr + t * d, d, d / 2, px, rope_freqs + d / 4);
                     rope_half(kr + t * d, d, 0, py, rope_freqs);
@@ -412,12 +441,12 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v, co
             for (size_t ti = 0; ti < HW; ++ti) {
                 const size_t tok = (size_t)b * HW + ti;
                 const int yi = (int)(ti / W), xi = (int)(ti % W);
-                const int sy = oracle_segment_of(M, s, yi), sx = oracle_segment_of(M, s, xi);
+                const int sy = win_of(part, H, M, s, yi), sx = win_of(part, W, M, s, xi);
                 int nk = 0;
                 for (int y = 0; y < H; ++y) {
-                    if (oracle_segment_of(M, s, y) != sy) continue;
+                    if (win_of(part, H, M, s, y) != sy) continue;
                     for (int x = 0; x < W; ++x) {
-                        if (oracle_segment_of(M, s, x) != sx) continue;
+                        if (win_of(part, W, M, s, x) != sx) continue;
                         ky[nk] = y; kx[nk] = x; ++nk;
                     }
                 }
@@ -445,7 +474,7 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v, co
                         lg = dot * rsd;
                     }
                     if (mode != 2 && table)
-                        lg += table[(size_t)((yi - ky[j] + M - 1) * R + (xi - kx[j] + M - 1)) * heads + h];
+                        lg += table[(size_t)((off_of(part, H, M, s, yi, ky[j]) + M - 1) * R + (off_of(part, W, M, s, xi, kx[j]) + M - 1)) * heads + h];
                     pw[j] = lg;
                     if (lg > mx) mx = lg;
                 }
@@ -490,12 +519,12 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v, co
                         }
                     }
                     if (mode != 2 && my_dtable)
-                        my_dtable[(size_t)((yi - ky[j] + M - 1) * R + (xi - kx[j] + M - 1)) * heads + h] += dl;
+                        my_dtable[(size_t)((off_of(part, H, M, s, yi, ky[j]) + M - 1) * R + (off_of(part, W, M, s, xi, kx[j]) + M - 1)) * heads + h] += dl;
                 }
                 /* gq is the gradient of the (rotated, in mode 2) query */
                 double* dqi = dq + tok * C + (size_t)h * d;
                 if (mode == 2) {
-                    const int pos[2] = {((yi - s) % M + M) % M, ((xi - s) % M + M) % M};
+                    const int pos[2] = {loc_of(part, H, M, s, yi), loc_of(part, W, M, s, xi)};
                     for (int half = 0; half < 2; ++half)
                         for (int t = 0; t < d / 4; ++t) {
                             const int e0 = half * (d / 2) + 2 * t;
@@ -518,7 +547,7 @@ int oracle_window_attn_bwd(const double* q, const double* k, const double* v, co
                 const double* g2 = dkr + tj * d;
                 if (mode == 2) {
                     const int y = (int)(tj / W), x = (int)(tj % W);
-                    const int pos[2] = {((y - s) % M + M) % M, ((x - s) % M + M) % M};
+                    const int pos[2] = {loc_of(part, H, M, s, y), loc_of(part, W, M, s, x)};
                     const double* kj = kr + tj * d;
                     for (int half = 0; half < 2; ++half)
                         for (int t = 0; t < d / 4; ++t) {

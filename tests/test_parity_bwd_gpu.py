@@ -3,7 +3,9 @@ against the oracle's gradients, on the same seeded inputs: dq, dk, dv and the
 parameter gradients (bias table, tau, RoPE frequencies) within
 max|gpu - oracle| / rms(oracle) <= 1e-5 (fp32 tensors) and 2e-2 (bf16
 tensors, checked on fp32 gradients; the bf16 gradients must then be their
-round-to-nearest-even rounding bit for bit)."""
+round-to-nearest-even rounding bit for bit).  The parameter gradients are
+summed by double atomic additions and rounded once: between calls they may
+differ in the last fp32 bit, never more."""
 import dataclasses
 
 import numpy as np
@@ -87,7 +89,11 @@ def check_case(w, shift, B=None, H=None, W=None, seed=None, mutate=None):
         assert torch.equal(g32[n].to(torch.bfloat16).view(torch.int16), g16[n].view(torch.int16)), n
     for n in ("dtable", "dtau", "drope"):
         if n in g32:
-            assert torch.equal(g32[n], g16[n]), n
+            # double atomic sums rounded once to fp32: the order of the
+            # additions varies between calls, so the last fp32 bit may too
+            a, b = g32[n].cpu().numpy(), g16[n].cpu().numpy()
+            ulp = np.spacing(np.maximum(np.abs(a), np.abs(b)).astype(np.float32))
+            assert np.all(np.abs(a - b) <= ulp + 1e-9 * np.abs(a).max()), n
     return compare(g32, want, TOL_BF16), g32, want
 
 
