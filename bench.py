@@ -18,7 +18,11 @@ traffic from the committed ncu summary of the same kernel source, and
 ``exp_bound``: the share of the all-MUFU exponential bound it reaches) and
 ``e2e`` (host buffers, copies in the timed region).  ``workloads`` repeats
 those figures for every bf16 workload (headline first; --only skips the
-others), with the CPB kernel's time in both forms where a workload has one.
+others), with the CPB kernel's time in both forms where a workload has one;
+a workload the tensor-core kernel does not take (Iwin's interleaved windows)
+is measured against the CUDA cores' fp32 peak ("bound": "alu").
+``backward`` times swin_window_attn_bwd on the same workloads (--no-backward
+skips it).
 Also: SM clocks sampled during the timed loops, the number of this library's
 kernel launches timed, and ``cpu_baseline`` (the oracle on the host cores and
 on one core).  ``--impl reference`` times the CPU oracle (the project's plain
@@ -68,11 +72,22 @@ def _window_counts(L, M, s):
     return out
 
 
+def _interleaved_lengths(L, M):
+    """Tokens per interleaved window along one axis: G = ceil(L/M) windows,
+    window a holds a + G i inside the axis."""
+    G = -(-L // M)
+    return [-(-(L - a) // G) for a in range(G)]
+
+
 def work(w: syn.Workload, B=None):
     B = w.B if B is None else B
     s = w.shifts[0]
-    win = sum(n * n for n in _window_counts(w.H, w.M, s)) * sum(n * n for n in _window_counts(w.W, w.M, s))
-    exact = sum(n * n for n in _seg_lengths(w.H, w.M, s)) * sum(n * n for n in _seg_lengths(w.W, w.M, s))
+    if w.partition == 1:  # interleaved windows: no padding, no mask
+        win = exact = (sum(n * n for n in _interleaved_lengths(w.H, w.M)) *
+                       sum(n * n for n in _interleaved_lengths(w.W, w.M)))
+    else:
+        win = sum(n * n for n in _window_counts(w.H, w.M, s)) * sum(n * n for n in _window_counts(w.W, w.M, s))
+        exact = sum(n * n for n in _seg_lengths(w.H, w.M, s)) * sum(n * n for n in _seg_lengths(w.W, w.M, s))
     C = w.heads * w.d
     esz = 4 if w.dtype == "f32" else 2
     return {
@@ -215,10 +230,26 @@ def whole_job(wk: dict, world: int, ms_max: float) -> dict:
             "tflops_exact": wk["flops_exact"] * world / sec / 1e12}
 
 
+FP32_LANES_PER_SM = 128  # B200: fp32 FMA lanes per SM per clock
+
+
+def on_tensor_cores(w: syn.Workload) -> bool:
+    """Whether the library runs this workload's forward on the tensor-core
+    kernel (bf16, d = 32, shifted windows, no bias table above M = 32)."""
+    has_table = w.mode != 2 and w.bias
+    return w.dtype == "bf16" and w.d == 32 and w.partition == 0 and (not has_table or w.M <= 32)
+
+
+def alu_peak_tflops(sms: int, clock_mhz: float) -> float:
+    """fp32 FMA peak of the CUDA cores: SMs x 128 lanes x 2 flop x SM clock."""
+    return sms * FP32_LANES_PER_SM * 2 * clock_mhz * 1e6 / 1e12
+
+
 def config_of(w: syn.Workload, world: int) -> dict:
     """The workload as both arms name it (same keys and values)."""
     return {"workload": w.name, "B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d, "M": w.M,
             "shift": w.shifts[0], "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode],
+            "partition": ["shifted", "interleaved"][w.partition],
             "global_batch": w.B * world, "parallelism": "replicas x%d" % world,
             "l2": "flushed before every timed step (256 MB write)", "timing": "median of per-step CUDA events"}
 
@@ -266,7 +297,8 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
     launches_per_step = 2 if "cpb" in kw else 1
 
     def step():
-        sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, workspace=ws, stream=stream, **kw)
+        sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, workspace=ws, stream=stream,
+                                partition=w.partition, **kw)
 
     timer.loop(step, max(args.warmup, 3))
     if sa.swin_stream_status(stream) != 0:
@@ -288,7 +320,8 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
         kw_k["bias_table"] = table
 
         def kstep():
-            sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, stream=stream, **kw_k)
+            sa.swin_window_attn_fwd(q, k, v, w.M, s, w.mode, out=out, stream=stream, partition=w.partition,
+                                    **kw_k)
         timer.loop(kstep, 3)
         ktimes = timer.loop(kstep, args.steps)
         launches += args.steps
@@ -305,16 +338,22 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
     k_ms = max_over_ranks(_median(ktimes), world, device)
     achieved = wk["flops_std"] / (k_ms * 1e-3) / 1e12
     hbm = wk["bytes"] / (k_ms * 1e-3) / 1e9
-    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": read_traffic("attn_tc", w), "peak_source": peaks["source"] + " (burst)",
+    if on_tensor_cores(w):
+        peak, bound, src, kname = peaks["bf16_tflops"], "tensor", peaks["source"] + " (burst)", "attn_tc"
+    else:  # the CUDA-core kernel: fp32 FMA lanes
+        peak, bound, kname = alu_peak_tflops(sms, clock_mhz), "alu", "attn_simt"
+        src = "derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz" % (sms, FP32_LANES_PER_SM, clock_mhz)
+    roofline = {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "traffic": read_traffic(kname, w), "peak_source": src, "kernel": kname,
                 "kernel_ms": round(k_ms, 5), "algorithmic_bytes": wk["bytes"],
                 "hbm_achieved_gbs": round(hbm, 1), "hbm_frac": round(hbm / peaks["hbm_gbs"], 4),
-                "attainable_frac": round(achieved / min(peaks["bf16_tflops"],
-                                                        peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3), 4),
+                "attainable_frac": round(achieved / min(peak, peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3),
+                                         4),
                 "exp_bound": exp_bound(wk, sms, clock_mhz, k_ms)}
     entry = {"workload": w.name, "config": {"B": w.B, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d, "M": w.M,
-                                            "shift": s, "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode]},
+                                            "shift": s, "mode": ["dot+bias", "cosine+cpb", "rope"][w.mode],
+                                            "partition": ["shifted", "interleaved"][w.partition]},
              "ms_per_step": round(ms, 5), "tokens_per_s": round(job["tokens_per_s"], 1),
              "tflops": round(job["tflops"], 2), "tflops_exact_pairs": round(job["tflops_exact"], 2),
              "roofline": roofline}
@@ -346,6 +385,48 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
     return entry, launches
 
 
+def time_backward(w: syn.Workload, args, timer, rank: int, world: int, sms: int, clock_mhz: float):
+    """The backward pass (swin_window_attn_bwd: dq, dk, dv and the parameter
+    gradients, softmax recomputed) of one workload, bf16 gradients.  Its
+    algorithmic work is five products of 2 d flops per attended pair (S, dP,
+    dV, dK, dQ), measured against the CUDA cores' fp32 FMA peak, where it
+    runs.  Returns (entry, launches)."""
+    import torch
+    from vision_transformer_shifted_window_b200 import swin_attn as sa
+    device, stream = timer.device, timer.stream
+    s = w.shifts[0]
+    q, k, v, kw = make_device_inputs(w, device, rank)
+    g = torch.from_numpy(syn.make_dout(w, seed=5000 + w.index + 7919 * rank)).to(device).to(q.dtype)
+    if "cpb" in kw:
+        kw["bias_table"] = sa.swin_cpb_eval(w.M, w.heads, *kw.pop("cpb"), stream=stream)
+    ws = torch.empty(sa.swin_window_attn_bwd_workspace_size(*q.shape, w.M), dtype=torch.uint8, device=device)
+    params = ("bias_table" in kw) or w.mode != 0
+
+    def step():
+        sa.swin_window_attn_bwd(q, k, v, g, w.M, s, w.mode, workspace=ws, stream=stream, partition=w.partition,
+                                **kw)
+    n = max(3, min(args.steps, 10))
+    timer.loop(step, 2)
+    times = timer.loop(step, n)
+    if sa.swin_stream_status(stream) != 0:
+        raise RuntimeError("device status after the backward of %s" % w.name)
+    ms = max_over_ranks(_median(times), world, device)
+    wk = work(w)
+    flops = 2.5 * wk["flops_exact"]
+    achieved = flops / (ms * 1e-3) / 1e12
+    peak = alu_peak_tflops(sms, clock_mhz)
+    entry = {"workload": w.name, "ms_per_step": round(ms, 4),
+             "tokens_per_s": round(wk["tokens"] * world / (ms * 1e-3), 1),
+             "roofline": {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                          "frac": round(achieved / peak, 4), "traffic": None, "kernel": "attn_bwd (q and kv passes)",
+                          "algorithmic_flops": flops,
+                          "peak_source": "derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz"
+                                         % (sms, FP32_LANES_PER_SM, clock_mhz)}}
+    del q, k, v, g, ws
+    torch.cuda.empty_cache()
+    return entry, (n + 2) * (3 if params else 2)
+
+
 def run_native(args, rank: int, world: int, local_rank: int):
     import torch
     from vision_transformer_shifted_window_b200 import build as swin_build
@@ -372,11 +453,27 @@ def run_native(args, rank: int, world: int, local_rank: int):
         e, n = time_workload(syn.WORKLOADS[idx], args, timer, rank, world, peaks, sms, clock_guess, False)
         other_entries.append(e)
         launches += n
+    bwd_entries = []
+    if not args.no_backward:
+        for idx in [args.workload] + others:
+            e, n = time_backward(syn.WORKLOADS[idx], args, timer, rank, world, sms, clock_guess)
+            bwd_entries.append(e)
+            launches += n
     clocks = sampler.stop()
     sm_mhz = float(clocks["sm_mhz"] or clocks["sm_max_mhz"] or clock_guess)
     wk = work(headline)
     for e, w in [(entry, headline)] + [(o, syn.WORKLOADS[i]) for o, i in zip(other_entries, others)]:
         e["roofline"]["exp_bound"] = exp_bound(work(w), sms, sm_mhz, e["roofline"]["kernel_ms"])
+        if e["roofline"]["bound"] == "alu":  # the derived peak at the sampled clock
+            pk = alu_peak_tflops(sms, sm_mhz)
+            e["roofline"].update(peak=round(pk, 1), frac=round(e["roofline"]["achieved"] / pk, 4),
+                                 peak_source="derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz (sampled)"
+                                             % (sms, FP32_LANES_PER_SM, sm_mhz))
+    for e in bwd_entries:
+        pk = alu_peak_tflops(sms, sm_mhz)
+        e["roofline"].update(peak=round(pk, 1), frac=round(e["roofline"]["achieved"] / pk, 4),
+                             peak_source="derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz (sampled)"
+                                         % (sms, FP32_LANES_PER_SM, sm_mhz))
     line = {
         "metric": METRIC, "value": entry["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": entry["ms_per_step"],
@@ -388,6 +485,7 @@ def run_native(args, rank: int, world: int, local_rank: int):
         "e2e": entry["e2e"],
         "clocks": clocks, "gpu_launches": launches,
         "workloads": [{k: v for k, v in entry.items() if k != "e2e"}] + other_entries,
+        "backward": bwd_entries,
     }
     return line, headline
 
@@ -422,7 +520,8 @@ def run_cpu_baseline(w: syn.Workload, budget_s: float):
         ids = np.sort(rng.choice(n_all, size=min(nq, n_all), replace=False))
         t0 = time.perf_counter()
         oracle.window_attn(inp["q"], inp["k"], inp["v"], w.M, s, w.mode, tau=inp.get("tau"), table=table,
-                           rope_freqs=inp.get("rope_freqs"), queries=ids, nthreads=nthreads)
+                           rope_freqs=inp.get("rope_freqs"), queries=ids, nthreads=nthreads,
+                           partition=w.partition)
         return len(ids), time.perf_counter() - t0
 
     def sized(budget, nthreads):
@@ -452,6 +551,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work to time")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true", help="time the headline workload alone")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurements")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -72,6 +72,20 @@ typedef enum {
 
 typedef enum { SWIN_F32 = 0, SWIN_BF16 = 1 } swin_dtype;
 
+/* How an axis of length L is cut into windows of M tokens.
+ *   SWIN_PARTITION_SHIFTED      segments with boundaries at shift + kM (Swin's
+ *        shifted windows; the page's window partition, described above);
+ *        window-local coordinate (y - shift) mod M.
+ *   SWIN_PARTITION_INTERLEAVED  G = ceil(L / M) windows per axis; window a
+ *        holds the tokens a + G i, i < M, inside the axis ("Iwin Transformer:
+ *        Hierarchical Vision Transformer using Interleaved Windows", abstract:
+ *        interleaved window attention; the pages give no index formula, this
+ *        strided grid is the reading taken); window-local coordinate i; shift
+ *        must be 0.  A window then spans the whole image.
+ * Bias-table offsets and RoPE positions use the window-local coordinates in
+ * both partitions. */
+typedef enum { SWIN_PARTITION_SHIFTED = 0, SWIN_PARTITION_INTERLEAVED = 1 } swin_partition;
+
 /* Weights of the Log-CPB meta network G ("Swin Transformer V2", §3.3, eq. 3):
  *   G(dx_hat, dy_hat) = w2 . relu(w1 . (dx_hat, dy_hat) + b1) + b2
  * with dx_hat = sign(dx) * ln(1 + |dx|) (eq. 4).  All device fp32:
@@ -160,6 +174,20 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
                                  void* workspace, size_t workspace_bytes,
                                  swin_stream_t stream);
 
+/* swin_window_attn_fwd_ex — swin_window_attn_fwd with a choice of window
+ * partition (a swin_partition; swin_window_attn_fwd is this call with
+ * SWIN_PARTITION_SHIFTED).  Interleaved windows run on the CUDA cores for
+ * every dtype (the tensor-core path gathers contiguous rectangles only).
+ * Arguments, layout, workspace and errors otherwise as swin_window_attn_fwd;
+ * an unknown partition, or a non-zero shift with interleaved windows, returns
+ * SWIN_ERR_INVALID_ARG. */
+swin_status swin_window_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
+                                    swin_dtype dt, swin_dtype out_dt, int B, int H, int W, int heads,
+                                    int d, int M, int shift, swin_partition partition, swin_mode mode,
+                                    const float* tau, const float* bias_table,
+                                    const swin_cpb_weights* cpb, const float* rope_freqs,
+                                    void* workspace, size_t workspace_bytes, swin_stream_t stream);
+
 /* swin_window_attn_fwd_noalloc — the same forward pass for callers that
  * cannot allocate device memory (a framework that owns every device byte
  * through its own pool, code running under stream capture, an embedding that
@@ -211,6 +239,7 @@ size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int hav
  *   B, H, W, heads, d, M, shift, mode, tau, rope_freqs
  *                    as swin_window_attn_fwd, except that d may be 8, 16, 32
  *                    or 64 for both dtypes
+ *   partition        a swin_partition, as swin_window_attn_fwd_ex
  *   bias_table       device fp32 [(2M-1)^2][heads] or NULL, modes 0 and 1
  *                    (mode 1 takes the table, not the CPB weights)
  *   dtable           device fp32 [(2M-1)^2][heads] or NULL; needs bias_table
@@ -227,8 +256,9 @@ size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int hav
 swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, const void* dout,
                                  void* dq, void* dk, void* dv, swin_dtype dt, swin_dtype grad_dt,
                                  int B, int H, int W, int heads, int d, int M, int shift,
-                                 swin_mode mode, const float* tau, const float* bias_table,
-                                 const float* rope_freqs, float* dtable, float* dtau, float* drope,
+                                 swin_partition partition, swin_mode mode, const float* tau,
+                                 const float* bias_table, const float* rope_freqs, float* dtable,
+                                 float* dtau, float* drope,
                                  void* workspace, size_t workspace_bytes, swin_stream_t stream);
 
 /* Bytes of workspace swin_window_attn_bwd needs: 16 per query row and head

@@ -210,7 +210,7 @@ def window_attn(q, k, v, M: int, shift: int, mode: int, tau=None, table=None,
 def window_attn_bwd(q, k, v, dout, M: int, shift: int, mode: int, tau=None, table=None, rope_freqs=None,
                     nthreads: int = 0, partition: int = PARTITION_SHIFTED) -> dict:
     """Gradients of L = sum(dout * window_attn(...)) in float64: dq, dk, dv
-    ([B, H, W, heads, d]), dtable ([(2M-1)^2, heads], modes 0 and 1), dtau
+    ([B, H, W, heads, d]), dtable ([(2M-1)^2, heads], modes 0 and 1 with a table), dtau
     ([heads], mode 1), drope ([2, d/4], mode 2)."""
     q, k, v, dout = (_f64(a) for a in (q, k, v, dout))
     B, H, W, heads, d = q.shape
@@ -218,7 +218,7 @@ def window_attn_bwd(q, k, v, dout, M: int, shift: int, mode: int, tau=None, tabl
     tau, table, rope_freqs = _f64(tau), _f64(table), _f64(rope_freqs)
     R = 2 * M - 1
     dq, dk, dv = (np.zeros_like(q) for _ in range(3))
-    dtable = np.zeros((R * R, heads)) if mode != 2 else None
+    dtable = np.zeros((R * R, heads)) if mode != 2 and table is not None else None
     dtau = np.zeros(heads) if mode == 1 else None
     drope = np.zeros((2, d // 4)) if mode == 2 else None
     rc = _load().oracle_window_attn_bwd(

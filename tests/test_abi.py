@@ -139,12 +139,13 @@ def test_bwd_workspace_size(L):
 
 def call_bwd(L, **kw):
     a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, dout=FAKE * 4, dq=FAKE * 64, dk=FAKE * 65, dv=FAKE * 66,
-             dt=sa.SWIN_F32, gdt=None, B=1, H=8, W=8, heads=1, d=32, M=4, shift=2, mode=sa.SWIN_MODE_DOT_BIAS,
+             dt=sa.SWIN_F32, gdt=None, B=1, H=8, W=8, heads=1, d=32, M=4, shift=2, part=0,
+             mode=sa.SWIN_MODE_DOT_BIAS,
              tau=None, table=None, rope=None, dtable=None, dtau=None, drope=None, ws=FAKE * 128, wsb=1 << 20)
     a.update(kw)
     return L.swin_window_attn_bwd(a["q"], a["k"], a["v"], a["dout"], a["dq"], a["dk"], a["dv"], a["dt"],
                                   a["dt"] if a["gdt"] is None else a["gdt"], a["B"], a["H"], a["W"], a["heads"],
-                                  a["d"], a["M"], a["shift"], a["mode"], a["tau"], a["table"], a["rope"],
+                                  a["d"], a["M"], a["shift"], a["part"], a["mode"], a["tau"], a["table"], a["rope"],
                                   a["dtable"], a["dtau"], a["drope"], a["ws"], a["wsb"], None)
 
 
@@ -157,7 +158,18 @@ def call_bwd(L, **kw):
     (dict(dtau=FAKE * 7), 1, "dtau"), (dict(drope=FAKE * 7), 1, "drope"),
     (dict(dt=0, gdt=1), 1, "output dtype"), (dict(d=24), 2, "d in"), (dict(ws=None), 1, "workspace"),
     (dict(wsb=256), 1, "workspace"), (dict(ws=FAKE * 128 + 16), 1, "256-byte"),
+    (dict(part=2), 1, "partition"), (dict(part=1), 1, "no shift"),
 ])
 def test_bwd_rejects_bad_arguments(L, kw, status, why):
     assert call_bwd(L, **kw) == status
     assert why in L.swin_last_error().decode()
+
+
+def test_fwd_ex_rejects_bad_partitions(L):
+    def call(part, shift):
+        return L.swin_window_attn_fwd_ex(FAKE, FAKE * 2, FAKE * 3, FAKE * 64, sa.SWIN_BF16, sa.SWIN_BF16, 1, 8, 8, 1,
+                                         32, 4, shift, part, sa.SWIN_MODE_DOT_BIAS, None, None, None, None, None, 0,
+                                         None)
+    assert call(2, 0) == sa.SWIN_ERR_INVALID_ARG and "partition" in L.swin_last_error().decode()
+    assert call(1, 2) == sa.SWIN_ERR_INVALID_ARG and "no shift" in L.swin_last_error().decode()
+    assert call(-1, 0) == sa.SWIN_ERR_INVALID_ARG

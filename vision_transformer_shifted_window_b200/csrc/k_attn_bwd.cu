@@ -25,7 +25,8 @@
 //      of 128 threads per image, head, rectangle and block of 128 queries).
 //      Pass 1 recomputes the row's log-sum-exp and D_i = g_i . o_i by an online
 //      softmax over the rectangle's keys, and stores both; pass 2 forms dl,
-//      accumulates dqt in registers and the bias gradient in shared memory.
+//      accumulates dqt in registers and the bias gradient in shared memory
+//      (in double).
 //   2. bwd_kv: one thread per key row; queries stream through shared memory
 //      with their stored statistics; accumulates dkt and dv in registers.
 //   3. bwd_finish: converts the double accumulators of the parameter
@@ -200,16 +201,30 @@ __device__ __forceinline__ void rope_grad(const A* xt, const A* g, int py, int p
   }
 }
 
-// Sum of v over the CTA into *dst (global double), v = 0 on idle threads.
+// Adds the warp's sum of v (v = 0 on idle threads) to a double in shared
+// memory.  Parameter-gradient partials are kept in double whatever the
+// arithmetic type, so the varying order of the atomic additions moves the
+// result by far less than one fp32 ulp.
 template <typename A>
-__device__ __forceinline__ void warp_sum_to(A v, A* smem_slot) {
+__device__ __forceinline__ void warp_sum_to(A v, double* smem_slot) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((threadIdx.x & 31) == 0) atomicAdd(smem_slot, v);
+  if ((threadIdx.x & 31) == 0) atomicAdd(smem_slot, (double)v);
 }
 
+// The CTA's rectangle (one window per axis) and its block of 128 rows.  Row
+// kk of the rectangle is the token (Y(kk), X(kk)) with window-local
+// coordinates (PY(kk), PX(kk)); offsets are differences of kk / lx, kk % lx.
 struct Geometry {
-  int y0, ly, x0, lx, n, chunk;
+  SwinAxis ay, ax;
+  int lx, n, chunk;
+  __device__ __forceinline__ int Y(int kk) const { return ay.start + ay.stride * (kk / lx); }
+  __device__ __forceinline__ int X(int kk) const { return ax.start + ax.stride * (kk % lx); }
+  __device__ __forceinline__ int PY(int kk) const { return ay.base + kk / lx; }
+  __device__ __forceinline__ int PX(int kk) const { return ax.base + kk % lx; }
+  __device__ __forceinline__ int rel(int qq, int kk, int M) const {
+    return swin_rel_row(qq / lx - kk / lx, qq % lx - kk % lx, M);
+  }
 };
 
 __device__ __forceinline__ Geometry geometry(const BwdArgs& a, int nsx, int chunks) {
@@ -217,11 +232,10 @@ __device__ __forceinline__ Geometry geometry(const BwdArgs& a, int nsx, int chun
   const int rect = blockIdx.x / chunks;
   g.chunk = blockIdx.x % chunks;
   const int sy = rect / nsx, sx = rect % nsx;
-  g.y0 = swin_seg_start(sy, a.M, a.shift);
-  g.ly = swin_seg_len(sy, a.H, a.M, a.shift);
-  g.x0 = swin_seg_start(sx, a.M, a.shift);
-  g.lx = swin_seg_len(sx, a.W, a.M, a.shift);
-  g.n = g.ly * g.lx;
+  g.ay = swin_axis(a.part, sy, a.H, a.M, a.shift);
+  g.ax = swin_axis(a.part, sx, a.W, a.M, a.shift);
+  g.lx = g.ax.len;
+  g.n = g.ay.len * g.lx;
   return g;
 }
 
@@ -236,19 +250,19 @@ struct Smem {
   A st0[kTile], st1[kTile];  // bwd_kv: lse and D of the query tile
   A rc[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
   A rs[(MODE == 2) ? 2 * kMaxM * (D / 4) : 1];
-  A red[1 + D / 2];  // CTA sums: d(tau), d(omega)
+  double red[1 + D / 2];  // CTA sums: d(tau), d(omega)
 };
 
 template <typename T, typename TG, typename A, int D, int MODE>
 __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int chunks) {
   constexpr int kTile = tile_rows<A, D>();
-  extern __shared__ __align__(16) unsigned char dyn[];  // A[(2M-1)^2]: this head's d(table)
+  extern __shared__ __align__(16) unsigned char dyn[];  // double[(2M-1)^2]: this head's d(table)
   __shared__ Smem<A, D, MODE> sm;
   const Geometry G = geometry(a, nsx, chunks);
   if (G.chunk * kThreads >= G.n) return;  // whole CTA idle (uniform)
   const int M = a.M, s = a.shift, h = blockIdx.y, b = blockIdx.z, R = 2 * M - 1;
   const bool want_T = MODE != 2 && a.acc_table != nullptr;
-  A* sT = reinterpret_cast<A*>(dyn);
+  double* sT = reinterpret_cast<double*>(dyn);
   if (want_T)
     for (int i = threadIdx.x; i < R * R; i += kThreads) sT[i] = 0;
   for (int i = threadIdx.x; i < 1 + D / 2; i += kThreads) sm.red[i] = 0;
@@ -261,8 +275,9 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
   const T* GO = static_cast<const T*>(a.dout);
   const int qi = G.chunk * kThreads + threadIdx.x;
   const bool active = qi < G.n;
-  const int yq = G.y0 + (active ? qi / G.lx : 0), xq = G.x0 + (active ? qi % G.lx : 0);
-  const int pyq = swin_local_coord(yq, M, s), pxq = swin_local_coord(xq, M, s);
+  const int qrow = active ? qi : 0;
+  const int yq = G.Y(qrow), xq = G.X(qrow);
+  const int pyq = G.PY(qrow), pxq = G.PX(qrow);
   const A t = MODE == 1 ? tau_eff<A>(a.tau, h) : (A)1;
   A qt[D], g[D];
   {
@@ -281,19 +296,18 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
     __syncthreads();
     for (int i = threadIdx.x; i < nk * D; i += kThreads) {
       const int j = i / D, e = i % D, kk = j0 + j;
-      const size_t off = row_off(a, b, G.y0 + kk / G.lx, G.x0 + kk % G.lx, h, D) + e;
+      const size_t off = row_off(a, b, G.Y(kk), G.X(kk), h, D) + e;
       sm.kv0[j][e] = (A)ld(K + off);
       sm.kv1[j][e] = (A)ld(V + off);
     }
     __syncthreads();
     if (MODE != 0 && threadIdx.x < nk) {
       const int kk = j0 + threadIdx.x;
-      const int yk = G.y0 + kk / G.lx, xk = G.x0 + kk % G.lx;
       A row[D];
 #pragma unroll
       for (int e = 0; e < D; ++e) row[e] = sm.kv0[threadIdx.x][e];
       bool c;
-      prep_k<A, D, MODE>(row, swin_local_coord(yk, M, s), swin_local_coord(xk, M, s), sm.rc, sm.rs, c);
+      prep_k<A, D, MODE>(row, G.PY(kk), G.PX(kk), sm.rc, sm.rs, c);
 #pragma unroll
       for (int e = 0; e < D; ++e) sm.kv0[threadIdx.x][e] = row[e];
     }
@@ -304,8 +318,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
 #pragma unroll
     for (int e = 0; e < D; ++e) dot += qt[e] * sm.kv0[j][e];
     if (MODE != 2 && a.table) {
-      const int r = swin_rel_row(yq - (G.y0 + kk / G.lx), xq - (G.x0 + kk % G.lx), M);
-      dot += (A)__ldg(a.table + (size_t)r * a.heads + h);
+      dot += (A)__ldg(a.table + (size_t)G.rel(qrow, kk, M) * a.heads + h);
     }
     return dot;
   };
@@ -356,7 +369,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
       const A dl = p * (gdotv(j) - Dq);
 #pragma unroll
       for (int e = 0; e < D; ++e) dqt[e] += dl * sm.kv0[j][e];
-      if (want_T) atomicAdd(&sT[swin_rel_row(yq - (G.y0 + kk / G.lx), xq - (G.x0 + kk % G.lx), M)], dl);
+      if (want_T) atomicAdd(&sT[G.rel(qrow, kk, M)], (double)dl);
     }
   }
 
@@ -406,10 +419,9 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
   __syncthreads();
   if (want_T)
     for (int i = threadIdx.x; i < R * R; i += kThreads)
-      if (sT[i] != (A)0) atomicAdd(a.acc_table + (size_t)i * a.heads + h, (double)sT[i]);
-  if (MODE == 1 && a.acc_tau && threadIdx.x == 0) atomicAdd(a.acc_tau + h, (double)sm.red[0]);
-  if (MODE == 2 && a.acc_rope && threadIdx.x < D / 2)
-    atomicAdd(a.acc_rope + threadIdx.x, (double)sm.red[1 + threadIdx.x]);
+      if (sT[i] != 0.0) atomicAdd(a.acc_table + (size_t)i * a.heads + h, sT[i]);
+  if (MODE == 1 && a.acc_tau && threadIdx.x == 0) atomicAdd(a.acc_tau + h, sm.red[0]);
+  if (MODE == 2 && a.acc_rope && threadIdx.x < D / 2) atomicAdd(a.acc_rope + threadIdx.x, sm.red[1 + threadIdx.x]);
 }
 
 template <typename T, typename TG, typename A, int D, int MODE>
@@ -429,8 +441,9 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
   const T* GO = static_cast<const T*>(a.dout);
   const int kj = G.chunk * kThreads + threadIdx.x;
   const bool active = kj < G.n;
-  const int yk = G.y0 + (active ? kj / G.lx : 0), xk = G.x0 + (active ? kj % G.lx : 0);
-  const int pyk = swin_local_coord(yk, M, s), pxk = swin_local_coord(xk, M, s);
+  const int krow = active ? kj : 0;
+  const int yk = G.Y(krow), xk = G.X(krow);
+  const int pyk = G.PY(krow), pxk = G.PX(krow);
   const A t = MODE == 1 ? tau_eff<A>(a.tau, h) : (A)1;
   A kt[D], vr[D];
   {
@@ -452,25 +465,24 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
     __syncthreads();
     for (int i = threadIdx.x; i < nq * D; i += kThreads) {
       const int r = i / D, e = i % D, qq = i0 + r;
-      const size_t off = row_off(a, b, G.y0 + qq / G.lx, G.x0 + qq % G.lx, h, D) + e;
+      const size_t off = row_off(a, b, G.Y(qq), G.X(qq), h, D) + e;
       sm.kv0[r][e] = (A)ld(Q + off);
       sm.kv1[r][e] = (A)ld(GO + off);
     }
     if (threadIdx.x < nq) {
       const int qq = i0 + threadIdx.x;
-      const double2 st = a.stats[(((size_t)b * a.H + G.y0 + qq / G.lx) * a.W + G.x0 + qq % G.lx) * a.heads + h];
+      const double2 st = a.stats[(((size_t)b * a.H + G.Y(qq)) * a.W + G.X(qq)) * a.heads + h];
       sm.st0[threadIdx.x] = (A)st.x;
       sm.st1[threadIdx.x] = (A)st.y;
     }
     __syncthreads();
     if (threadIdx.x < nq) {
       const int qq = i0 + threadIdx.x;
-      const int yq = G.y0 + qq / G.lx, xq = G.x0 + qq % G.lx;
       A row[D];
 #pragma unroll
       for (int e = 0; e < D; ++e) row[e] = sm.kv0[threadIdx.x][e];
       bool c;
-      prep_q<A, D, MODE>(row, t, swin_local_coord(yq, M, s), swin_local_coord(xq, M, s), sm.rc, sm.rs, c);
+      prep_q<A, D, MODE>(row, t, G.PY(qq), G.PX(qq), sm.rc, sm.rs, c);
 #pragma unroll
       for (int e = 0; e < D; ++e) sm.kv0[threadIdx.x][e] = row[e];
     }
@@ -485,8 +497,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
         gv += sm.kv1[i][e] * vr[e];
       }
       if (MODE != 2 && a.table) {
-        const int r = swin_rel_row(G.y0 + qq / G.lx - yk, G.x0 + qq % G.lx - xk, M);
-        dot += (A)__ldg(a.table + (size_t)r * a.heads + h);
+        dot += (A)__ldg(a.table + (size_t)G.rel(qq, krow, M) * a.heads + h);
       }
       const A p = a_exp(dot - sm.st0[i]);
       const A dl = p * (gv - sm.st1[i]);
@@ -536,7 +547,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
 #pragma unroll
     for (int e = 0; e < D / 2; ++e) warp_sum_to(drope[e], &sm.red[1 + e]);
     __syncthreads();
-    if (threadIdx.x < D / 2) atomicAdd(a.acc_rope + threadIdx.x, (double)sm.red[1 + threadIdx.x]);
+    if (threadIdx.x < D / 2) atomicAdd(a.acc_rope + threadIdx.x, sm.red[1 + threadIdx.x]);
   }
 }
 
@@ -557,10 +568,10 @@ __global__ void bwd_finish_kernel(const double* acc, int n_table, int n_tau, int
 
 template <typename T, typename TG, typename A, int D, int MODE>
 swin_status launch_mode(const BwdArgs& a, cudaStream_t stream) {
-  const int nsy = swin_nseg(a.H, a.M, a.shift), nsx = swin_nseg(a.W, a.M, a.shift);
+  const int nsy = swin_nwin(a.part, a.H, a.M, a.shift), nsx = swin_nwin(a.part, a.W, a.M, a.shift);
   const int chunks = (a.M * a.M + kThreads - 1) / kThreads;
   const dim3 grid(nsy * nsx * chunks, a.heads, a.B);
-  const size_t dyn = (MODE != 2 && a.acc_table) ? sizeof(A) * (size_t)(2 * a.M - 1) * (2 * a.M - 1) : 0;
+  const size_t dyn = (MODE != 2 && a.acc_table) ? sizeof(double) * (size_t)(2 * a.M - 1) * (2 * a.M - 1) : 0;
   auto kq = bwd_q_kernel<T, TG, A, D, MODE>;
   if (dyn > 0) {  // static plus dynamic shared memory may pass the 48 KB default
     cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);

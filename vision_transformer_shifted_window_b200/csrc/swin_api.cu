@@ -137,9 +137,28 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
                                  const float* bias_table, const swin_cpb_weights* cpb,
                                  const float* rope_freqs, void* workspace,
                                  size_t workspace_bytes, swin_stream_t stream) {
+  return swin_window_attn_fwd_ex(q, k, v, out, dt, out_dt, B, H, W, heads, d, M, shift, SWIN_PARTITION_SHIFTED,
+                                 mode, tau, bias_table, cpb, rope_freqs, workspace, workspace_bytes, stream);
+}
+
+static swin_status check_partition(swin_partition partition, int shift) {
+  if (partition != SWIN_PARTITION_SHIFTED && partition != SWIN_PARTITION_INTERLEAVED)
+    return fail(SWIN_ERR_INVALID_ARG, "unknown partition %d", (int)partition);
+  if (partition == SWIN_PARTITION_INTERLEAVED && shift != 0)
+    return fail(SWIN_ERR_INVALID_ARG, "interleaved windows take no shift (got %d)", shift);
+  return SWIN_OK;
+}
+
+swin_status swin_window_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, swin_dtype dt,
+                                    swin_dtype out_dt, int B, int H, int W, int heads, int d, int M, int shift,
+                                    swin_partition partition, swin_mode mode, const float* tau,
+                                    const float* bias_table, const swin_cpb_weights* cpb, const float* rope_freqs,
+                                    void* workspace, size_t workspace_bytes, swin_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   swin_status vs = swin::check_fwd_args(q, k, v, out, dt, out_dt, B, H, W, heads, d, M, shift, mode, tau,
                                         bias_table, cpb, rope_freqs);
+  if (vs != SWIN_OK) return vs;
+  vs = check_partition(partition, shift);
   if (vs != SWIN_OK) return vs;
 
   const float* table = bias_table;
@@ -159,11 +178,13 @@ swin_status swin_window_attn_fwd(const void* q, const void* k, const void* v, vo
   swin::AttnArgs a;
   a.q = q; a.k = k; a.v = v; a.out = out;
   a.B = B; a.H = H; a.W = W; a.heads = heads; a.d = d; a.M = M; a.shift = shift; a.mode = (int)mode;
+  a.part = (int)partition;
   a.tau = tau; a.table = table; a.rope = rope_freqs;
   a.status = swin::status_word();
   if (!a.status) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
-  // tensor-core path: bf16, d = 32; a bias table must fit its shared-memory slot (M <= 32)
-  if (dt == SWIN_BF16 && d == 32 && (table == nullptr || M <= 32))
+  // tensor-core path: bf16, d = 32, shifted windows; a bias table must fit its
+  // shared-memory slot (M <= 32)
+  if (dt == SWIN_BF16 && d == 32 && partition == SWIN_PARTITION_SHIFTED && (table == nullptr || M <= 32))
     return swin::launch_attn_tc(a, out_dt == SWIN_F32, st);
   return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
 }
@@ -181,13 +202,16 @@ size_t swin_window_attn_bwd_workspace_size(int B, int H, int W, int heads, int d
 
 swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, const void* dout, void* dq,
                                  void* dk, void* dv, swin_dtype dt, swin_dtype grad_dt, int B, int H, int W,
-                                 int heads, int d, int M, int shift, swin_mode mode, const float* tau,
+                                 int heads, int d, int M, int shift, swin_partition partition, swin_mode mode,
+                                 const float* tau,
                                  const float* bias_table, const float* rope_freqs, float* dtable, float* dtau,
                                  float* drope, void* workspace, size_t workspace_bytes, swin_stream_t stream) {
   // the forward's checks with dq standing for out (dtype, shape, alignment,
   // mode parameters, dq against q, k, v)
   swin_status vs = swin::check_fwd_args(q, k, v, dq, dt, grad_dt, B, H, W, heads, d, M, shift, mode, tau,
                                         bias_table, nullptr, rope_freqs);
+  if (vs != SWIN_OK) return vs;
+  vs = check_partition(partition, shift);
   if (vs != SWIN_OK) return vs;
   if (!dout || !dk || !dv) return fail(SWIN_ERR_INVALID_ARG, "dout, dk and dv must be non-NULL");
   if (!aligned16(dout) || !aligned16(dk) || !aligned16(dv))
@@ -218,6 +242,7 @@ swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, co
   swin::BwdArgs a;
   a.q = q; a.k = k; a.v = v; a.dout = dout; a.dq = dq; a.dk = dk; a.dv = dv;
   a.B = B; a.H = H; a.W = W; a.heads = heads; a.d = d; a.M = M; a.shift = shift; a.mode = (int)mode;
+  a.part = (int)partition;
   a.tau = tau; a.table = mode == SWIN_MODE_ROPE ? nullptr : bias_table; a.rope = rope_freqs;
   size_t slot = 0;
   a.acc_base = acc;

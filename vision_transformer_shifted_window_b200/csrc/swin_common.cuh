@@ -36,6 +36,7 @@ struct AttnArgs {
   const void* v;
   void* out;
   int B, H, W, heads, d, M, shift, mode;
+  int part;  // SwinPartition (the tensor-core path takes kPartShifted only)
   const float* tau;
   const float* table;  // [(2M-1)^2][heads] or nullptr
   const float* rope;   // [2][d/4] or nullptr
@@ -54,6 +55,7 @@ struct BwdArgs {
   void* dk;
   void* dv;
   int B, H, W, heads, d, M, shift, mode;
+  int part;  // SwinPartition
   const float* tau;
   const float* table;  // [(2M-1)^2][heads] or nullptr
   const float* rope;   // [2][d/4] or nullptr

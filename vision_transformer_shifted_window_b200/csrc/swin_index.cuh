@@ -69,3 +69,39 @@ SWIN_HD SwinRolled swin_rolled(int y, int x, int H, int W, int M, int s) {
   r.local = (u % M) * M + (v % M);
   return r;
 }
+
+// Partitions an axis can be cut into (see include/swin_attn.h).
+enum SwinPartition : int { kPartShifted = 0, kPartInterleaved = 1 };
+
+// One window along an axis: its tokens are start + stride * i for i < len,
+// and the window-local coordinate of token i is base + i.  Shifted windows
+// are the segments above (stride 1; base = (start - s) mod M, so the local
+// coordinates of a segment run without a wrap up to M - 1).  Interleaved
+// windows ("Iwin Transformer", abstract: interleaved window attention) take
+// G = ceil(L / M) windows per axis; window k holds k + G i inside the axis
+// (len = ceil((L - k) / G) <= M) and its local coordinate is i.  Offsets of
+// two tokens of one window are differences of their i in either partition.
+struct SwinAxis {
+  int start, stride, len, base;
+};
+
+SWIN_HD int swin_nwin(int part, int L, int M, int s) {
+  return part == kPartInterleaved ? (L + M - 1) / M : swin_nseg(L, M, s);
+}
+
+SWIN_HD SwinAxis swin_axis(int part, int k, int L, int M, int s) {
+  SwinAxis a;
+  if (part == kPartInterleaved) {
+    const int G = (L + M - 1) / M;
+    a.start = k;
+    a.stride = G;
+    a.len = (L - k + G - 1) / G;
+    a.base = 0;
+  } else {
+    a.start = swin_seg_start(k, M, s);
+    a.stride = 1;
+    a.len = swin_seg_len(k, L, M, s);
+    a.base = swin_local_coord(a.start, M, s);
+  }
+  return a;
+}

@@ -32,8 +32,12 @@ SWIN_BF16 = 1
 SWIN_CPB_PAPER = 0
 SWIN_CPB_CODE = 1
 
+SWIN_PARTITION_SHIFTED = 0
+SWIN_PARTITION_INTERLEAVED = 1
+
 #: every symbol include/swin_attn.h declares
-EXPORTED = ("swin_cpb_eval", "swin_cpb_eval_form", "swin_window_attn_fwd", "swin_window_attn_fwd_noalloc",
+EXPORTED = ("swin_cpb_eval", "swin_cpb_eval_form", "swin_window_attn_fwd", "swin_window_attn_fwd_ex",
+            "swin_window_attn_fwd_noalloc",
             "swin_window_attn_workspace_size", "swin_window_attn_bwd", "swin_window_attn_bwd_workspace_size",
             "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version",
             "swin_debug_set")
@@ -70,12 +74,15 @@ def lib():
                                            ctypes.POINTER(swin_cpb_weights), vp, vp,
                                            ctypes.c_size_t, st]
         L.swin_window_attn_fwd.restype = i
+        L.swin_window_attn_fwd_ex.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, i, vp, vp,
+                                              ctypes.POINTER(swin_cpb_weights), vp, vp, ctypes.c_size_t, st]
+        L.swin_window_attn_fwd_ex.restype = i
         L.swin_window_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp,
                                                    vp, ctypes.POINTER(swin_cpb_weights), vp, st]
         L.swin_window_attn_fwd_noalloc.restype = i
         L.swin_window_attn_workspace_size.argtypes = [i, i, i, i]
         L.swin_window_attn_workspace_size.restype = ctypes.c_size_t
-        L.swin_window_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, vp, vp,
+        L.swin_window_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, i, i, vp, vp,
                                            vp, vp, vp, vp, vp, ctypes.c_size_t, st]
         L.swin_window_attn_bwd.restype = i
         L.swin_window_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
@@ -209,10 +216,13 @@ def swin_window_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: i
                          rope_freqs: Optional[torch.Tensor] = None,
                          out: Optional[torch.Tensor] = None,
                          workspace: Optional[torch.Tensor] = None, stream=None,
-                         out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
+                         out_dtype: Optional[torch.dtype] = None,
+                         partition: int = SWIN_PARTITION_SHIFTED) -> torch.Tensor:
     """Shifted-window attention forward; q, k, v, out are [B, H, W, heads, d].
 
-    ``out_dtype`` (or the dtype of ``out``) may be float32 for bfloat16 inputs."""
+    ``out_dtype`` (or the dtype of ``out``) may be float32 for bfloat16 inputs;
+    ``partition`` SWIN_PARTITION_INTERLEAVED (with shift 0) selects Iwin's
+    interleaved windows (swin_window_attn_fwd_ex)."""
     if q.dtype == torch.float32:
         dt = SWIN_F32
     elif q.dtype == torch.bfloat16:
@@ -226,11 +236,11 @@ def swin_window_attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: i
     B, H, W, heads, d = q.shape
     with _on(stream):
         return _fwd_on_stream(q, k, v, M, shift, mode, dt, B, H, W, heads, d, tau, bias_table, cpb, rope_freqs,
-                              out, workspace, stream, out_dtype)
+                              out, workspace, stream, out_dtype, partition)
 
 
 def _fwd_on_stream(q, k, v, M, shift, mode, dt, B, H, W, heads, d, tau, bias_table, cpb, rope_freqs, out,
-                   workspace, stream, out_dtype):
+                   workspace, stream, out_dtype, partition=SWIN_PARTITION_SHIFTED):
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if out.shape != q.shape:
@@ -245,8 +255,8 @@ def _fwd_on_stream(q, k, v, M, shift, mode, dt, B, H, W, heads, d, tau, bias_tab
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib().swin_window_attn_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, mode,
+    rc = lib().swin_window_attn_fwd_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), dt, odt, B, H, W, heads, d, M, shift, int(partition), mode,
         _ptr(tau), _ptr(bias_table), ctypes.byref(cs) if cs is not None else None,
         _ptr(rope_freqs), _ptr(workspace), ws_bytes, _stream(stream))
     _check(rc)
@@ -295,7 +305,7 @@ def swin_window_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout
                          bias_table: Optional[torch.Tensor] = None,
                          rope_freqs: Optional[torch.Tensor] = None, param_grads: bool = True,
                          grad_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
-                         stream=None) -> dict:
+                         stream=None, partition: int = SWIN_PARTITION_SHIFTED) -> dict:
     """Gradients of sum(dout * swin_window_attn_fwd(...)): a dict with dq, dk, dv
     ([B, H, W, heads, d], dtype ``grad_dtype`` or q's) and, when ``param_grads``,
     dtable (with a bias table), dtau (mode 1) and drope (mode 2), fp32."""
@@ -326,7 +336,7 @@ def swin_window_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         rc = lib().swin_window_attn_bwd(
             _ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), dt, gcode,
-            B, H, W, heads, d, M, shift, mode, _ptr(tau), _ptr(bias_table), _ptr(rope_freqs),
+            B, H, W, heads, d, M, shift, int(partition), mode, _ptr(tau), _ptr(bias_table), _ptr(rope_freqs),
             _ptr(g.get("dtable")), _ptr(g.get("dtau")), _ptr(g.get("drope")), _ptr(workspace),
             workspace.numel() * workspace.element_size(), _stream(stream))
         _check(rc)

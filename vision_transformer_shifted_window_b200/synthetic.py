@@ -13,8 +13,9 @@ where the workload says so; RoPE frequencies are 100^(-t/(d/4)) per axis.
 
 The shapes follow the workloads the pages describe: Swin-T stage 1 (56x56, C=96,
 M=7), SwinV2-T at 256 px (64x64, M=16), FlashSwin-T with dense p=2 tokens
-(112x112, M=32), and a SwinV2-G-like stage 1 at 1536 px (384x384, C=512, M=24);
-no dataset is read.
+(112x112, M=32), a SwinV2-G-like stage 1 at 1536 px (384x384, C=512, M=24),
+and Iwin-T's stage 1 (Swin-T's shape with interleaved windows and no position
+bias); no dataset is read.
 """
 from __future__ import annotations
 
@@ -44,6 +45,8 @@ class Workload:
     tau: Optional[Tuple[float, float]] = None  # fixed value (a, a) or U(a, b)
     cpb_hidden: int = 0  # 0: a bias table is drawn instead (modes 0 and 1)
     rope_base: float = 0.0
+    partition: int = 0  # 0 shifted windows, 1 interleaved windows (shift 0)
+    bias: bool = True  # False: no bias table (position-free attention)
 
     @property
     def tokens(self) -> int:
@@ -60,6 +63,10 @@ WORKLOADS: Dict[int, Workload] = {
                 MODE_ROPE, rope_base=100.0),
     4: Workload(4, "swinv2-g-stage1-384x384-M24", "bf16", 2, 384, 384, 16, 32, 24, (12,),
                 MODE_COSINE_CPB, tau=(0.05, 0.2), cpb_hidden=512),
+    # Iwin-T stage 1 at 224 px: Swin-T's shape, interleaved windows, no
+    # position bias (the depthwise convolution beside it is not attention)
+    5: Workload(5, "iwin-t-stage1-56x56-M7-interleaved", "bf16", 32, 56, 56, 3, 32, 7, (0,), MODE_DOT_BIAS,
+                partition=1, bias=False),
 }
 
 
@@ -88,7 +95,7 @@ def make_inputs(w: Workload, B: Optional[int] = None, H: Optional[int] = None,
         x = g.standard_normal(shape, dtype=np.float32)
         out[name] = round_to_bf16(x) if w.dtype == "bf16" else x
     R = 2 * w.M - 1
-    if w.mode in (MODE_DOT_BIAS, MODE_COSINE_CPB):
+    if w.mode in (MODE_DOT_BIAS, MODE_COSINE_CPB) and w.bias:
         if w.cpb_hidden:
             hid = w.cpb_hidden
             out["w1"] = (0.02 * gens[3].standard_normal((hid, 2))).astype(np.float32)
