@@ -18,6 +18,12 @@ Every function states the passage it follows:
   the same definition; see the C source for the formulas).
 * ``index_tables`` — the Swin bookkeeping (window, band, local index, relative
   index) built by literally rolling a padded grid.
+* ``block`` (a submodule, plain numpy) — the projections and the residual
+  post-norm around the attention: "Swin Transformer V2", Method item 1, §3.2,
+  fig. 1, ``swin_v2_block`` pseudocode.
+* ``window_attn`` / ``window_attn_bwd`` with ``partition`` =
+  PARTITION_INTERLEAVED — the interleaved windows of the "Iwin Transformer"
+  abstract (the strided index map is a reading; see the C source).
 """
 from __future__ import annotations
 
