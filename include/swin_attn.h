@@ -266,6 +266,73 @@ swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, co
  * accumulators of the parameter gradients, rounded up to 256. */
 size_t swin_window_attn_bwd_workspace_size(int B, int H, int W, int heads, int d, int M);
 
+/* The steps either side of the attention in a Swin V2 block ("Swin
+ * Transformer V2" wiki card, Method item 1 "Residual post-norm", §3.2,
+ * fig. 1, and the swin_v2_block pseudocode): the block input x is projected
+ * to q, k and v; after the attention, its output a is projected back and
+ * layer-normalised before joining the residual path (post-norm: the norm sits
+ * on the branch's output, not on its input).  All tensors are device arrays,
+ * dense row-major, of dtype dt (fp32 or bf16), with C = heads * d channels per
+ * token; the token order is the caller's ([B][H][W] for the attention).
+ * Weights follow the usual linear-layer layout [out][in]; biases, gamma and
+ * beta are fp32.  The projections are cuBLASLt GEMMs with fp32 accumulation
+ * into the caller's workspace (fp32); the bias, the post-norm and the
+ * residual add are this library's kernels, in fp32, and every output element
+ * is rounded once: outputs of dtype out_dt (== dt, or SWIN_F32 for SWIN_BF16
+ * inputs; a bf16 output is the fp32 one rounded to nearest even).  Pointers
+ * 16-byte aligned, workspaces 256-byte aligned; C a multiple of 8.
+ * Asynchronous on the stream. */
+
+/* q = x Wq^T + bq, k = x Wk^T + bk, v = x Wv^T + bv, with
+ *   x        [tokens][C]
+ *   w_qkv    [3C][C]: the rows of Wq, then Wk, then Wv
+ *   b_qkv    fp32 [3C] or NULL (no bias)
+ *   q, k, v  [tokens][C] each (= [B][H][W][heads][d]) of dtype out_dt; must
+ *            not overlap x, each other or the workspace
+ *   workspace  swin_qkv_proj_workspace_size(tokens, C) bytes (tokens x 3C
+ *            fp32: the product before the bias) */
+swin_status swin_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
+                          swin_dtype dt, swin_dtype out_dt, int tokens, int C, void* workspace,
+                          size_t workspace_bytes, swin_stream_t stream);
+size_t swin_qkv_proj_workspace_size(int tokens, int C);
+
+/* out = x + LN(a Wo^T + bo), LN(y) = (y - mean(y)) / sqrt(var(y) + eps) *
+ * gamma + beta over the C channels of each token (biased variance), with
+ *   a        [tokens][C], the attention output
+ *   w_o      [C][C];  b_o fp32 [C] or NULL
+ *   x        [tokens][C], the residual path (the block's input)
+ *   gamma, beta  fp32 [C] or NULL (1 and 0);  eps > 0 (1e-5 is the usual)
+ *   out      [tokens][C] of dtype out_dt; must not overlap x, a or the
+ *            workspace; C <= 1024
+ *   workspace  swin_proj_postnorm_workspace_size(tokens, C) bytes (the fp32
+ *            projection) */
+swin_status swin_proj_postnorm_residual(const void* a, const void* w_o, const float* b_o, const void* x,
+                                        const float* gamma, const float* beta, float eps, void* out, swin_dtype dt,
+                                        swin_dtype out_dt, int tokens, int C, void* workspace, size_t workspace_bytes,
+                                        swin_stream_t stream);
+size_t swin_proj_postnorm_workspace_size(int tokens, int C);
+
+/* The attention half of a Swin V2 block (the swin_v2_block pseudocode's first
+ * two lines): swin_qkv_proj, swin_window_attn_fwd_ex, then
+ * swin_proj_postnorm_residual, on one stream.  x and out are
+ * [B][H][W][heads * d], out of dtype out_dt; the attention arguments are
+ * swin_window_attn_fwd_ex's; out must not overlap x.  q, k, v and the
+ * attention output are stored in dtype dt between the steps.  The workspace
+ * (swin_attn_block_workspace_size bytes, 256-byte aligned) holds them, the
+ * fp32 projections and the attention's own workspace.  Every argument is
+ * checked before the first launch. */
+swin_status swin_attn_block_fwd(const void* x, const void* w_qkv, const float* b_qkv, const void* w_o,
+                                const float* b_o, const float* gamma, const float* beta, float eps, void* out,
+                                swin_dtype dt, swin_dtype out_dt, int B, int H, int W, int heads, int d, int M,
+                                int shift,
+                                swin_partition partition, swin_mode mode, const float* tau, const float* bias_table,
+                                const swin_cpb_weights* cpb, const float* rope_freqs, void* workspace,
+                                size_t workspace_bytes, swin_stream_t stream);
+
+/* Bytes of workspace swin_attn_block_fwd needs (0 for invalid sizes). */
+size_t swin_attn_block_workspace_size(int B, int H, int W, int heads, int d, int M, swin_mode mode, int have_table,
+                                      swin_dtype dt);
+
 /* swin_index_tables — Swin's bookkeeping for an HxW grid in the rolled frame
  * (pad to Hp = ceil(H/M)*M, Wp likewise; roll by -shift; cut MxM windows), as
  * the kernels' index arithmetic sees it.  For testing; any output may be NULL.

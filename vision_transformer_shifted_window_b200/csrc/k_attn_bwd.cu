@@ -240,6 +240,7 @@ __device__ __forceinline__ Geometry geometry(const BwdArgs& a, int nsx, int chun
 }
 
 __device__ __forceinline__ size_t row_off(const BwdArgs& a, int b, int y, int x, int h, int D) {
+  SWIN_DCHECK(a.status, b >= 0 && b < a.B && y >= 0 && y < a.H && x >= 0 && x < a.W && h >= 0 && h < a.heads);
   return (((size_t)b * a.H + y) * a.W + x) * (size_t)a.heads * D + (size_t)h * D;
 }
 
@@ -369,6 +370,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
       const A dl = p * (gdotv(j) - Dq);
 #pragma unroll
       for (int e = 0; e < D; ++e) dqt[e] += dl * sm.kv0[j][e];
+      SWIN_DCHECK(a.status, !want_T || (G.rel(qrow, kk, M) >= 0 && G.rel(qrow, kk, M) < R * R));
       if (want_T) atomicAdd(&sT[G.rel(qrow, kk, M)], (double)dl);
     }
   }

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
       const int j = i / D, e = i % D, kk = j0 + j;
       const int yk = ay.start + ay.stride * (kk / lx), xk = ax.start + ax.stride * (kk % lx);
       const size_t off = (((size_t)b * a.H + yk) * a.W + xk) * C + (size_t)h * D + e;
+      SWIN_DCHECK(a.status, yk >= 0 && yk < a.H && xk >= 0 && xk < a.W && off < (size_t)a.B * a.H * a.W * C);
       ks[j][e] = (A)load_elem(K + off);
       vs[j][e] = load_elem(V + off);
     }
@@ -184,6 +185,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
   }
   if (active) {
     const A inv = (A)1 / l;
+    SWIN_DCHECK(a.status, yq >= 0 && yq < a.H && xq >= 0 && xq < a.W);
     TO* dst = O + (((size_t)b * a.H + yq) * a.W + xq) * C + (size_t)h * D;
 #pragma unroll
     for (int e = 0; e < D; ++e) dst[e] = store_conv<TO>((double)(o[e] * inv));

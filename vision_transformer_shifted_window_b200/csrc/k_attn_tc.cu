@@ -498,6 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             const int qs = qu[g] & 1;
             if (qu[g] >= 2) ok = wait_bar(&bars->q_empty[g][qs], ((qu[g] >> 1) - 1) & 1, ctl);
             if (!ok) break;
+            SWIN_DCHECK(p.status, t.h >= 0 && t.h < p.heads && r.x0 >= 0 && r.x0 + r.lx <= p.W && t.b >= 0 &&
+                                      t.b < p.B && t.y0 + r.tile * r.R >= 0 && t.y0 + r.tile * r.R < p.H);
             ptx::mbar_arrive_expect_tx(&bars->q_full[g][qs], (uint32_t)(64 * r.lx * r.R));
             ptx::tma_load_5d(qbuf + (g * 2 + qs) * kTileBytes, &p.tmap[0][r.cls], &bars->q_full[g][qs], 0, t.h,
                              r.x0, t.y0 + r.tile * r.R, t.b);
@@ -510,6 +512,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             if (ku >= (uint32_t)kStages) ok = wait_bar(&bars->kv_empty[st], ((ku / kStages) - 1) & 1, ctl);
             if (!ok) break;
             uint8_t* kb = kvbuf + st * 2 * kTileBytes;
+            SWIN_DCHECK(p.status, t.h >= 0 && t.h < p.heads && r.x0 >= 0 && r.x0 + r.lx <= p.W && t.b >= 0 &&
+                                      t.b < p.B && t.y0 + j * r.Rk >= 0 && t.y0 + j * r.Rk < p.H);
             ptx::mbar_arrive_expect_tx(&bars->kv_full[st], (uint32_t)(2 * 64 * r.lx * r.Rk));
             ptx::tma_load_5d(kb, &p.tmap[1][r.cls], &bars->kv_full[st], 0, t.h, r.x0, t.y0 + j * r.Rk, t.b);
             ptx::tma_load_5d(kb + kTileBytes, &p.tmap[2][r.cls], &bars->kv_full[st], 0, t.h, r.x0,
@@ -739,6 +743,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
     // O / l of one row to global memory (32 values; column 32 holds l)
     auto store_rows = [&](const uint32_t (&o)[32], uint32_t l, size_t off, bool row_valid) {
       if (!row_valid) return;
+#if SWIN_DEBUG_BUILD
+      if (off % 32 != 0 || off + 32 > (size_t)p.B * p.H * p.W * p.heads * 32) {
+        atomicOr(p.status, kStatusRangeCheck);
+        return;
+      }
+#endif
       const float inv = 1.0f / __uint_as_float(l);  // row sum of the fp16 P
       if (OUT_F32) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + off);
@@ -892,6 +902,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
               }
               const int4 ko = kof4[c4];  // broadcast; keys 4 c4 .. 4 c4 + 3 share a row pairwise
+#if SWIN_DEBUG_BUILD
+              // unmasked keys of a valid row read inside this warpgroup's slot
+              if (row_ok && 4 * c4 < nk) {
+                const long long i0 = (long long)(pb - ko.x - slot);
+                SWIN_DCHECK(p.status, i0 >= 0 && i0 + 1 < kSlotFloats);
+              }
+              if (row_ok && 4 * c4 + 2 < nk) {
+                const long long i1 = (long long)(pb - ko.z - slot);
+                SWIN_DCHECK(p.status, i1 >= 0 && i1 + 1 < kSlotFloats);
+              }
+#endif
               const float2 b0 = *reinterpret_cast<const float2*>(pb - ko.x);  // (bias key+1, bias key)
               const float2 b1 = *reinterpret_cast<const float2*>(pb - ko.z);
               x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(b0.y, b0.x));
@@ -909,6 +930,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
                 s1 = __fmul2_rn(make_float2(kc.z, kc.w), s1);
               }
               const int4 ko = kof4[c4];
+#if SWIN_DEBUG_BUILD
+              {
+                const int kk[4] = {ko.x, ko.y, ko.z, ko.w};
+                for (int e = 0; e < 4; ++e)
+                  if (row_ok && 4 * c4 + e < nk) {
+                    const long long ii = (long long)(hb - kk[e] - slot);
+                    SWIN_DCHECK(p.status, ii >= 0 && ii < kSlotFloats);
+                  }
+              }
+#endif
               x[2 * c4] = __ffma2_rn(x[2 * c4], s0, make_float2(hb[-ko.x], hb[-ko.y]));
               x[2 * c4 + 1] = __ffma2_rn(x[2 * c4 + 1], s1, make_float2(hb[-ko.z], hb[-ko.w]));
             }

@@ -1,0 +1,228 @@
+// The steps either side of the window attention in a Swin V2 block
+// ("Swin Transformer V2" wiki card, Method item 1 "Residual post-norm", §3.2,
+// fig. 1, and the swin_v2_block pseudocode): the projection of the block's
+// input into q, k and v, and after the attention the output projection, whose
+// result is layer-normalised before it joins the residual path:
+//   q | k | v = x W_qkv^T + b_qkv
+//   out       = x + LN(a W_o^T + b_o) * gamma + beta
+// The projections are plain GEMMs (cuBLASLt, fp32 accumulation, no cuBLAS
+// workspace) whose fp32 results land in the caller's workspace; the bias, the
+// post-norm and the residual add are this file's kernels, in fp32, and each
+// output element is rounded once (a bf16 output is the fp32 one rounded to
+// nearest even).
+#include <cublasLt.h>
+
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "swin_common.cuh"
+
+namespace swin {
+namespace {
+
+std::mutex g_lt_mu;
+cublasLtHandle_t g_lt = nullptr;
+
+// (dtype, m, n, k) -> heuristic algorithm; a GEMM shape is planned once.
+std::map<std::tuple<int, int, int, int>, cublasLtMatmulAlgo_t> g_algos;
+
+swin_status lt_fail(const char* what, cublasStatus_t st) {
+  return fail(SWIN_ERR_CUDA, "cuBLASLt %s failed (status %d)", what, (int)st);
+}
+
+// Y[rows][n] = X[rows][k] W[n][k]^T (row-major, dense), fp32 accumulation;
+// X and W fp32 or bf16, Y fp32.
+swin_status gemm_xwt(const void* X, const void* Wt, float* Y, bool bf16, int rows, int n, int k,
+                     cudaStream_t stream) {
+  std::lock_guard<std::mutex> lock(g_lt_mu);
+  cublasStatus_t st;
+  if (!g_lt) {
+    st = cublasLtCreate(&g_lt);
+    if (st != CUBLAS_STATUS_SUCCESS) return lt_fail("create", st);
+  }
+  const cudaDataType_t t = bf16 ? CUDA_R_16BF : CUDA_R_32F, to = CUDA_R_32F;
+  // Column-major view: Y^T (n x rows) = W (n x k) . X^T (k x rows), where the
+  // row-major W buffer is W^T in column-major (k x n), hence op(A) = T.
+  cublasLtMatmulDesc_t op = nullptr;
+  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  swin_status ret = SWIN_OK;
+  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
+  const float one = 1.0f, zero = 0.0f;
+  do {
+    if ((st = cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F)) != CUBLAS_STATUS_SUCCESS) {
+      ret = lt_fail("descriptor", st);
+      break;
+    }
+    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta));
+    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb));
+    if ((st = cublasLtMatrixLayoutCreate(&la, t, k, n, k)) != CUBLAS_STATUS_SUCCESS ||
+        (st = cublasLtMatrixLayoutCreate(&lb, t, k, rows, k)) != CUBLAS_STATUS_SUCCESS ||
+        (st = cublasLtMatrixLayoutCreate(&lc, to, n, rows, n)) != CUBLAS_STATUS_SUCCESS) {
+      ret = lt_fail("layout", st);
+      break;
+    }
+    const auto key = std::make_tuple((int)bf16, n, rows, k);
+    auto it = g_algos.find(key);
+    if (it == g_algos.end()) {
+      cublasLtMatmulPreference_t pref = nullptr;
+      size_t zero_ws = 0;
+      cublasLtMatmulPreferenceCreate(&pref);
+      cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &zero_ws,
+                                           sizeof(zero_ws));
+      cublasLtMatmulHeuristicResult_t res;
+      int found = 0;
+      st = cublasLtMatmulAlgoGetHeuristic(g_lt, op, la, lb, lc, lc, pref, 1, &res, &found);
+      cublasLtMatmulPreferenceDestroy(pref);
+      if (st != CUBLAS_STATUS_SUCCESS || found < 1) {
+        ret = fail(SWIN_ERR_UNSUPPORTED, "cuBLASLt has no algorithm for a %d x %d x %d GEMM", rows, n, k);
+        break;
+      }
+      it = g_algos.emplace(key, res.algo).first;
+    }
+    st = cublasLtMatmul(g_lt, op, &one, Wt, la, X, lb, &zero, Y, lc, Y, lc, &it->second, nullptr, 0, stream);
+    if (st != CUBLAS_STATUS_SUCCESS) ret = lt_fail("matmul", st);
+  } while (false);
+  if (lc) cublasLtMatrixLayoutDestroy(lc);
+  if (lb) cublasLtMatrixLayoutDestroy(lb);
+  if (la) cublasLtMatrixLayoutDestroy(la);
+  if (op) cublasLtMatmulDescDestroy(op);
+  return ret;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// q, k, v = the fp32 product y [tokens][3C] plus b (NULL: 0), split by
+// channel thirds and rounded once to T (grid-stride over tokens x C).
+template <typename T>
+__global__ void bias_split_kernel(const float* __restrict__ y, const float* b, T* q, T* k, T* v, long long n,
+                                  int C) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long t = i / C;
+    const int c = (int)(i - t * C);
+    const float* yr = y + t * 3 * C;
+    q[i] = from_f<T>(yr[c] + (b ? __ldg(b + c) : 0.f));
+    k[i] = from_f<T>(yr[C + c] + (b ? __ldg(b + C + c) : 0.f));
+    v[i] = from_f<T>(yr[2 * C + c] + (b ? __ldg(b + 2 * C + c) : 0.f));
+  }
+}
+
+// out[t] = x[t] + gamma * (y[t] + b - mean) / sqrt(var + eps) + beta, one warp
+// per token row; y is the fp32 projection.  Mean and variance are two passes
+// over the row held in registers (fp32; the row is at most kMaxC channels).
+constexpr int kMaxC = 1024;
+
+template <typename T, typename TO>
+__global__ void postnorm_residual_kernel(const T* __restrict__ x, const float* __restrict__ yall, TO* out,
+                                         const float* b, const float* gamma, const float* beta, float eps,
+                                         long long tokens, int C) {
+  constexpr int kPer = kMaxC / 32;
+  const int lane = threadIdx.x & 31;
+  const long long warp = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long t = warp; t < tokens; t += nwarps) {
+    const float* yr = yall + t * C;
+    TO* row = out + t * C;
+    float y[kPer];
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int c = lane + 32 * j;
+      y[j] = 0.f;
+      if (c < C) {
+        y[j] = yr[c] + (b ? __ldg(b + c) : 0.f);
+        s += y[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / (float)C;
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int c = lane + 32 * j;
+      if (c < C) ss += (y[j] - mean) * (y[j] - mean);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = rsqrtf(ss / (float)C + eps);
+    const T* xr = x + t * C;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int c = lane + 32 * j;
+      if (c < C) {
+        const float g = gamma ? __ldg(gamma + c) : 1.f, be = beta ? __ldg(beta + c) : 0.f;
+        row[c] = from_f<TO>(to_f(xr[c]) + (y[j] - mean) * rstd * g + be);
+      }
+    }
+  }
+}
+
+int grid_for(long long work, int per_block) {
+  long long g = (work + per_block - 1) / per_block;
+  return (int)(g < 148 * 16 ? (g < 1 ? 1 : g) : 148 * 16);
+}
+
+}  // namespace
+
+swin_status launch_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
+                            bool bf16, bool f32_out, int tokens, int C, float* y, cudaStream_t stream) {
+  swin_status s = gemm_xwt(x, w_qkv, y, bf16, tokens, 3 * C, C, stream);
+  if (s != SWIN_OK) return s;
+  const long long n = (long long)tokens * C;
+  if (bf16 && !f32_out)
+    bias_split_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, stream>>>(
+        y, b_qkv, static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(v), n,
+        C);
+  else
+    bias_split_kernel<float><<<grid_for(n, 256), 256, 0, stream>>>(
+        y, b_qkv, static_cast<float*>(q), static_cast<float*>(k), static_cast<float*>(v), n, C);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "bias launch: %s", cudaGetErrorString(e));
+  return SWIN_OK;
+}
+
+swin_status launch_proj_postnorm(const void* a, const void* w_o, const float* b_o, const void* x,
+                                 const float* gamma, const float* beta, float eps, void* out, bool bf16, bool f32_out,
+                                 int tokens, int C, float* y, cudaStream_t stream) {
+  if (C > kMaxC) return fail(SWIN_ERR_UNSUPPORTED, "post-norm supports C <= %d, got %d", kMaxC, C);
+  swin_status s = gemm_xwt(a, w_o, y, bf16, tokens, C, C, stream);
+  if (s != SWIN_OK) return s;
+  const int blocks = grid_for((long long)tokens, 8);
+  using bf = __nv_bfloat16;
+  if (bf16 && !f32_out)
+    postnorm_residual_kernel<bf, bf><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y, static_cast<bf*>(out),
+                                                                 b_o, gamma, beta, eps, tokens, C);
+  else if (bf16)
+    postnorm_residual_kernel<bf, float><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y,
+                                                                    static_cast<float*>(out), b_o, gamma, beta, eps,
+                                                                    tokens, C);
+  else
+    postnorm_residual_kernel<float, float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), y,
+                                                                       static_cast<float*>(out), b_o, gamma, beta,
+                                                                       eps, tokens, C);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "post-norm launch: %s", cudaGetErrorString(e));
+  return SWIN_OK;
+}
+
+}  // namespace swin

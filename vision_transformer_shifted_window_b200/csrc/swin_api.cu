@@ -252,8 +252,131 @@ swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, co
   slot += dtau ? (size_t)heads : 0;
   a.acc_rope = drope ? acc + slot : nullptr;
   a.stats = reinterpret_cast<double2*>(static_cast<char*>(workspace) + acc_bytes);
+  a.status = swin::status_word();
+  if (!a.status) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
   return swin::launch_attn_bwd(a, dt == SWIN_BF16, grad_dt == SWIN_F32, dtable, dtau, drope,
                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+static swin_status check_proj(const void* const* ptrs, int n, swin_dtype dt, swin_dtype out_dt, int tokens, int C) {
+  for (int i = 0; i < n; ++i)
+    if (!ptrs[i]) return fail(SWIN_ERR_INVALID_ARG, "tensor arguments must be non-NULL");
+  for (int i = 0; i < n; ++i)
+    if (!aligned16(ptrs[i])) return fail(SWIN_ERR_INVALID_ARG, "tensor arguments must be 16-byte aligned");
+  if (dt != SWIN_F32 && dt != SWIN_BF16) return fail(SWIN_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+  if (out_dt != dt && !(dt == SWIN_BF16 && out_dt == SWIN_F32))
+    return fail(SWIN_ERR_INVALID_ARG, "output dtype %d not allowed for input dtype %d", (int)out_dt, (int)dt);
+  if (tokens < 1 || C < 1) return fail(SWIN_ERR_INVALID_ARG, "tokens and C must be >= 1");
+  if ((long long)tokens * C * 3 >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "tokens*3C must be < 2^31");
+  if (C % 8 != 0) return fail(SWIN_ERR_INVALID_ARG, "C must be a multiple of 8 (16-byte rows), got %d", C);
+  return SWIN_OK;
+}
+
+static size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+static swin_status check_ws(void* ws, size_t have, size_t need) {
+  if (!ws || have < need) return fail(SWIN_ERR_INVALID_ARG, "workspace of %zu bytes needed, got %zu", need, have);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(SWIN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  return SWIN_OK;
+}
+
+size_t swin_qkv_proj_workspace_size(int tokens, int C) {
+  if (tokens < 1 || C < 1) return 0;
+  return align256(sizeof(float) * (size_t)tokens * 3 * C);
+}
+
+size_t swin_proj_postnorm_workspace_size(int tokens, int C) {
+  if (tokens < 1 || C < 1) return 0;
+  return align256(sizeof(float) * (size_t)tokens * C);
+}
+
+swin_status swin_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
+                          swin_dtype dt, swin_dtype out_dt, int tokens, int C, void* workspace,
+                          size_t workspace_bytes, swin_stream_t stream) {
+  const void* ptrs[5] = {x, w_qkv, q, k, v};
+  swin_status vs = check_proj(ptrs, 5, dt, out_dt, tokens, C);
+  if (vs != SWIN_OK) return vs;
+  const size_t need = swin_qkv_proj_workspace_size(tokens, C);
+  if ((vs = check_ws(workspace, workspace_bytes, need)) != SWIN_OK) return vs;
+  const size_t xb = (size_t)tokens * C * (dt == SWIN_F32 ? 4 : 2), ob = (size_t)tokens * C * (out_dt == SWIN_F32 ? 4 : 2);
+  const void* outs[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    if (overlaps(outs[i], ob, x, xb) || overlaps(outs[i], ob, workspace, need))
+      return fail(SWIN_ERR_INVALID_ARG, "q, k and v must not overlap x or the workspace");
+    for (int j = i + 1; j < 3; ++j)
+      if (overlaps(outs[i], ob, outs[j], ob)) return fail(SWIN_ERR_INVALID_ARG, "q, k and v must not overlap");
+  }
+  return swin::launch_qkv_proj(x, w_qkv, b_qkv, q, k, v, dt == SWIN_BF16, out_dt == SWIN_F32, tokens, C,
+                               static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+swin_status swin_proj_postnorm_residual(const void* a, const void* w_o, const float* b_o, const void* x,
+                                        const float* gamma, const float* beta, float eps, void* out, swin_dtype dt,
+                                        swin_dtype out_dt, int tokens, int C, void* workspace, size_t workspace_bytes,
+                                        swin_stream_t stream) {
+  const void* ptrs[4] = {a, w_o, x, out};
+  swin_status vs = check_proj(ptrs, 4, dt, out_dt, tokens, C);
+  if (vs != SWIN_OK) return vs;
+  if (!(eps > 0.0f)) return fail(SWIN_ERR_INVALID_ARG, "eps must be > 0");
+  if (C > 1024) return fail(SWIN_ERR_UNSUPPORTED, "post-norm supports C <= 1024, got %d", C);
+  const size_t need = swin_proj_postnorm_workspace_size(tokens, C);
+  if ((vs = check_ws(workspace, workspace_bytes, need)) != SWIN_OK) return vs;
+  const size_t xb = (size_t)tokens * C * (dt == SWIN_F32 ? 4 : 2), ob = (size_t)tokens * C * (out_dt == SWIN_F32 ? 4 : 2);
+  if (overlaps(out, ob, x, xb) || overlaps(out, ob, a, xb) || overlaps(out, ob, workspace, need))
+    return fail(SWIN_ERR_INVALID_ARG, "out must not overlap x, a or the workspace");
+  return swin::launch_proj_postnorm(a, w_o, b_o, x, gamma, beta, eps, out, dt == SWIN_BF16, out_dt == SWIN_F32,
+                                    tokens, C, static_cast<float*>(workspace), reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t swin_attn_block_workspace_size(int B, int H, int W, int heads, int d, int M, swin_mode mode, int have_table,
+                                      swin_dtype dt) {
+  if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1) return 0;
+  const size_t tokens = (size_t)B * H * W, C = (size_t)heads * d;
+  const size_t tb = align256(tokens * C * (dt == SWIN_F32 ? 4 : 2));
+  return 4 * tb + align256(sizeof(float) * tokens * 3 * C) + swin_window_attn_workspace_size(M, heads, mode, have_table);
+}
+
+swin_status swin_attn_block_fwd(const void* x, const void* w_qkv, const float* b_qkv, const void* w_o,
+                                const float* b_o, const float* gamma, const float* beta, float eps, void* out,
+                                swin_dtype dt, swin_dtype out_dt, int B, int H, int W, int heads, int d, int M,
+                                int shift, swin_partition partition, swin_mode mode, const float* tau,
+                                const float* bias_table, const swin_cpb_weights* cpb, const float* rope_freqs,
+                                void* workspace, size_t workspace_bytes, swin_stream_t stream) {
+  if (B < 1 || H < 1 || W < 1 || heads < 1 || d < 1) return fail(SWIN_ERR_INVALID_ARG, "B, H, W, heads and d must be >= 1");
+  const long long tokens = (long long)B * H * W;
+  if (tokens >= (1ll << 31)) return fail(SWIN_ERR_UNSUPPORTED, "B*H*W must be < 2^31");
+  const int C = heads * d;
+  const void* ptrs[4] = {x, w_qkv, w_o, out};
+  swin_status st = check_proj(ptrs, 4, dt, out_dt, (int)tokens, C);
+  if (st != SWIN_OK) return st;
+  const size_t need = swin_attn_block_workspace_size(B, H, W, heads, d, M, mode, bias_table != nullptr, dt);
+  if ((st = check_ws(workspace, workspace_bytes, need)) != SWIN_OK) return st;
+  const size_t tb = align256((size_t)tokens * C * (dt == SWIN_F32 ? 4 : 2));
+  const size_t yb = align256(sizeof(float) * (size_t)tokens * 3 * C);
+  const size_t ob = (size_t)tokens * C * (out_dt == SWIN_F32 ? 4 : 2);
+  char* ws = static_cast<char*>(workspace);
+  void *q = ws, *k = ws + tb, *v = ws + 2 * tb, *att = ws + 3 * tb;
+  float* y = reinterpret_cast<float*>(ws + 4 * tb);
+  if (overlaps(out, ob, x, (size_t)tokens * C * (dt == SWIN_F32 ? 4 : 2)))
+    return fail(SWIN_ERR_INVALID_ARG, "out must not overlap x");
+  if (overlaps(out, ob, workspace, need) || overlaps(x, tb, workspace, need))
+    return fail(SWIN_ERR_INVALID_ARG, "x and out must not overlap the workspace");
+  // every attention argument is checked before the first launch
+  st = swin::check_fwd_args(q, k, v, att, dt, dt, B, H, W, heads, d, M, shift, mode, tau, bias_table, cpb,
+                            rope_freqs);
+  if (st != SWIN_OK) return st;
+  st = check_partition(partition, shift);
+  if (st != SWIN_OK) return st;
+  if (!(eps > 0.0f)) return fail(SWIN_ERR_INVALID_ARG, "eps must be > 0");
+  if (C > 1024) return fail(SWIN_ERR_UNSUPPORTED, "post-norm supports C <= 1024, got %d", C);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = swin::launch_qkv_proj(x, w_qkv, b_qkv, q, k, v, dt == SWIN_BF16, false, (int)tokens, C, y, s);
+  if (st != SWIN_OK) return st;
+  st = swin_window_attn_fwd_ex(q, k, v, att, dt, dt, B, H, W, heads, d, M, shift, partition, mode, tau, bias_table,
+                               cpb, rope_freqs, ws + 4 * tb + yb, workspace_bytes - 4 * tb - yb, stream);
+  if (st != SWIN_OK) return st;
+  return swin::launch_proj_postnorm(att, w_o, b_o, x, gamma, beta, eps, out, dt == SWIN_BF16, out_dt == SWIN_F32,
+                                    (int)tokens, C, y, s);
 }
 
 swin_status swin_index_tables(int H, int W, int M, int shift, int32_t* tok_window,
@@ -282,6 +405,9 @@ swin_status swin_stream_status(swin_stream_t stream) {
   if (cudaMemcpy(&val, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
       cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return fail(SWIN_ERR_CUDA, "reading the device status word failed");
+  if (val & swin::kStatusRangeCheck)
+    return fail(SWIN_ERR_CUDA, "a range check of the SWIN_DEBUG build failed (an index outside its buffer; "
+                               "the access was skipped)");
   if (val & SWIN_ERR_TIMEOUT) return fail(SWIN_ERR_TIMEOUT, "a kernel's bounded wait ran out");
   if (val & SWIN_ERR_UNSUPPORTED)
     return fail(SWIN_ERR_UNSUPPORTED, "an operand left the fp16 range on the tensor-core path (a RoPE-rotated k or a V entry of magnitude >= 65504)");

@@ -25,6 +25,23 @@ swin_status check_fwd_args(const void* q, const void* k, const void* v, const vo
                            swin_mode mode, const float* tau, const float* bias_table,
                            const swin_cpb_weights* cpb, const float* rope_freqs);
 
+// Status bit a SWIN_DEBUG build's kernels OR into the status word when an
+// index check fails (the access is then skipped where skipping is safe);
+// swin_stream_status reports it.  Release builds compile the checks away.
+constexpr int kStatusRangeCheck = 0x100;
+#ifdef SWIN_DEBUG
+#define SWIN_DCHECK(status_ptr, cond)                                  \
+  do {                                                                 \
+    if (!(cond)) atomicOr((status_ptr), ::swin::kStatusRangeCheck);    \
+  } while (0)
+#define SWIN_DEBUG_BUILD 1
+#else
+#define SWIN_DCHECK(status_ptr, cond) \
+  do {                                \
+  } while (0)
+#define SWIN_DEBUG_BUILD 0
+#endif
+
 // fp32 RoPE tables are built in the kernels from the caller's frequencies.
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kTauMin = 0.01f;
@@ -64,6 +81,7 @@ struct BwdArgs {
   double* acc_tau;
   double* acc_rope;
   double2* stats;  // [B][H][W][heads]: (log-sum-exp, D) of each query row
+  int* status;     // device status word (range checks of a SWIN_DEBUG build)
 };
 
 // Launchers (one per translation unit).
@@ -74,6 +92,12 @@ swin_status launch_index_tables(int H, int W, int M, int shift, int32_t* tw, int
 swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream);
 void tc_set_debug(int flags, long long wait_limit);
 swin_status launch_attn_simt(const AttnArgs& a, bool bf16_in, bool f32_out, cudaStream_t stream);
+// y: fp32 scratch of tokens x 3C (qkv) or tokens x C (post-norm) floats.
+swin_status launch_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
+                            bool bf16, bool f32_out, int tokens, int C, float* y, cudaStream_t stream);
+swin_status launch_proj_postnorm(const void* a, const void* w_o, const float* b_o, const void* x,
+                                 const float* gamma, const float* beta, float eps, void* out, bool bf16, bool f32_out,
+                                 int tokens, int C, float* y, cudaStream_t stream);
 swin_status launch_attn_bwd(const BwdArgs& a, bool bf16_in, bool f32_grad, float* dtable, float* dtau,
                             float* drope, cudaStream_t stream);
 

@@ -15,7 +15,9 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libswinattn.so")
+#: SWIN_ATTN_DEBUG=1 selects the range-checking build (build.py --debug)
+DEBUG_BUILD = os.environ.get("SWIN_ATTN_DEBUG", "0") == "1"
+LIB_PATH = os.path.join(_PKG, "libswinattn_debug.so" if DEBUG_BUILD else "libswinattn.so")
 
 SWIN_OK = 0
 SWIN_ERR_INVALID_ARG = 1
@@ -39,6 +41,8 @@ SWIN_PARTITION_INTERLEAVED = 1
 EXPORTED = ("swin_cpb_eval", "swin_cpb_eval_form", "swin_window_attn_fwd", "swin_window_attn_fwd_ex",
             "swin_window_attn_fwd_noalloc",
             "swin_window_attn_workspace_size", "swin_window_attn_bwd", "swin_window_attn_bwd_workspace_size",
+            "swin_qkv_proj", "swin_proj_postnorm_residual", "swin_attn_block_fwd", "swin_attn_block_workspace_size",
+            "swin_qkv_proj_workspace_size", "swin_proj_postnorm_workspace_size",
             "swin_index_tables", "swin_stream_status", "swin_last_error", "swin_version",
             "swin_debug_set")
 
@@ -62,8 +66,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError("libswinattn.so is not built; run "
-                               "`python -m vision_transformer_shifted_window_b200.build`")
+            raise RuntimeError("%s is not built; run `python -m vision_transformer_shifted_window_b200.build%s`"
+                               % (os.path.basename(LIB_PATH), " --debug" if DEBUG_BUILD else ""))
         L = ctypes.CDLL(LIB_PATH)
         vp, i, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p
         L.swin_cpb_eval.argtypes = [i, i, ctypes.POINTER(swin_cpb_weights), vp, st]
@@ -87,6 +91,21 @@ def lib():
         L.swin_window_attn_bwd.restype = i
         L.swin_window_attn_bwd_workspace_size.argtypes = [i, i, i, i, i, i]
         L.swin_window_attn_bwd_workspace_size.restype = ctypes.c_size_t
+        L.swin_qkv_proj.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, vp, ctypes.c_size_t, st]
+        L.swin_qkv_proj.restype = i
+        L.swin_qkv_proj_workspace_size.argtypes = [i, i]
+        L.swin_qkv_proj_workspace_size.restype = ctypes.c_size_t
+        L.swin_proj_postnorm_residual.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, i, i, i, i, vp,
+                                                  ctypes.c_size_t, st]
+        L.swin_proj_postnorm_residual.restype = i
+        L.swin_proj_postnorm_workspace_size.argtypes = [i, i]
+        L.swin_proj_postnorm_workspace_size.restype = ctypes.c_size_t
+        L.swin_attn_block_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, i, i, i, i, i, i, i, i,
+                                          i, i, i, vp, vp, ctypes.POINTER(swin_cpb_weights), vp, vp,
+                                          ctypes.c_size_t, st]
+        L.swin_attn_block_fwd.restype = i
+        L.swin_attn_block_workspace_size.argtypes = [i, i, i, i, i, i, i, i, i]
+        L.swin_attn_block_workspace_size.restype = ctypes.c_size_t
         L.swin_index_tables.argtypes = [i, i, i, i, vp, vp, vp, vp, st]
         L.swin_index_tables.restype = i
         L.swin_stream_status.argtypes = [st]
@@ -341,6 +360,114 @@ def swin_window_attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, dout
             workspace.numel() * workspace.element_size(), _stream(stream))
         _check(rc)
     return g
+
+
+def _dtcode(t: torch.Tensor) -> int:
+    dt = {torch.float32: SWIN_F32, torch.bfloat16: SWIN_BF16}.get(t.dtype)
+    if dt is None:
+        raise ValueError("tensors must be float32 or bfloat16")
+    return dt
+
+
+def _scratch(workspace, need, device):
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def swin_qkv_proj(x: torch.Tensor, w_qkv: torch.Tensor, b_qkv: Optional[torch.Tensor] = None,
+                  out_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """q, k, v = x W^T + b split three ways: x [..., C], w_qkv [3C, C] (x's
+    dtype), b_qkv fp32 [3C] or None.  Returns three tensors of x's shape
+    (dtype ``out_dtype``: x's, or float32 for bfloat16 x)."""
+    dt = _dtcode(x)
+    C = int(x.shape[-1])
+    tokens = x.numel() // C
+    _shape("w_qkv", w_qkv, (3 * C, C))
+    if w_qkv.dtype != x.dtype:
+        raise ValueError("w_qkv must have x's dtype")
+    odt = out_dtype or x.dtype
+    with _on(stream):
+        b_qkv = _f32(b_qkv)
+        _shape("b_qkv", b_qkv, (3 * C,))
+        q, k, v = (torch.empty(x.shape, dtype=odt, device=x.device) for _ in range(3))
+        ws, wsb = _scratch(workspace, int(lib().swin_qkv_proj_workspace_size(tokens, C)), x.device)
+        _check(lib().swin_qkv_proj(_ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(q), _ptr(k), _ptr(v), dt, _dtcode(q),
+                                   tokens, C, _ptr(ws), wsb, _stream(stream)))
+    return q, k, v
+
+
+def swin_proj_postnorm_residual(a: torch.Tensor, w_o: torch.Tensor, b_o: Optional[torch.Tensor], x: torch.Tensor,
+                                gamma: Optional[torch.Tensor] = None, beta: Optional[torch.Tensor] = None,
+                                eps: float = 1e-5, out: Optional[torch.Tensor] = None,
+                                out_dtype: Optional[torch.dtype] = None, workspace: Optional[torch.Tensor] = None,
+                                stream=None) -> torch.Tensor:
+    """out = x + LayerNorm(a W_o^T + b_o) (gamma, beta fp32 [C]); a, x [..., C];
+    out of dtype ``out_dtype`` (x's, or float32 for bfloat16 x)."""
+    dt = _dtcode(x)
+    C = int(x.shape[-1])
+    tokens = x.numel() // C
+    if a.shape != x.shape or a.dtype != x.dtype or w_o.dtype != x.dtype:
+        raise ValueError("a must match x; w_o must have x's dtype")
+    _shape("w_o", w_o, (C, C))
+    with _on(stream):
+        b_o, gamma, beta = _f32(b_o), _f32(gamma), _f32(beta)
+        for n, t in (("b_o", b_o), ("gamma", gamma), ("beta", beta)):
+            _shape(n, t, (C,))
+        if out is None:
+            out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+        ws, wsb = _scratch(workspace, int(lib().swin_proj_postnorm_workspace_size(tokens, C)), x.device)
+        _check(lib().swin_proj_postnorm_residual(_ptr(a), _ptr(w_o), _ptr(b_o), _ptr(x), _ptr(gamma), _ptr(beta),
+                                                 float(eps), _ptr(out), dt, _dtcode(out), tokens, C, _ptr(ws), wsb,
+                                                 _stream(stream)))
+    return out
+
+
+def swin_attn_block_workspace_size(B, H, W, heads, d, M, mode, have_table, dtype) -> int:
+    return int(lib().swin_attn_block_workspace_size(B, H, W, heads, d, M, mode, int(bool(have_table)),
+                                                    SWIN_F32 if dtype == torch.float32 else SWIN_BF16))
+
+
+def swin_attn_block_fwd(x: torch.Tensor, heads: int, w_qkv: torch.Tensor, b_qkv: Optional[torch.Tensor],
+                        w_o: torch.Tensor, b_o: Optional[torch.Tensor], gamma: Optional[torch.Tensor],
+                        beta: Optional[torch.Tensor], M: int, shift: int, mode: int, eps: float = 1e-5,
+                        tau=None, bias_table=None, cpb=None, rope_freqs=None, partition: int = SWIN_PARTITION_SHIFTED,
+                        out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                        stream=None, out_dtype: Optional[torch.dtype] = None) -> torch.Tensor:
+    """x + LN(proj(window_attention(qkv(x)))) for x [B, H, W, C], C = heads * d;
+    out of dtype ``out_dtype`` (x's, or float32 for bfloat16 x)."""
+    dt = _dtcode(x)
+    if x.dim() != 4:
+        raise ValueError("x must be [B, H, W, C]")
+    B, H, W, C = x.shape
+    if C % heads:
+        raise ValueError("C must be a multiple of heads")
+    d = C // heads
+    _shape("w_qkv", w_qkv, (3 * C, C))
+    _shape("w_o", w_o, (C, C))
+    if w_qkv.dtype != x.dtype or w_o.dtype != x.dtype:
+        raise ValueError("weights must have x's dtype")
+    with _on(stream):
+        b_qkv, b_o, gamma, beta = _f32(b_qkv), _f32(b_o), _f32(gamma), _f32(beta)
+        _shape("b_qkv", b_qkv, (3 * C,))
+        for n, t in (("b_o", b_o), ("gamma", gamma), ("beta", beta)):
+            _shape(n, t, (C,))
+        tau, bias_table, rope_freqs = _f32(tau), _f32(bias_table), _f32(rope_freqs)
+        _param_shapes(M, heads, d, tau, bias_table, rope_freqs)
+        cs, keep = _cpb_struct(cpb, heads)
+        need = swin_attn_block_workspace_size(B, H, W, heads, d, M, mode, bias_table is not None, x.dtype)
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+        if out is None:
+            out = torch.empty(x.shape, dtype=out_dtype or x.dtype, device=x.device)
+        _check(lib().swin_attn_block_fwd(
+            _ptr(x), _ptr(w_qkv), _ptr(b_qkv), _ptr(w_o), _ptr(b_o), _ptr(gamma), _ptr(beta), float(eps), _ptr(out),
+            dt, _dtcode(out), B, H, W, heads, d, M, shift, int(partition), mode, _ptr(tau), _ptr(bias_table),
+            ctypes.byref(cs) if cs is not None else None, _ptr(rope_freqs), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream)))
+        del keep
+    return out
 
 
 def swin_index_tables(H: int, W: int, M: int, shift: int, device="cuda", stream=None):

@@ -126,3 +126,31 @@ def make_dout(w: Workload, B: Optional[int] = None, H: Optional[int] = None, W: 
     g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(5000 + w.index if seed is None else seed)))
     x = g.standard_normal((B, H, W, w.heads, w.d), dtype=np.float32)
     return round_to_bf16(x) if w.dtype == "bf16" else x
+
+
+def make_block_inputs(w: Workload, B: Optional[int] = None, H: Optional[int] = None, W: Optional[int] = None,
+                      seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Block input x [B, H, W, C] ~ N(0, 1) and the parameters around the
+    attention (SeedSequence(9000 + index) unless ``seed``, spawned into eight
+    streams in this order): w_qkv [3C, C] and w_o [C, C] ~ N(0, 1/C) (so q, k,
+    v and the projection keep unit scale), b_qkv [3C] and b_o [C] ~ N(0, 0.02),
+    gamma ~ 1 + N(0, 0.1) and beta ~ N(0, 0.1) over C; x and the weights are
+    rounded to bf16 for bf16 workloads, biases and norm parameters stay fp32.
+    The attention's own parameters come from ``make_inputs``."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    W = w.W if W is None else W
+    C = w.heads * w.d
+    ss = np.random.SeedSequence(9000 + w.index if seed is None else seed)
+    g = [np.random.Generator(np.random.PCG64(c)) for c in ss.spawn(8)]
+    rb = (lambda a: round_to_bf16(a)) if w.dtype == "bf16" else (lambda a: a)
+    f32 = lambda a: a.astype(np.float32)
+    return {
+        "x": rb(g[0].standard_normal((B, H, W, C), dtype=np.float32)),
+        "w_qkv": rb(f32(g[1].standard_normal((3 * C, C)) / np.sqrt(C))),
+        "b_qkv": f32(0.02 * g[2].standard_normal(3 * C)),
+        "w_o": rb(f32(g[3].standard_normal((C, C)) / np.sqrt(C))),
+        "b_o": f32(0.02 * g[4].standard_normal(C)),
+        "gamma": f32(1.0 + 0.1 * g[5].standard_normal(C)),
+        "beta": f32(0.1 * g[6].standard_normal(C)),
+    }
