@@ -22,7 +22,8 @@ others), with the CPB kernel's time in both forms where a workload has one;
 a workload the tensor-core kernel does not take (Iwin's interleaved windows)
 is measured against the CUDA cores' fp32 peak ("bound": "alu").
 ``backward`` times swin_window_attn_bwd on the same workloads (--no-backward
-skips it).
+skips it); ``block`` times the attention half of a Swin V2 block
+(swin_attn_block_fwd) and its projection steps against HBM (--no-block).
 Also: SM clocks sampled during the timed loops, the number of this library's
 kernel launches timed, and ``cpu_baseline`` (the oracle on the host cores and
 on one core).  ``--impl reference`` times the CPU oracle (the project's plain
@@ -424,7 +425,73 @@ def time_backward(w: syn.Workload, args, timer, rank: int, world: int, sms: int,
                                          % (sms, FP32_LANES_PER_SM, clock_mhz)}}
     del q, k, v, g, ws
     torch.cuda.empty_cache()
-    return entry, (n + 2) * (3 if params else 2)
+    return entry, n * (3 if params else 2)
+
+
+def time_block(w: syn.Workload, args, timer, rank: int, world: int, peaks: dict):
+    """The attention half of a Swin V2 block on one workload (swin_attn_block_fwd:
+    qkv projection, the attention, output projection with the residual
+    post-norm), bf16, and its two projection steps alone.  The projections
+    are memory-bound at these widths (K = C <= 512), so each step is set
+    against HBM: its algorithmic bytes are the tensors it must read and write
+    once (x and W in, q, k, v out; a, x and W_o in, out out).  Returns
+    (entry, launches)."""
+    import torch
+    from vision_transformer_shifted_window_b200 import swin_attn as sa
+    device, stream = timer.device, timer.stream
+    s = w.shifts[0]
+    _, _, _, kw = make_device_inputs(w, device, rank)
+    p = syn.make_block_inputs(w, seed=9000 + w.index + 7919 * rank)
+    dev = lambda a, dt=None: torch.from_numpy(np.ascontiguousarray(a)).to(device).to(dt or torch.float32)
+    bf = torch.bfloat16
+    x, wq, wo = dev(p["x"], bf), dev(p["w_qkv"], bf), dev(p["w_o"], bf)
+    bq, bo, ga, be = (dev(p[n]) for n in ("b_qkv", "b_o", "gamma", "beta"))
+    B, H, W, C = x.shape
+    tokens = B * H * W
+    out = torch.empty_like(x)
+    ws = torch.empty(sa.swin_attn_block_workspace_size(B, H, W, w.heads, w.d, w.M, w.mode, "bias_table" in kw, bf),
+                     dtype=torch.uint8, device=device)
+    q, k, v, a = (torch.empty_like(x) for _ in range(4))
+    wsq = torch.empty(max(sa.lib().swin_qkv_proj_workspace_size(tokens, C), 256), dtype=torch.uint8, device=device)
+    wsp = torch.empty(max(sa.lib().swin_proj_postnorm_workspace_size(tokens, C), 256), dtype=torch.uint8,
+                      device=device)
+    n = max(3, min(args.steps, 20))
+
+    def block():
+        sa.swin_attn_block_fwd(x, w.heads, wq, bq, wo, bo, ga, be, w.M, s, w.mode, out=out, workspace=ws,
+                               stream=stream, partition=w.partition, **kw)
+
+    def qkv():
+        sa.swin_qkv_proj(x, wq, bq, workspace=wsq, stream=stream)
+
+    def post():
+        sa.swin_proj_postnorm_residual(a, wo, bo, x, ga, be, out=out, workspace=wsp, stream=stream)
+    res = {}
+    for name, fn in (("block", block), ("qkv_proj", qkv), ("proj_postnorm", post)):
+        timer.loop(fn, 2)
+        res[name] = max_over_ranks(_median(timer.loop(fn, n)), world, device)
+    if sa.swin_stream_status(stream) != 0:
+        raise RuntimeError("device status after the block of %s" % w.name)
+    e = 2  # bf16 bytes
+    bytes_qkv = tokens * C * e * 4 + 3 * C * C * e
+    bytes_post = tokens * C * e * 3 + C * C * e
+    hbm = peaks["hbm_gbs"]
+    gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+    entry = {"workload": w.name, "block_ms": round(res["block"], 4),
+             "block_tokens_per_s": round(tokens * world / (res["block"] * 1e-3), 1),
+             "qkv_proj": {"ms": round(res["qkv_proj"], 4), "algorithmic_bytes": bytes_qkv,
+                          "achieved_gbs": round(gbs(bytes_qkv, res["qkv_proj"]), 1),
+                          "frac_hbm": round(gbs(bytes_qkv, res["qkv_proj"]) / hbm, 4)},
+             "proj_postnorm": {"ms": round(res["proj_postnorm"], 4), "algorithmic_bytes": bytes_post,
+                               "achieved_gbs": round(gbs(bytes_post, res["proj_postnorm"]), 1),
+                               "frac_hbm": round(gbs(bytes_post, res["proj_postnorm"]) / hbm, 4)},
+             "peak": {"hbm_gbs": hbm, "source": peaks["source"]}}
+    # this library's kernels per timed call (the cuBLASLt GEMMs are not counted):
+    # block = split, [CPB,] attention, post-norm; each projection step = 1
+    mine_block = 3 + (1 if "cpb" in kw else 0)
+    del x, out, ws, q, k, v, a, wsq, wsp
+    torch.cuda.empty_cache()
+    return entry, n * (mine_block + 1 + 1)
 
 
 def run_native(args, rank: int, world: int, local_rank: int):
@@ -453,6 +520,12 @@ def run_native(args, rank: int, world: int, local_rank: int):
         e, n = time_workload(syn.WORKLOADS[idx], args, timer, rank, world, peaks, sms, clock_guess, False)
         other_entries.append(e)
         launches += n
+    block_entries = []
+    if not args.no_block:
+        for idx in [args.workload] + others:
+            e, n = time_block(syn.WORKLOADS[idx], args, timer, rank, world, peaks)
+            block_entries.append(e)
+            launches += n
     bwd_entries = []
     if not args.no_backward:
         for idx in [args.workload] + others:
@@ -486,6 +559,7 @@ def run_native(args, rank: int, world: int, local_rank: int):
         "clocks": clocks, "gpu_launches": launches,
         "workloads": [{k: v for k, v in entry.items() if k != "e2e"}] + other_entries,
         "backward": bwd_entries,
+        "block": block_entries,
     }
     return line, headline
 
@@ -552,6 +626,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--only", action="store_true", help="time the headline workload alone")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurements")
+    ap.add_argument("--no-block", action="store_true", help="skip the block (projections + post-norm) measurements")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -128,14 +128,16 @@ __global__ void bias_split_kernel(const float* __restrict__ y, const float* b, T
 
 // out[t] = x[t] + gamma * (y[t] + b - mean) / sqrt(var + eps) + beta, one warp
 // per token row; y is the fp32 projection.  Mean and variance are two passes
-// over the row held in registers (fp32; the row is at most kMaxC channels).
+// over the row held in registers (fp32): kPer values per lane, the row's C
+// channels rounded up to a multiple of 32, so a narrow row keeps few
+// registers and many warps resident (C <= kMaxC).
 constexpr int kMaxC = 1024;
 
-template <typename T, typename TO>
-__global__ void postnorm_residual_kernel(const T* __restrict__ x, const float* __restrict__ yall, TO* out,
-                                         const float* b, const float* gamma, const float* beta, float eps,
-                                         long long tokens, int C) {
-  constexpr int kPer = kMaxC / 32;
+template <typename T, typename TO, int kPer>
+__global__ void __launch_bounds__(256) postnorm_residual_kernel(const T* __restrict__ x,
+                                                                const float* __restrict__ yall, TO* out,
+                                                                const float* b, const float* gamma, const float* beta,
+                                                                float eps, long long tokens, int C) {
   const int lane = threadIdx.x & 31;
   const long long warp = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
@@ -182,6 +184,26 @@ int grid_for(long long work, int per_block) {
   return (int)(g < 148 * 16 ? (g < 1 ? 1 : g) : 148 * 16);
 }
 
+template <int kPer>
+void launch_postnorm(const void* x, const float* y, void* out, const float* b_o, const float* gamma,
+                     const float* beta, float eps, bool bf16, bool f32_out, int tokens, int C, cudaStream_t stream) {
+  using bf = __nv_bfloat16;
+  // 8 warps per block, one token per warp at a time; every token in one wave
+  const int blocks = (int)(((long long)tokens + 7) / 8);
+  if (bf16 && !f32_out)
+    postnorm_residual_kernel<bf, bf, kPer><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y,
+                                                                       static_cast<bf*>(out), b_o, gamma, beta, eps,
+                                                                       tokens, C);
+  else if (bf16)
+    postnorm_residual_kernel<bf, float, kPer><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y,
+                                                                          static_cast<float*>(out), b_o, gamma, beta,
+                                                                          eps, tokens, C);
+  else
+    postnorm_residual_kernel<float, float, kPer><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), y,
+                                                                             static_cast<float*>(out), b_o, gamma,
+                                                                             beta, eps, tokens, C);
+}
+
 }  // namespace
 
 swin_status launch_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
@@ -207,19 +229,15 @@ swin_status launch_proj_postnorm(const void* a, const void* w_o, const float* b_
   if (C > kMaxC) return fail(SWIN_ERR_UNSUPPORTED, "post-norm supports C <= %d, got %d", kMaxC, C);
   swin_status s = gemm_xwt(a, w_o, y, bf16, tokens, C, C, stream);
   if (s != SWIN_OK) return s;
-  const int blocks = grid_for((long long)tokens, 8);
-  using bf = __nv_bfloat16;
-  if (bf16 && !f32_out)
-    postnorm_residual_kernel<bf, bf><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y, static_cast<bf*>(out),
-                                                                 b_o, gamma, beta, eps, tokens, C);
-  else if (bf16)
-    postnorm_residual_kernel<bf, float><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y,
-                                                                    static_cast<float*>(out), b_o, gamma, beta, eps,
-                                                                    tokens, C);
-  else
-    postnorm_residual_kernel<float, float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), y,
-                                                                       static_cast<float*>(out), b_o, gamma, beta,
-                                                                       eps, tokens, C);
+  const int per = (C + 31) / 32;
+  switch (per <= 2 ? 2 : per <= 3 ? 3 : per <= 4 ? 4 : per <= 8 ? 8 : per <= 16 ? 16 : 32) {
+    case 2: launch_postnorm<2>(x, y, out, b_o, gamma, beta, eps, bf16, f32_out, tokens, C, stream); break;
+    case 3: launch_postnorm<3>(x, y, out, b_o, gamma, beta, eps, bf16, f32_out, tokens, C, stream); break;
+    case 4: launch_postnorm<4>(x, y, out, b_o, gamma, beta, eps, bf16, f32_out, tokens, C, stream); break;
+    case 8: launch_postnorm<8>(x, y, out, b_o, gamma, beta, eps, bf16, f32_out, tokens, C, stream); break;
+    case 16: launch_postnorm<16>(x, y, out, b_o, gamma, beta, eps, bf16, f32_out, tokens, C, stream); break;
+    default: launch_postnorm<32>(x, y, out, b_o, gamma, beta, eps, bf16, f32_out, tokens, C, stream); break;
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "post-norm launch: %s", cudaGetErrorString(e));
   return SWIN_OK;
