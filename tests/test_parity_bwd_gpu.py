@@ -191,3 +191,46 @@ def test_bf16_workload_full_size_every_window(idx):
     w = syn.WORKLOADS[idx]
     errs, _, _ = check_case(w, w.shifts[0])
     print(w.name, errs)
+
+
+# ---------------------------------------------------------------------------
+# the tensor-core backward (bf16, d = 32, M <= 32): tiling shapes
+# ---------------------------------------------------------------------------
+TC_SHAPES = [  # B, H, W, heads, M, s
+    (1, 16, 16, 1, 8, 4), (2, 20, 13, 2, 7, 3), (1, 40, 36, 3, 16, 8), (1, 33, 70, 2, 24, 12),
+    (1, 64, 64, 1, 32, 16), (1, 50, 45, 2, 32, 5), (1, 5, 130, 1, 3, 1), (3, 6, 7, 2, 1, 0),
+    (1, 24, 24, 4, 12, 6), (2, 17, 23, 1, 11, 10),
+]
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+@pytest.mark.parametrize("B,H,W,heads,M,s", TC_SHAPES)
+def test_bf16_tensor_core_backward_shapes(B, H, W, heads, M, s, mode):
+    """Every rectangle width class, partial query tiles (128 tokens) and key
+    blocks (64), odd and large windows, H != W, M = 1; tables with large
+    entries so the bias gradient matters."""
+    w = syn.Workload(90, "bwd-tc", "bf16", B, H, W, heads, 32, M, (s,), mode,
+                     tau=(0.05, 0.2) if mode == 1 else None, rope_base=100.0 if mode == 2 else 0.0)
+
+    def mutate(inp):
+        if "table" in inp:
+            inp["table"] = (0.5 * np.random.default_rng(M).standard_normal(inp["table"].shape)).astype(np.float32)
+
+    check_case(w, s, seed=7 * H + W + 100 * mode + M, mutate=mutate)
+
+
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_bf16_tensor_core_backward_interleaved(mode):
+    w = syn.Workload(91, "bwd-tc-il", "bf16", 2, 30, 27, 2, 32, 8, (0,), mode,
+                     tau=(0.05, 0.2) if mode == 1 else None, rope_base=100.0 if mode == 2 else 0.0, partition=1)
+    inp = syn.make_inputs(w, seed=5 + mode)
+    dout = syn.make_dout(w, seed=6 + mode)
+    kw = dict(tau=dev(inp["tau"]) if "tau" in inp else None,
+              bias_table=dev(inp["table"]) if "table" in inp else None,
+              rope_freqs=dev(inp["rope_freqs"]) if "rope_freqs" in inp else None)
+    q, k, v, g = (dev(a).to(torch.bfloat16) for a in (inp["q"], inp["k"], inp["v"], dout))
+    got = sa.swin_window_attn_bwd(q, k, v, g, w.M, 0, mode, grad_dtype=torch.float32, partition=1, **kw)
+    assert sa.swin_stream_status() == 0
+    want = oracle.window_attn_bwd(inp["q"], inp["k"], inp["v"], dout, w.M, 0, mode, tau=inp.get("tau"),
+                                  table=inp.get("table"), rope_freqs=inp.get("rope_freqs"), partition=1)
+    compare(got, want, TOL_BF16)

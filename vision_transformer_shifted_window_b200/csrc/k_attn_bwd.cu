@@ -22,7 +22,8 @@
 // Nothing is kept from the forward pass: the softmax statistics are
 // recomputed.  Three launches, all on the caller's stream:
 //   1. bwd_q: one thread per query row (the forward's decomposition: one CTA
-//      of 128 threads per image, head, rectangle and block of 128 queries).
+//      of 128 threads, 64 for windows of <= 64 tokens, per image, head,
+//      rectangle and block of queries).
 //      Pass 1 recomputes the row's log-sum-exp and D_i = g_i . o_i by an online
 //      softmax over the rectangle's keys, and stores both; pass 2 forms dl,
 //      accumulates dqt in registers and the bias gradient in shared memory
@@ -104,7 +105,7 @@ __device__ __forceinline__ __nv_bfloat16 st_conv<__nv_bfloat16>(double x) {
 template <typename A, int D>
 __device__ void build_rope_tables(const float* freqs, int M, A* rc, A* rs) {
   constexpr int Qd = D / 4;
-  for (int i = threadIdx.x; i < 2 * M * Qd; i += kThreads) {
+  for (int i = threadIdx.x; i < 2 * M * Qd; i += blockDim.x) {
     const int axis = i / (M * Qd), p = (i / Qd) % M, t = i % Qd;
     double sv, cv;
     sincos((double)p * (double)freqs[axis * Qd + t], &sv, &cv);
@@ -227,6 +228,16 @@ struct Geometry {
   }
 };
 
+// Dot product of two rows, one FMA chain: split chains cost registers that
+// lowered the occupancy of these kernels by a third and measured slower.
+template <typename A, int D>
+__device__ __forceinline__ A row_dot(const A* x, const A* y) {
+  A d = 0;
+#pragma unroll
+  for (int e = 0; e < D; ++e) d += x[e] * y[e];
+  return d;
+}
+
 __device__ __forceinline__ Geometry geometry(const BwdArgs& a, int nsx, int chunks) {
   Geometry g;
   const int rect = blockIdx.x / chunks;
@@ -254,19 +265,23 @@ struct Smem {
   double red[1 + D / 2];  // CTA sums: d(tau), d(omega)
 };
 
-template <typename T, typename TG, typename A, int D, int MODE>
-__global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int chunks) {
+// NT threads per CTA (128, or 64 for windows of <= 64 tokens).  The register
+// bound keeps three 128-thread CTAs per SM for fp32 arithmetic (170
+// registers); one more register per thread would drop it to two.
+template <typename T, typename TG, typename A, int D, int MODE, int NT>
+__global__ void __launch_bounds__(NT, sizeof(A) == 4 ? 384 / NT : 1) bwd_q_kernel(BwdArgs a, int nsx, int chunks) {
   constexpr int kTile = tile_rows<A, D>();
   extern __shared__ __align__(16) unsigned char dyn[];  // double[(2M-1)^2]: this head's d(table)
   __shared__ Smem<A, D, MODE> sm;
   const Geometry G = geometry(a, nsx, chunks);
-  if (G.chunk * kThreads >= G.n) return;  // whole CTA idle (uniform)
+  constexpr int nt = NT;
+  if (G.chunk * nt >= G.n) return;  // whole CTA idle (uniform)
   const int M = a.M, s = a.shift, h = blockIdx.y, b = blockIdx.z, R = 2 * M - 1;
   const bool want_T = MODE != 2 && a.acc_table != nullptr;
   double* sT = reinterpret_cast<double*>(dyn);
   if (want_T)
-    for (int i = threadIdx.x; i < R * R; i += kThreads) sT[i] = 0;
-  for (int i = threadIdx.x; i < 1 + D / 2; i += kThreads) sm.red[i] = 0;
+    for (int i = threadIdx.x; i < R * R; i += nt) sT[i] = 0;
+  for (int i = threadIdx.x; i < 1 + D / 2; i += nt) sm.red[i] = 0;
   if (MODE == 2) build_rope_tables<A, D>(a.rope, M, sm.rc, sm.rs);
   __syncthreads();
 
@@ -274,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
   const T* K = static_cast<const T*>(a.k);
   const T* V = static_cast<const T*>(a.v);
   const T* GO = static_cast<const T*>(a.dout);
-  const int qi = G.chunk * kThreads + threadIdx.x;
+  const int qi = G.chunk * nt + threadIdx.x;
   const bool active = qi < G.n;
   const int qrow = active ? qi : 0;
   const int yq = G.Y(qrow), xq = G.X(qrow);
@@ -295,7 +310,7 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
   // One tile of the rectangle's keys: kt into kv0, v into kv1.
   auto load_tile = [&](int j0, int nk) {
     __syncthreads();
-    for (int i = threadIdx.x; i < nk * D; i += kThreads) {
+    for (int i = threadIdx.x; i < nk * D; i += nt) {
       const int j = i / D, e = i % D, kk = j0 + j;
       const size_t off = row_off(a, b, G.Y(kk), G.X(kk), h, D) + e;
       sm.kv0[j][e] = (A)ld(K + off);
@@ -315,20 +330,13 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
     __syncthreads();
   };
   auto logit = [&](int j, int kk) {
-    A dot = 0;
-#pragma unroll
-    for (int e = 0; e < D; ++e) dot += qt[e] * sm.kv0[j][e];
+    A dot = row_dot<A, D>(qt, sm.kv0[j]);
     if (MODE != 2 && a.table) {
       dot += (A)__ldg(a.table + (size_t)G.rel(qrow, kk, M) * a.heads + h);
     }
     return dot;
   };
-  auto gdotv = [&](int j) {
-    A dp = 0;
-#pragma unroll
-    for (int e = 0; e < D; ++e) dp += g[e] * sm.kv1[j][e];
-    return dp;
-  };
+  auto gdotv = [&](int j) { return row_dot<A, D>(g, sm.kv1[j]); };
 
   // pass 1: log-sum-exp and D = g . o by an online softmax
   A m = -INFINITY, l = 0, u = 0;
@@ -420,20 +428,21 @@ __global__ void __launch_bounds__(kThreads) bwd_q_kernel(BwdArgs a, int nsx, int
     for (int e = 0; e < D / 2; ++e) warp_sum_to(drope[e], &sm.red[1 + e]);
   __syncthreads();
   if (want_T)
-    for (int i = threadIdx.x; i < R * R; i += kThreads)
+    for (int i = threadIdx.x; i < R * R; i += nt)
       if (sT[i] != 0.0) atomicAdd(a.acc_table + (size_t)i * a.heads + h, sT[i]);
   if (MODE == 1 && a.acc_tau && threadIdx.x == 0) atomicAdd(a.acc_tau + h, sm.red[0]);
   if (MODE == 2 && a.acc_rope && threadIdx.x < D / 2) atomicAdd(a.acc_rope + threadIdx.x, sm.red[1 + threadIdx.x]);
 }
 
-template <typename T, typename TG, typename A, int D, int MODE>
-__global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, int chunks) {
+template <typename T, typename TG, typename A, int D, int MODE, int NT>
+__global__ void __launch_bounds__(NT, sizeof(A) == 4 ? 256 / NT : 1) bwd_kv_kernel(BwdArgs a, int nsx, int chunks) {
   constexpr int kTile = tile_rows<A, D>();
   __shared__ Smem<A, D, MODE> sm;
   const Geometry G = geometry(a, nsx, chunks);
-  if (G.chunk * kThreads >= G.n) return;
+  constexpr int nt = NT;
+  if (G.chunk * nt >= G.n) return;
   const int M = a.M, s = a.shift, h = blockIdx.y, b = blockIdx.z;
-  for (int i = threadIdx.x; i < 1 + D / 2; i += kThreads) sm.red[i] = 0;
+  for (int i = threadIdx.x; i < 1 + D / 2; i += nt) sm.red[i] = 0;
   if (MODE == 2) build_rope_tables<A, D>(a.rope, M, sm.rc, sm.rs);
   __syncthreads();
 
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
   const T* K = static_cast<const T*>(a.k);
   const T* V = static_cast<const T*>(a.v);
   const T* GO = static_cast<const T*>(a.dout);
-  const int kj = G.chunk * kThreads + threadIdx.x;
+  const int kj = G.chunk * nt + threadIdx.x;
   const bool active = kj < G.n;
   const int krow = active ? kj : 0;
   const int yk = G.Y(krow), xk = G.X(krow);
@@ -465,7 +474,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
   for (int i0 = 0; i0 < G.n; i0 += kTile) {
     const int nq = min(kTile, G.n - i0);
     __syncthreads();
-    for (int i = threadIdx.x; i < nq * D; i += kThreads) {
+    for (int i = threadIdx.x; i < nq * D; i += nt) {
       const int r = i / D, e = i % D, qq = i0 + r;
       const size_t off = row_off(a, b, G.Y(qq), G.X(qq), h, D) + e;
       sm.kv0[r][e] = (A)ld(Q + off);
@@ -492,12 +501,7 @@ __global__ void __launch_bounds__(kThreads) bwd_kv_kernel(BwdArgs a, int nsx, in
     if (!active) continue;
     for (int i = 0; i < nq; ++i) {
       const int qq = i0 + i;
-      A dot = 0, gv = 0;
-#pragma unroll
-      for (int e = 0; e < D; ++e) {
-        dot += sm.kv0[i][e] * kt[e];
-        gv += sm.kv1[i][e] * vr[e];
-      }
+      A dot = row_dot<A, D>(sm.kv0[i], kt), gv = row_dot<A, D>(sm.kv1[i], vr);
       if (MODE != 2 && a.table) {
         dot += (A)__ldg(a.table + (size_t)G.rel(qq, krow, M) * a.heads + h);
       }
@@ -568,22 +572,30 @@ __global__ void bwd_finish_kernel(const double* acc, int n_table, int n_tau, int
   }
 }
 
-template <typename T, typename TG, typename A, int D, int MODE>
-swin_status launch_mode(const BwdArgs& a, cudaStream_t stream) {
+template <typename T, typename TG, typename A, int D, int MODE, int NT>
+swin_status launch_nt(const BwdArgs& a, cudaStream_t stream) {
   const int nsy = swin_nwin(a.part, a.H, a.M, a.shift), nsx = swin_nwin(a.part, a.W, a.M, a.shift);
-  const int chunks = (a.M * a.M + kThreads - 1) / kThreads;
+  constexpr int nt = NT;
+  const int chunks = (a.M * a.M + nt - 1) / nt;
   const dim3 grid(nsy * nsx * chunks, a.heads, a.B);
   const size_t dyn = (MODE != 2 && a.acc_table) ? sizeof(double) * (size_t)(2 * a.M - 1) * (2 * a.M - 1) : 0;
-  auto kq = bwd_q_kernel<T, TG, A, D, MODE>;
+  auto kq = bwd_q_kernel<T, TG, A, D, MODE, NT>;
   if (dyn > 0) {  // static plus dynamic shared memory may pass the 48 KB default
     cudaError_t e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
     if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_bwd smem attribute: %s", cudaGetErrorString(e));
   }
-  kq<<<grid, kThreads, dyn, stream>>>(a, nsx, chunks);
-  bwd_kv_kernel<T, TG, A, D, MODE><<<grid, kThreads, 0, stream>>>(a, nsx, chunks);
+  kq<<<grid, nt, dyn, stream>>>(a, nsx, chunks);
+  bwd_kv_kernel<T, TG, A, D, MODE, NT><<<grid, nt, 0, stream>>>(a, nsx, chunks);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_bwd launch: %s", cudaGetErrorString(e));
   return SWIN_OK;
+}
+
+template <typename T, typename TG, typename A, int D, int MODE>
+swin_status launch_mode(const BwdArgs& a, cudaStream_t stream) {
+  // windows of <= 64 tokens: 64 threads, so fewer of them idle
+  return a.M * a.M <= 64 ? launch_nt<T, TG, A, D, MODE, 64>(a, stream)
+                         : launch_nt<T, TG, A, D, MODE, kThreads>(a, stream);
 }
 
 template <typename T, typename TG, typename A, int D>
@@ -622,7 +634,9 @@ swin_status launch_attn_bwd(const BwdArgs& a, bool bf16_in, bool f32_grad, float
     if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_bwd memset: %s", cudaGetErrorString(e));
   }
   swin_status st;
-  if (!bf16_in)
+  if (attn_bwd_tc_supported(a, bf16_in))
+    st = launch_attn_bwd_tc(a, f32_grad, stream);
+  else if (!bf16_in)
     st = launch_typed<float, float, double>(a, stream);
   else if (f32_grad)
     st = launch_typed<__nv_bfloat16, float, float>(a, stream);

@@ -14,18 +14,20 @@
 // softmax is the exact online form FlashSwin relies on: a running maximum and
 // rescaled running sums, so no score row is stored.
 //
-// Decomposition: one CTA of 128 threads per (image, head, rectangle, block of
-// 128 queries); a rectangle is one window per axis, a segment of the shifted
-// partition or a strided window of the interleaved one (see swin_index.cuh),
-// i.e. one independent attention problem of up to M*M tokens.  Each thread owns one query row; keys and values stream through
-// shared memory 16 at a time (normalised or rotated once per key), and every
-// thread reads them as broadcasts.
+// Decomposition: one CTA per (image, head, rectangle, block of queries), of
+// 128 threads, or 64 when a window has at most 64 tokens (M <= 8); a
+// rectangle is one window per axis, a segment of the shifted partition or a
+// strided window of the interleaved one (see swin_index.cuh), i.e. one
+// independent attention problem of up to M*M tokens.  Each thread owns one
+// query row; keys and values stream through shared memory 16 at a time
+// (normalised or rotated once per key), and every thread reads them as
+// broadcasts; each logit is four independent FMA chains.
 #include "swin_common.cuh"
 
 namespace swin {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 128;  // threads per CTA (64 when a window has at most 64 tokens)
 constexpr int kKeyTile = 16;
 constexpr int kMaxM = 64;
 
@@ -82,7 +84,8 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
   const SwinAxis ay = swin_axis(a.part, sy, a.H, M, s), ax = swin_axis(a.part, sx, a.W, M, s);
   const int ly = ay.len, lx = ax.len;
   const int n = ly * lx;
-  if (chunk * kThreads >= n) return;  // whole CTA idle (uniform)
+  const int nt = blockDim.x;
+  if (chunk * nt >= n) return;  // whole CTA idle (uniform)
   const int C = a.heads * D;
   const T* Q = static_cast<const T*>(a.q);
   const T* K = static_cast<const T*>(a.k);
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
 
   if (MODE == 2) {
     constexpr int Qd = D / 4;
-    for (int i = threadIdx.x; i < 2 * M * Qd; i += kThreads) {
+    for (int i = threadIdx.x; i < 2 * M * Qd; i += nt) {
       const int axis = i / (M * Qd), p = (i / Qd) % M, t = i % Qd;
       double sv, cv;
       sincos((double)p * (double)a.rope[axis * Qd + t], &sv, &cv);
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
     __syncthreads();
   }
 
-  const int qi = chunk * kThreads + threadIdx.x;
+  const int qi = chunk * nt + threadIdx.x;
   const bool active = qi < n;
   const int iyq = active ? qi / lx : 0, ixq = active ? qi % lx : 0;
   const int yq = ay.start + ay.stride * iyq, xq = ax.start + ax.stride * ixq;
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
   for (int j0 = 0; j0 < n; j0 += kKeyTile) {
     const int nk = min(kKeyTile, n - j0);
     __syncthreads();
-    for (int i = threadIdx.x; i < nk * D; i += kThreads) {
+    for (int i = threadIdx.x; i < nk * D; i += nt) {
       const int j = i / D, e = i % D, kk = j0 + j;
       const int yk = ay.start + ay.stride * (kk / lx), xk = ax.start + ax.stride * (kk % lx);
       const size_t off = (((size_t)b * a.H + yk) * a.W + xk) * C + (size_t)h * D + e;
@@ -160,10 +163,16 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
     __syncthreads();
     if (!active) continue;
     for (int j = 0; j < nk; ++j) {
-      A dot = 0;
+      // four partial sums: independent FMA chains
+      A d0 = 0, d1 = 0, d2 = 0, d3 = 0;
 #pragma unroll
-      for (int e = 0; e < D; ++e) dot = fma(q[e], ks[j][e], dot);
-      A lg = dot * scale;
+      for (int e = 0; e < D; e += 4) {
+        d0 = fma(q[e], ks[j][e], d0);
+        d1 = fma(q[e + 1], ks[j][e + 1], d1);
+        d2 = fma(q[e + 2], ks[j][e + 2], d2);
+        d3 = fma(q[e + 3], ks[j][e + 3], d3);
+      }
+      A lg = ((d0 + d1) + (d2 + d3)) * scale;
       if (MODE != 2 && a.table) {
         const int kk = j0 + j;
         const int r = swin_rel_row(iyq - kk / lx, ixq - kk % lx, M);
@@ -195,13 +204,14 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, int nsx
 template <typename T, typename TO, typename A, int D>
 swin_status launch_typed(const AttnArgs& a, cudaStream_t stream) {
   const int nsy = swin_nwin(a.part, a.H, a.M, a.shift), nsx = swin_nwin(a.part, a.W, a.M, a.shift);
-  const int chunks = (a.M * a.M + kThreads - 1) / kThreads;
+  const int nt = a.M * a.M <= 64 ? 64 : kThreads;
+  const int chunks = (a.M * a.M + nt - 1) / nt;
   dim3 grid(nsy * nsx * chunks, a.heads, a.B);
   switch (a.mode) {
-    case 0: attn_simt_kernel<T, TO, A, D, 0><<<grid, kThreads, 0, stream>>>(a, nsx, chunks); break;
-    case 1: attn_simt_kernel<T, TO, A, D, 1><<<grid, kThreads, 0, stream>>>(a, nsx, chunks); break;
+    case 0: attn_simt_kernel<T, TO, A, D, 0><<<grid, nt, 0, stream>>>(a, nsx, chunks); break;
+    case 1: attn_simt_kernel<T, TO, A, D, 1><<<grid, nt, 0, stream>>>(a, nsx, chunks); break;
     default:
-      if constexpr (D % 4 == 0) attn_simt_kernel<T, TO, A, D, 2><<<grid, kThreads, 0, stream>>>(a, nsx, chunks);
+      if constexpr (D % 4 == 0) attn_simt_kernel<T, TO, A, D, 2><<<grid, nt, 0, stream>>>(a, nsx, chunks);
       break;
   }
   cudaError_t e = cudaGetLastError();

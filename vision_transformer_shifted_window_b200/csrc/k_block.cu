@@ -111,18 +111,42 @@ __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
 }
 
+// Four consecutive values of T from fp32, rounded once each.
+__device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
+__device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 w;
+  w.x = *reinterpret_cast<uint32_t*>(&lo);
+  w.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(dst) = w;
+}
+
 // q, k, v = the fp32 product y [tokens][3C] plus b (NULL: 0), split by
-// channel thirds and rounded once to T (grid-stride over tokens x C).
+// channel thirds and rounded once to T; each thread takes four consecutive
+// channels (C % 8 == 0: every 16-byte load and store is aligned), grid-stride
+// over tokens x C / 4.
 template <typename T>
 __global__ void bias_split_kernel(const float* __restrict__ y, const float* b, T* q, T* k, T* v, long long n,
                                   int C) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const long long t = i / C;
-    const int c = (int)(i - t * C);
-    const float* yr = y + t * 3 * C;
-    q[i] = from_f<T>(yr[c] + (b ? __ldg(b + c) : 0.f));
-    k[i] = from_f<T>(yr[C + c] + (b ? __ldg(b + C + c) : 0.f));
-    v[i] = from_f<T>(yr[2 * C + c] + (b ? __ldg(b + 2 * C + c) : 0.f));
+  const long long n4 = n / 4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long e = 4 * i, t = e / C;
+    const int c = (int)(e - t * C);
+    const float* yr = y + t * 3 * C + c;
+    T* outs[3] = {q + e, k + e, v + e};
+#pragma unroll
+    for (int part = 0; part < 3; ++part) {
+      float4 val = *reinterpret_cast<const float4*>(yr + part * C);
+      if (b) {
+        const float* bb = b + part * C + c;
+        val.x += __ldg(bb);
+        val.y += __ldg(bb + 1);
+        val.z += __ldg(bb + 2);
+        val.w += __ldg(bb + 3);
+      }
+      store4(outs[part], val);
+    }
   }
 }
 
@@ -133,7 +157,9 @@ __global__ void bias_split_kernel(const float* __restrict__ y, const float* b, T
 // registers and many warps resident (C <= kMaxC).
 constexpr int kMaxC = 1024;
 
-template <typename T, typename TO, int kPer>
+// kTok tokens per warp at a time, all their loads issued before the first
+// reduction (kTok x kPer values per lane in flight).
+template <typename T, typename TO, int kPer, int kTok>
 __global__ void __launch_bounds__(256) postnorm_residual_kernel(const T* __restrict__ x,
                                                                 const float* __restrict__ yall, TO* out,
                                                                 const float* b, const float* gamma, const float* beta,
@@ -141,40 +167,42 @@ __global__ void __launch_bounds__(256) postnorm_residual_kernel(const T* __restr
   const int lane = threadIdx.x & 31;
   const long long warp = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long t = warp; t < tokens; t += nwarps) {
-    const float* yr = yall + t * C;
-    TO* row = out + t * C;
-    float y[kPer];
-    float s = 0.f;
+  for (long long t0 = warp * kTok; t0 < tokens; t0 += nwarps * kTok) {
+    float y[kTok][kPer], xv[kTok][kPer];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int c = lane + 32 * j;
-      y[j] = 0.f;
-      if (c < C) {
-        y[j] = yr[c] + (b ? __ldg(b + c) : 0.f);
-        s += y[j];
+    for (int u = 0; u < kTok; ++u)
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        const int c = lane + 32 * j;
+        const bool ok = c < C && t0 + u < tokens;
+        y[u][j] = ok ? yall[(t0 + u) * C + c] + (b ? __ldg(b + c) : 0.f) : 0.f;
+        xv[u][j] = ok ? to_f(x[(t0 + u) * C + c]) : 0.f;
       }
+    float mean[kTok], rstd[kTok];
+#pragma unroll
+    for (int u = 0; u < kTok; ++u) {
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) s += y[u][j];  // padding lanes hold 0
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      mean[u] = s / (float)C;
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j)
+        if (lane + 32 * j < C) ss += (y[u][j] - mean[u]) * (y[u][j] - mean[u]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      rstd[u] = rsqrtf(ss / (float)C + eps);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float mean = s / (float)C;
-    float ss = 0.f;
-#pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int c = lane + 32 * j;
-      if (c < C) ss += (y[j] - mean) * (y[j] - mean);
-    }
+      if (c >= C) continue;
+      const float g = gamma ? __ldg(gamma + c) : 1.f, be = beta ? __ldg(beta + c) : 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rstd = rsqrtf(ss / (float)C + eps);
-    const T* xr = x + t * C;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      const int c = lane + 32 * j;
-      if (c < C) {
-        const float g = gamma ? __ldg(gamma + c) : 1.f, be = beta ? __ldg(beta + c) : 0.f;
-        row[c] = from_f<TO>(to_f(xr[c]) + (y[j] - mean) * rstd * g + be);
-      }
+      for (int u = 0; u < kTok; ++u)
+        if (t0 + u < tokens) out[(t0 + u) * C + c] = from_f<TO>(xv[u][j] + (y[u][j] - mean[u]) * rstd[u] * g + be);
     }
   }
 }
@@ -188,20 +216,19 @@ template <int kPer>
 void launch_postnorm(const void* x, const float* y, void* out, const float* b_o, const float* gamma,
                      const float* beta, float eps, bool bf16, bool f32_out, int tokens, int C, cudaStream_t stream) {
   using bf = __nv_bfloat16;
-  // 8 warps per block, one token per warp at a time; every token in one wave
-  const int blocks = (int)(((long long)tokens + 7) / 8);
+  // one token per warp: batching 2-4 tokens per warp measured slower (fewer
+  // warps in flight); 8 warps per block, every token in one wave
+  constexpr int kTok = 1;
+  const int blocks = (int)(((long long)tokens + 8 * kTok - 1) / (8 * kTok));
   if (bf16 && !f32_out)
-    postnorm_residual_kernel<bf, bf, kPer><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y,
-                                                                       static_cast<bf*>(out), b_o, gamma, beta, eps,
-                                                                       tokens, C);
+    postnorm_residual_kernel<bf, bf, kPer, kTok><<<blocks, 256, 0, stream>>>(
+        static_cast<const bf*>(x), y, static_cast<bf*>(out), b_o, gamma, beta, eps, tokens, C);
   else if (bf16)
-    postnorm_residual_kernel<bf, float, kPer><<<blocks, 256, 0, stream>>>(static_cast<const bf*>(x), y,
-                                                                          static_cast<float*>(out), b_o, gamma, beta,
-                                                                          eps, tokens, C);
+    postnorm_residual_kernel<bf, float, kPer, kTok><<<blocks, 256, 0, stream>>>(
+        static_cast<const bf*>(x), y, static_cast<float*>(out), b_o, gamma, beta, eps, tokens, C);
   else
-    postnorm_residual_kernel<float, float, kPer><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), y,
-                                                                             static_cast<float*>(out), b_o, gamma,
-                                                                             beta, eps, tokens, C);
+    postnorm_residual_kernel<float, float, kPer, kTok><<<blocks, 256, 0, stream>>>(
+        static_cast<const float*>(x), y, static_cast<float*>(out), b_o, gamma, beta, eps, tokens, C);
 }
 
 }  // namespace
@@ -212,11 +239,11 @@ swin_status launch_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv
   if (s != SWIN_OK) return s;
   const long long n = (long long)tokens * C;
   if (bf16 && !f32_out)
-    bias_split_kernel<__nv_bfloat16><<<grid_for(n, 256), 256, 0, stream>>>(
+    bias_split_kernel<__nv_bfloat16><<<grid_for(n / 4, 256), 256, 0, stream>>>(
         y, b_qkv, static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), static_cast<__nv_bfloat16*>(v), n,
         C);
   else
-    bias_split_kernel<float><<<grid_for(n, 256), 256, 0, stream>>>(
+    bias_split_kernel<float><<<grid_for(n / 4, 256), 256, 0, stream>>>(
         y, b_qkv, static_cast<float*>(q), static_cast<float*>(k), static_cast<float*>(v), n, C);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "bias launch: %s", cudaGetErrorString(e));

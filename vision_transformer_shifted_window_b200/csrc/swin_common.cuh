@@ -100,5 +100,9 @@ swin_status launch_proj_postnorm(const void* a, const void* w_o, const float* b_
                                  int tokens, int C, float* y, cudaStream_t stream);
 swin_status launch_attn_bwd(const BwdArgs& a, bool bf16_in, bool f32_grad, float* dtable, float* dtau,
                             float* drope, cudaStream_t stream);
+// The tensor-core backward (bf16, d = 32, M <= 32): dq, dk, dv and the
+// parameter-gradient accumulators, with the statistics in a.stats.
+bool attn_bwd_tc_supported(const BwdArgs& a, bool bf16_in);
+swin_status launch_attn_bwd_tc(const BwdArgs& a, bool f32_grad, cudaStream_t stream);
 
 }  // namespace swin
