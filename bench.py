@@ -386,12 +386,20 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
     return entry, launches
 
 
-def time_backward(w: syn.Workload, args, timer, rank: int, world: int, sms: int, clock_mhz: float):
+def bwd_on_tensor_cores(w: syn.Workload) -> bool:
+    """Whether the library runs this workload's backward on the tensor cores
+    (bf16, d = 32, M <= 32, either partition)."""
+    return w.dtype == "bf16" and w.d == 32 and w.M <= 32
+
+
+def time_backward(w: syn.Workload, args, timer, rank: int, world: int, sms: int, clock_mhz: float, peaks: dict):
     """The backward pass (swin_window_attn_bwd: dq, dk, dv and the parameter
     gradients, softmax recomputed) of one workload, bf16 gradients.  Its
     algorithmic work is five products of 2 d flops per attended pair (S, dP,
-    dV, dK, dQ), measured against the CUDA cores' fp32 FMA peak, where it
-    runs.  Returns (entry, launches)."""
+    dV, dK, dQ), measured against the bf16 tensor peak where the tensor-core
+    kernels run (else the CUDA cores' fp32 FMA peak); its exponentials, three
+    per pair (the statistics pass and both gradient passes), give the MUFU
+    bound beside it.  Returns (entry, launches)."""
     import torch
     from vision_transformer_shifted_window_b200 import swin_attn as sa
     device, stream = timer.device, timer.stream
@@ -415,17 +423,22 @@ def time_backward(w: syn.Workload, args, timer, rank: int, world: int, sms: int,
     wk = work(w)
     flops = 2.5 * wk["flops_exact"]
     achieved = flops / (ms * 1e-3) / 1e12
-    peak = alu_peak_tflops(sms, clock_mhz)
+    tc = bwd_on_tensor_cores(w)
+    if tc:
+        peak, bound, kname, src = peaks["bf16_tflops"], "tensor", "bwd_tc_q + bwd_tc_kv", peaks["source"] + " (burst)"
+    else:
+        peak, bound, kname = alu_peak_tflops(sms, clock_mhz), "alu", "bwd_q + bwd_kv (CUDA cores)"
+        src = "derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz" % (sms, FP32_LANES_PER_SM, clock_mhz)
+    exps = dict(wk, exps=3 * wk["exps"])
     entry = {"workload": w.name, "ms_per_step": round(ms, 4),
              "tokens_per_s": round(wk["tokens"] * world / (ms * 1e-3), 1),
-             "roofline": {"bound": "alu", "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-                          "frac": round(achieved / peak, 4), "traffic": None, "kernel": "attn_bwd (q and kv passes)",
-                          "algorithmic_flops": flops,
-                          "peak_source": "derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz"
-                                         % (sms, FP32_LANES_PER_SM, clock_mhz)}}
+             "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+                          "frac": round(achieved / peak, 4), "traffic": None, "kernel": kname,
+                          "algorithmic_flops": flops, "peak_source": src, "kernel_ms": round(ms, 5),
+                          "exp_bound": exp_bound(exps, sms, clock_mhz, ms)}}
     del q, k, v, g, ws
     torch.cuda.empty_cache()
-    return entry, n * (3 if params else 2)
+    return entry, n * ((3 if params else 2))
 
 
 def time_block(w: syn.Workload, args, timer, rank: int, world: int, peaks: dict):
@@ -516,20 +529,20 @@ def run_native(args, rank: int, world: int, local_rank: int):
     clock_guess = 1965.0
     entry, launches = time_workload(headline, args, timer, rank, world, peaks, sms, clock_guess, with_e2e=True)
     other_entries = []
-    for idx in others:
+    for idx in (others if args.part in ("all", "fwd") else []):
         e, n = time_workload(syn.WORKLOADS[idx], args, timer, rank, world, peaks, sms, clock_guess, False)
         other_entries.append(e)
         launches += n
     block_entries = []
-    if not args.no_block:
+    if not args.no_block and args.part in ("all", "block"):
         for idx in [args.workload] + others:
             e, n = time_block(syn.WORKLOADS[idx], args, timer, rank, world, peaks)
             block_entries.append(e)
             launches += n
     bwd_entries = []
-    if not args.no_backward:
+    if not args.no_backward and args.part in ("all", "bwd"):
         for idx in [args.workload] + others:
-            e, n = time_backward(syn.WORKLOADS[idx], args, timer, rank, world, sms, clock_guess)
+            e, n = time_backward(syn.WORKLOADS[idx], args, timer, rank, world, sms, clock_guess, peaks)
             bwd_entries.append(e)
             launches += n
     clocks = sampler.stop()
@@ -542,11 +555,15 @@ def run_native(args, rank: int, world: int, local_rank: int):
             e["roofline"].update(peak=round(pk, 1), frac=round(e["roofline"]["achieved"] / pk, 4),
                                  peak_source="derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz (sampled)"
                                              % (sms, FP32_LANES_PER_SM, sm_mhz))
-    for e in bwd_entries:
-        pk = alu_peak_tflops(sms, sm_mhz)
-        e["roofline"].update(peak=round(pk, 1), frac=round(e["roofline"]["achieved"] / pk, 4),
-                             peak_source="derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz (sampled)"
-                                         % (sms, FP32_LANES_PER_SM, sm_mhz))
+    for e, i in zip(bwd_entries, [args.workload] + others):
+        w = syn.WORKLOADS[i]
+        e["roofline"]["exp_bound"] = exp_bound(dict(work(w), exps=3 * work(w)["exps"]), sms, sm_mhz,
+                                               e["roofline"]["kernel_ms"])
+        if e["roofline"]["bound"] == "alu":
+            pk = alu_peak_tflops(sms, sm_mhz)
+            e["roofline"].update(peak=round(pk, 1), frac=round(e["roofline"]["achieved"] / pk, 4),
+                                 peak_source="derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz (sampled)"
+                                             % (sms, FP32_LANES_PER_SM, sm_mhz))
     line = {
         "metric": METRIC, "value": entry["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": entry["ms_per_step"],
@@ -627,6 +644,9 @@ def main():
     ap.add_argument("--only", action="store_true", help="time the headline workload alone")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward-pass measurements")
     ap.add_argument("--no-block", action="store_true", help="skip the block (projections + post-norm) measurements")
+    ap.add_argument("--part", default="all", choices=("all", "fwd", "bwd", "block"),
+                    help="time one part only (for profiling captures): the forward lines, the backward or the block "
+                         "(the JSON line then carries the forward headline plus that part)")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

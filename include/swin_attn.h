@@ -247,10 +247,17 @@ size_t swin_window_attn_workspace_size(int M, int heads, swin_mode mode, int hav
  *   drope            device fp32 [2][d/4] or NULL; mode 2 only
  *   workspace        device scratch of swin_window_attn_bwd_workspace_size
  *                    bytes, 256-byte aligned
- * Arithmetic: double for SWIN_F32 tensors, fp32 for SWIN_BF16 tensors, on
- * the CUDA cores.  dq, dk, dv are deterministic.  Parameter gradients are
- * summed by double atomic additions and rounded once to fp32; the order of
- * the additions varies, so between calls they may differ in the last bit.
+ * Arithmetic.  SWIN_BF16 tensors with d == 32 and M <= 32 (either
+ * partition): the tensor cores (tcgen05), the five products with fp16
+ * operands and fp32 accumulation — q, k, v, dout converted exactly from bf16
+ * inside fp16's range, RoPE-rotated q and k carried as fp16 hi + lo parts,
+ * probabilities and dS in fp16 — and the softmax in fp32; an operand at or
+ * beyond fp16's range saturates and the call reports SWIN_ERR_UNSUPPORTED
+ * through swin_stream_status.  Otherwise the CUDA cores: double arithmetic
+ * for SWIN_F32 tensors, fp32 for SWIN_BF16.  dq, dk, dv are deterministic.
+ * Parameter gradients are summed by double atomic additions and rounded once
+ * to fp32; the order of the additions varies, so between calls they may
+ * differ in the last bit.
  * Errors as swin_window_attn_fwd: argument errors return before anything is
  * enqueued. */
 swin_status swin_window_attn_bwd(const void* q, const void* k, const void* v, const void* dout,

@@ -156,6 +156,7 @@ __device__ __forceinline__ float clamped_norm(const float (&v)[kD], bool& clampe
 struct TcBwd {
   const __nv_bfloat16 *q, *k, *v, *dout;
   void *dq, *dk, *dv;
+  void* out;  // the forward kernel's output
   int B, H, W, heads, M, shift, part;
   const float* tau;
   const float* table;
@@ -788,6 +789,212 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
   }
 }
 
+// ============================================================== forward
+// The forward pass over arbitrary rectangles (used for interleaved windows,
+// whose strided windows the TMA kernel does not gather): one CTA per query
+// tile, S = Q K^T per 64-key block (RoPE operands split into fp16 hi + lo as
+// in the backward), the softmax in fp32 with the running maximum kept until a
+// block exceeds it by more than 8 (log2 units; probabilities then <= 2^8,
+// exact in fp16's range), P as fp16 into TMEM and O += P V on the tensor
+// cores.  The row sum is taken from the same fp16 probabilities that weight
+// V, so O / l normalises exactly the weights applied.  128 TMEM columns
+// (S 64, P 32, O 32) per CTA.
+template <int MODE, bool TABLE, typename TO>
+__global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ TcBwd p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint8_t* qs = smem;
+  uint8_t* ks = qs + kTileB;
+  uint8_t* vs = ks + kBlkB;
+  uint8_t* qlo = vs + kBlkB;
+  uint8_t* klo = qlo + kTileB;
+  SmemCommon* sc = reinterpret_cast<SmemCommon*>(klo + kBlkB);
+  float* tab = reinterpret_cast<float*>(sc + 1);
+  const int R = 2 * p.M - 1, RR = R * R;
+
+  const int rect = blockIdx.x / p.tiles, tile = blockIdx.x % p.tiles;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const Rect rc = rect_of(p, rect);
+  const int t0 = tile * kRows;
+  if (t0 >= rc.n) return;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tq = t0 + tid;
+  const bool row_ok = tq < rc.n;
+
+  if (tid == 0) {
+    ptx::mbar_init(&sc->mma_bar, 1);
+    ptx::fence_mbar_init();
+    sc->range_hit = 0;
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(&sc->tmem_base, 128);
+    ptx::tmem_relinquish();
+  }
+  if (MODE == 2) build_rope(p.rope, p.M, sc->rc, sc->rs);
+  if (TABLE)
+    for (int i = tid; i < RR; i += kThreads) tab[i] = __ldg(p.table + (size_t)i * p.heads + h) * kLog2e;
+  __syncthreads();
+
+  const float t_eff = MODE == 1 ? fmaxf(__ldg(p.tau + h), kTauMin) : 1.f;
+  float qn = 1.f;
+  {
+    bool hit = false;
+    if (row_ok) {
+      float qrow[kD];
+      load_row(p.q + tok_off(p, b, rc.Y(tq), rc.X(tq), h), qrow);
+      bool c;
+      if (MODE == 1) qn = clamped_norm(qrow, c);
+      prep_row<MODE>(qrow, rc.PY(tq), rc.PX(tq), sc->rc, sc->rs);
+      hit = MODE == 2 ? store_row_f16_split(qs, qlo, tid, qrow) : store_row_f16(qs, tid, qrow);
+    } else {
+      zero_row(qs, tid);
+      if (MODE == 2) zero_row(qlo, tid);
+    }
+    if (hit) sc->range_hit = 1;
+  }
+  const float srow = MODE == 1 ? kLog2e / (qn * t_eff) : kLog2e * rsqrtf((float)kD);
+  const int qbase = rc.off(row_ok ? tq : t0, R) + (p.M - 1) * (R + 1);
+
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tbase = sc->tmem_base;
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const uint32_t tS = tbase, tP = tbase + 64, tO = tbase + 96;
+  constexpr uint32_t idS = ptx::idesc_f16(0, 0, 0, 0, kBlk, kRows);
+  constexpr uint32_t idO = ptx::idesc_f16(0, 0, 0, 1, kD, kRows);
+  const uint64_t qd = ptx::smem_desc(ptx::smem_addr(qs), 16, 512, ptx::kSwizzle64B);
+  const uint64_t kd = ptx::smem_desc(ptx::smem_addr(ks), 16, 512, ptx::kSwizzle64B);
+  const uint64_t vd = ptx::smem_desc(ptx::smem_addr(vs), 16, 512, ptx::kSwizzle64B);
+  const uint64_t qld = ptx::smem_desc(ptx::smem_addr(qlo), 16, 512, ptx::kSwizzle64B);
+  const uint64_t kld = ptx::smem_desc(ptx::smem_addr(klo), 16, 512, ptx::kSwizzle64B);
+  uint32_t phase = 0;
+  bool ok = true;
+  float m2 = -INFINITY, l = 0.f;
+  const int nkb = (rc.n + kBlk - 1) / kBlk;
+  for (int kb = 0; kb < nkb && ok; ++kb) {
+    const int k0 = kb * kBlk, nk = min(kBlk, rc.n - k0);
+    {
+      const int r = tid & (kBlk - 1);
+      const bool isk = tid < kBlk;
+      const int tk = k0 + r;
+      if (isk) sc->coff[r] = rc.off(min(tk, rc.n - 1), R);
+      bool hit = false;
+      if (r < nk) {
+        float v[kD];
+        const size_t off = tok_off(p, b, rc.Y(tk), rc.X(tk), h);
+        if (isk) {
+          load_row(p.k + off, v);
+          if (MODE == 1) {
+            bool c;
+            sc->colf[r] = 1.f / clamped_norm(v, c);
+          }
+          prep_row<MODE>(v, rc.PY(tk), rc.PX(tk), sc->rc, sc->rs);
+          hit = MODE == 2 ? store_row_f16_split(ks, klo, r, v) : store_row_f16(ks, r, v);
+        } else {
+          load_row(p.v + off, v);
+          hit = store_row_f16(vs, r, v);
+        }
+      } else {
+        zero_row(isk ? ks : vs, r);
+        if (isk && MODE == 2) zero_row(klo, r);
+        if (isk && MODE == 1) sc->colf[r] = 0.f;
+      }
+      if (hit) sc->range_hit = 1;
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      ptx::mma_ss(tS, qd, kd, idS, 0);
+      ptx::mma_ss(tS, qd + 2, kd + 2, idS, 1);
+      if (MODE == 2) {
+        ptx::mma_ss(tS, qld, kd, idS, 1);
+        ptx::mma_ss(tS, qld + 2, kd + 2, idS, 1);
+        ptx::mma_ss(tS, qd, kld, idS, 1);
+        ptx::mma_ss(tS, qd + 2, kld + 2, idS, 1);
+      }
+      ptx::mma_commit(&sc->mma_bar);
+    }
+    ok = wait_mma(&sc->mma_bar, phase, p.status);
+    phase ^= 1;
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    ptx::tc_fence_after();
+    uint32_t sr[2][32];
+    ptx::tmem_ld32(tS + lane_off, sr[0]);
+    ptx::tmem_ld32(tS + 32 + lane_off, sr[1]);
+    ptx::tmem_wait_ld();
+    auto logit = [&](int jj) {
+      const float sv = __uint_as_float(sr[jj >> 5][jj & 31]);
+      float xv = MODE == 1 ? sv * srow * sc->colf[jj] : sv * srow;
+      if (TABLE) xv += tab[qbase - sc->coff[jj]];
+      return jj < nk ? xv : -INFINITY;
+    };
+    float mb = -INFINITY;
+#pragma unroll
+    for (int jj = 0; jj < kBlk; ++jj) mb = fmaxf(mb, logit(jj));
+    // lazy maximum: raised only when this block exceeds it by more than 8
+    float c = 1.f;
+    if (mb > m2 + 8.f) {
+      c = ptx::ex2_approx(m2 - mb);  // 0 at the first block
+      m2 = mb;
+      l *= c;
+    }
+    if (kb > 0 && __any_sync(0xffffffffu, c != 1.f)) {  // rescale O (the previous PV has completed)
+      uint32_t o[32];
+      ptx::tmem_ld32(tO + lane_off, o);
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * c);
+      ptx::tmem_st32(tO + lane_off, o);
+    }
+    uint32_t pk[32];
+#pragma unroll
+    for (int jj = 0; jj < kBlk; jj += 2) {
+      const uint32_t w2 = ptx::pack_f16x2(ptx::ex2_approx(logit(jj) - m2), ptx::ex2_approx(logit(jj + 1) - m2));
+      const __half2 hp = *reinterpret_cast<const __half2*>(&w2);
+      l += __low2float(hp) + __high2float(hp);  // the weights V receives
+      pk[jj / 2] = w2;
+    }
+    ptx::tmem_st32(tP + lane_off, pk);
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kBlk / 16; ++kk)
+        ptx::mma_ts(tO, tP + kk * 8, vd + (uint64_t)(kk * 1024 >> 4), idO, (kb > 0 || kk > 0) ? 1u : 0u);
+      ptx::mma_commit(&sc->mma_bar);
+    }
+    ok = wait_mma(&sc->mma_bar, phase, p.status);
+    phase ^= 1;
+    ok = __syncthreads_and(ok);
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
+  if (ok) {
+    ptx::tc_fence_after();
+    uint32_t o[32];
+    ptx::tmem_ld32(tO + lane_off, o);
+    ptx::tmem_wait_ld();
+    const float inv = 1.f / l;
+    float g[kD];
+#pragma unroll
+    for (int e = 0; e < kD; ++e) g[e] = __uint_as_float(o[e]) * inv;
+    if (row_ok) store_grad<TO>(static_cast<TO*>(p.out) + tok_off(p, b, rc.Y(tq), rc.X(tq), h), g);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && sc->range_hit) atomicOr(p.status, (int)SWIN_ERR_UNSUPPORTED);
+  if (warp == 0) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tbase, 128);
+  }
+}
+
 size_t smem_q(int M, bool table) {
   const int RR = (2 * M - 1) * (2 * M - 1);
   size_t s = 3 * kTileB + 3 * kBlkB + sizeof(SmemCommon);
@@ -830,14 +1037,65 @@ swin_status launch_tg(const TcBwd& p, int mode, bool table, cudaStream_t stream)
   }
 }
 
+template <int MODE, bool TABLE, typename TO>
+swin_status launch_fwd_rect(const TcBwd& p, cudaStream_t stream) {
+  const int nsy = swin_nwin(p.part, p.H, p.M, p.shift);
+  const dim3 grid(nsy * p.nsx * p.tiles, p.heads, p.B);
+  auto kf = fwd_tc_rect<MODE, TABLE, TO>;
+  const int RR = (2 * p.M - 1) * (2 * p.M - 1);
+  // 128 TMEM columns per CTA: at most four CTAs per SM (57 KB of shared memory or more)
+  const size_t sm = std::max<size_t>(2 * kTileB + 3 * kBlkB + sizeof(SmemCommon) + (TABLE ? sizeof(float) * RR : 0),
+                                     57 * 1024);
+  cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_fwd_rect smem attribute: %s", cudaGetErrorString(e));
+  kf<<<grid, kThreads, sm, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_fwd_rect launch: %s", cudaGetErrorString(e));
+  return SWIN_OK;
+}
+
+template <typename TO>
+swin_status launch_fwd_to(const TcBwd& p, int mode, bool table, cudaStream_t stream) {
+  switch (mode) {
+    case 0: return table ? launch_fwd_rect<0, true, TO>(p, stream) : launch_fwd_rect<0, false, TO>(p, stream);
+    case 1: return table ? launch_fwd_rect<1, true, TO>(p, stream) : launch_fwd_rect<1, false, TO>(p, stream);
+    default: return launch_fwd_rect<2, false, TO>(p, stream);
+  }
+}
+
 }  // namespace
+
+swin_status launch_attn_fwd_tc_rect(const AttnArgs& a, bool f32_out, cudaStream_t stream) {
+  if (a.d != kD || a.M > 32) return fail(SWIN_ERR_UNSUPPORTED, "rectangle tensor-core path: d = 32, M <= 32");
+  TcBwd p = {};
+  p.q = static_cast<const __nv_bfloat16*>(a.q);
+  p.k = static_cast<const __nv_bfloat16*>(a.k);
+  p.v = static_cast<const __nv_bfloat16*>(a.v);
+  p.out = a.out;
+  p.B = a.B;
+  p.H = a.H;
+  p.W = a.W;
+  p.heads = a.heads;
+  p.M = a.M;
+  p.shift = a.shift;
+  p.part = a.part;
+  p.tau = a.tau;
+  p.table = a.mode == 2 ? nullptr : a.table;
+  p.rope = a.rope;
+  p.status = a.status;
+  p.nsx = swin_nwin(a.part, a.W, a.M, a.shift);
+  p.tiles = (a.M * a.M + kRows - 1) / kRows;
+  const bool table = p.table != nullptr;
+  return f32_out ? launch_fwd_to<float>(p, a.mode, table, stream)
+                 : launch_fwd_to<__nv_bfloat16>(p, a.mode, table, stream);
+}
 
 bool attn_bwd_tc_supported(const BwdArgs& a, bool bf16_in) {
   return bf16_in && a.d == kD && a.M <= 32;
 }
 
 swin_status launch_attn_bwd_tc(const BwdArgs& a, bool f32_grad, cudaStream_t stream) {
-  TcBwd p;
+  TcBwd p = {};
   p.q = static_cast<const __nv_bfloat16*>(a.q);
   p.k = static_cast<const __nv_bfloat16*>(a.k);
   p.v = static_cast<const __nv_bfloat16*>(a.v);

@@ -186,6 +186,9 @@ swin_status swin_window_attn_fwd_ex(const void* q, const void* k, const void* v,
   // shared-memory slot (M <= 32)
   if (dt == SWIN_BF16 && d == 32 && partition == SWIN_PARTITION_SHIFTED && (table == nullptr || M <= 32))
     return swin::launch_attn_tc(a, out_dt == SWIN_F32, st);
+  // interleaved windows: the tensor-core kernel over strided rectangles
+  if (dt == SWIN_BF16 && d == 32 && partition == SWIN_PARTITION_INTERLEAVED && M <= 32)
+    return swin::launch_attn_fwd_tc_rect(a, out_dt == SWIN_F32, st);
   return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
 }
 

@@ -103,6 +103,9 @@ swin_status launch_attn_bwd(const BwdArgs& a, bool bf16_in, bool f32_grad, float
 // The tensor-core backward (bf16, d = 32, M <= 32): dq, dk, dv and the
 // parameter-gradient accumulators, with the statistics in a.stats.
 bool attn_bwd_tc_supported(const BwdArgs& a, bool bf16_in);
+// The tensor-core forward over arbitrary rectangles (bf16, d = 32, M <= 32),
+// used for the interleaved partition.
+swin_status launch_attn_fwd_tc_rect(const AttnArgs& a, bool f32_out, cudaStream_t stream);
 swin_status launch_attn_bwd_tc(const BwdArgs& a, bool f32_grad, cudaStream_t stream);
 
 }  // namespace swin
