@@ -234,11 +234,21 @@ def whole_job(wk: dict, world: int, ms_max: float) -> dict:
 FP32_LANES_PER_SM = 128  # B200: fp32 FMA lanes per SM per clock
 
 
-def on_tensor_cores(w: syn.Workload) -> bool:
-    """Whether the library runs this workload's forward on the tensor-core
-    kernel (bf16, d = 32, shifted windows, no bias table above M = 32)."""
+def fwd_kernel(w: syn.Workload) -> str:
+    """The kernel the library runs this workload's forward on: the TMA
+    tensor-core kernel (bf16, d = 32, shifted windows, no bias table above
+    M = 32), the rectangle tensor-core kernel (bf16, d = 32, interleaved
+    windows, M <= 32) or the CUDA cores."""
     has_table = w.mode != 2 and w.bias
-    return w.dtype == "bf16" and w.d == 32 and w.partition == 0 and (not has_table or w.M <= 32)
+    if w.dtype == "bf16" and w.d == 32 and w.partition == 0 and (not has_table or w.M <= 32):
+        return "attn_tc"
+    if w.dtype == "bf16" and w.d == 32 and w.partition == 1 and w.M <= 32:
+        return "fwd_tc_rect"
+    return "attn_simt"
+
+
+def on_tensor_cores(w: syn.Workload) -> bool:
+    return fwd_kernel(w) != "attn_simt"
 
 
 def alu_peak_tflops(sms: int, clock_mhz: float) -> float:
@@ -339,14 +349,16 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
     k_ms = max_over_ranks(_median(ktimes), world, device)
     achieved = wk["flops_std"] / (k_ms * 1e-3) / 1e12
     hbm = wk["bytes"] / (k_ms * 1e-3) / 1e9
+    kname = fwd_kernel(w)
     if on_tensor_cores(w):
-        peak, bound, src, kname = peaks["bf16_tflops"], "tensor", peaks["source"] + " (burst)", "attn_tc"
+        peak, bound, src = peaks["bf16_tflops"], "tensor", peaks["source"] + " (burst)"
     else:  # the CUDA-core kernel: fp32 FMA lanes
-        peak, bound, kname = alu_peak_tflops(sms, clock_mhz), "alu", "attn_simt"
+        peak, bound = alu_peak_tflops(sms, clock_mhz), "alu"
         src = "derived: %d SMs x %d fp32 lanes x 2 flop x %.0f MHz" % (sms, FP32_LANES_PER_SM, clock_mhz)
     roofline = {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1),
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "traffic": read_traffic(kname, w), "peak_source": src, "kernel": kname,
+                "traffic": read_traffic(kname, w),
+                "peak_source": src, "kernel": kname,
                 "kernel_ms": round(k_ms, 5), "algorithmic_bytes": wk["bytes"],
                 "hbm_achieved_gbs": round(hbm, 1), "hbm_frac": round(hbm / peaks["hbm_gbs"], 4),
                 "attainable_frac": round(achieved / min(peak, peaks["hbm_gbs"] * wk["flops_std"] / wk["bytes"] / 1e3),
@@ -433,7 +445,8 @@ def time_backward(w: syn.Workload, args, timer, rank: int, world: int, sms: int,
     entry = {"workload": w.name, "ms_per_step": round(ms, 4),
              "tokens_per_s": round(wk["tokens"] * world / (ms * 1e-3), 1),
              "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-                          "frac": round(achieved / peak, 4), "traffic": None, "kernel": kname,
+                          "frac": round(achieved / peak, 4),
+                          "traffic": read_traffic("attn_bwd_tc", w) if tc else None, "kernel": kname,
                           "algorithmic_flops": flops, "peak_source": src, "kernel_ms": round(ms, 5),
                           "exp_bound": exp_bound(exps, sms, clock_mhz, ms)}}
     del q, k, v, g, ws
