@@ -78,6 +78,27 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16* src, float (&v)[kD
   }
 }
 
+// One token's head row (32 bf16) as raw 16-byte words, loaded ahead of use.
+struct RawRow {
+  uint4 w[4];
+};
+__device__ __forceinline__ void fetch_row(const __nv_bfloat16* src, RawRow& r) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) r.w[c] = __ldg(s4 + c);
+}
+__device__ __forceinline__ void unpack_row(const RawRow& r, float (&v)[32]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t u[4] = {r.w[c].x, r.w[c].y, r.w[c].z, r.w[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * c + 2 * e] = __uint_as_float(u[e] << 16);
+      v[8 * c + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+  }
+}
+
 // A row of 32 values as fp16 into a swizzled tile; returns whether an entry
 // reached fp16's range limit (saturated).
 __device__ __forceinline__ bool store_row_f16(uint8_t* tile, int row, const float (&v)[kD]) {
@@ -192,17 +213,23 @@ __device__ __forceinline__ size_t tok_off(const TcBwd& p, int b, int y, int x, i
   return (((size_t)b * p.H + y) * p.W + x) * (size_t)p.heads * kD + (size_t)h * kD;
 }
 
-// Bounded wait on phase `parity` of the MMA barrier; false (and the status
-// recorded) if it gave up.
+// Bounded wait on phase `parity` of the MMA barrier, by thread 0 alone (the
+// issuer; it sleeps in hardware between probes) while the other threads wait
+// at the CTA barrier that follows, issuing nothing; every thread then orders
+// its TMEM reads after the MMAs with tcgen05.fence::after_thread_sync.  Returns
+// false on every thread (and records the status) if the wait gave up.
 __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t parity, int* status) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!ptx::mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitLimit) {
-      atomicOr(status, (int)SWIN_ERR_TIMEOUT);
-      return false;
-    }
-  return true;
+  bool ok = true;
+  if (threadIdx.x == 0 && !ptx::mbar_try_wait(bar, parity)) {
+    const long long t0 = clock64();
+    while (!ptx::mbar_try_wait_sleep(bar, parity, 20000u))
+      if (clock64() - t0 > kWaitLimit) {
+        atomicOr(status, (int)SWIN_ERR_TIMEOUT);
+        ok = false;
+        break;
+      }
+  }
+  return __syncthreads_and(ok);
 }
 
 template <typename TG>
@@ -225,9 +252,10 @@ __device__ __forceinline__ void store_grad<__nv_bfloat16>(__nv_bfloat16* dst, co
 // Shared memory common to both kernels, after the operand tiles.
 struct SmemCommon {
   float rc[2 * 64 * 8], rs[2 * 64 * 8];  // RoPE cos / sin [axis][p][t]
-  float colf[kBlk];                      // per block column: 1/|k| (q kernel) or 1/(tau |q|) (kv kernel)
-  int coff[kBlk];                        // per block column: iy (2M-1) + ix of its token in the rectangle
-  float lse2[kBlk], dsum[kBlk];          // kv kernel: statistics of the block's queries
+  // per block column, double-buffered with the operand blocks:
+  float colf[2][kBlk];                   // 1/|k| (q kernel) or 1/(tau |q|) (kv kernel)
+  int coff[2][kBlk];                     // iy (2M-1) + ix of its token in the rectangle
+  float lse2[2][kBlk], dsum[2][kBlk];    // kv kernel: statistics of the block's queries
   double red[1 + 16];                    // CTA sums: d(tau), d(omega)
   uint64_t mma_bar;
   uint32_t tmem_base;
@@ -267,11 +295,9 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_q(const __grid_constant__ TcB
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* qs = smem;                  // Q tile, fp16 (128 rows)
   uint8_t* gs = qs + kTileB;           // dO tile, fp16
-  uint8_t* ks = gs + kTileB;           // K block, fp16 (64 rows)
-  uint8_t* vs = ks + kBlkB;            // V block, fp16
-  uint8_t* qlo = vs + kBlkB;           // mode 2: lo parts of the rotated Q tile
-  uint8_t* klo = qlo + kTileB;         //         and K block
-  SmemCommon* sc = reinterpret_cast<SmemCommon*>(klo + kBlkB);
+  uint8_t* qlo = gs + kTileB;          // mode 2: lo parts of the rotated Q tile
+  uint8_t* kvb = qlo + kTileB;         // two buffers of [K block | V block | K lo parts] (64 rows each)
+  SmemCommon* sc = reinterpret_cast<SmemCommon*>(kvb + 2 * 3 * kBlkB);
   float* tab = reinterpret_cast<float*>(sc + 1);  // (2M-1)^2 table entries x log2 e (TABLE)
   const int R = 2 * p.M - 1, RR = R * R;
   double* dtab = reinterpret_cast<double*>(tab + (TABLE ? ((RR + 1) & ~1) : 0));  // d(table) sums
@@ -346,152 +372,173 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_q(const __grid_constant__ TcB
   constexpr uint32_t idDQ = ptx::idesc_f16(0, 0, 0, 1, kD, kRows);
   const uint64_t qd = ptx::smem_desc(ptx::smem_addr(qs), 16, 512, ptx::kSwizzle64B);
   const uint64_t gd = ptx::smem_desc(ptx::smem_addr(gs), 16, 512, ptx::kSwizzle64B);
-  const uint64_t kd = ptx::smem_desc(ptx::smem_addr(ks), 16, 512, ptx::kSwizzle64B);
-  const uint64_t vd = ptx::smem_desc(ptx::smem_addr(vs), 16, 512, ptx::kSwizzle64B);
   const uint64_t qld = ptx::smem_desc(ptx::smem_addr(qlo), 16, 512, ptx::kSwizzle64B);
-  const uint64_t kld = ptx::smem_desc(ptx::smem_addr(klo), 16, 512, ptx::kSwizzle64B);
+  // buffer x: K at kvb + 3 x kBlkB, V after it, K lo parts after that
+  auto kbuf = [&](int x) { return kvb + 3 * x * kBlkB; };
+  auto kdesc = [&](int x, int part) {
+    return ptx::smem_desc(ptx::smem_addr(kbuf(x) + part * kBlkB), 16, 512, ptx::kSwizzle64B);
+  };
   uint32_t phase = 0;
   bool ok = true;
 
   float m2 = -INFINITY, l = 0.f, u = 0.f;  // pass 1: running max (log2), sum, sum of p dP
   float lse2 = 0.f, Dv = 0.f;
   const int nkb = (rc.n + kBlk - 1) / kBlk;
-  for (int pass = 0; pass < 2 && ok; ++pass) {
-    for (int kb = 0; kb < nkb && ok; ++kb) {
-      const int k0 = kb * kBlk, nk = min(kBlk, rc.n - k0);
-      // ---- K and V rows of the block: threads 0-63 take K, 64-127 V
-      {
-        const int r = tid & (kBlk - 1);
-        const bool isk = tid < kBlk;
-        const int tk = k0 + r;
-        if (isk) sc->coff[r] = rc.off(min(tk, rc.n - 1), R);  // masked keys: a valid row, weight 0
-        bool hit = false;
-        if (r < nk) {
-          float v[kD];
-          const size_t off = tok_off(p, b, rc.Y(tk), rc.X(tk), h);
-          if (isk) {
-            load_row(p.k + off, v);
-            if (MODE == 1) {
-              bool c;
-              sc->colf[r] = 1.f / clamped_norm(v, c);
-            }
-            prep_row<MODE>(v, rc.PY(tk), rc.PX(tk), sc->rc, sc->rs);
-            hit = MODE == 2 ? store_row_f16_split(ks, klo, r, v) : store_row_f16(ks, r, v);
-          } else {
-            load_row(p.v + off, v);
-            hit = store_row_f16(vs, r, v);
-          }
-        } else {
-          zero_row(isk ? ks : vs, r);
-          if (isk && MODE == 2) zero_row(klo, r);
-          if (isk && MODE == 1) sc->colf[r] = 0.f;
+  const int nsteps = 2 * nkb;  // pass 1 then pass 2 over the key blocks; step g uses buffer g & 1
+  // Threads 0-63 carry K rows of a block, 64-127 V rows.  A step's rows are
+  // fetched (registers) while the previous step computes, and stored once its
+  // buffer is free: the wait on a step's S / dP commit also covers the dQ
+  // MMAs issued before it, the last readers of the other buffer.
+  const int lr = tid & (kBlk - 1);
+  const bool isk = tid < kBlk;
+  RawRow pre;
+  auto fetch = [&](int g) {
+    const int tk = (g % nkb) * kBlk + lr;
+    if (tk < rc.n) fetch_row((isk ? p.k : p.v) + tok_off(p, b, rc.Y(tk), rc.X(tk), h), pre);
+  };
+  auto stash = [&](int g) {
+    const int x = g & 1, tk = (g % nkb) * kBlk + lr;
+    uint8_t* kt = kbuf(x);
+    bool hit = false;
+    if (isk) sc->coff[x][lr] = rc.off(min(tk, rc.n - 1), R);  // masked keys: a valid row, weight 0
+    if (tk < rc.n) {
+      float v[kD];
+      unpack_row(pre, v);
+      if (isk) {
+        if (MODE == 1) {
+          bool c;
+          sc->colf[x][lr] = 1.f / clamped_norm(v, c);
         }
-        if (hit) sc->range_hit = 1;
+        prep_row<MODE>(v, rc.PY(tk), rc.PX(tk), sc->rc, sc->rs);
+        hit = MODE == 2 ? store_row_f16_split(kt, kt + 2 * kBlkB, lr, v) : store_row_f16(kt, lr, v);
+      } else {
+        hit = store_row_f16(kt + kBlkB, lr, v);
       }
-      ptx::fence_proxy_async_smem();
+    } else {
+      zero_row(isk ? kt : kt + kBlkB, lr);
+      if (isk && MODE == 2) zero_row(kt + 2 * kBlkB, lr);
+      if (isk && MODE == 1) sc->colf[x][lr] = 0.f;
+    }
+    if (hit) sc->range_hit = 1;
+  };
+  fetch(0);
+  stash(0);
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  for (int g = 0; g < nsteps && ok; ++g) {
+    const int x = g & 1, pass = g / nkb, kb = g % nkb;
+    const int k0 = kb * kBlk, nk = min(kBlk, rc.n - k0);
+    const uint64_t kd = kdesc(x, 0), vd = kdesc(x, 1), kld = kdesc(x, 2);
+    // ---- S = Q K^T, dP = dO V^T (the commit also covers the previous dQ MMAs)
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      ptx::mma_ss(tS, qd, kd, idS, 0);
+      ptx::mma_ss(tS, qd + 2, kd + 2, idS, 1);
+      if (MODE == 2) {  // + Q_lo K_hi^T + Q_hi K_lo^T
+        ptx::mma_ss(tS, qld, kd, idS, 1);
+        ptx::mma_ss(tS, qld + 2, kd + 2, idS, 1);
+        ptx::mma_ss(tS, qd, kld, idS, 1);
+        ptx::mma_ss(tS, qd + 2, kld + 2, idS, 1);
+      }
+      ptx::mma_ss(tP, gd, vd, idS, 0);
+      ptx::mma_ss(tP, gd + 2, vd + 2, idS, 1);
+      ptx::mma_commit(&sc->mma_bar);
+    }
+    if (g + 1 < nsteps) fetch(g + 1);  // in flight during the MMAs and the softmax
+    ok = wait_mma(&sc->mma_bar, phase, p.status);
+    phase ^= 1;
+    if (!ok) break;
+    ptx::tc_fence_after();
+    const float* colf = sc->colf[x];
+    const int* coff = sc->coff[x];
+    // the block's 64 keys in two halves of 32 (TMEM columns 32 hf ..)
+    for (int hf = 0; hf < 2; ++hf) {
+      uint32_t sr[32], dr[32];
+      ptx::tmem_ld32(tS + 32 * hf + lane_off, sr);
+      ptx::tmem_ld32(tP + 32 * hf + lane_off, dr);
+      ptx::tmem_wait_ld();
+      // logit of key j of this half in the log2 domain; masked keys -inf
+      auto logit = [&](int j) {
+        const int jj = 32 * hf + j;
+        float xv = MODE == 1 ? __uint_as_float(sr[j]) * srow * colf[jj] : __uint_as_float(sr[j]) * srow;
+        SWIN_DCHECK(p.status, !TABLE || (qbase - coff[jj] >= 0 && qbase - coff[jj] < RR));
+        if (TABLE) xv += tab[qbase - coff[jj]];
+        return jj < nk ? xv : -INFINITY;
+      };
+      if (pass == 0) {
+        float mb = m2;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mb = fmaxf(mb, logit(j));
+        const float c = ptx::ex2_approx(m2 - mb);  // 0 at the first half (m2 = -inf)
+        l *= c;
+        u *= c;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float pj = ptx::ex2_approx(logit(j) - mb);
+          l += pj;
+          u = fmaf(pj, __uint_as_float(dr[j]), u);
+        }
+        m2 = mb;
+      } else {
+        // dl = P (dP - D); dS = dl * (d logit / d raw product), fp16 into TMEM
+        uint32_t pk[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          float dl[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int jj = 32 * hf + j + e;
+            const float pj = ptx::ex2_approx(logit(j + e) - lse2);  // 0 for masked keys
+            dl[e] = row_ok ? pj * (__uint_as_float(dr[j + e]) - Dv) : 0.f;
+            if (want_T && row_ok && jj < nk) atomicAdd(&dtab[qbase - coff[jj]], (double)dl[e]);
+          }
+          float a0 = dl[0] * dscale, a1 = dl[1] * dscale;
+          if (MODE == 1) {
+            a0 *= colf[32 * hf + j];
+            a1 *= colf[32 * hf + j + 1];
+          }
+          if (fabsf(a0) >= 65504.f || fabsf(a1) >= 65504.f) sc->range_hit = 1;
+          pk[j / 2] = ptx::pack_f16x2_sat(a0, a1);
+        }
+        ptx::tmem_st16(tDS + 16 * hf + lane_off, pk);
+      }
+    }
+    if (pass == 0 && kb == nkb - 1) {
+      lse2 = m2 + __log2f(l);
+      Dv = u / l;
+      if (row_ok)
+        p.stats[(((size_t)b * p.H + rc.Y(tq)) * p.W + rc.X(tq)) * p.heads + h] = make_double2((double)lse2, (double)Dv);
+    }
+    if (pass == 1) {
+      ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncthreads();
-      // ---- S = Q K^T, dP = dO V^T
+      // ---- dQ += dS K (A = dS from TMEM, B = K as MN-major [keys x d]); not
+      // waited for here: the next step's S / dP commit covers it
       if (tid == 0) {
         ptx::tc_fence_after();
-        ptx::mma_ss(tS, qd, kd, idS, 0);
-        ptx::mma_ss(tS, qd + 2, kd + 2, idS, 1);
-        if (MODE == 2) {  // + Q_lo K_hi^T + Q_hi K_lo^T
-          ptx::mma_ss(tS, qld, kd, idS, 1);
-          ptx::mma_ss(tS, qld + 2, kd + 2, idS, 1);
-          ptx::mma_ss(tS, qd, kld, idS, 1);
-          ptx::mma_ss(tS, qd + 2, kld + 2, idS, 1);
-        }
-        ptx::mma_ss(tP, gd, vd, idS, 0);
-        ptx::mma_ss(tP, gd + 2, vd + 2, idS, 1);
-        ptx::mma_commit(&sc->mma_bar);
-      }
-      ok = wait_mma(&sc->mma_bar, phase, p.status);
-      phase ^= 1;
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-      ptx::tc_fence_after();
-      // the block's 64 keys in two halves of 32 (TMEM columns 32 hf ..)
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t sr[32], dr[32];
-        ptx::tmem_ld32(tS + 32 * hf + lane_off, sr);
-        ptx::tmem_ld32(tP + 32 * hf + lane_off, dr);
-        ptx::tmem_wait_ld();
-        // logit of key j of this half in the log2 domain; masked keys -inf
-        auto logit = [&](int j) {
-          const int jj = 32 * hf + j;
-          float xv = MODE == 1 ? __uint_as_float(sr[j]) * srow * sc->colf[jj] : __uint_as_float(sr[j]) * srow;
-          SWIN_DCHECK(p.status, !TABLE || (qbase - sc->coff[jj] >= 0 && qbase - sc->coff[jj] < RR));
-          if (TABLE) xv += tab[qbase - sc->coff[jj]];
-          return jj < nk ? xv : -INFINITY;
-        };
-        if (pass == 0) {
-          float mb = m2;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) mb = fmaxf(mb, logit(j));
-          const float c = ptx::ex2_approx(m2 - mb);  // 0 at the first half (m2 = -inf)
-          l *= c;
-          u *= c;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float pj = ptx::ex2_approx(logit(j) - mb);
-            l += pj;
-            u = fmaf(pj, __uint_as_float(dr[j]), u);
-          }
-          m2 = mb;
-        } else {
-          // dl = P (dP - D); dS = dl * (d logit / d raw product), fp16 into TMEM
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float dl[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int jj = 32 * hf + j + e;
-              const float pj = ptx::ex2_approx(logit(j + e) - lse2);  // 0 for masked keys
-              dl[e] = row_ok ? pj * (__uint_as_float(dr[j + e]) - Dv) : 0.f;
-              if (want_T && row_ok && jj < nk) atomicAdd(&dtab[qbase - sc->coff[jj]], (double)dl[e]);
-            }
-            float a0 = dl[0] * dscale, a1 = dl[1] * dscale;
-            if (MODE == 1) {
-              a0 *= sc->colf[32 * hf + j];
-              a1 *= sc->colf[32 * hf + j + 1];
-            }
-            if (fabsf(a0) >= 65504.f || fabsf(a1) >= 65504.f) sc->range_hit = 1;
-            pk[j / 2] = ptx::pack_f16x2_sat(a0, a1);
-          }
-          ptx::tmem_st16(tDS + 16 * hf + lane_off, pk);
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          ptx::mma_ts(tDQ, tDS + kk * 8, kd + (uint64_t)(kk * 1024 >> 4), idDQ, (kb > 0 || kk > 0) ? 1u : 0u);
+          if (MODE == 2) ptx::mma_ts(tDQ, tDS + kk * 8, kld + (uint64_t)(kk * 1024 >> 4), idDQ, 1u);
         }
       }
-      if (pass == 0 && kb == nkb - 1) {
-        lse2 = m2 + __log2f(l);
-        Dv = u / l;
-        if (row_ok)
-          p.stats[(((size_t)b * p.H + rc.Y(tq)) * p.W + rc.X(tq)) * p.heads + h] =
-              make_double2((double)lse2, (double)Dv);
-      }
-      if (pass == 1) {
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncthreads();
-        // ---- dQ += dS K (A = dS from TMEM, B = K as MN-major [keys x d])
-        if (tid == 0) {
-          ptx::tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {
-            ptx::mma_ts(tDQ, tDS + kk * 8, kd + (uint64_t)(kk * 1024 >> 4), idDQ, (kb > 0 || kk > 0) ? 1u : 0u);
-            if (MODE == 2) ptx::mma_ts(tDQ, tDS + kk * 8, kld + (uint64_t)(kk * 1024 >> 4), idDQ, 1u);
-          }
-          ptx::mma_commit(&sc->mma_bar);
-        }
-        ok = wait_mma(&sc->mma_bar, phase, p.status);
-        phase ^= 1;
-        ok = __syncthreads_and(ok);
-      }
-      // the next block overwrites K / V in shared memory and S / dP in TMEM
-      ptx::tc_fence_before();
-      __syncthreads();
     }
+    // the next step's buffer: its last readers (step g - 1's MMAs) are complete
+    if (g + 1 < nsteps) stash(g + 1);
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
+  // the last dQ MMAs
+  if (ok) {
+    if (tid == 0) {
+      ptx::tc_fence_after();
+      ptx::mma_commit(&sc->mma_bar);
+    }
+    ok = wait_mma(&sc->mma_bar, phase, p.status);
+    phase ^= 1;
   }
 
   // ---- epilogue: dq from the accumulated gradient of the prepared q
@@ -547,11 +594,9 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* ks = smem;          // K tile, fp16 (128 rows)
   uint8_t* vs = ks + kTileB;   // V tile, fp16
-  uint8_t* qs = vs + kTileB;   // Q block, fp16 (64 rows)
-  uint8_t* gs = qs + kBlkB;    // dO block, fp16
-  uint8_t* klo = gs + kBlkB;   // mode 2: lo parts of the rotated K tile
-  uint8_t* qlo = klo + kTileB; //         and Q block
-  SmemCommon* sc = reinterpret_cast<SmemCommon*>(qlo + kBlkB);
+  uint8_t* klo = vs + kTileB;  // mode 2: lo parts of the rotated K tile
+  uint8_t* qgb = klo + kTileB; // two buffers of [Q block | dO block | Q lo parts] (64 rows each)
+  SmemCommon* sc = reinterpret_cast<SmemCommon*>(qgb + 2 * 3 * kBlkB);
   float* tab = reinterpret_cast<float*>(sc + 1);
   const int R = 2 * p.M - 1, RR = R * R;
 
@@ -622,56 +667,71 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
   constexpr uint32_t idAcc = ptx::idesc_f16(0, 0, 0, 1, kD, kRows);
   const uint64_t kd = ptx::smem_desc(ptx::smem_addr(ks), 16, 512, ptx::kSwizzle64B);
   const uint64_t vd = ptx::smem_desc(ptx::smem_addr(vs), 16, 512, ptx::kSwizzle64B);
-  const uint64_t qd = ptx::smem_desc(ptx::smem_addr(qs), 16, 512, ptx::kSwizzle64B);
-  const uint64_t gd = ptx::smem_desc(ptx::smem_addr(gs), 16, 512, ptx::kSwizzle64B);
   const uint64_t kld = ptx::smem_desc(ptx::smem_addr(klo), 16, 512, ptx::kSwizzle64B);
-  const uint64_t qld = ptx::smem_desc(ptx::smem_addr(qlo), 16, 512, ptx::kSwizzle64B);
+  auto qbuf = [&](int x) { return qgb + 3 * x * kBlkB; };
+  auto qdesc = [&](int x, int part) {
+    return ptx::smem_desc(ptx::smem_addr(qbuf(x) + part * kBlkB), 16, 512, ptx::kSwizzle64B);
+  };
   uint32_t phase = 0;
   bool ok = true;
 
   const int nqb = (rc.n + kBlk - 1) / kBlk;
-  for (int qb = 0; qb < nqb && ok; ++qb) {
-    const int q0 = qb * kBlk, nq = min(kBlk, rc.n - q0);
-    // ---- Q and dO rows of the block (threads 0-63 Q, 64-127 dO) and statistics
-    {
-      const int r = tid & (kBlk - 1);
-      const bool isq = tid < kBlk;
-      const int tq = q0 + r;
-      if (isq) sc->coff[r] = rc.off(min(tq, rc.n - 1), R);
-      bool hit = false;
-      if (r < nq) {
-        float v[kD];
-        const size_t off = tok_off(p, b, rc.Y(tq), rc.X(tq), h);
-        if (isq) {
-          load_row(p.q + off, v);
-          if (MODE == 1) {
-            bool c;
-            sc->colf[r] = 1.f / (clamped_norm(v, c) * t_eff);
-          }
-          prep_row<MODE>(v, rc.PY(tq), rc.PX(tq), sc->rc, sc->rs);
-          hit = MODE == 2 ? store_row_f16_split(qs, qlo, r, v) : store_row_f16(qs, r, v);
-          const double2 st = p.stats[(((size_t)b * p.H + rc.Y(tq)) * p.W + rc.X(tq)) * p.heads + h];
-          sc->lse2[r] = (float)st.x;
-          sc->dsum[r] = (float)st.y;
-        } else {
-          load_row(p.dout + off, v);
-          hit = store_row_f16(gs, r, v);
-        }
-      } else {
-        zero_row(isq ? qs : gs, r);
-        if (isq && MODE == 2) zero_row(qlo, r);
-        if (isq) {
-          sc->colf[r] = 0.f;
-          sc->lse2[r] = INFINITY;  // exp2(x - inf) = 0: no weight for padding columns
-          sc->dsum[r] = 0.f;
-        }
-      }
-      if (hit) sc->range_hit = 1;
+  // Threads 0-63 carry Q rows (and their statistics) of a query block, 64-127
+  // dO rows; block qb + 1 is fetched while qb computes and stored once its
+  // buffer is free (the wait on S^T / dP^T of qb covers the dV / dK MMAs of
+  // qb - 1, that buffer's last readers).
+  const int lr = tid & (kBlk - 1);
+  const bool isq = tid < kBlk;
+  RawRow pre;
+  double2 pst = make_double2(0.0, 0.0);
+  auto fetch = [&](int qb) {
+    const int tq = qb * kBlk + lr;
+    if (tq < rc.n) {
+      const size_t off = tok_off(p, b, rc.Y(tq), rc.X(tq), h);
+      fetch_row((isq ? p.q : p.dout) + off, pre);
+      if (isq) pst = p.stats[(((size_t)b * p.H + rc.Y(tq)) * p.W + rc.X(tq)) * p.heads + h];
     }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-    // ---- S^T = K Q^T, dP^T = V dO^T
+  };
+  auto stash = [&](int qb) {
+    const int x = qb & 1, tq = qb * kBlk + lr;
+    uint8_t* qt = qbuf(x);
+    bool hit = false;
+    if (isq) sc->coff[x][lr] = rc.off(min(tq, rc.n - 1), R);
+    if (tq < rc.n) {
+      float v[kD];
+      unpack_row(pre, v);
+      if (isq) {
+        if (MODE == 1) {
+          bool c;
+          sc->colf[x][lr] = 1.f / (clamped_norm(v, c) * t_eff);
+        }
+        prep_row<MODE>(v, rc.PY(tq), rc.PX(tq), sc->rc, sc->rs);
+        hit = MODE == 2 ? store_row_f16_split(qt, qt + 2 * kBlkB, lr, v) : store_row_f16(qt, lr, v);
+        sc->lse2[x][lr] = (float)pst.x;
+        sc->dsum[x][lr] = (float)pst.y;
+      } else {
+        hit = store_row_f16(qt + kBlkB, lr, v);
+      }
+    } else {
+      zero_row(isq ? qt : qt + kBlkB, lr);
+      if (isq && MODE == 2) zero_row(qt + 2 * kBlkB, lr);
+      if (isq) {
+        sc->colf[x][lr] = 0.f;
+        sc->lse2[x][lr] = INFINITY;  // exp2(x - inf) = 0: no weight for padding columns
+        sc->dsum[x][lr] = 0.f;
+      }
+    }
+    if (hit) sc->range_hit = 1;
+  };
+  fetch(0);
+  stash(0);
+  ptx::fence_proxy_async_smem();
+  ptx::tc_fence_before();
+  __syncthreads();
+  for (int qb = 0; qb < nqb && ok; ++qb) {
+    const int x = qb & 1;
+    const uint64_t qd = qdesc(x, 0), gd = qdesc(x, 1), qld = qdesc(x, 2);
+    // ---- S^T = K Q^T, dP^T = V dO^T (the commit also covers the previous dV / dK MMAs)
     if (tid == 0) {
       ptx::tc_fence_after();
       ptx::mma_ss(tS, kd, qd, idS, 0);
@@ -686,11 +746,15 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
       ptx::mma_ss(tP, vd + 2, gd + 2, idS, 1);
       ptx::mma_commit(&sc->mma_bar);
     }
+    if (qb + 1 < nqb) fetch(qb + 1);  // in flight during the MMAs and the softmax
     ok = wait_mma(&sc->mma_bar, phase, p.status);
     phase ^= 1;
-    ok = __syncthreads_and(ok);
     if (!ok) break;
     ptx::tc_fence_after();
+    const float* colf = sc->colf[x];
+    const int* coff = sc->coff[x];
+    const float* lse2 = sc->lse2[x];
+    const float* dsum = sc->dsum[x];
     // the block's 64 queries in two halves of 32
     for (int hf = 0; hf < 2; ++hf) {
       uint32_t sr[32], dr[32];
@@ -704,14 +768,14 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int ii = 32 * hf + i + e;
-          const float s = __uint_as_float(sr[i + e]);
-          float x = MODE == 1 ? s * srow * sc->colf[ii] : s * srow;
-          SWIN_DCHECK(p.status, !TABLE || (sc->coff[ii] - kbase >= 0 && sc->coff[ii] - kbase < RR));
-          if (TABLE) x += tab[sc->coff[ii] - kbase];
-          const float pj = row_ok ? ptx::ex2_approx(x - sc->lse2[ii]) : 0.f;
-          const float dl = pj * (__uint_as_float(dr[i + e]) - sc->dsum[ii]);
+          const float sv = __uint_as_float(sr[i + e]);
+          float xv = MODE == 1 ? sv * srow * colf[ii] : sv * srow;
+          SWIN_DCHECK(p.status, !TABLE || (coff[ii] - kbase >= 0 && coff[ii] - kbase < RR));
+          if (TABLE) xv += tab[coff[ii] - kbase];
+          const float pj = row_ok ? ptx::ex2_approx(xv - lse2[ii]) : 0.f;
+          const float dl = pj * (__uint_as_float(dr[i + e]) - dsum[ii]);
           pv[e] = pj;
-          dsv[e] = MODE == 1 ? dl * sc->colf[ii] : dl * dscale;
+          dsv[e] = MODE == 1 ? dl * colf[ii] : dl * dscale;
         }
         if (fabsf(dsv[0]) >= 65504.f || fabsf(dsv[1]) >= 65504.f) sc->range_hit = 1;
         pk[i / 2] = ptx::pack_f16x2(pv[0], pv[1]);
@@ -723,7 +787,8 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
     __syncthreads();
-    // ---- dV += P^T dO, dK += dS^T Q (B operands MN-major [queries x d])
+    // ---- dV += P^T dO, dK += dS^T Q (B operands MN-major [queries x d]); not
+    // waited for here: the next block's S^T / dP^T commit covers them
     if (tid == 0) {
       ptx::tc_fence_after();
 #pragma unroll
@@ -733,13 +798,20 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
         ptx::mma_ts(tDK, tDS + kk * 8, qd + (uint64_t)(kk * 1024 >> 4), idAcc, acc);
         if (MODE == 2) ptx::mma_ts(tDK, tDS + kk * 8, qld + (uint64_t)(kk * 1024 >> 4), idAcc, 1u);
       }
+    }
+    if (qb + 1 < nqb) stash(qb + 1);
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
+  // the last dV / dK MMAs
+  if (ok) {
+    if (tid == 0) {
+      ptx::tc_fence_after();
       ptx::mma_commit(&sc->mma_bar);
     }
     ok = wait_mma(&sc->mma_bar, phase, p.status);
     phase ^= 1;
-    ok = __syncthreads_and(ok);
-    ptx::tc_fence_before();
-    __syncthreads();
   }
 
   float drope[16];
@@ -878,7 +950,7 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
       const int r = tid & (kBlk - 1);
       const bool isk = tid < kBlk;
       const int tk = k0 + r;
-      if (isk) sc->coff[r] = rc.off(min(tk, rc.n - 1), R);
+      if (isk) sc->coff[0][r] = rc.off(min(tk, rc.n - 1), R);
       bool hit = false;
       if (r < nk) {
         float v[kD];
@@ -887,7 +959,7 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
           load_row(p.k + off, v);
           if (MODE == 1) {
             bool c;
-            sc->colf[r] = 1.f / clamped_norm(v, c);
+            sc->colf[0][r] = 1.f / clamped_norm(v, c);
           }
           prep_row<MODE>(v, rc.PY(tk), rc.PX(tk), sc->rc, sc->rs);
           hit = MODE == 2 ? store_row_f16_split(ks, klo, r, v) : store_row_f16(ks, r, v);
@@ -898,7 +970,7 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
       } else {
         zero_row(isk ? ks : vs, r);
         if (isk && MODE == 2) zero_row(klo, r);
-        if (isk && MODE == 1) sc->colf[r] = 0.f;
+        if (isk && MODE == 1) sc->colf[0][r] = 0.f;
       }
       if (hit) sc->range_hit = 1;
     }
@@ -919,7 +991,6 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
     }
     ok = wait_mma(&sc->mma_bar, phase, p.status);
     phase ^= 1;
-    ok = __syncthreads_and(ok);
     if (!ok) break;
     ptx::tc_fence_after();
     uint32_t sr[2][32];
@@ -928,8 +999,8 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
     ptx::tmem_wait_ld();
     auto logit = [&](int jj) {
       const float sv = __uint_as_float(sr[jj >> 5][jj & 31]);
-      float xv = MODE == 1 ? sv * srow * sc->colf[jj] : sv * srow;
-      if (TABLE) xv += tab[qbase - sc->coff[jj]];
+      float xv = MODE == 1 ? sv * srow * sc->colf[0][jj] : sv * srow;
+      if (TABLE) xv += tab[qbase - sc->coff[0][jj]];
       return jj < nk ? xv : -INFINITY;
     };
     float mb = -INFINITY;
@@ -971,7 +1042,6 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
     }
     ok = wait_mma(&sc->mma_bar, phase, p.status);
     phase ^= 1;
-    ok = __syncthreads_and(ok);
     ptx::tc_fence_before();
     __syncthreads();
   }
@@ -997,14 +1067,14 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
 
 size_t smem_q(int M, bool table) {
   const int RR = (2 * M - 1) * (2 * M - 1);
-  size_t s = 3 * kTileB + 3 * kBlkB + sizeof(SmemCommon);
+  size_t s = 3 * kTileB + 6 * kBlkB + sizeof(SmemCommon);
   if (table) s += sizeof(float) * ((RR + 1) & ~1) + sizeof(double) * RR;
   return s;
 }
 
 size_t smem_kv(int M, bool table) {
   const int RR = (2 * M - 1) * (2 * M - 1);
-  return 3 * kTileB + 3 * kBlkB + sizeof(SmemCommon) + (table ? sizeof(float) * RR : 0);
+  return 3 * kTileB + 6 * kBlkB + sizeof(SmemCommon) + (table ? sizeof(float) * RR : 0);
 }
 
 template <int MODE, bool TABLE, typename TG>
