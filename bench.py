@@ -235,15 +235,15 @@ FP32_LANES_PER_SM = 128  # B200: fp32 FMA lanes per SM per clock
 
 
 def fwd_kernel(w: syn.Workload) -> str:
-    """The kernel the library runs this workload's forward on: the TMA
-    tensor-core kernel (bf16, d = 32, shifted windows, no bias table above
-    M = 32), the rectangle tensor-core kernel (bf16, d = 32, interleaved
-    windows, M <= 32) or the CUDA cores."""
+    """The kernel the library runs this workload's forward on: the rectangle
+    tensor-core kernel (bf16, d = 32, M <= 32, interleaved windows or M <= 8),
+    the TMA tensor-core kernel (other bf16, d = 32 shifted windows, no bias
+    table above M = 32) or the CUDA cores."""
     has_table = w.mode != 2 and w.bias
+    if w.dtype == "bf16" and w.d == 32 and w.M <= 32 and (w.partition == 1 or w.M <= 8):
+        return "fwd_tc_rect"
     if w.dtype == "bf16" and w.d == 32 and w.partition == 0 and (not has_table or w.M <= 32):
         return "attn_tc"
-    if w.dtype == "bf16" and w.d == 32 and w.partition == 1 and w.M <= 32:
-        return "fwd_tc_rect"
     return "attn_simt"
 
 

@@ -156,11 +156,13 @@ swin_status swin_cpb_eval_form(int M, int heads, const swin_cpb_weights* g, swin
  * Asynchronous; q/k/v must stay valid until the stream reaches the call.
  *
  * Arithmetic of the bf16, d == 32 path (tcgen05 tensor cores; taken when
- * there is no bias table or M <= 32, else the CUDA-core path runs): q.k
- * products of the bf16 inputs accumulate in fp32 (modes 0 and 1; mode 1
- * applies 1/|q|, 1/|k| and 1/tau in fp32 afterwards, and the bias is added in
- * fp32); mode 2 rotates q and k in fp32 and multiplies them as fp16, q scaled
- * by an exact power of two.  Probabilities (at most 2^8 times the running
+ * there is no bias table or M <= 32, else the CUDA-core path runs; windows of
+ * at most 64 tokens, M <= 8, use a kernel that loads rows into shared memory
+ * instead of TMA tiles): q.k products of the bf16 inputs accumulate in fp32
+ * (modes 0 and 1; mode 1 applies 1/|q|, 1/|k| and 1/tau in fp32 afterwards,
+ * and the bias is added in fp32); mode 2 rotates q and k in fp32 and
+ * multiplies them as fp16 (q scaled by an exact power of two; for M <= 8 as
+ * fp16 hi + lo parts).  Probabilities (at most 2^8 times the running
  * maximum's) and V are carried in fp16, sums in fp32, and the row sum is
  * accumulated from the same fp16 probabilities that weight V.  A rotated k
  * entry or a V entry of magnitude 65504 or more saturates; the kernel then

@@ -182,13 +182,15 @@ swin_status swin_window_attn_fwd_ex(const void* q, const void* k, const void* v,
   a.tau = tau; a.table = table; a.rope = rope_freqs;
   a.status = swin::status_word();
   if (!a.status) return fail(SWIN_ERR_CUDA, "could not resolve the device status word");
-  // tensor-core path: bf16, d = 32, shifted windows; a bias table must fit its
-  // shared-memory slot (M <= 32)
+  // tensor cores, bf16 and d = 32.  Interleaved windows, and windows of at most
+  // 64 tokens (M <= 8: one query tile and one key block each, where the
+  // rectangle kernel measured faster, 0.134 against 0.145 ms on Swin-T stage 1),
+  // take the kernel over row-loaded rectangles; other shifted windows the TMA
+  // kernel, whose bias-table slot holds M <= 32.
+  if (dt == SWIN_BF16 && d == 32 && M <= 32 && (partition == SWIN_PARTITION_INTERLEAVED || M <= 8))
+    return swin::launch_attn_fwd_tc_rect(a, out_dt == SWIN_F32, st);
   if (dt == SWIN_BF16 && d == 32 && partition == SWIN_PARTITION_SHIFTED && (table == nullptr || M <= 32))
     return swin::launch_attn_tc(a, out_dt == SWIN_F32, st);
-  // interleaved windows: the tensor-core kernel over strided rectangles
-  if (dt == SWIN_BF16 && d == 32 && partition == SWIN_PARTITION_INTERLEAVED && M <= 32)
-    return swin::launch_attn_fwd_tc_rect(a, out_dt == SWIN_F32, st);
   return swin::launch_attn_simt(a, dt == SWIN_BF16, out_dt == SWIN_F32, st);
 }
 
