@@ -22,10 +22,12 @@ namespace swin {
 namespace {
 
 std::mutex g_lt_mu;
-cublasLtHandle_t g_lt = nullptr;
+constexpr int kMaxDevices = 64;
+cublasLtHandle_t g_lt[kMaxDevices] = {};  // one per device ordinal
 
-// (dtype, m, n, k) -> heuristic algorithm; a GEMM shape is planned once.
-std::map<std::tuple<int, int, int, int>, cublasLtMatmulAlgo_t> g_algos;
+// (device, dtype, m, n, k) -> heuristic algorithm; a GEMM shape is planned
+// once per device.
+std::map<std::tuple<int, int, int, int, int>, cublasLtMatmulAlgo_t> g_algos;
 
 swin_status lt_fail(const char* what, cublasStatus_t st) {
   return fail(SWIN_ERR_CUDA, "cuBLASLt %s failed (status %d)", what, (int)st);
@@ -35,12 +37,16 @@ swin_status lt_fail(const char* what, cublasStatus_t st) {
 // X and W fp32 or bf16, Y fp32.
 swin_status gemm_xwt(const void* X, const void* Wt, float* Y, bool bf16, int rows, int n, int k,
                      cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return fail(SWIN_ERR_CUDA, "could not resolve the current device");
   std::lock_guard<std::mutex> lock(g_lt_mu);
   cublasStatus_t st;
-  if (!g_lt) {
-    st = cublasLtCreate(&g_lt);
+  if (!g_lt[dev]) {
+    st = cublasLtCreate(&g_lt[dev]);
     if (st != CUBLAS_STATUS_SUCCESS) return lt_fail("create", st);
   }
+  cublasLtHandle_t lt = g_lt[dev];
   const cudaDataType_t t = bf16 ? CUDA_R_16BF : CUDA_R_32F, to = CUDA_R_32F;
   // Column-major view: Y^T (n x rows) = W (n x k) . X^T (k x rows), where the
   // row-major W buffer is W^T in column-major (k x n), hence op(A) = T.
@@ -62,7 +68,7 @@ swin_status gemm_xwt(const void* X, const void* Wt, float* Y, bool bf16, int row
       ret = lt_fail("layout", st);
       break;
     }
-    const auto key = std::make_tuple((int)bf16, n, rows, k);
+    const auto key = std::make_tuple(dev, (int)bf16, n, rows, k);
     auto it = g_algos.find(key);
     if (it == g_algos.end()) {
       cublasLtMatmulPreference_t pref = nullptr;
@@ -72,7 +78,7 @@ swin_status gemm_xwt(const void* X, const void* Wt, float* Y, bool bf16, int row
                                            sizeof(zero_ws));
       cublasLtMatmulHeuristicResult_t res;
       int found = 0;
-      st = cublasLtMatmulAlgoGetHeuristic(g_lt, op, la, lb, lc, lc, pref, 1, &res, &found);
+      st = cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, lc, lc, pref, 1, &res, &found);
       cublasLtMatmulPreferenceDestroy(pref);
       if (st != CUBLAS_STATUS_SUCCESS || found < 1) {
         ret = fail(SWIN_ERR_UNSUPPORTED, "cuBLASLt has no algorithm for a %d x %d x %d GEMM", rows, n, k);
@@ -80,7 +86,7 @@ swin_status gemm_xwt(const void* X, const void* Wt, float* Y, bool bf16, int row
       }
       it = g_algos.emplace(key, res.algo).first;
     }
-    st = cublasLtMatmul(g_lt, op, &one, Wt, la, X, lb, &zero, Y, lc, Y, lc, &it->second, nullptr, 0, stream);
+    st = cublasLtMatmul(lt, op, &one, Wt, la, X, lb, &zero, Y, lc, Y, lc, &it->second, nullptr, 0, stream);
     if (st != CUBLAS_STATUS_SUCCESS) ret = lt_fail("matmul", st);
   } while (false);
   if (lc) cublasLtMatrixLayoutDestroy(lc);
