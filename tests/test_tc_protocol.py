@@ -7,6 +7,9 @@ in any order, each issuer's MMA commits complete in issue order, and the
 online-softmax rescale happens at random.  Random interleavings over the real
 per-CTA work-item sequences of every workload must finish with no deadlock and
 with no wait whose parity could match a phase two or more completions old.
+The tensor-memory hazard is checked too: S(b) overwrites the buffer that
+holds P(b - 2), so PV(b - 2) must be issued before it (a thread's MMAs run in
+issue order).
 """
 import random
 
@@ -95,7 +98,7 @@ class Deadlock(Exception):
     pass
 
 
-def run(items, mode, seed, rescale_p=0.2, early_pv=True):
+def run(items, mode, seed, rescale_p=0.2, early_pv=True, pv_lag=2):
     rng = random.Random(seed)
     bars = {}
 
@@ -162,12 +165,13 @@ def run(items, mode, seed, rescale_p=0.2, early_pv=True):
             rel2 = not shared
             for j, uu in enumerate(mine):
                 st = uu % S
-                while npv + 2 <= b:
+                while npv + pv_lag <= b:
                     yield from issue_pv(npv); npv += 1
                 if early_pv and npv < b and u_last + S <= uu:
                     yield from issue_pv(npv); npv += 1
                 if j == 0: yield W(("q_ready", g, qs), qpar)
                 yield W(("kv_ready", st), uu // S)
+                assert npv + 2 > b, "S(%d) issued before PV(%d)" % (b, b - 2)
                 c = [("s_full", g, b & 1)]
                 if j == len(mine) - 1: c.append(("q_empty", g, qs))
                 mmaq[g].append(c)
@@ -281,3 +285,11 @@ def test_model_catches_the_deadlock_it_guards_against():
             run(items, 2, seed, early_pv=False)
     for seed in range(4):
         run(items, 2, seed)
+
+
+def test_model_catches_the_tmem_hazard():
+    """An issuer that lets PV fall three blocks behind would overwrite P(b - 2)
+    with S(b) before PV(b - 2) read it; the model rejects it."""
+    items = items_for(16, 112, 112, 3, 32, 16, 0, 148)
+    with pytest.raises(AssertionError):
+        run(items, 2, 0, pv_lag=3)

@@ -19,9 +19,9 @@
 //               [B][H][W][heads][d] with 64-byte swizzle, no multicast
 //   warps 1, 2  tcgen05.mma issuers, one thread each: warp 1 + g issues the
 //               MMAs of softmax warpgroup g; warp 1 owns TMEM
-//   warps 3, 12-15  operand prep in shared memory: K unit-normalisation
-//               (mode 1), RoPE rotation of Q and K (mode 2), per-row
-//               1/(tau |q|) (mode 1), V to fp16
+//   warps 3, 12-15  operand prep in shared memory, one row per thread: K
+//               unit-normalisation (mode 1), RoPE rotation of Q and K
+//               (mode 2), per-row 1/(tau |q|) (mode 1), V to fp16
 //   warps 4-7   softmax of warpgroup 0 (one TMEM lane = one query row)
 //   warps 8-11  softmax of warpgroup 1
 // TMEM per softmax warpgroup g (128 lanes): two score buffers X0, X1 of 96
@@ -34,11 +34,12 @@
 //
 // Softmax: online, with the running maximum kept until a block exceeds it by
 // more than 8 (log2 units), so O is rescaled rarely; P in fp16 (values up to
-// 2^8) keeps that accurate.  V is converted to fp16 by the prep warps; the
-// constant column c = 1 of [V | c] makes the same MMAs accumulate the row sum
-// of the fp16 P, so O / l uses exactly the probabilities that weighted V.
-// V entries of magnitude 65504 or more saturate and record
-// SWIN_ERR_UNSUPPORTED in the status word.
+// 2^8) keeps that accurate: bf16 P, which would spare the V conversion, leaves
+// errors of 2.6 % of the output RMS on sharp cosine attention.  V is converted
+// to fp16 by the prep warps; the constant column c = 1 of [V | c] makes the
+// same MMAs accumulate the row sum of the fp16 P, so O / l uses exactly the
+// probabilities that weighted V.  V entries of magnitude 65504 or more
+// saturate and record SWIN_ERR_UNSUPPORTED in the status word.
 //
 // Precision of the score operands: mode 0 multiplies the bf16 inputs as they
 // are; mode 1 also multiplies the raw inputs and applies 1/|q| (per row),
@@ -623,7 +624,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
       // 160 threads (warps 3 and 12-15); work in half rows (16 channels):
       // the two halves of a row sit in adjacent lanes, and each half of a
       // RoPE row rotates along one axis only.
-      const int pt = warp < 4 ? (int)threadIdx.x - 96 : (int)threadIdx.x - 384 + 32;  // 0..159
+      // Row work goes to warps 12-15, one per SM sub-partition, so that every
+      // softmax warp shares its sub-partition with the same prep load (warp 3
+      // only takes part in the arrivals): query row (warp - 12) * 32 + lane,
+      // key row (warp - 12) * 24 + lane.
+      const int prow_q = warp >= 12 ? (warp - 12) * 32 + lane : 1 << 20;
+      const int prow_k = warp >= 12 && lane < 24 ? (warp - 12) * 24 + lane : 1 << 20;
       uint32_t qu[2] = {0, 0}, ku = 0;
       bool ok = true;
       bool range_hit = false;  // a rotated K or a V entry saturated the fp16 range
@@ -645,31 +651,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           uint8_t* tile = qbuf + (g * 2 + qs) * kTileBytes;
           const float te = MODE == 1 ? fmaxf(__ldg(p.tau + t.h), kTauMin) : 1.f;
           if (MODE != 0) {
-#pragma unroll 1
-            for (int u = pt; u < 2 * 128; u += kPrepThreads) {  // uniform trip count per lane pair
-              const int r = u >> 1, h = u & 1;
-              const bool act = r < qrows;
-              float v[16];
-              if (act) load_half_bf16(tile, r, h, v);
-              else for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            // one query row per thread (a tile has at most 128 rows)
+            const int r = prow_q;
+            if (r < qrows) {
+              float v0[16], v1[16];
+              load_half_bf16(tile, r, 0, v0);
+              load_half_bf16(tile, r, 1, v1);
               if (MODE == 1) {
-                float ss = half_sumsq(v);
-                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-                if (act && h == 0)
-                  qscale[(g * 2 + qs) * 128 + r] = kLog2eF / (fmaxf(sqrtf(ss), kNormEps) * te);
+                const float ss = half_sumsq(v0) + half_sumsq(v1);
+                qscale[(g * 2 + qs) * 128 + r] = kLog2eF / (fmaxf(sqrtf(ss), kNormEps) * te);
               } else {
-                if (act) {
-                  const int pr = rp[r];
-                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + rq.tile * rq.R + (pr & 0xFFFF), 63), rcos,
-                            rsin);
-                }
-                float m = half_absmax(v);
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                const float sc = pow2_scale(m);  // exact per-row scale, undone in the softmax
-                if (act) {
-                  store_half_f16(tile, r, h, v, sc);
-                  if (h == 0) qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
-                }
+                // the row's scale needs both halves rotated: the first half is
+                // rotated again for the store (fewer live registers)
+                const int pr = rp[r];
+                const int pos0 = min(py0 + rq.tile * rq.R + (pr & 0xFFFF), 63), pos1 = px0 + (pr >> 16);
+                rope_half(v0, 0, pos0, rcos, rsin);
+                rope_half(v1, 1, pos1, rcos, rsin);
+                const float sc = pow2_scale(fmaxf(half_absmax(v0), half_absmax(v1)));  // exact, undone in the softmax
+                store_half_f16(tile, r, 1, v1, sc);
+                load_half_bf16(tile, r, 0, v0);
+                rope_half(v0, 0, pos0, rcos, rsin);
+                store_half_f16(tile, r, 0, v0, sc);
+                qscale[(g * 2 + qs) * 128 + r] = kLog2eF * rsqrtf(32.0f) / sc;
               }
             }
             ptx::fence_proxy_async_smem();
@@ -688,34 +691,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           if (!ok) break;
           uint8_t* ktile = kvbuf + st * 2 * kTileBytes;
           uint8_t* vtile = ktile + kTileBytes;
-          // units: half h of K row r and half h of V row r (r < krows <= 96);
-          // fp16 with saturation, a saturated entry is reported after the loop.
-          // Trip counts are uniform per warp (the shuffle below needs all lanes).
+          // one key row per thread (a block has at most 96 rows)
+          {
+            const int r = prow_k;
+            if (r < krows) {
 #pragma unroll 1
-          for (int un = pt; un < 2 * kBlk; un += kPrepThreads) {
-          const int r = un >> 1, h = un & 1;
-          const bool act = r < krows;
-          if (MODE != 0) {
-            float v[16];
-            if (act) load_half_bf16(ktile, r, h, v);
-            else for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            if (MODE == 1) {
-              float ss = half_sumsq(v);
-              ss += __shfl_xor_sync(0xffffffffu, ss, 1);
-              if (act && h == 0) kcol[st * 128 + r] = 1.0f / fmaxf(sqrtf(ss), kNormEps);
-            } else if (act) {
-              const int pr = rp[r];
-              rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + j * rk.Rk + (pr & 0xFFFF), 63), rcos, rsin);
-              range_hit |= half_absmax(v) >= 65504.0f;
-              store_half_f16(ktile, r, h, v, 1.0f);
+              for (int h = 0; h < 2; ++h) {
+                float v[16];
+                load_half_bf16(vtile, r, h, v);
+                range_hit |= half_absmax(v) >= 65504.0f;
+                store_half_f16(vtile, r, h, v, 1.0f);
+              }
             }
           }
-          if (act) {
-            float v[16];
-            load_half_bf16(vtile, r, h, v);
-            range_hit |= half_absmax(v) >= 65504.0f;
-            store_half_f16(vtile, r, h, v, 1.0f);
-          }
+          if (MODE != 0) {
+            const int r = prow_k;
+            if (r < krows) {
+              if (MODE == 1) {
+                float v0[16], v1[16];
+                load_half_bf16(ktile, r, 0, v0);
+                load_half_bf16(ktile, r, 1, v1);
+                kcol[st * 128 + r] = 1.0f / fmaxf(sqrtf(half_sumsq(v0) + half_sumsq(v1)), kNormEps);
+              } else {
+                const int pr = rp[r];
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                  float v[16];
+                  load_half_bf16(ktile, r, h, v);
+                  rope_half(v, h, h ? px0 + (pr >> 16) : min(py0 + j * rk.Rk + (pr & 0xFFFF), 63), rcos, rsin);
+                  range_hit |= half_absmax(v) >= 65504.0f;
+                  store_half_f16(ktile, r, h, v, 1.0f);
+                }
+              }
+            }
           }
           ptx::fence_proxy_async_smem();
           ptx::mbar_arrive(&bars->kv_ready[st]);
@@ -843,7 +851,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
         if (!ok) break;
         SWIN_TC_MARK(1);
         ptx::tc_fence_after();
-        const uint32_t tS = tX + (blk & 1) * kBlk;
+        const uint32_t tS = tX + (blk & 1) * kBlk, tP = tS;  // P written over the scores
         float2 x[kBlk / 2];  // scores as packed pairs (keys 2c, 2c+1)
         {
           uint32_t r0[32], r1[32], r2[32];
@@ -990,7 +998,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
           const float2 e = __ffma2_rn(x[c], make_float2(ea, ea), make_float2(eb, eb));
           pa[c] = ptx::pack_f16x2(ptx::ex2_approx(e.x), ptx::ex2_approx(e.y));
         }
-        ptx::tmem_st32(tS, pa);
+        ptx::tmem_st32(tP, pa);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const float2 e = __ffma2_rn(x[32 + c], make_float2(ea, ea), make_float2(eb, eb));
@@ -1021,7 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
             ptx::tmem_st1(tO + 32, __float_as_uint(__uint_as_float(pl) * factor));
           }
         }
-        ptx::tmem_st16(tS + 32, pb);
+        ptx::tmem_st16(tP + 32, pb);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[g][blk & 1]);
