@@ -57,6 +57,7 @@
 
 #include "sm100_ptx.cuh"
 #include "swin_common.cuh"
+#include "tma_encode.cuh"
 
 // Phase markers for external timing builds; they compile to nothing here.
 #ifndef SWIN_TC_MARK
@@ -1071,26 +1072,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const __grid_const
 }
 
 // ------------------------------------------------------------------ host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// The driver entry point, looked up once; a function-local static with an
-// initialiser is thread-safe in C++11 and later.
-EncodeTiledFn encode_fn() {
-  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      return reinterpret_cast<EncodeTiledFn>(p);
-    return nullptr;
-  }();
-  return fn;
-}
-
 bool encode_map(CUtensorMap* m, const void* base, const AttnArgs& a, int lx, int R) {
-  EncodeTiledFn fn = encode_fn();
+  EncodeTiledFn fn = tma_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[5] = {32, (cuuint64_t)a.heads, (cuuint64_t)a.W, (cuuint64_t)a.H, (cuuint64_t)a.B};
   const cuuint64_t row = 64;  // bytes of one head
@@ -1115,6 +1098,20 @@ swin_status launch_mode(const TcParams& p, int grid, cudaStream_t stream) {
 }
 
 }  // namespace
+
+// The driver entry point, looked up once; a function-local static with an
+// initialiser is thread-safe in C++11 and later.
+EncodeTiledFn tma_encode_fn() {
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
+  return fn;
+}
 
 static long long g_tc_wait_limit = 4000000000ll;  // ~2 s at 2 GHz
 static int g_tc_debug_flags = 0;

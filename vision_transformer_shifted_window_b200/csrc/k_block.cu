@@ -5,11 +5,14 @@
 // result is layer-normalised before it joins the residual path:
 //   q | k | v = x W_qkv^T + b_qkv
 //   out       = x + LN(a W_o^T + b_o) * gamma + beta
-// The projections are plain GEMMs (cuBLASLt, fp32 accumulation, no cuBLAS
-// workspace) whose fp32 results land in the caller's workspace; the bias, the
-// post-norm and the residual add are this file's kernels, in fp32, and each
-// output element is rounded once (a bf16 output is the fp32 one rounded to
-// nearest even).
+// bf16 inputs with C = heads * d a multiple of 32 up to 128 (96 for the qkv
+// projection, whose weights must stay in shared memory) take the fused
+// tensor-core kernels of k_block_tc.cu.  Otherwise the projections are plain
+// GEMMs (cuBLASLt, fp32 accumulation, no cuBLAS workspace) whose fp32 results
+// land in the caller's workspace, and the bias, the post-norm and the
+// residual add are this file's kernels.  Either way the arithmetic after the
+// products is fp32 and each output element is rounded once (a bf16 output is
+// the fp32 one rounded to nearest even).
 #include <cublasLt.h>
 
 #include <map>
@@ -241,6 +244,7 @@ void launch_postnorm(const void* x, const float* y, void* out, const float* b_o,
 
 swin_status launch_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
                             bool bf16, bool f32_out, int tokens, int C, float* y, cudaStream_t stream) {
+  if (block_tc_supported(C, bf16, false)) return launch_qkv_proj_tc(x, w_qkv, b_qkv, q, k, v, f32_out, tokens, C, stream);
   swin_status s = gemm_xwt(x, w_qkv, y, bf16, tokens, 3 * C, C, stream);
   if (s != SWIN_OK) return s;
   const long long n = (long long)tokens * C;
@@ -260,6 +264,8 @@ swin_status launch_proj_postnorm(const void* a, const void* w_o, const float* b_
                                  const float* gamma, const float* beta, float eps, void* out, bool bf16, bool f32_out,
                                  int tokens, int C, float* y, cudaStream_t stream) {
   if (C > kMaxC) return fail(SWIN_ERR_UNSUPPORTED, "post-norm supports C <= %d, got %d", kMaxC, C);
+  if (block_tc_supported(C, bf16, true))
+    return launch_proj_postnorm_tc(a, w_o, b_o, x, gamma, beta, eps, out, f32_out, tokens, C, stream);
   swin_status s = gemm_xwt(a, w_o, y, bf16, tokens, C, C, stream);
   if (s != SWIN_OK) return s;
   const int per = (C + 31) / 32;

@@ -106,6 +106,14 @@ bool attn_bwd_tc_supported(const BwdArgs& a, bool bf16_in);
 // The tensor-core forward over arbitrary rectangles (bf16, d = 32, M <= 32),
 // used for the interleaved partition.
 swin_status launch_attn_fwd_tc_rect(const AttnArgs& a, bool f32_out, cudaStream_t stream);
+// Fused tensor-core block steps (k_block_tc.cu): bf16 inputs, C % 32 == 0,
+// C <= 128, weights and tiles within shared memory.
+bool block_tc_supported(int C, bool bf16_in, bool postnorm);
+swin_status launch_qkv_proj_tc(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
+                               bool f32_out, int tokens, int C, cudaStream_t stream);
+swin_status launch_proj_postnorm_tc(const void* a, const void* w_o, const float* b_o, const void* x,
+                                    const float* gamma, const float* beta, float eps, void* out, bool f32_out,
+                                    int tokens, int C, cudaStream_t stream);
 swin_status launch_attn_bwd_tc(const BwdArgs& a, bool f32_grad, cudaStream_t stream);
 
 }  // namespace swin
