@@ -284,13 +284,17 @@ size_t swin_window_attn_bwd_workspace_size(int B, int H, int W, int heads, int d
  * dense row-major, of dtype dt (fp32 or bf16), with C = heads * d channels per
  * token; the token order is the caller's ([B][H][W] for the attention).
  * Weights follow the usual linear-layer layout [out][in]; biases, gamma and
- * beta are fp32.  The projections are cuBLASLt GEMMs with fp32 accumulation
- * into the caller's workspace (fp32); the bias, the post-norm and the
- * residual add are this library's kernels, in fp32, and every output element
- * is rounded once: outputs of dtype out_dt (== dt, or SWIN_F32 for SWIN_BF16
- * inputs; a bf16 output is the fp32 one rounded to nearest even).  Pointers
- * 16-byte aligned, workspaces 256-byte aligned; C a multiple of 8.
- * Asynchronous on the stream. */
+ * beta are fp32.  For bf16 inputs with C a multiple of 32 (at most 96 for
+ * the qkv projection, 128 for the post-norm) each step is one tensor-core
+ * kernel (tcgen05, bf16 products, fp32 accumulation, the epilogue in fp32)
+ * that leaves the workspace untouched; otherwise the projection is a
+ * cuBLASLt GEMM with fp32 accumulation into the caller's workspace (fp32)
+ * and the bias, the post-norm and the residual add are this library's
+ * kernels, in fp32.  Either way every output element is rounded once:
+ * outputs of dtype out_dt (== dt, or SWIN_F32 for SWIN_BF16 inputs; a bf16
+ * output is the fp32 one rounded to nearest even).  Pointers 16-byte
+ * aligned, workspaces 256-byte aligned; C a multiple of 8.  Asynchronous on
+ * the stream. */
 
 /* q = x Wq^T + bq, k = x Wk^T + bk, v = x Wv^T + bv, with
  *   x        [tokens][C]
