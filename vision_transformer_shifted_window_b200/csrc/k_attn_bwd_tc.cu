@@ -63,6 +63,25 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
 
+// One token's head row (32 bf16) as four 16-byte words, and those words as floats.
+__device__ __forceinline__ void load_raw(const __nv_bfloat16* src, uint4 (&w)[4]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) w[c] = __ldg(s4 + c);
+}
+
+__device__ __forceinline__ void unpack_row(const uint4 (&w)[4], float (&v)[kD]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t u[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[8 * c + 2 * e] = __uint_as_float(u[e] << 16);
+      v[8 * c + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+    }
+  }
+}
+
 // One token's head row (32 bf16) into floats.
 __device__ __forceinline__ void load_row(const __nv_bfloat16* src, float (&v)[kD]) {
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
@@ -862,17 +881,21 @@ __global__ void __launch_bounds__(kThreads) bwd_tc_kv(const __grid_constant__ Tc
 }
 
 // ============================================================== forward
-// The forward pass over arbitrary rectangles (used for interleaved windows,
-// whose strided windows the TMA kernel does not gather): one CTA per query
-// tile, S = Q K^T per 64-key block (RoPE operands split into fp16 hi + lo as
-// in the backward), the softmax in fp32 with the running maximum kept until a
-// block exceeds it by more than 8 (log2 units; probabilities then <= 2^8,
-// exact in fp16's range), P as fp16 into TMEM and O += P V on the tensor
-// cores.  The row sum is taken from the same fp16 probabilities that weight
-// V, so O / l normalises exactly the weights applied.  128 TMEM columns
-// (S 64, P 32, O 32) per CTA.
+// The forward pass over arbitrary rectangles (interleaved windows, whose
+// strided windows the TMA kernel does not gather, and windows of at most 64
+// tokens): persistent CTAs, each walking work items (one query tile of one
+// rectangle of one (image, head); heads outermost, so the bias table of a
+// head is loaded once for several items).  Per item: the Q rows and the first
+// K / V block's rows are loaded together, then S = Q K^T per 64-key block
+// (RoPE operands split into fp16 hi + lo as in the backward), the softmax in
+// fp32 with the running maximum kept until a block exceeds it by more than 8
+// (log2 units; probabilities then <= 2^8, exact in fp16's range), P as fp16
+// into TMEM and O += P V on the tensor cores.  The row sum is taken from the
+// same fp16 probabilities that weight V, so O / l normalises exactly the
+// weights applied.  128 TMEM columns (S 64, P 32, O 32) per CTA, allocated
+// once.
 template <int MODE, bool TABLE, typename TO>
-__global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ TcBwd p) {
+__global__ void __launch_bounds__(kThreads, 4) fwd_tc_rect(const __grid_constant__ TcBwd p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* qs = smem;
   uint8_t* ks = qs + kTileB;
@@ -882,15 +905,7 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
   SmemCommon* sc = reinterpret_cast<SmemCommon*>(klo + kBlkB);
   float* tab = reinterpret_cast<float*>(sc + 1);
   const int R = 2 * p.M - 1, RR = R * R;
-
-  const int rect = blockIdx.x / p.tiles, tile = blockIdx.x % p.tiles;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const Rect rc = rect_of(p, rect);
-  const int t0 = tile * kRows;
-  if (t0 >= rc.n) return;
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int tq = t0 + tid;
-  const bool row_ok = tq < rc.n;
 
   if (tid == 0) {
     ptx::mbar_init(&sc->mma_bar, 1);
@@ -902,31 +917,6 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
     ptx::tmem_relinquish();
   }
   if (MODE == 2) build_rope(p.rope, p.M, sc->rc, sc->rs);
-  if (TABLE)
-    for (int i = tid; i < RR; i += kThreads) tab[i] = __ldg(p.table + (size_t)i * p.heads + h) * kLog2e;
-  __syncthreads();
-
-  const float t_eff = MODE == 1 ? fmaxf(__ldg(p.tau + h), kTauMin) : 1.f;
-  float qn = 1.f;
-  {
-    bool hit = false;
-    if (row_ok) {
-      float qrow[kD];
-      load_row(p.q + tok_off(p, b, rc.Y(tq), rc.X(tq), h), qrow);
-      bool c;
-      if (MODE == 1) qn = clamped_norm(qrow, c);
-      prep_row<MODE>(qrow, rc.PY(tq), rc.PX(tq), sc->rc, sc->rs);
-      hit = MODE == 2 ? store_row_f16_split(qs, qlo, tid, qrow) : store_row_f16(qs, tid, qrow);
-    } else {
-      zero_row(qs, tid);
-      if (MODE == 2) zero_row(qlo, tid);
-    }
-    if (hit) sc->range_hit = 1;
-  }
-  const float srow = MODE == 1 ? kLog2e / (qn * t_eff) : kLog2e * rsqrtf((float)kD);
-  const int qbase = rc.off(row_ok ? tq : t0, R) + (p.M - 1) * (R + 1);
-
-  ptx::fence_proxy_async_smem();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -940,112 +930,163 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
   const uint64_t vd = ptx::smem_desc(ptx::smem_addr(vs), 16, 512, ptx::kSwizzle64B);
   const uint64_t qld = ptx::smem_desc(ptx::smem_addr(qlo), 16, 512, ptx::kSwizzle64B);
   const uint64_t kld = ptx::smem_desc(ptx::smem_addr(klo), 16, 512, ptx::kSwizzle64B);
+  const int nrect = swin_nwin(p.part, p.H, p.M, p.shift) * p.nsx;
+  const long long n_items = (long long)nrect * p.tiles * p.heads * p.B;
   uint32_t phase = 0;
   bool ok = true;
-  float m2 = -INFINITY, l = 0.f;
-  const int nkb = (rc.n + kBlk - 1) / kBlk;
-  for (int kb = 0; kb < nkb && ok; ++kb) {
-    const int k0 = kb * kBlk, nk = min(kBlk, rc.n - k0);
+  int cur_h = -1;
+
+  for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    const int tile = (int)(it % p.tiles);
+    long long rest = it / p.tiles;
+    const int rect = (int)(rest % nrect);
+    rest /= nrect;
+    const int b = (int)(rest % p.B), h = (int)(rest / p.B);
+    const Rect rc = rect_of(p, rect);
+    const int t0 = tile * kRows;
+    if (t0 >= rc.n) continue;  // uniform: the rectangle has fewer tiles
+    const int tq = t0 + tid;
+    const bool row_ok = tq < rc.n;
+    // this thread's rows of the item, loaded together: its Q row and its K
+    // (threads 0-63) or V (64-127) row of the first block
+    const int kr = tid & (kBlk - 1);
+    const bool isk = tid < kBlk;
+    uint4 qraw[4], kvraw[4];
+    if (row_ok) load_raw(p.q + tok_off(p, b, rc.Y(tq), rc.X(tq), h), qraw);
+    if (kr < rc.n) load_raw((isk ? p.k : p.v) + tok_off(p, b, rc.Y(kr), rc.X(kr), h), kvraw);
+    if (TABLE && h != cur_h) {  // uniform: every thread walks the same items
+      for (int i = tid; i < RR; i += kThreads) tab[i] = __ldg(p.table + (size_t)i * p.heads + h) * kLog2e;
+      cur_h = h;
+      __syncthreads();
+    }
+
+    const float t_eff = MODE == 1 ? fmaxf(__ldg(p.tau + h), kTauMin) : 1.f;
+    float qn = 1.f;
     {
-      const int r = tid & (kBlk - 1);
-      const bool isk = tid < kBlk;
-      const int tk = k0 + r;
-      if (isk) sc->coff[0][r] = rc.off(min(tk, rc.n - 1), R);
       bool hit = false;
-      if (r < nk) {
-        float v[kD];
-        const size_t off = tok_off(p, b, rc.Y(tk), rc.X(tk), h);
-        if (isk) {
-          load_row(p.k + off, v);
-          if (MODE == 1) {
-            bool c;
-            sc->colf[0][r] = 1.f / clamped_norm(v, c);
-          }
-          prep_row<MODE>(v, rc.PY(tk), rc.PX(tk), sc->rc, sc->rs);
-          hit = MODE == 2 ? store_row_f16_split(ks, klo, r, v) : store_row_f16(ks, r, v);
-        } else {
-          load_row(p.v + off, v);
-          hit = store_row_f16(vs, r, v);
-        }
+      if (row_ok) {
+        float qrow[kD];
+        unpack_row(qraw, qrow);
+        bool c;
+        if (MODE == 1) qn = clamped_norm(qrow, c);
+        prep_row<MODE>(qrow, rc.PY(tq), rc.PX(tq), sc->rc, sc->rs);
+        hit = MODE == 2 ? store_row_f16_split(qs, qlo, tid, qrow) : store_row_f16(qs, tid, qrow);
       } else {
-        zero_row(isk ? ks : vs, r);
-        if (isk && MODE == 2) zero_row(klo, r);
-        if (isk && MODE == 1) sc->colf[0][r] = 0.f;
+        zero_row(qs, tid);
+        if (MODE == 2) zero_row(qlo, tid);
       }
       if (hit) sc->range_hit = 1;
     }
-    ptx::fence_proxy_async_smem();
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      ptx::tc_fence_after();
-      ptx::mma_ss(tS, qd, kd, idS, 0);
-      ptx::mma_ss(tS, qd + 2, kd + 2, idS, 1);
-      if (MODE == 2) {
-        ptx::mma_ss(tS, qld, kd, idS, 1);
-        ptx::mma_ss(tS, qld + 2, kd + 2, idS, 1);
-        ptx::mma_ss(tS, qd, kld, idS, 1);
-        ptx::mma_ss(tS, qd + 2, kld + 2, idS, 1);
+    const float srow = MODE == 1 ? kLog2e / (qn * t_eff) : kLog2e * rsqrtf((float)kD);
+    const int qbase = rc.off(row_ok ? tq : t0, R) + (p.M - 1) * (R + 1);
+
+    float m2 = -INFINITY, l = 0.f;
+    const int nkb = (rc.n + kBlk - 1) / kBlk;
+    for (int kb = 0; kb < nkb && ok; ++kb) {
+      const int k0 = kb * kBlk, nk = min(kBlk, rc.n - k0);
+      {
+        const int tk = k0 + kr;
+        if (isk) sc->coff[0][kr] = rc.off(min(tk, rc.n - 1), R);
+        bool hit = false;
+        if (kr < nk) {
+          float v[kD];
+          if (kb == 0) {
+            unpack_row(kvraw, v);
+          } else {
+            const size_t off = tok_off(p, b, rc.Y(tk), rc.X(tk), h);
+            load_row((isk ? p.k : p.v) + off, v);
+          }
+          if (isk) {
+            if (MODE == 1) {
+              bool c;
+              sc->colf[0][kr] = 1.f / clamped_norm(v, c);
+            }
+            prep_row<MODE>(v, rc.PY(tk), rc.PX(tk), sc->rc, sc->rs);
+            hit = MODE == 2 ? store_row_f16_split(ks, klo, kr, v) : store_row_f16(ks, kr, v);
+          } else {
+            hit = store_row_f16(vs, kr, v);
+          }
+        } else {
+          zero_row(isk ? ks : vs, kr);
+          if (isk && MODE == 2) zero_row(klo, kr);
+          if (isk && MODE == 1) sc->colf[0][kr] = 0.f;
+        }
+        if (hit) sc->range_hit = 1;
       }
-      ptx::mma_commit(&sc->mma_bar);
-    }
-    ok = wait_mma(&sc->mma_bar, phase, p.status);
-    phase ^= 1;
-    if (!ok) break;
-    ptx::tc_fence_after();
-    uint32_t sr[2][32];
-    ptx::tmem_ld32(tS + lane_off, sr[0]);
-    ptx::tmem_ld32(tS + 32 + lane_off, sr[1]);
-    ptx::tmem_wait_ld();
-    auto logit = [&](int jj) {
-      const float sv = __uint_as_float(sr[jj >> 5][jj & 31]);
-      float xv = MODE == 1 ? sv * srow * sc->colf[0][jj] : sv * srow;
-      if (TABLE) xv += tab[qbase - sc->coff[0][jj]];
-      return jj < nk ? xv : -INFINITY;
-    };
-    float mb = -INFINITY;
-#pragma unroll
-    for (int jj = 0; jj < kBlk; ++jj) mb = fmaxf(mb, logit(jj));
-    // lazy maximum: raised only when this block exceeds it by more than 8
-    float c = 1.f;
-    if (mb > m2 + 8.f) {
-      c = ptx::ex2_approx(m2 - mb);  // 0 at the first block
-      m2 = mb;
-      l *= c;
-    }
-    if (kb > 0 && __any_sync(0xffffffffu, c != 1.f)) {  // rescale O (the previous PV has completed)
-      uint32_t o[32];
-      ptx::tmem_ld32(tO + lane_off, o);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * c);
-      ptx::tmem_st32(tO + lane_off, o);
-    }
-    uint32_t pk[32];
-#pragma unroll
-    for (int jj = 0; jj < kBlk; jj += 2) {
-      const uint32_t w2 = ptx::pack_f16x2(ptx::ex2_approx(logit(jj) - m2), ptx::ex2_approx(logit(jj + 1) - m2));
-      const __half2 hp = *reinterpret_cast<const __half2*>(&w2);
-      l += __low2float(hp) + __high2float(hp);  // the weights V receives
-      pk[jj / 2] = w2;
-    }
-    ptx::tmem_st32(tP + lane_off, pk);
-    ptx::tmem_wait_st();
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        ptx::tc_fence_after();
+        ptx::mma_ss(tS, qd, kd, idS, 0);
+        ptx::mma_ss(tS, qd + 2, kd + 2, idS, 1);
+        if (MODE == 2) {
+          ptx::mma_ss(tS, qld, kd, idS, 1);
+          ptx::mma_ss(tS, qld + 2, kd + 2, idS, 1);
+          ptx::mma_ss(tS, qd, kld, idS, 1);
+          ptx::mma_ss(tS, qd + 2, kld + 2, idS, 1);
+        }
+        ptx::mma_commit(&sc->mma_bar);
+      }
+      ok = wait_mma(&sc->mma_bar, phase, p.status);
+      phase ^= 1;
+      if (!ok) break;
       ptx::tc_fence_after();
+      uint32_t sr[2][32];
+      ptx::tmem_ld32(tS + lane_off, sr[0]);
+      ptx::tmem_ld32(tS + 32 + lane_off, sr[1]);
+      ptx::tmem_wait_ld();
+      // log2-domain logits, formed once (the score registers are reused)
+      float xl[kBlk];
+      float mb = -INFINITY;
 #pragma unroll
-      for (int kk = 0; kk < kBlk / 16; ++kk)
-        ptx::mma_ts(tO, tP + kk * 8, vd + (uint64_t)(kk * 1024 >> 4), idO, (kb > 0 || kk > 0) ? 1u : 0u);
-      ptx::mma_commit(&sc->mma_bar);
+      for (int jj = 0; jj < kBlk; ++jj) {
+        const float sv = __uint_as_float(sr[jj >> 5][jj & 31]);
+        float xv = MODE == 1 ? sv * srow * sc->colf[0][jj] : sv * srow;
+        if (TABLE) xv += tab[qbase - sc->coff[0][jj]];
+        xl[jj] = jj < nk ? xv : -INFINITY;
+        mb = fmaxf(mb, xl[jj]);
+      }
+      // lazy maximum: raised only when this block exceeds it by more than 8
+      float c = 1.f;
+      if (mb > m2 + 8.f) {
+        c = ptx::ex2_approx(m2 - mb);  // 0 at the first block
+        m2 = mb;
+        l *= c;
+      }
+      if (kb > 0 && __any_sync(0xffffffffu, c != 1.f)) {  // rescale O (the previous PV has completed)
+        uint32_t o[32];
+        ptx::tmem_ld32(tO + lane_off, o);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * c);
+        ptx::tmem_st32(tO + lane_off, o);
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int jj = 0; jj < kBlk; jj += 2) {
+        const uint32_t w2 = ptx::pack_f16x2(ptx::ex2_approx(xl[jj] - m2), ptx::ex2_approx(xl[jj + 1] - m2));
+        const __half2 hp = *reinterpret_cast<const __half2*>(&w2);
+        l += __low2float(hp) + __high2float(hp);  // the weights V receives
+        pk[jj / 2] = w2;
+      }
+      ptx::tmem_st32(tP + lane_off, pk);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncthreads();
+      if (tid == 0) {
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          ptx::mma_ts(tO, tP + kk * 8, vd + (uint64_t)(kk * 1024 >> 4), idO, (kb > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(&sc->mma_bar);
+      }
+      ok = wait_mma(&sc->mma_bar, phase, p.status);
+      phase ^= 1;
+      ptx::tc_fence_before();
+      __syncthreads();
     }
-    ok = wait_mma(&sc->mma_bar, phase, p.status);
-    phase ^= 1;
-    ptx::tc_fence_before();
-    __syncthreads();
-  }
-  if (ok) {
+    if (!ok) break;
     ptx::tc_fence_after();
     uint32_t o[32];
     ptx::tmem_ld32(tO + lane_off, o);
@@ -1055,6 +1096,10 @@ __global__ void __launch_bounds__(kThreads) fwd_tc_rect(const __grid_constant__ 
 #pragma unroll
     for (int e = 0; e < kD; ++e) g[e] = __uint_as_float(o[e]) * inv;
     if (row_ok) store_grad<TO>(static_cast<TO*>(p.out) + tok_off(p, b, rc.Y(tq), rc.X(tq), h), g);
+    // the next item's first PV overwrites O: every thread has read it
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -1109,15 +1154,24 @@ swin_status launch_tg(const TcBwd& p, int mode, bool table, cudaStream_t stream)
 
 template <int MODE, bool TABLE, typename TO>
 swin_status launch_fwd_rect(const TcBwd& p, cudaStream_t stream) {
-  const int nsy = swin_nwin(p.part, p.H, p.M, p.shift);
-  const dim3 grid(nsy * p.nsx * p.tiles, p.heads, p.B);
+  const long long items = (long long)swin_nwin(p.part, p.H, p.M, p.shift) * p.nsx * p.tiles * p.heads * p.B;
+  if (items == 0) return SWIN_OK;
   auto kf = fwd_tc_rect<MODE, TABLE, TO>;
   const int RR = (2 * p.M - 1) * (2 * p.M - 1);
-  // 128 TMEM columns per CTA: at most four CTAs per SM (57 KB of shared memory or more)
+  // 128 TMEM columns per CTA: at most four CTAs per SM, which 50 KB of shared
+  // memory or more ensures (a fifth would wait in its TMEM allocation)
   const size_t sm = std::max<size_t>(2 * kTileB + 3 * kBlkB + sizeof(SmemCommon) + (TABLE ? sizeof(float) * RR : 0),
-                                     57 * 1024);
+                                     50 * 1024);
   cudaError_t e = cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  // the occupancy below (and at launch) assumes the largest shared-memory carveout
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kf, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_fwd_rect smem attribute: %s", cudaGetErrorString(e));
+  // persistent: four CTAs per SM, all resident at once (128 registers and at
+  // most ~56 KB of shared memory each)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)std::min<long long>(items, 4LL * sms);
   kf<<<grid, kThreads, sm, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail(SWIN_ERR_CUDA, "attn_fwd_rect launch: %s", cudaGetErrorString(e));
