@@ -3,10 +3,11 @@ host.
 
 Roles: the TMA producer (weights once, then one input tile per work item into
 a ring of S stages), the MMA issuer (one product per output into a ring of
-TMEM accumulator slots) and the epilogue (reads each product's slot, then
-stores).  Each role is a program of mbarrier arrivals and parity waits in the
-kernel's order; TMA copies complete in any order and the issuer's MMA commits
-complete in issue order.  Random interleavings must finish with no deadlock,
+TMEM accumulator slots) and one or two epilogue warpgroups (warpgroup e reads
+the slots of products u with u % nepi == e, then stores).  Each role is a
+program of mbarrier arrivals and parity waits in the kernel's order; TMA
+copies complete in any order and the issuer's MMA commits complete in issue
+order.  Random interleavings must finish with no deadlock,
 no wait whose parity could match a phase two or more completions old, and no
 tensor-memory or shared-memory hazard: a product never overwrites a slot the
 epilogue has not finished reading, and a stage is never reloaded while its
@@ -33,7 +34,7 @@ class Deadlock(Exception):
     pass
 
 
-def run(ntiles, nparts, S, NS, postnorm, seed, slot_wait=True):
+def run(ntiles, nparts, S, NS, postnorm, seed, slot_wait=True, nepi=1):
     rng = random.Random(seed)
     bars = {("w_full",): Bar("w_full", 1)}
     for s in range(S):
@@ -49,7 +50,7 @@ def run(ntiles, nparts, S, NS, postnorm, seed, slot_wait=True):
     tma = []
     mmaq = []  # FIFO of commit lists (in issue order)
     slot_owner = {}  # slot -> product index whose accumulator it holds
-    slot_reading = set()  # slots the epilogue is reading
+    slot_reading = set()  # slots an epilogue warpgroup is reading
     stage_tile = {}  # stage -> tile whose input it holds
     stage_in_use = {}  # stage -> count of readers (MMA, epilogue residual)
 
@@ -81,27 +82,34 @@ def run(ntiles, nparts, S, NS, postnorm, seed, slot_wait=True):
                 u += 1
             mmaq.append([("release", s), ("in_empty", s)])
 
-    def epilogue():
+    def epilogue(ew):
         u = 0
         for i in range(ntiles):
             s = i % S
-            if postnorm:
-                yield W(("in_full", s), i // S)
-                stage_in_use[s] = stage_in_use.get(s, 0) + 1
+            mine = False
             for part in range(nparts):
+                if u % nepi != ew:
+                    u += 1
+                    continue
+                mine = True
                 k = u % NS
                 yield W(("slot_full", k), u // NS)
+                if postnorm:
+                    yield W(("in_full", s), i // S)
+                    stage_in_use[s] = stage_in_use.get(s, 0) + 1
                 assert slot_owner[k] == u, "slot %d holds product %d, expected %d" % (k, slot_owner[k], u)
                 slot_reading.add(k)
                 yield None  # the reads take time
                 slot_reading.discard(k)
                 bars[("slot_empty", k)].arrive(4)
                 u += 1
-            if postnorm:
+            if postnorm and mine:
                 stage_in_use[s] -= 1
                 bars[("in_empty", s)].arrive()
 
-    roles = {"producer": producer(), "mma": mma(), "epilogue": epilogue()}
+    roles = {"producer": producer(), "mma": mma()}
+    for ew in range(nepi):
+        roles["epilogue%d" % ew] = epilogue(ew)
     waiting = {r: None for r in roles}
     alive = set(roles)
 
@@ -142,14 +150,16 @@ PLANS = [(32, 3, 3, 6, False), (64, 3, 3, 6, False), (96, 3, 3, 5, False), (32, 
          (96, 1, 3, 5, True), (128, 1, 2, 4, True)]
 
 
+@pytest.mark.parametrize("nepi", [1, 2])
 @pytest.mark.parametrize("C,nparts,S,NS,postnorm", PLANS)
 @pytest.mark.parametrize("ntiles", [1, 2, 7, 11])
-def test_block_protocol(C, nparts, S, NS, postnorm, ntiles):
+def test_block_protocol(C, nparts, S, NS, postnorm, ntiles, nepi):
     for seed in range(6):
-        run(ntiles, nparts, S, NS, postnorm, seed)
+        run(ntiles, nparts, S, NS, postnorm, seed, nepi=nepi)
 
 
-def test_model_catches_a_missing_slot_wait():
+@pytest.mark.parametrize("nepi", [1, 2])
+def test_model_catches_a_missing_slot_wait(nepi):
     with pytest.raises(AssertionError):
         for seed in range(20):
-            run(11, 3, 3, 5, False, seed, slot_wait=False)
+            run(11, 3, 3, 5, False, seed, slot_wait=False, nepi=nepi)

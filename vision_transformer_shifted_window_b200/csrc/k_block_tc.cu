@@ -16,8 +16,10 @@
 // fp32 one rounded to nearest even.
 //
 // Warps: 0 TMA producer (weights once, then input tiles into a ring of
-// stages), 1 MMA issuer (and TMEM owner), 2-5 epilogue (warp w reads TMEM
-// lanes 32 (w % 4) ...).  Every wait is bounded; on time-out the kernel
+// stages), 1 MMA issuer (and TMEM owner), 2-5 and 6-9 two epilogue
+// warpgroups taking alternate products (warp w reads TMEM lanes
+// 32 (w % 4) ...; one warpgroup where shared memory holds a single set of
+// staging tiles).  Every wait is bounded; on time-out the kernel
 // records SWIN_ERR_TIMEOUT, drains what it issued and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,7 +33,7 @@ namespace {
 
 constexpr int kTok = 128;                // tokens per tile
 constexpr int kChunk = kTok * 64;        // one column chunk of a tile: 128 rows x 64 bytes
-constexpr int kThreadsBlk = 192;
+constexpr int kThreadsBlk = 320;
 constexpr int kMaxSmem = 227 * 1024;
 constexpr long long kWaitLimit = 4000000000ll;  // clock64 cycles (~2 s)
 constexpr int kMaxSlots = 6;                    // TMEM accumulator slots
@@ -45,7 +47,8 @@ struct BlkParams {
   const float* gamma;      // [C] or null (post-norm)
   const float* beta;       // [C] or null (post-norm)
   float eps;
-  int C, nparts, ntiles, nstages, nout;  // nout: staging buffers (1 or 2)
+  int C, nparts, ntiles, nstages, nout;  // nout: staging buffers per epilogue warpgroup (1 or 2)
+  int nepi;                              // epilogue warpgroups (1 or 2)
   int nslots;                            // TMEM accumulator slots of C columns
   int off_w, off_in, off_res, off_out, off_vec, off_bar;
   uint32_t tmem_cols;
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kThreadsBlk, 1) block_tc_kernel(const __grid_c
   uint8_t* sw = smem + p.off_w;      // [KC][N rows][64 B]
   uint8_t* sin = smem + p.off_in;    // [S][KC][128 rows][64 B]
   uint8_t* sres = smem + p.off_res;  // [S][KC][128 rows][64 B]  (post-norm)
-  uint8_t* sout = smem + p.off_out;  // [nout][C * out bytes / 64][128 rows][64 B]
+  uint8_t* sout = smem + p.off_out;  // [nepi][nout][C * out bytes / 64][128 rows][64 B]
   float* sbias = reinterpret_cast<float*>(smem + p.off_vec);  // [N]
   float* sgam = sbias + N;                                    // [C] (post-norm)
   float* sbet = sgam + C;
@@ -244,21 +247,27 @@ __global__ void __launch_bounds__(kThreadsBlk, 1) block_tc_kernel(const __grid_c
       ptx::mma_commit(drain);
       wait_drain(drain, 0);
     }
-  } else {
+  } else if ((warp - 2) >> 2 < p.nepi) {
     // ================================================================ epilogue
-    const int et = threadIdx.x - 64;            // 0..127
+    const int ew = (warp - 2) >> 2;             // epilogue warpgroup: products u with u % nepi == ew
+    const int et = (threadIdx.x - 64) & 127;    // 0..127 within the warpgroup
+    const int bar = 1 + ew;                     // its named barrier
     const int lg = warp & 3;                    // TMEM lane group of this warp
     const int r = lg * 32 + lane;               // row of the tile
     const uint32_t tl = tmem_base + ((uint32_t)(lg * 32) << 16);
+    uint8_t* sout_w = sout + ew * p.nout * stage_bytes;
     int ob = 0;
     bool ok = true;
-    int i = 0, u = 0;  // tiles, (tile, output) products read
+    int i = 0, u = 0;  // tiles, (tile, output) products
     for (int tile = blockIdx.x; tile < p.ntiles && ok; tile += gridDim.x, ++i) {
       const int s = i % S;
+      bool mine_tile = false;  // this warpgroup read the tile's residual rows
       for (int part = 0; part < p.nparts; ++part, ++u) {
+        if (u % p.nepi != ew) continue;
+        mine_tile = true;
         const int k = u % NS;
         ok = __all_sync(0xffffffffu, wait(slot_full + k, (u / NS) & 1) && (!PN || wait(in_full + s, (i / S) & 1)));
-        ok = ptx::named_bar_and(1, 128, ok);
+        ok = ptx::named_bar_and(bar, 128, ok);
         if (!ok) break;
         ptx::tc_fence_after();
         const uint32_t ts = tl + k * C;  // this product's accumulator slot
@@ -286,13 +295,13 @@ __global__ void __launch_bounds__(kThreadsBlk, 1) block_tc_kernel(const __grid_c
           }
           rstd = rsqrtf(ss / (float)C + p.eps);
         }
-        uint8_t* stage = sout + ob * stage_bytes;
+        uint8_t* stage = sout_w + ob * stage_bytes;
         // the store that last read this staging buffer has finished reading it
         if (et == 0) {
           if (p.nout == 2) bulk_wait_read1();
           else bulk_wait_read0();
         }
-        ptx::named_bar_sync(1, 128);
+        ptx::named_bar_sync(bar, 128);
         for (int cc = 0; cc < KC; ++cc) {
           uint32_t v[32];
           ptx::tmem_ld32(ts + cc * 32, v);
@@ -324,7 +333,7 @@ __global__ void __launch_bounds__(kThreadsBlk, 1) block_tc_kernel(const __grid_c
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(slot_empty + k);
         ptx::fence_proxy_async_smem();
-        ptx::named_bar_sync(1, 128);
+        ptx::named_bar_sync(bar, 128);
         if (et == 0) {
           const int nbox = F32 ? C / 16 : C / 32, bw = F32 ? 16 : 32;
           for (int c = 0; c < nbox; ++c) tma_store_2d(&p.map_out[part], stage + c * kChunk, c * bw, tile * kTok);
@@ -333,7 +342,7 @@ __global__ void __launch_bounds__(kThreadsBlk, 1) block_tc_kernel(const __grid_c
         if (p.nout == 2) ob ^= 1;
       }
       if (!ok) break;
-      if (PN && et == 0) ptx::mbar_arrive(in_empty + s);  // residual rows read (the barrier above)
+      if (PN && mine_tile && et == 0) ptx::mbar_arrive(in_empty + s);  // residual rows read (the barrier above)
     }
     if (et == 0) bulk_wait_all();
   }
@@ -372,10 +381,12 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 }  // namespace
 
 // Shared-memory plan: weights, `stages` input (and residual) tiles, `nout`
-// staging tiles, the bias / gamma / beta vectors and the barriers; the ring
-// and staging depths are the largest (3 / 2 at most) that fit.
+// staging tiles per epilogue warpgroup, the bias / gamma / beta vectors and
+// the barriers; two epilogue warpgroups where they fit, then the deepest ring
+// (3 stages at most) and staging (2 tiles at most).
 static bool plan_smem(BlkParams& p, bool pn, bool f32_out) {
   const int C = p.C, N = p.nparts * C;
+  for (int nepi = 2; nepi >= 1; --nepi)
   for (int S = 3; S >= 2; --S)
     for (int nout = 2; nout >= 1; --nout) {
       int off = 0;
@@ -386,7 +397,7 @@ static bool plan_smem(BlkParams& p, bool pn, bool f32_out) {
       p.off_res = off;
       if (pn) off += S * C * kTok * 2;
       p.off_out = off;
-      off += nout * C * kTok * (f32_out ? 4 : 2);
+      off += nepi * nout * C * kTok * (f32_out ? 4 : 2);
       p.off_vec = off;
       off += ((N + 2 * C) * 4 + 15) / 16 * 16;
       p.off_bar = off;
@@ -394,6 +405,7 @@ static bool plan_smem(BlkParams& p, bool pn, bool f32_out) {
       if (off + 1024 <= kMaxSmem) {
         p.nstages = S;
         p.nout = nout;
+        p.nepi = nepi;
         return true;
       }
     }
