@@ -131,3 +131,35 @@ def test_block_rejects_before_launch():
         sa.swin_attn_block_fwd(x, 3, w3, None, w1, None, None, None, 4, 4, 0)
     with pytest.raises(sa.SwinError, match="no shift"):
         sa.swin_attn_block_fwd(x, 3, w3, None, w1, None, None, None, 4, 2, 0, partition=1)
+
+
+@pytest.mark.parametrize("C", [32, 64, 96, 128])
+@pytest.mark.parametrize("tokens", [1, 127, 128, 129, 300, 2000])
+def test_fused_block_kernels_tiles_and_optional_parameters(C, tokens):
+    """The fused tensor-core block kernels (bf16, C a multiple of 32): partial
+    and single tiles, several tiles per CTA, every supported C, with and
+    without bias, gamma and beta; fp32 output against the oracle and the bf16
+    output its RNE, bit for bit."""
+    w = case("bf16", C // 32, 32)
+    p = syn.make_block_inputs(w, B=1, H=1, W=tokens, seed=7 * C + tokens)
+    a = syn.make_block_inputs(w, B=1, H=1, W=tokens, seed=7 * C + tokens + 1)["x"]
+    x = dev(p["x"]).to(torch.bfloat16)
+    wq, wo = dev(p["w_qkv"]).to(torch.bfloat16), dev(p["w_o"]).to(torch.bfloat16)
+    for with_params in (True, False):
+        bq = dev(p["b_qkv"]) if with_params else None
+        got = sa.swin_qkv_proj(x, wq, bq, out_dtype=torch.float32)
+        want = block.qkv_proj(p["x"], p["w_qkv"], p["b_qkv"] if with_params else None)
+        for g, ref in zip(got, want):
+            assert rel_err(g.cpu().numpy(), ref) <= TOL_BF16
+        for g16, g32 in zip(sa.swin_qkv_proj(x, wq, bq), got):
+            assert torch.equal(g32.to(torch.bfloat16).view(torch.int16), g16.view(torch.int16))
+        bo, gam, bet = ((dev(p["b_o"]), dev(p["gamma"]), dev(p["beta"])) if with_params else (None, None, None))
+        args = (dev(a).to(torch.bfloat16), wo, bo, x, gam, bet)
+        got = sa.swin_proj_postnorm_residual(*args, eps=1e-5, out_dtype=torch.float32)
+        want = block.proj_postnorm_residual(a, p["w_o"], p["b_o"] if with_params else None, p["x"],
+                                            p["gamma"] if with_params else None, p["beta"] if with_params else None,
+                                            1e-5)
+        assert rel_err(got.cpu().numpy(), want) <= TOL_BF16
+        g16 = sa.swin_proj_postnorm_residual(*args, eps=1e-5)
+        assert torch.equal(got.to(torch.bfloat16).view(torch.int16), g16.view(torch.int16))
+    assert sa.swin_stream_status() == sa.SWIN_OK
