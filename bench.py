@@ -16,7 +16,12 @@ unless --workload) gives ``value`` (whole-job tokens/s), ``tflops``,
 ``roofline`` (the attention kernel against the measured bf16 peak, DRAM
 traffic from the committed ncu summary of the same kernel source, and
 ``exp_bound``: the share of the all-MUFU exponential bound it reaches) and
-``e2e`` (host buffers, copies in the timed region).  ``workloads`` repeats
+``e2e`` (host buffers, every step's copies in the timed region: the H2D copy
+of q, k, v from pinned host memory and the D2H copy of the output, on their
+own streams with two device buffer sets, so one step's copies overlap its
+neighbours' copies and kernels; steady-state time per step over the loop;
+``e2e.serial_ms_per_step`` is the same step with copies and call in one
+stream).  ``workloads`` repeats
 those figures for every bf16 workload (headline first; --only skips the
 others), with the CPB kernel's time in both forms where a workload has one;
 a workload the tensor-core kernel does not take (Iwin's interleaved windows)
@@ -387,10 +392,52 @@ def time_workload(w: syn.Workload, args, timer, rank: int, world: int, peaks: di
         n_e2e = max(3, min(args.steps, 20))
         etimes = timer.loop(e2e_step, n_e2e, flush_l2=False)
         launches += launches_per_step * n_e2e
-        e_ms = max_over_ranks(_median(etimes), world, device)
+        serial_ms = max_over_ranks(_median(etimes), world, device)
+        # pipelined: step i copies into buffer set i % 2 on the H2D stream,
+        # computes on the library's stream, copies back on the D2H stream;
+        # events order every reuse of a buffer set after its previous step
+        sets = [(q, k, v, out, ws)] + [tuple(torch.empty_like(t) for t in (q, k, v, out)) + (torch.empty_like(ws),)]
+        h2d, d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev = lambda: torch.cuda.Event()
+        in_ready, computed, out_read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+        def pipelined(n):
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            h2d.wait_event(t0)
+            d2h.wait_event(t0)
+            for i in range(n):
+                j = i & 1
+                qq, kk, vv, oo, ww = sets[j]
+                if i >= 2:
+                    h2d.wait_event(computed[j])  # the call of step i - 2 has read this set
+                with torch.cuda.stream(h2d):
+                    qq.copy_(hq, non_blocking=True)
+                    kk.copy_(hk, non_blocking=True)
+                    vv.copy_(hv, non_blocking=True)
+                    in_ready[j].record(h2d)
+                stream.wait_event(in_ready[j])
+                if i >= 2:
+                    stream.wait_event(out_read[j])  # the D2H of step i - 2 has read this output
+                sa.swin_window_attn_fwd(qq, kk, vv, w.M, s, w.mode, out=oo, workspace=ww, stream=stream,
+                                        partition=w.partition, **kw)
+                computed[j].record(stream)
+                d2h.wait_event(computed[j])
+                with torch.cuda.stream(d2h):
+                    hout.copy_(oo, non_blocking=True)
+                    out_read[j].record(d2h)
+            stream.wait_event(out_read[(n - 1) & 1])
+            stream.wait_event(in_ready[(n - 1) & 1])
+            t1.record(stream)
+            torch.cuda.synchronize(device)
+            return t0.elapsed_time(t1) / n
+        pipelined(3)
+        e_ms = max_over_ranks(pipelined(n_e2e), world, device)
+        launches += launches_per_step * n_e2e
         entry["e2e"] = {"value": round(wk["tokens"] * world / (e_ms * 1e-3), 1), "unit": "tokens/s",
                         "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
-                        "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": round(e_ms, 4)}
+                        "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": round(e_ms, 4),
+                        "serial_ms_per_step": round(serial_ms, 4)}
     if sa.swin_stream_status(stream) != 0:
         raise RuntimeError("device status after the timed loops of %s" % w.name)
     del q, k, v, out, ws
