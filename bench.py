@@ -24,8 +24,10 @@ neighbours' copies and kernels; steady-state time per step over the loop;
 stream).  ``workloads`` repeats
 those figures for every bf16 workload (headline first; --only skips the
 others), with the CPB kernel's time in both forms where a workload has one;
-a workload the tensor-core kernel does not take (Iwin's interleaved windows)
-is measured against the CUDA cores' fp32 peak ("bound": "alu").
+every bf16, d = 32 workload runs on a tensor-core kernel (the TMA kernel, or
+the rectangle kernel for interleaved and small windows) and is set against
+the bf16 peak; one that ran on the CUDA cores would be set against their fp32
+peak ("bound": "alu").
 ``backward`` times swin_window_attn_bwd on the same workloads (--no-backward
 skips it); ``block`` times the attention half of a Swin V2 block
 (swin_attn_block_fwd) and its projection steps against HBM (--no-block).
