@@ -37,7 +37,7 @@ def seg_len(k, L, M, s):
     return min(b, L) - a
 
 
-def items_for(B, H, W, heads, M, s, cta, grid):
+def items_for(B, H, W, heads, M, s, cta, grid, pos_major=False):
     """Work items of CTA `cta` in the kernel's order: heads outermost, then
     image, then rows of rectangles; item i of a row takes tiles 2i and 2i+1 of
     the row's tile list (rectangles left to right, each split into query
@@ -65,6 +65,8 @@ def items_for(B, H, W, heads, M, s, cta, grid):
             else:
                 per_hb.append((a[1], 0, False))
     n_items = B * heads * len(per_hb)
+    if pos_major:  # item i: position i // (B heads) of (head, image) i % (B heads)
+        return [per_hb[it // (B * heads)] for it in range(cta, n_items, grid)]
     return [per_hb[it % len(per_hb)] for it in range(cta, n_items, grid)]
 
 
@@ -264,12 +266,15 @@ WORKLOADS = {  # B, H, W, heads, M, shift, mode
 }
 
 
+@pytest.mark.parametrize("pos_major", [False, True])
 @pytest.mark.parametrize("name", sorted(WORKLOADS))
-def test_protocol_no_deadlock_no_parity_alias(name):
+def test_protocol_no_deadlock_no_parity_alias(name, pos_major):
+    """Both item orders: heads outermost (a bias table per head) and
+    position-major (no table)."""
     B, H, W, heads, M, s, mode = WORKLOADS[name]
     grid = 148 if B * H * W > 20000 else 8
     for cta in (0, 1, grid // 3, grid - 1):
-        items = items_for(B, H, W, heads, M, s, cta, grid)
+        items = items_for(B, H, W, heads, M, s, cta, grid, pos_major)
         for seed in range(4):
             run(items, mode, seed)
 

@@ -89,6 +89,8 @@ __device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
 struct TcParams {
   CUtensorMap tmap[3][3];  // [tensor q/k/v][x-class first/middle/last]
   FastDiv div_ipb, div_B, div_mid_items, div_mid_tiles[3];
+  FastDiv div_hb;  // B * heads
+  int pos_major;   // walk items position-major (see decode)
   int lx[3], R[3], Rk[3];  // per x-class: segment width, rows per query tile, rows per K/V block
   // per row class (first, middle, last row of rectangles): height, items,
   // and per x-class the query tiles and K/V blocks of one rectangle
@@ -191,6 +193,15 @@ struct Task {
 __device__ __forceinline__ Task decode(const TcParams& p, long long item) {
   Task t;
   uint32_t i = (uint32_t)item;
+  if (p.pos_major) {
+    // item i is position i / (B heads) of (head, image) i % (B heads): the
+    // round-robin CTAs then see every position class evenly (tile pairs of
+    // full and edge rectangles cost up to 3x apart) instead of a run of
+    // consecutive positions; used without a bias table, whose per-head
+    // reload favours heads outermost
+    const uint32_t pos = fdiv(i, p.div_hb);
+    i = (i - pos * p.div_hb.d) * p.div_ipb.d + pos;
+  }
   uint32_t q = fdiv(i, p.div_ipb);
   uint32_t rem = i - q * p.div_ipb.d;  // item within (head, image)
   i = q;
@@ -1198,6 +1209,8 @@ swin_status launch_attn_tc(const AttnArgs& a, bool f32_out, cudaStream_t stream)
   p.div_ipb = make_fastdiv((uint32_t)ipb);
   p.div_mid_items = make_fastdiv((uint32_t)p.row_items[1]);
   p.div_B = make_fastdiv((uint32_t)a.B);
+  p.div_hb = make_fastdiv((uint32_t)(a.B * a.heads));
+  p.pos_major = a.mode == 2 || a.table == nullptr;  // no per-head bias table to keep
   p.out = a.out;
   p.tau = a.tau;
   p.table = a.table;
