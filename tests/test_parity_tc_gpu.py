@@ -102,3 +102,19 @@ def test_tc_v_out_of_fp16_range_reports_unsupported():
     assert sa.swin_stream_status() == sa.SWIN_ERR_UNSUPPORTED
     sa.swin_window_attn_fwd(q, k, v, 8, 4, 0)
     assert sa.swin_stream_status() == sa.SWIN_OK
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("B,H,W,heads,M,s", [(2, 40, 36, 3, 16, 8), (1, 50, 45, 2, 32, 5), (3, 24, 24, 4, 12, 6)])
+def test_tc_no_bias_table_position_major(B, H, W, heads, M, s, mode):
+    """Without a bias table the kernel walks its work items position-major
+    (all heads and images of one item position, then the next): dot-product
+    and cosine scores with no relative bias, ragged and multi-head shapes."""
+    w = syn.Workload(86, "tc", "bf16", B, H, W, heads, 32, M, (s,), mode, tau=(0.05, 0.2))
+    inp = syn.make_inputs(w, seed=13 * H + W + mode)
+    inp.pop("table", None)
+    for key in ("w1", "b1", "w2", "b2"):
+        inp.pop(key, None)
+    got = gpu_run_bf16_checked(inp, w, s).cpu().numpy()
+    want = oracle_run(inp, w, s)
+    assert rel_err(got, want) <= TOL_BF16
